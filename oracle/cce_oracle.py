@@ -1,0 +1,240 @@
+"""Plain, slow, fp64 CPU oracle for the Cut Cross-Entropy hot path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
+execute this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.  It shares
+no code with the CUDA library (``linear_cross_entropy_cce_b200``) and imports
+nothing from it.
+
+Sources (web pages, cited by title and section):
+  [LM]  "The loss and the mask: Cut Cross-Entropy + FlexAttention (2 papers)",
+        part "Cut Your Losses in Large-Vocabulary Language Models (CCE)":
+        §Contribution, §What transfers to us.
+  [MAP] "Cut Your Losses in Large-Vocabulary Language Models" (research-map
+        entry): §Approach, §Key results, §Limitations.
+  [DE]  "The Defensive Edit: Chunking Cross-Entropy Loss After an OOM Wake-Up
+        Call": §The Trade-Off Analysis / §Assumptions (Assumption 2).
+
+What it computes.  The cross-entropy of row i is the log-sum-exp of its logits
+minus its correct-token logit, the logits being plain dot products
+z_ij = <h_i, e_j> ([LM] §Contribution).  The oracle materialises the logits in
+row slices (the position-chunked CE of [DE]), which the method itself never
+does; that is the point of an oracle.  The backward is the exact gradient of
+sum_i dloss_i * loss_i; with gradient filtering on, softmax entries below the
+threshold are dropped element by element ([LM] §Contribution; [MAP] §Approach).
+A composite head is a list of segments on the logical vocabulary; ids that no
+segment covers form the dead gap whose logits are -inf ([LM] §What transfers
+to us, third bullet).
+
+Readings where the pages are silent (each also listed in the design doc):
+  * no bias, temperature or soft-capping on the logits;
+  * ignored rows (y == ignore_index) have loss = lse = 0 and zero gradient;
+  * a target outside [0, V) or inside the gap yields NaN loss/lse for its row;
+  * the filter drops p_ij < filter_eps (strict), decided on the softmax p
+    itself, never on the target's one-hot term; filter_eps <= 0 means off.
+
+Inputs are bf16 bit patterns (uint16 arrays), widened exactly to fp64; fp64
+arrays are accepted as they are (the finite-difference pin needs them).
+Every function below is pinned by the ``-m "not gpu"`` tests in
+``tests/test_oracle_pins.py``; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, List, Sequence, Tuple
+
+import numpy as np
+
+SLICE_ROWS = 512  # rows per materialised slice ([DE]: chunk the positions)
+
+
+def widen_bf16(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float64, exactly (bf16 is the top half of fp32)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def as_f64(x: np.ndarray) -> np.ndarray:
+    """fp64 arrays pass through (finite-difference tests); bf16 bits widen."""
+    x = np.asarray(x)
+    return x if x.dtype == np.float64 else widen_bf16(x)
+
+
+def _segments_f64(segments) -> List[Tuple[int, int, np.ndarray]]:
+    out = []
+    for begin, end, E in segments:
+        E64 = as_f64(E)
+        assert E64.shape[0] == end - begin
+        out.append((int(begin), int(end), E64))
+    return out
+
+
+def logits_rows(H64: np.ndarray, segs64, V: int) -> np.ndarray:
+    """Logical logit rows z[r, j] = <h_r, e_j>; ids in no segment are -inf.
+
+    [LM] §Contribution (dot-product logits); [LM] §What transfers to us (a
+    dead gap contributes -inf).  Written out on the logical vocabulary on
+    purpose: the segment composition by log-add-exp is *not* reused here.
+    """
+    Z = np.full((H64.shape[0], V), -np.inf)
+    for begin, end, E64 in segs64:
+        Z[:, begin:end] = H64 @ E64.T
+    return Z
+
+
+def logsumexp_rows(Z: np.ndarray) -> np.ndarray:
+    """lse_r = m_r + log sum_j exp(z_rj - m_r), m_r the row max (textbook)."""
+    m = Z.max(axis=1)
+    return m + np.log(np.exp(Z - m[:, None]).sum(axis=1))
+
+
+def _valid_targets(y: np.ndarray, V: int, ignore_index: int, segs64):
+    live = np.zeros(V, dtype=bool)
+    for begin, end, _ in segs64:
+        live[begin:end] = True
+    y = np.asarray(y, dtype=np.int64)
+    ignored = y == ignore_index
+    in_range = (y >= 0) & (y < V)
+    good = np.zeros_like(ignored)
+    good[in_range] = live[y[in_range]]
+    good &= ~ignored
+    bad = ~ignored & ~good
+    return ignored, good, bad
+
+
+def forward(H, segments, y, V: int, ignore_index: int = -100,
+            rows: Iterable[int] | None = None,
+            slice_rows: int = SLICE_ROWS) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-row loss and lse in fp64 for ``rows`` (default: all rows).
+
+    segments: sequence of (vocab_begin, vocab_end, E_bits[end-begin, D]).
+    loss_i = lse_i - z_{i, y_i}  ([LM] §Contribution).
+    Returns arrays indexed like ``rows``.
+    """
+    segs64 = _segments_f64(segments)
+    y = np.asarray(y, dtype=np.int64)
+    rows = np.arange(y.shape[0]) if rows is None else np.asarray(list(rows), dtype=np.int64)
+    ignored, good, bad = _valid_targets(y[rows], V, ignore_index, segs64)
+    loss = np.zeros(rows.shape[0])
+    lse = np.zeros(rows.shape[0])
+    for s in range(0, rows.shape[0], slice_rows):
+        r = rows[s:s + slice_rows]
+        Z = logits_rows(as_f64(H[r]), segs64, V)
+        l = logsumexp_rows(Z)
+        g = good[s:s + slice_rows]
+        zy = np.zeros(r.shape[0])
+        zy[g] = Z[np.nonzero(g)[0], y[r][g]]
+        loss[s:s + slice_rows] = np.where(g, l - zy, 0.0)
+        lse[s:s + slice_rows] = np.where(g, l, 0.0)
+    loss[bad] = np.nan
+    lse[bad] = np.nan
+    return loss, lse
+
+
+def dlogits(Z: np.ndarray, lse: np.ndarray, y_rows: np.ndarray,
+            dloss_rows: np.ndarray, filter_eps: float = 0.0) -> np.ndarray:
+    """G = dloss_i * (softmax_ij * keep_ij - [j == y_i]) on a logit slice.
+
+    keep_ij = softmax_ij >= filter_eps when filter_eps > 0 (softmax entries
+    below the threshold carry no gradient: [LM] §Contribution, [MAP]
+    §Approach); the one-hot term is never filtered.  Rows with y < 0 are
+    treated as having no target (callers zero their dloss).
+    """
+    P = np.exp(Z - lse[:, None])
+    if filter_eps > 0.0:
+        P = np.where(P >= filter_eps, P, 0.0)
+    G = P
+    has_t = y_rows >= 0
+    G[np.nonzero(has_t)[0], y_rows[has_t]] -= 1.0
+    return dloss_rows[:, None] * G
+
+
+def backward(H, segments, y, V: int, dloss, ignore_index: int = -100,
+             filter_eps: float = 0.0, slice_rows: int = SLICE_ROWS):
+    """Exact gradients of sum_i dloss_i * loss_i w.r.t. H and each E segment.
+
+    Returns (dH[N, D] fp64, [dE_s[n_s, D] fp64 per segment]).  Ignored rows
+    get a zero dH row and contribute nothing to dE.  [LM] §Contribution,
+    [MAP] §Approach (the method recomputes these blockwise; the oracle just
+    forms them slice by slice).
+    """
+    segs64 = _segments_f64(segments)
+    y = np.asarray(y, dtype=np.int64)
+    N, D = H.shape
+    dloss = np.asarray(dloss, dtype=np.float64)
+    ignored, good, bad = _valid_targets(y, V, ignore_index, segs64)
+    dH = np.zeros((N, D))
+    dE = [np.zeros_like(E64) for _, _, E64 in segs64]
+    for s in range(0, N, slice_rows):
+        r = np.arange(s, min(N, s + slice_rows))
+        g = good[r]
+        if not g.any():
+            continue
+        r = r[g]
+        H64 = as_f64(H[r])
+        Z = logits_rows(H64, segs64, V)
+        G = dlogits(Z, logsumexp_rows(Z), y[r], dloss[r], filter_eps)
+        acc = np.zeros((r.shape[0], D))
+        for k, (begin, end, E64) in enumerate(segs64):
+            Gs = G[:, begin:end]
+            acc += Gs @ E64
+            dE[k] += Gs.T @ H64
+        dH[r] = acc
+    dH[bad] = np.nan
+    return dH, dE
+
+
+def softmax_rows(H, segments, V: int, rows) -> np.ndarray:
+    """Softmax over the logical vocabulary for the given rows (gap = 0)."""
+    segs64 = _segments_f64(segments)
+    Z = logits_rows(as_f64(H[np.asarray(rows)]), segs64, V)
+    return np.exp(Z - logsumexp_rows(Z)[:, None])
+
+
+def dE_columns(H, segments, y, V: int, dloss, cols: Sequence[int],
+               ignore_index: int = -100, filter_eps: float = 0.0,
+               slice_rows: int = SLICE_ROWS) -> np.ndarray:
+    """Rows of dE for a few logical vocab ids (needs every row's lse).
+
+    dE_j = sum_i G_ij h_i; the lse of every valid row comes from the oracle's
+    own forward over all rows.  Used for sampled checks at full size.
+    """
+    segs64 = _segments_f64(segments)
+    y = np.asarray(y, dtype=np.int64)
+    N, D = H.shape
+    cols = np.asarray(cols, dtype=np.int64)
+    ignored, good, bad = _valid_targets(y, V, ignore_index, segs64)
+    out = np.zeros((cols.shape[0], D))
+    dloss = np.asarray(dloss, dtype=np.float64)
+    for s in range(0, N, slice_rows):
+        r = np.arange(s, min(N, s + slice_rows))
+        r = r[good[r]]
+        if r.shape[0] == 0:
+            continue
+        H64 = as_f64(H[r])
+        Z = logits_rows(H64, segs64, V)
+        lse = logsumexp_rows(Z)
+        Zc = Z[:, cols]
+        P = np.exp(Zc - lse[:, None])
+        if filter_eps > 0.0:
+            P = np.where(P >= filter_eps, P, 0.0)
+        P -= (y[r][:, None] == cols[None, :])
+        out += (dloss[r][:, None] * P).T @ H64
+    return out
+
+
+def mean_loss(loss: np.ndarray, valid: np.ndarray) -> float:
+    """Mean over valid rows, exactly rounded (math.fsum); N_v = 0 gives NaN."""
+    n_v = int(np.count_nonzero(valid))
+    if n_v == 0:
+        return float("nan")
+    return math.fsum(np.asarray(loss, dtype=np.float64)[valid].tolist()) / n_v
+
+
+def kahan_reference(parts: Sequence[np.ndarray]) -> np.ndarray:
+    """Exact (fp64) sum of several gradient contributions, the target that a
+    compensated accumulation approaches ([MAP] §Limitations, Kahan variants)."""
+    acc = np.zeros_like(parts[0], dtype=np.float64)
+    for p in parts:
+        acc += p
+    return acc

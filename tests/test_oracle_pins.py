@@ -1,0 +1,305 @@
+"""Pins for the fp64 oracle: each test ties it to something other than itself.
+
+Closed forms, invariants, a library routine (torch fp64 on the CPU), brute
+force on tiny inputs and central finite differences.  A dropped term, a wrong
+sign or index, or a transposed operand anywhere in the oracle fails at least
+one of them (see the "catches" note on each test).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_cross_entropy_cce_b200 import synthetic as syn
+
+IGN = -100
+
+
+def _small(N=37, D=24, V=53, std=2.0, seed=1, ignore=0.2, segments=None):
+    wl = syn.Workload("t", N=N, D=D, V=V, logit_std=std, ignore_frac=ignore,
+                      segments=tuple(segments) if segments else (),
+                      segment_mix=(0.6, 0.4) if segments else ())
+    return syn.make_inputs(wl, seed=seed)
+
+
+# ---------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("V", [7, 4096, 256000])
+def test_zero_E_gives_lnV_exactly(V):
+    """E = 0: every logit is 0, sum exp = V exactly, loss = lse = ln V bitwise.
+    Catches: a missing/extra term in the lse, a wrong max shift."""
+    N, D = 5, 8
+    H = syn.fp32_to_bf16_bits(np.random.default_rng(0).standard_normal((N, D)).astype(np.float32))
+    E = np.zeros((V, D), dtype=np.uint16)
+    y = np.array([0, V - 1, 3 % V, IGN, 1], dtype=np.int32)
+    loss, lse = oracle.forward(H, [(0, V, E)], y, V, IGN)
+    valid = y != IGN
+    assert np.all(loss[valid] == np.log(V)) and np.all(lse[valid] == np.log(V))
+    assert loss[~valid] == 0 and lse[~valid] == 0
+
+
+def test_zero_E_composite_counts_only_live_ids():
+    """With a dead gap and E = 0 the loss is ln(V_live): the gap adds nothing
+    (its logits are -inf).  Catches: a gap filled with 0 instead of -inf."""
+    V, D = 40, 4
+    segs = [(0, 17, np.zeros((17, D), np.uint16)), (25, 40, np.zeros((15, D), np.uint16))]
+    H = np.zeros((3, D), np.uint16)
+    y = np.array([0, 30, 16], np.int32)
+    loss, lse = oracle.forward(H, segs, y, V, IGN)
+    assert np.all(loss == np.log(32.0))
+
+
+def test_two_class_is_softplus():
+    """V = 2: CE reduces to softplus(z_other - z_target) (textbook logistic loss).
+    Catches: sign errors, using the wrong logit as the target."""
+    rng = np.random.default_rng(3)
+    H = rng.standard_normal((9, 3))
+    E = rng.standard_normal((2, 3))
+    y = rng.integers(0, 2, 9).astype(np.int32)
+    loss, _ = oracle.forward(H, [(0, 2, E)], y, 2, IGN)
+    Z = H @ E.T
+    d = Z[np.arange(9), 1 - y] - Z[np.arange(9), y]
+    assert np.allclose(loss, np.log1p(np.exp(d)), rtol=1e-13, atol=1e-15)
+
+
+def test_identity_head_matches_library_logsumexp():
+    """E = I (D = V): logits are H itself, so lse must equal the library's
+    scipy.special.logsumexp of H's rows.  Catches: transposed H/E."""
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(4)
+    V = 11
+    H = rng.standard_normal((6, V)) * 5
+    E = np.eye(V)
+    y = rng.integers(0, V, 6).astype(np.int32)
+    loss, lse = oracle.forward(H, [(0, V, E)], y, V, IGN)
+    assert np.allclose(lse, logsumexp(H, axis=1), rtol=1e-14, atol=0)
+    assert np.allclose(loss, lse - H[np.arange(6), y], rtol=1e-13, atol=1e-14)
+
+
+# ------------------------------------------------------------------ invariants
+def test_shift_invariance():
+    """Adding c to every logit (extra column h=1, e=c) leaves the loss unchanged.
+    Catches: lse without the max term cancelling, a target logit taken from
+    the wrong place."""
+    x = _small()
+    c = syn.fp32_to_bf16_bits(np.array([3.0], np.float32))[0]
+    H2 = np.concatenate([x.H, np.full((x.H.shape[0], 1), syn.fp32_to_bf16_bits(np.array([1.0], np.float32))[0], np.uint16)], 1)
+    E = x.segments[0][2]
+    E2 = np.concatenate([E, np.full((E.shape[0], 1), c, np.uint16)], 1)
+    l1, s1 = oracle.forward(x.H, x.segments, x.y, x.wl.V, IGN)
+    l2, s2 = oracle.forward(H2, [(0, x.wl.V, E2)], x.y, x.wl.V, IGN)
+    v = x.valid
+    assert np.allclose(l1[v], l2[v], rtol=1e-12, atol=1e-12)
+    assert np.allclose(s2[v] - s1[v], 3.0, rtol=0, atol=1e-12)
+
+
+def test_dlogit_rows_sum_to_zero():
+    """Unfiltered, sum_j dloss*(p_ij - onehot_ij) = 0 for every row.
+    Catches: a missing one-hot term, a softmax that does not normalise."""
+    x = _small()
+    H64 = oracle.widen_bf16(x.H[x.valid])
+    Z = oracle.logits_rows(H64, [(0, x.wl.V, oracle.widen_bf16(x.segments[0][2]))], x.wl.V)
+    G = oracle.dlogits(Z, oracle.logsumexp_rows(Z), x.y[x.valid].astype(np.int64),
+                       np.ones(H64.shape[0]))
+    assert np.max(np.abs(G.sum(1))) <= 1e-12
+
+
+def test_gradient_pairing_identity():
+    """<dH, H>_F = <dE, E>_F: both equal sum_ij G_ij z_ij.
+    Catches: a transposed operand in either contraction, a wrong row scatter."""
+    x = _small(N=64, D=16, V=40, std=3.0)
+    dl = x.dloss_mean()
+    dH, dE = oracle.backward(x.H, x.segments, x.y, x.wl.V, dl, IGN)
+    a = np.sum(dH * oracle.widen_bf16(x.H))
+    b = np.sum(dE[0] * oracle.widen_bf16(x.segments[0][2]))
+    assert abs(a - b) <= 1e-12 * max(1.0, abs(a))
+
+
+def test_softmax_rows_sum_to_one_and_gap_is_zero():
+    x = _small(N=8, D=8, V=30, segments=[(0, 10), (14, 30)])
+    P = oracle.softmax_rows(x.H, x.segments, 30, np.arange(8))
+    assert np.allclose(P.sum(1), 1.0, rtol=0, atol=1e-14)
+    assert np.all(P[:, 10:14] == 0.0)
+
+
+# ----------------------------------------------------------- finite differences
+def test_central_finite_differences():
+    """dH, dE against central differences of sum_i dloss_i loss_i on N=3, D=5,
+    V=7 in fp64.  Catches: any sign/index/scale error in the backward."""
+    rng = np.random.default_rng(5)
+    N, D, V = 3, 5, 7
+    H = rng.standard_normal((N, D))
+    E = rng.standard_normal((V, D))
+    y = np.array([2, 6, 0], np.int32)
+    dl = np.array([0.7, -1.3, 0.25])
+
+    def f(Hx, Ex):
+        loss, _ = oracle.forward(Hx, [(0, V, Ex)], y, V, IGN)
+        return float(np.dot(dl, loss))
+
+    dH, dE = oracle.backward(H, [(0, V, E)], y, V, dl, IGN)
+    h = 1e-6
+    for arr, grad in ((H, dH), (E, dE[0])):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            old = arr[idx]
+            arr[idx] = old + h
+            fp = f(H, E)
+            arr[idx] = old - h
+            fm = f(H, E)
+            arr[idx] = old
+            num[idx] = (fp - fm) / (2 * h)
+        rel = np.linalg.norm(num - grad) / np.linalg.norm(grad)
+        assert rel <= 1e-7, rel
+
+
+# ------------------------------------------------------------------ brute force
+def _brute(H, E, y, dl, eps=0.0):
+    N, D = len(H), len(H[0])
+    V = len(E)
+    loss, dH, dE = [], [[0.0] * D for _ in range(N)], [[0.0] * D for _ in range(V)]
+    for i in range(N):
+        z = [sum(H[i][d] * E[j][d] for d in range(D)) for j in range(V)]
+        m = max(z)
+        lse = m + math.log(sum(math.exp(zj - m) for zj in z))
+        loss.append(lse - z[y[i]])
+        for j in range(V):
+            p = math.exp(z[j] - lse)
+            if eps > 0 and p < eps:
+                p = 0.0
+            g = dl[i] * (p - (1.0 if j == y[i] else 0.0))
+            for d in range(D):
+                dH[i][d] += g * E[j][d]
+                dE[j][d] += g * H[i][d]
+    return np.array(loss), np.array(dH), np.array(dE)
+
+
+@pytest.mark.parametrize("eps", [0.0, 0.05])
+def test_brute_force_triple_loop(eps):
+    """Pure-Python loops on N=4, D=8, V=16, with and without the filter."""
+    rng = np.random.default_rng(6)
+    H = oracle.widen_bf16(syn.fp32_to_bf16_bits(rng.standard_normal((4, 8)).astype(np.float32)))
+    E = oracle.widen_bf16(syn.fp32_to_bf16_bits(rng.standard_normal((16, 8)).astype(np.float32)))
+    y = np.array([3, 0, 15, 7], np.int32)
+    dl = np.array([0.25, 0.25, -0.5, 1.0])
+    bl, bdH, bdE = _brute(H.tolist(), E.tolist(), y.tolist(), dl.tolist(), eps)
+    loss, _ = oracle.forward(H, [(0, 16, E)], y, 16, IGN)
+    dH, dE = oracle.backward(H, [(0, 16, E)], y, 16, dl, IGN, filter_eps=eps)
+    assert np.allclose(loss, bl, rtol=1e-12, atol=1e-12)
+    assert np.allclose(dH, bdH, rtol=1e-12, atol=1e-12)
+    assert np.allclose(dE[0], bdE, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------- library routine
+def test_matches_torch_cross_entropy_fp64_on_tiny():
+    """Tiny workload vs torch.nn.functional.cross_entropy (CPU, fp64,
+    reduction='none', ignore_index=-100) and torch.autograd for dH, dE."""
+    x = syn.make_inputs(syn.WORKLOADS["tiny"], seed=0)
+    V = x.wl.V
+    Ht = torch.tensor(oracle.widen_bf16(x.H), requires_grad=True)
+    Et = torch.tensor(oracle.widen_bf16(x.segments[0][2]), requires_grad=True)
+    yt = torch.tensor(x.y.astype(np.int64))
+    ref = torch.nn.functional.cross_entropy(Ht @ Et.T, yt, reduction="none", ignore_index=IGN)
+    dl = x.dloss_mean().astype(np.float64)
+    (ref * torch.tensor(dl)).sum().backward()
+    loss, lse = oracle.forward(x.H, x.segments, x.y, V, IGN)
+    assert np.allclose(loss, ref.detach().numpy(), rtol=1e-12, atol=1e-12)
+    lse_t = torch.logsumexp(Ht.detach() @ Et.detach().T, 1).numpy()
+    assert np.allclose(lse[x.valid], lse_t[x.valid], rtol=1e-13, atol=1e-13)
+    dH, dE = oracle.backward(x.H, x.segments, x.y, V, dl, IGN)
+    assert np.allclose(dH, Ht.grad.numpy(), rtol=1e-12, atol=1e-14)
+    assert np.allclose(dE[0], Et.grad.numpy(), rtol=1e-12, atol=1e-14)
+    # mean over valid rows, exactly rounded, equals torch's 'mean' reduction
+    m = torch.nn.functional.cross_entropy(Ht.detach() @ Et.detach().T, yt, ignore_index=IGN).item()
+    assert abs(oracle.mean_loss(loss, x.valid) - m) <= 1e-13 * abs(m)
+
+
+# ------------------------------------------------------------ chunking / segments
+def test_row_chunking_does_not_change_results():
+    """Position-chunked CE summed equals the unchunked CE (rows are independent)."""
+    x = _small(N=70, D=16, V=33)
+    a = oracle.forward(x.H, x.segments, x.y, 33, IGN, slice_rows=1)
+    b = oracle.forward(x.H, x.segments, x.y, 33, IGN, slice_rows=512)
+    c = oracle.forward(x.H, x.segments, x.y, 33, IGN, slice_rows=16)
+    for u, v in ((a, b), (b, c)):
+        assert np.allclose(u[0], v[0], rtol=1e-14, atol=1e-14)
+        assert np.allclose(u[1], v[1], rtol=1e-14, atol=1e-14)
+    dl = x.dloss_mean()
+    g1 = oracle.backward(x.H, x.segments, x.y, 33, dl, IGN, slice_rows=7)
+    g2 = oracle.backward(x.H, x.segments, x.y, 33, dl, IGN, slice_rows=512)
+    assert np.allclose(g1[0], g2[0], rtol=1e-13, atol=1e-16)
+    assert np.allclose(g1[1][0], g2[1][0], rtol=1e-13, atol=1e-16)
+
+
+def test_vocab_chunked_logaddexp_equals_full_lse():
+    """lse over the whole vocabulary equals log-add-exp of per-chunk lse values."""
+    x = _small(N=20, D=16, V=301, std=6.0)
+    Z = oracle.logits_rows(oracle.widen_bf16(x.H), [(0, 301, oracle.widen_bf16(x.segments[0][2]))], 301)
+    full = oracle.logsumexp_rows(Z)
+    parts = [oracle.logsumexp_rows(Z[:, a:a + 64]) for a in range(0, 301, 64)]
+    comp = parts[0]
+    for p in parts[1:]:
+        comp = np.logaddexp(comp, p)
+    assert np.allclose(comp, full, rtol=1e-13, atol=0)
+
+
+def test_segmented_with_gap_equals_compact_head():
+    """Segments with a -inf gap == one compact head [E_A; E_B] with targets of
+    segment B shifted down by the gap width."""
+    segs = [(0, 40), (47, 90)]
+    x = _small(N=50, D=12, V=90, std=4.0, segments=segs)
+    EA, EB = x.segments[0][2], x.segments[1][2]
+    compact = [(0, 83, np.concatenate([EA, EB], 0))]
+    y2 = x.y.copy()
+    y2[x.y >= 47] -= 7
+    l1, s1 = oracle.forward(x.H, x.segments, x.y, 90, IGN)
+    l2, s2 = oracle.forward(x.H, compact, y2, 83, IGN)
+    assert np.allclose(l1, l2, rtol=1e-13, atol=1e-13)
+    assert np.allclose(s1, s2, rtol=1e-13, atol=1e-13)
+    dl = x.dloss_mean()
+    dH1, dE1 = oracle.backward(x.H, x.segments, x.y, 90, dl, IGN)
+    dH2, dE2 = oracle.backward(x.H, compact, y2, 83, dl, IGN)
+    assert np.allclose(dH1, dH2, rtol=1e-12, atol=1e-15)
+    assert np.allclose(np.concatenate(dE1, 0), dE2[0], rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------- edge cases
+def test_ignored_and_bad_targets():
+    V, D = 10, 4
+    rng = np.random.default_rng(8)
+    H = syn.fp32_to_bf16_bits(rng.standard_normal((5, D)).astype(np.float32))
+    segs = [(0, 6, syn.fp32_to_bf16_bits(rng.standard_normal((6, D)).astype(np.float32)))]
+    y = np.array([IGN, 10, 7, -3, 2], np.int32)   # ignored, out of range, in gap, negative, ok
+    loss, lse = oracle.forward(H, segs, y, V, IGN)
+    assert loss[0] == 0 and lse[0] == 0
+    assert np.all(np.isnan(loss[1:4])) and np.all(np.isnan(lse[1:4]))
+    assert np.isfinite(loss[4])
+    dH, dE = oracle.backward(H, segs, y, V, np.ones(5), IGN)
+    assert np.all(dH[0] == 0) and np.all(np.isnan(dH[1:4])) and np.all(np.isfinite(dH[4]))
+    assert math.isnan(oracle.mean_loss(loss, np.zeros(5, bool)))
+
+
+def test_filter_drops_exactly_the_small_softmax_entries():
+    """With filter_eps, dE of a column whose softmax is below eps in every row
+    equals the one-hot part only; a column at/above eps keeps its softmax part."""
+    x = _small(N=30, D=16, V=64, std=8.0, ignore=0.0)
+    eps = 2.0 ** -12
+    P = oracle.softmax_rows(x.H, x.segments, 64, np.arange(30))
+    dl = x.dloss_mean().astype(np.float64)
+    _, dE = oracle.backward(x.H, x.segments, x.y, 64, dl, IGN, filter_eps=eps)
+    H64 = oracle.widen_bf16(x.H)
+    for j in range(64):
+        keep = P[:, j] >= eps
+        expect = ((dl * np.where(keep, P[:, j], 0.0) - dl * (x.y == j))[:, None] * H64).sum(0)
+        assert np.allclose(dE[0][j], expect, rtol=1e-12, atol=1e-15)
+
+
+def test_dE_columns_match_backward():
+    x = _small(N=40, D=8, V=50, segments=[(0, 20), (26, 50)])
+    dl = x.dloss_mean()
+    _, dE = oracle.backward(x.H, x.segments, x.y, 50, dl, IGN, filter_eps=1e-3)
+    cols = [0, 19, 26, 49]
+    got = oracle.dE_columns(x.H, x.segments, x.y, 50, dl, cols, IGN, filter_eps=1e-3, slice_rows=9)
+    ref = np.stack([dE[0][0], dE[0][19], dE[1][0], dE[1][23]])
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-16)
