@@ -1,0 +1,186 @@
+/*
+ * libcce — Cut Cross-Entropy on NVIDIA B200 (sm_100a): the classifier matmul
+ * fused with cross-entropy over a large vocabulary, forward and backward,
+ * without ever writing the [N, V] logit matrix to device memory.
+ *
+ * What is computed (sources are web pages, cited by title and section):
+ *   "The loss and the mask: Cut Cross-Entropy + FlexAttention (2 papers)",
+ *   part "Cut Your Losses in Large-Vocabulary Language Models (CCE)",
+ *   §Contribution: the cross-entropy of row i needs only the correct-token
+ *   logit <h_i, e_{y_i}> (an indexed dot product) and the log-sum-exp of the
+ *   row's logits z_ij = <h_i, e_j>, computed blockwise on chip while streaming
+ *   over vocabulary tiles; loss_i = lse_i - <h_i, e_{y_i}>.  The backward
+ *   recomputes the logits blockwise and drops softmax entries below bf16
+ *   precision ("Cut Your Losses in Large-Vocabulary Language Models",
+ *   research-map entry, §Approach).  §What transfers to us (third bullet) of
+ *   the first page: a composite head composes the lse over several vocabulary
+ *   segments with log-add-exp, and a dead gap between segments contributes
+ *   -inf.
+ *
+ * Conventions shared by every entry point
+ *   - Layouts are row-major and dense: H [N, D] bf16, E [V_s, D] bf16 per
+ *     segment, y [N] int32.  D must be a positive multiple of 8 (16-byte rows,
+ *     a TMA requirement); every device pointer must be 16-byte aligned.
+ *   - All pointers except the ones marked "host" are device pointers.  The
+ *     caller owns every buffer, including the workspace; the library never
+ *     allocates device memory and never synchronises the stream.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is enqueued asynchronously on it.
+ *   - Return value: host-detectable errors (CCE_E*).  Errors found by the GPU
+ *     while running are OR-ed as CCE_STATUS_* bits into *status (device int32,
+ *     which the caller zeroes and reads after synchronising).  Device code
+ *     never traps; every wait inside a kernel is bounded and reports
+ *     CCE_STATUS_TIMEOUT instead of hanging.
+ *   - Rows whose target equals ignore_index are skipped before any math:
+ *     loss = lse = 0 and their dH row is 0.  A target outside [0, V) or inside
+ *     a gap sets CCE_STATUS_BADTARGET and yields NaN loss, lse and dH row.
+ */
+#ifndef CCE_H_
+#define CCE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes (host side). */
+#define CCE_OK 0
+#define CCE_EINVAL 1      /* bad shape, alignment, segment table or NULL pointer */
+#define CCE_EWORKSPACE 2  /* workspace NULL or smaller than *_workspace_size()  */
+#define CCE_ELAUNCH 3     /* a kernel launch or tensor-map encode failed          */
+#define CCE_EDEVICE 4     /* no sm_100 device / driver entry point unavailable     */
+
+/* Device status bits OR-ed into *status. */
+#define CCE_STATUS_BADTARGET 1
+#define CCE_STATUS_TIMEOUT 2
+
+/* cce_bwd flags. */
+#define CCE_KAHAN_DE 1u   /* dE += grad with a bf16 Kahan compensation buffer  */
+#define CCE_FP32_GRADS 2u /* dH and dE are written as fp32 instead of bf16     */
+
+#define CCE_MAX_SEGMENTS 8
+
+/*
+ * One live range of a composite classifier head.  Logical vocabulary ids
+ * [vocab_begin, vocab_end) are rows 0 .. vocab_end - vocab_begin - 1 of E.
+ * Ids covered by no segment form the dead gap (logit -inf).
+ *   E       [vocab_end - vocab_begin, D] bf16, read only.
+ *   dE      output of cce_bwd for this segment (bf16, or fp32 with
+ *           CCE_FP32_GRADS); may be NULL for cce_fwd.
+ *   dE_comp bf16 Kahan compensation, same shape as dE, read and updated
+ *           only with CCE_KAHAN_DE (else ignored).
+ * Segments must be sorted by vocab_begin, non-empty, non-overlapping and
+ * inside [0, V); at most CCE_MAX_SEGMENTS.
+ */
+typedef struct cce_segment {
+  int64_t vocab_begin;
+  int64_t vocab_end;
+  const void* E;
+  void* dE;
+  void* dE_comp;
+} cce_segment;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int cce_version(void);
+
+/* Static text for a CCE_* return code. */
+const char* cce_strerror(int code);
+
+/*
+ * Workspace bytes cce_fwd needs for these sizes (0 on invalid sizes).
+ * n_segs = 0 means one segment [0, V).
+ */
+size_t cce_fwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs);
+
+/*
+ * Forward: per-row loss and log-sum-exp (natural log), fp32.
+ *   H        [N, D] bf16 hidden states.
+ *   E        [V, D] bf16 classifier, used when segs == NULL (one segment
+ *            [0, V)); must be NULL when segs != NULL.
+ *   y        [N] int32 targets (logical ids) or ignore_index.
+ *   segs     host array of n_segs segments, or NULL / 0.
+ *   loss,lse [N] fp32 outputs.
+ *   colmax   optional [V_live] fp32 output, V_live = sum of segment sizes:
+ *            the largest logit each live vocabulary row reaches over the
+ *            valid rows (-inf if none), in segment order; the statistic
+ *            cce_vocab_sort can order the vocabulary by.  NULL to skip.
+ *   workspace, workspace_bytes  scratch of at least cce_fwd_workspace_size().
+ *   status   device int32, OR-ed with CCE_STATUS_* bits.
+ * Only rows with a valid target are computed; nothing of size N*V is ever
+ * allocated or written.
+ */
+int cce_fwd(const void* H, const void* E, const int32_t* y,
+            int64_t N, int64_t D, int64_t V, int32_t ignore_index,
+            const cce_segment* segs, int32_t n_segs,
+            float* loss, float* lse, float* colmax,
+            void* workspace, size_t workspace_bytes,
+            int32_t* status, void* stream);
+
+/* Workspace bytes cce_bwd needs (0 on invalid sizes). */
+size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs,
+                              uint32_t flags);
+
+/*
+ * Backward: gradients of sum_i dloss_i * loss_i.
+ *   H, E, y, N, D, V, ignore_index, segs, n_segs  as for cce_fwd.
+ *   lse      [N] fp32, the forward's lse output for the same inputs.
+ *   dloss    [N] fp32 upstream gradient per row (1/N_valid on valid rows for
+ *            a mean loss).
+ *   filter_eps  softmax entries p_ij < filter_eps carry no gradient
+ *            (element granularity; the target's one-hot term is never
+ *            dropped); <= 0 turns filtering off.  2^-12 is bf16 precision.
+ *            Tensor-core work is skipped on 16-wide blocks that are entirely
+ *            zero after filtering.
+ *   vocab_perm  optional [V_live] int32: for each segment, a permutation of
+ *            its local rows (entries [off_s, off_s + n_s) permute
+ *            0..n_s-1, off_s = sum of the sizes of earlier segments).  The
+ *            backward walks the vocabulary in that order so that surviving
+ *            blocks cluster; results do not depend on it beyond rounding.
+ *            NULL = identity.
+ *   flags    CCE_KAHAN_DE | CCE_FP32_GRADS.
+ *   dH       [N, D] output (bf16, or fp32 with CCE_FP32_GRADS).
+ *   dE       [V, D] output when segs == NULL (else per-segment dE).  Written
+ *            (overwritten) unless CCE_KAHAN_DE, in which case the new
+ *            gradient g is added into the bf16 running sum s with the bf16
+ *            compensation c (dE_comp): y' = g - c; t = s + y'; c = (t - s) - y';
+ *            s = t, in fp32 arithmetic, each element owned by one thread
+ *            (deterministic).  The caller zeroes s and c before the first
+ *            accumulation.
+ *   dE_comp  [V, D] bf16 compensation when segs == NULL and CCE_KAHAN_DE.
+ *   debug_keep  optional [debug_rows, ceil(V/32)] uint32 bitmask: bit j%32 of
+ *            word j/32 of row r is set when element (r, j) kept a non-zero
+ *            softmax gradient (not filtered).  Rows are original row ids
+ *            0..debug_rows-1.  NULL to skip.
+ */
+int cce_bwd(const void* H, const void* E, const int32_t* y,
+            const float* lse, const float* dloss,
+            int64_t N, int64_t D, int64_t V, int32_t ignore_index,
+            const cce_segment* segs, int32_t n_segs,
+            float filter_eps, const int32_t* vocab_perm, uint32_t flags,
+            void* dH, void* dE, void* dE_comp,
+            uint32_t* debug_keep, int64_t debug_rows,
+            void* workspace, size_t workspace_bytes,
+            int32_t* status, void* stream);
+
+/* Workspace bytes cce_vocab_sort needs. */
+size_t cce_vocab_sort_workspace_size(int64_t N, int64_t V, int32_t n_segs);
+
+/*
+ * Vocabulary sort ("Cut Your Losses in Large-Vocabulary Language Models",
+ * first page §Contribution: a vocabulary sort groups the surviving blocks).
+ * Writes vocab_perm [V_live] (layout as in cce_bwd): within each segment,
+ * local rows ordered by descending key, ties by ascending id (stable).  The
+ * key is colmax (from cce_fwd) when given, else the number of valid targets
+ * that hit the row.
+ */
+int cce_vocab_sort(const float* colmax, const int32_t* y, int64_t N, int64_t V,
+                   int32_t ignore_index, const cce_segment* segs, int32_t n_segs,
+                   int32_t* vocab_perm, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CCE_H_ */

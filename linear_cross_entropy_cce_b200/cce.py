@@ -1,0 +1,223 @@
+"""ctypes binding of libcce (argument marshalling only).
+
+Every step of the computation runs in libcce.so's CUDA kernels; torch is used
+for device memory, the current stream and dtype bookkeeping.  There is no CPU
+fallback: if the library is missing or no sm_100 GPU is present the calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcce.so")
+
+CCE_OK, CCE_EINVAL, CCE_EWORKSPACE, CCE_ELAUNCH, CCE_EDEVICE = 0, 1, 2, 3, 4
+STATUS_BADTARGET, STATUS_TIMEOUT = 1, 2
+KAHAN_DE, FP32_GRADS = 1, 2
+MAX_SEGMENTS = 8
+
+EXPORTS = ("cce_version", "cce_strerror", "cce_fwd_workspace_size", "cce_fwd",
+           "cce_bwd_workspace_size", "cce_bwd", "cce_vocab_sort_workspace_size",
+           "cce_vocab_sort")
+
+
+class CCEError(RuntimeError):
+    pass
+
+
+class Segment(ctypes.Structure):
+    _fields_ = [("vocab_begin", ctypes.c_int64), ("vocab_end", ctypes.c_int64),
+                ("E", ctypes.c_void_p), ("dE", ctypes.c_void_p), ("dE_comp", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcce.so (built in-tree by ``linear_cross_entropy_cce_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise CCEError(f"libcce.so not found at {LIB_PATH}; build it with "
+                       "`python -m linear_cross_entropy_cce_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    i64, i32, u32, vp, sz, fp = (ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32, ctypes.c_void_p,
+                                 ctypes.c_size_t, ctypes.c_float)
+    L.cce_version.restype = ctypes.c_int
+    L.cce_strerror.restype = ctypes.c_char_p
+    L.cce_strerror.argtypes = [ctypes.c_int]
+    L.cce_fwd_workspace_size.restype = sz
+    L.cce_fwd_workspace_size.argtypes = [i64, i64, i64, i32]
+    L.cce_fwd.restype = ctypes.c_int
+    L.cce_fwd.argtypes = [vp, vp, vp, i64, i64, i64, i32, ctypes.POINTER(Segment), i32,
+                          vp, vp, vp, vp, sz, vp, vp]
+    L.cce_bwd_workspace_size.restype = sz
+    L.cce_bwd_workspace_size.argtypes = [i64, i64, i64, i32, u32]
+    L.cce_bwd.restype = ctypes.c_int
+    L.cce_bwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, ctypes.POINTER(Segment), i32,
+                          fp, vp, u32, vp, vp, vp, vp, i64, vp, sz, vp, vp]
+    L.cce_vocab_sort_workspace_size.restype = sz
+    L.cce_vocab_sort_workspace_size.argtypes = [i64, i64, i32]
+    L.cce_vocab_sort.restype = ctypes.c_int
+    L.cce_vocab_sort.argtypes = [vp, vp, i64, i64, i32, ctypes.POINTER(Segment), i32, vp, vp, sz, vp]
+    _lib = L
+    return L
+
+
+def _check(rc: int, what: str):
+    if rc != CCE_OK:
+        raise CCEError(f"{what}: {lib().cce_strerror(rc).decode()} (code {rc})")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_ptr(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _require_cuda(*ts: torch.Tensor):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise CCEError("all tensors must be contiguous CUDA tensors")
+
+
+SegSpec = Tuple[int, int, torch.Tensor]  # (vocab_begin, vocab_end, E_s)
+
+
+def _seg_array(segments: Optional[Sequence], dEs=None, comps=None):
+    if not segments:
+        return None, 0
+    arr = (Segment * len(segments))()
+    for k, s in enumerate(segments):
+        b, e, E = s[0], s[1], s[2]
+        arr[k].vocab_begin, arr[k].vocab_end, arr[k].E = int(b), int(e), E.data_ptr()
+        arr[k].dE = dEs[k].data_ptr() if dEs is not None else None
+        arr[k].dE_comp = comps[k].data_ptr() if comps is not None else None
+    return arr, len(segments)
+
+
+def fwd_workspace_size(N: int, D: int, V: int, n_segs: int = 0) -> int:
+    return int(lib().cce_fwd_workspace_size(N, D, V, n_segs))
+
+
+def bwd_workspace_size(N: int, D: int, V: int, n_segs: int = 0, flags: int = 0) -> int:
+    return int(lib().cce_bwd_workspace_size(N, D, V, n_segs, flags))
+
+
+def vocab_sort_workspace_size(N: int, V: int, n_segs: int = 0) -> int:
+    return int(lib().cce_vocab_sort_workspace_size(N, V, n_segs))
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise CCEError("workspace too small")
+        return workspace
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def fwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, ignore_index: int = -100,
+        segments: Optional[Sequence[SegSpec]] = None, V: Optional[int] = None,
+        want_colmax: bool = False, workspace: Optional[torch.Tensor] = None,
+        status: Optional[torch.Tensor] = None):
+    """Per-row (loss, lse) fp32; optional colmax [V_live].  See cce_fwd."""
+    N, D = H.shape
+    if segments:
+        V = V if V is not None else int(segments[-1][1])
+        v_live = sum(int(e) - int(b) for b, e, *_ in segments)
+    else:
+        V = int(E.shape[0])
+        v_live = V
+    _require_cuda(H, E, y, *[s[2] for s in (segments or [])])
+    dev = H.device
+    loss = torch.empty(N, dtype=torch.float32, device=dev)
+    lse = torch.empty(N, dtype=torch.float32, device=dev)
+    colmax = torch.empty(v_live, dtype=torch.float32, device=dev) if want_colmax else None
+    segarr, nseg = _seg_array(segments)
+    ws = _workspace(fwd_workspace_size(N, D, V, nseg), dev, workspace)
+    st = status if status is not None else torch.zeros(1, dtype=torch.int32, device=dev)
+    rc = lib().cce_fwd(_ptr(H), _ptr(E) if not segments else None, _ptr(y), N, D, V, ignore_index,
+                       segarr, nseg, _ptr(loss), _ptr(lse), _ptr(colmax), _ptr(ws),
+                       ws.numel(), _ptr(st), _stream_ptr(dev))
+    _check(rc, "cce_fwd")
+    if want_colmax:
+        return loss, lse, colmax
+    return loss, lse
+
+
+def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.Tensor,
+        dloss: torch.Tensor, ignore_index: int = -100,
+        segments: Optional[Sequence[SegSpec]] = None, V: Optional[int] = None,
+        filter_eps: float = 0.0, vocab_perm: Optional[torch.Tensor] = None,
+        kahan: bool = False, fp32_grads: bool = False,
+        dE_out=None, dE_comp=None, debug_rows: int = 0,
+        workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
+    """Gradients (dH, dE) of sum_i dloss_i loss_i.  See cce_bwd.
+
+    dE is one tensor for a single head, a list (one per segment) otherwise.
+    With kahan=True, dE_out and dE_comp (bf16, same shape(s)) are required
+    and updated in place.  Returns (dH, dE, debug_keep or None).
+    """
+    N, D = H.shape
+    dev = H.device
+    _require_cuda(H, E, y, lse, dloss, vocab_perm)
+    gdt = torch.float32 if fp32_grads else torch.bfloat16
+    if segments:
+        V = V if V is not None else int(segments[-1][1])
+        shapes = [(int(e) - int(b), D) for b, e, *_ in segments]
+    else:
+        V = int(E.shape[0])
+        shapes = [(V, D)]
+    if dE_out is None:
+        if kahan:
+            raise CCEError("kahan accumulation needs dE_out and dE_comp")
+        dEs = [torch.empty(s, dtype=gdt, device=dev) for s in shapes]
+    else:
+        dEs = list(dE_out) if isinstance(dE_out, (list, tuple)) else [dE_out]
+    comps = None
+    if kahan:
+        comps = list(dE_comp) if isinstance(dE_comp, (list, tuple)) else [dE_comp]
+    dH = torch.empty((N, D), dtype=gdt, device=dev)
+    flags = (KAHAN_DE if kahan else 0) | (FP32_GRADS if fp32_grads else 0)
+    words = (V + 31) // 32
+    dbg = torch.empty((debug_rows, words), dtype=torch.int32, device=dev) if debug_rows > 0 else None
+    segarr, nseg = _seg_array(segments, dEs if segments else None, comps if segments else None)
+    ws = _workspace(bwd_workspace_size(N, D, V, nseg, flags), dev, workspace)
+    st = status if status is not None else torch.zeros(1, dtype=torch.int32, device=dev)
+    rc = lib().cce_bwd(_ptr(H), _ptr(E) if not segments else None, _ptr(y), _ptr(lse), _ptr(dloss),
+                       N, D, V, ignore_index, segarr, nseg, float(filter_eps), _ptr(vocab_perm),
+                       flags, _ptr(dH), None if segments else dEs[0].data_ptr(),
+                       None if (segments or not kahan) else comps[0].data_ptr(),
+                       _ptr(dbg), debug_rows, _ptr(ws), ws.numel(), _ptr(st), _stream_ptr(dev))
+    _check(rc, "cce_bwd")
+    return dH, (dEs if segments else dEs[0]), dbg
+
+
+def vocab_sort(colmax: Optional[torch.Tensor], y: torch.Tensor, V: int, ignore_index: int = -100,
+               segments: Optional[Sequence[SegSpec]] = None,
+               workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Per-segment permutation of live vocabulary rows by descending key."""
+    dev = y.device
+    v_live = sum(int(e) - int(b) for b, e, *_ in segments) if segments else V
+    perm = torch.empty(v_live, dtype=torch.int32, device=dev)
+    segarr, nseg = _seg_array(segments)
+    ws = _workspace(vocab_sort_workspace_size(y.numel(), V, nseg), dev, workspace)
+    rc = lib().cce_vocab_sort(_ptr(colmax), _ptr(y), y.numel(), V, ignore_index, segarr, nseg,
+                              _ptr(perm), _ptr(ws), ws.numel(), _stream_ptr(dev))
+    _check(rc, "cce_vocab_sort")
+    return perm
+
+
+def bf16_from_bits(bits, device) -> torch.Tensor:
+    """Upload uint16 bf16 bit patterns (numpy) as a bf16 CUDA tensor."""
+    import numpy as np
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.to(device).view(torch.bfloat16)

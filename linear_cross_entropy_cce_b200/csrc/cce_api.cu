@@ -1,0 +1,577 @@
+// Host side of libcce: argument validation, workspace layout, TMA tensor-map
+// encoding and kernel launches on the caller's stream.  See include/cce.h for
+// the contract of every entry point.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cub/device/device_radix_sort.cuh>
+
+#include "../../include/cce.h"
+#include "cce_kernels.cuh"
+
+using namespace cce;
+
+namespace {
+
+constexpr int kPlanSMs = 148;            // SM count the workspace plan assumes
+constexpr size_t kGBudgetBytes = 64ull << 20;  // bf16 G slab per vocabulary chunk
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------- driver API
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix with the given row
+// stride (elements), 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld,
+              uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  int major = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return -1;
+  if (major != 10) return -1;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return sms;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------ segment table
+struct Segs {
+  int n = 0;
+  cce_segment s[CCE_MAX_SEGMENTS];
+  int64_t live = 0;  // V_live
+};
+
+int build_segs(const void* E, int64_t V, const cce_segment* segs, int32_t n_segs, Segs& out) {
+  if (segs == nullptr || n_segs == 0) {
+    if (E == nullptr) return CCE_EINVAL;
+    out.n = 1;
+    out.s[0] = cce_segment{0, V, E, nullptr, nullptr};
+    out.live = V;
+    return CCE_OK;
+  }
+  if (E != nullptr || n_segs < 0 || n_segs > CCE_MAX_SEGMENTS) return CCE_EINVAL;
+  int64_t prev_end = 0;
+  out.n = n_segs;
+  out.live = 0;
+  for (int i = 0; i < n_segs; ++i) {
+    const cce_segment& g = segs[i];
+    if (g.vocab_begin < prev_end || g.vocab_end <= g.vocab_begin || g.vocab_end > V) return CCE_EINVAL;
+    if (g.E == nullptr || !aligned16(g.E)) return CCE_EINVAL;
+    if (g.vocab_end - g.vocab_begin > (int64_t)INT32_MAX) return CCE_EINVAL;
+    prev_end = g.vocab_end;
+    out.s[i] = g;
+    out.live += g.vocab_end - g.vocab_begin;
+  }
+  return CCE_OK;
+}
+
+SegTable dev_table(const Segs& g, int* T_v) {
+  SegTable t;
+  memset(&t, 0, sizeof(t));
+  t.n_segs = g.n;
+  int tiles = 0, live = 0;
+  for (int i = 0; i < g.n; ++i) {
+    SegDev& d = t.s[i];
+    d.begin = g.s[i].vocab_begin;
+    d.end = g.s[i].vocab_end;
+    d.n = (int)(d.end - d.begin);
+    d.tile_off = tiles;
+    d.live_off = live;
+    d.E = static_cast<const __nv_bfloat16*>(g.s[i].E);
+    tiles += (int)cdiv(d.n, BN);
+    live += d.n;
+  }
+  if (T_v) *T_v = tiles;
+  return t;
+}
+
+bool sizes_ok(int64_t N, int64_t D, int64_t V) {
+  return N >= 0 && N <= (int64_t)INT32_MAX - 256 && D > 0 && D % 8 == 0 && D <= 65536 && V > 0 &&
+         V <= (int64_t)INT32_MAX - 256;
+}
+
+// ------------------------------------------------------------ forward plan
+struct FwdPlan {
+  int64_t Npad;
+  int T_v_max, tpi, S_max;
+  size_t off_nvalid, off_idx, off_pos, off_hc, off_part, total;
+};
+
+FwdPlan plan_fwd(int64_t N, int64_t D, int64_t V, int32_t n_segs) {
+  FwdPlan p;
+  p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
+  p.T_v_max = (int)(cdiv(V, BN) + std::max(1, (int)n_segs));
+  const int64_t num_mb = p.Npad / BM;
+  p.tpi = (int)std::min<int64_t>(16, std::max<int64_t>(2, num_mb * p.T_v_max / (kPlanSMs * 24)));
+  p.S_max = (int)cdiv(p.T_v_max, p.tpi);
+  size_t o = 0;
+  p.off_nvalid = o; o += align_up(16);
+  p.off_idx = o; o += align_up(sizeof(int) * (size_t)std::max<int64_t>(N, 1));
+  p.off_pos = o; o += align_up(sizeof(int) * (size_t)std::max<int64_t>(N, 1));
+  p.off_hc = o; o += align_up((size_t)p.Npad * D * 2);
+  p.off_part = o; o += align_up((size_t)p.S_max * p.Npad * sizeof(float2));
+  p.total = o;
+  return p;
+}
+
+// ----------------------------------------------------------- backward plan
+struct BwdPlan {
+  int64_t Npad, Vc;
+  size_t off_nvalid, off_idx, off_pos, off_lse2, off_dl, off_tseg, off_tpos, off_inv, off_hc,
+      off_dh, off_g, off_ec, total;
+};
+
+BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V) {
+  BwdPlan p;
+  p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
+  int64_t vc = (int64_t)(kGBudgetBytes / (2 * (size_t)p.Npad)) / BN * BN;
+  p.Vc = std::max<int64_t>(BN, std::min<int64_t>(8192, vc));
+  p.Vc = std::min<int64_t>(p.Vc, cdiv(V, BN) * BN);
+  const size_t n4 = sizeof(int) * (size_t)std::max<int64_t>(N, 1);
+  size_t o = 0;
+  p.off_nvalid = o; o += align_up(16);
+  p.off_idx = o; o += align_up(n4);
+  p.off_pos = o; o += align_up(n4);
+  p.off_lse2 = o; o += align_up(n4);
+  p.off_dl = o; o += align_up(n4);
+  p.off_tseg = o; o += align_up(n4);
+  p.off_tpos = o; o += align_up(n4);
+  p.off_inv = o; o += align_up(sizeof(int) * (size_t)V);
+  p.off_hc = o; o += align_up((size_t)p.Npad * D * 2);
+  p.off_dh = o; o += align_up((size_t)p.Npad * D * 4);
+  p.off_g = o; o += align_up((size_t)p.Npad * p.Vc * 2);
+  p.off_ec = o; o += align_up((size_t)p.Vc * D * 2);
+  p.total = o;
+  return p;
+}
+
+template <class Policy>
+int launch_tc(const typename Policy::Params& prm, int grid, cudaStream_t st) {
+  auto k = tc_kernel<Policy>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+    return CCE_ELAUNCH;
+  k<<<grid, THREADS, SMEM_BYTES, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? CCE_OK : CCE_ELAUNCH;
+}
+
+int launched() { return cudaGetLastError() == cudaSuccess ? CCE_OK : CCE_ELAUNCH; }
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+// Compaction + H_c gather shared by forward and backward.
+int run_compaction(const CompactParams& cp, const void* H, int64_t Npad, int64_t D, int sms,
+                   __nv_bfloat16* Hc, cudaStream_t st) {
+  compact_kernel<<<1, COMPACT_THREADS, 0, st>>>(cp);
+  if (launched() != CCE_OK) return CCE_ELAUNCH;
+  gather_rows_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(H), cp.idx,
+                                              cp.n_valid, (int)Npad, (int)D, Hc);
+  return launched();
+}
+
+}  // namespace
+
+// ------------------------------------------------------------- vocab sort
+namespace {
+__global__ void target_hist_kernel(const int* y, int N, int ignore_index, SegTable t, float* key) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < N; i += gridDim.x * blockDim.x) {
+    const int v = y[i];
+    if (v == ignore_index) continue;
+    const int s = segment_of(t, (long long)v);
+    if (s >= 0) atomicAdd(&key[t.s[s].live_off + (v - (int)t.s[s].begin)], 1.0f);
+  }
+}
+__global__ void iota_kernel(int* a, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) a[i] = i;
+}
+
+struct SortPlan {
+  size_t off_key, off_key_out, off_ids, off_tmp, tmp_bytes, total;
+};
+SortPlan plan_sort(int64_t V) {
+  SortPlan p;
+  size_t o = 0;
+  p.off_key = o; o += align_up(sizeof(float) * (size_t)V);
+  p.off_key_out = o; o += align_up(sizeof(float) * (size_t)V);
+  p.off_ids = o; o += align_up(sizeof(int) * (size_t)V);
+  p.off_tmp = o;
+  // generous bound on cub's radix-sort scratch (checked again at run time)
+  p.tmp_bytes = align_up(3 * sizeof(float) * (size_t)V + (8u << 20));
+  o += p.tmp_bytes;
+  p.total = o;
+  return p;
+}
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+int cce_version(void) { return 10000; }
+
+const char* cce_strerror(int code) {
+  switch (code) {
+    case CCE_OK: return "ok";
+    case CCE_EINVAL: return "invalid argument (shape, alignment, segment table or NULL pointer)";
+    case CCE_EWORKSPACE: return "workspace missing or too small";
+    case CCE_ELAUNCH: return "kernel launch or tensor-map encoding failed";
+    case CCE_EDEVICE: return "no sm_100 device or driver entry point unavailable";
+    default: return "unknown error";
+  }
+}
+
+size_t cce_fwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs) {
+  if (!sizes_ok(N, D, V) || n_segs < 0 || n_segs > CCE_MAX_SEGMENTS) return 0;
+  return plan_fwd(N, D, V, n_segs).total;
+}
+
+size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs, uint32_t flags) {
+  (void)flags;
+  if (!sizes_ok(N, D, V) || n_segs < 0 || n_segs > CCE_MAX_SEGMENTS) return 0;
+  return plan_bwd(N, D, V).total;
+}
+
+int cce_fwd(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D, int64_t V,
+            int32_t ignore_index, const cce_segment* segs, int32_t n_segs, float* loss, float* lse,
+            float* colmax, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  if (!sizes_ok(N, D, V)) return CCE_EINVAL;
+  Segs sg;
+  if (int rc = build_segs(E, V, segs, n_segs, sg)) return rc;
+  if (N == 0) return CCE_OK;
+  if (!H || !y || !loss || !lse || !status || !aligned16(H)) return CCE_EINVAL;
+  const FwdPlan pl = plan_fwd(N, D, V, n_segs);
+  if (!workspace || workspace_bytes < pl.total) return CCE_EWORKSPACE;
+  const int sms = device_sms();
+  if (sms <= 0 || !encode_fn()) return CCE_EDEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  int T_v = 0;
+  const SegTable table = dev_table(sg, &T_v);
+  CompactParams cp;
+  memset(&cp, 0, sizeof(cp));
+  cp.y = y;
+  cp.N = (int)N;
+  cp.ignore_index = ignore_index;
+  cp.segs = table;
+  cp.idx = at<int>(workspace, pl.off_idx);
+  cp.pos_of_row = at<int>(workspace, pl.off_pos);
+  cp.n_valid = at<int>(workspace, pl.off_nvalid);
+  cp.status = status;
+  __nv_bfloat16* Hc = at<__nv_bfloat16>(workspace, pl.off_hc);
+  if (int rc = run_compaction(cp, H, pl.Npad, D, sms, Hc, st)) return rc;
+
+  if (colmax) {
+    colmax_init_kernel<<<sms, 256, 0, st>>>(reinterpret_cast<int*>(colmax), (int)sg.live);
+    if (launched()) return CCE_ELAUNCH;
+  }
+
+  FwdParams fp;
+  memset(&fp, 0, sizeof(fp));
+  if (!make_map(&fp.mapA, Hc, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
+  for (int s = 0; s < sg.n; ++s)
+    if (!make_map(&fp.mapB[s], sg.s[s].E, D, table.s[s].n, D, BK, BN)) return CCE_ELAUNCH;
+  fp.segs = table;
+  fp.T_v = T_v;
+  fp.tpi = pl.tpi;
+  fp.S = (int)cdiv(T_v, pl.tpi);
+  fp.Npad = (int)pl.Npad;
+  fp.nkb = (int)cdiv(D, BK);
+  fp.n_valid = cp.n_valid;
+  fp.part = at<float2>(workspace, pl.off_part);
+  fp.colmax = reinterpret_cast<int*>(colmax);
+  fp.status = status;
+  const int64_t items = (pl.Npad / BM) * fp.S;
+  if (int rc = launch_tc<FwdPolicy>(fp, (int)std::min<int64_t>(sms, items), st)) return rc;
+
+  FinParams fin;
+  fin.H = static_cast<const __nv_bfloat16*>(H);
+  fin.y = y;
+  fin.pos_of_row = cp.pos_of_row;
+  fin.part = fp.part;
+  fin.segs = table;
+  fin.N = (int)N;
+  fin.D = (int)D;
+  fin.S = fp.S;
+  fin.Npad = fp.Npad;
+  fin.loss = loss;
+  fin.lse = lse;
+  fwd_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, 8), sms * 8), 256, 0, st>>>(fin);
+  if (launched()) return CCE_ELAUNCH;
+  if (colmax) {
+    colmax_final_kernel<<<sms, 256, 0, st>>>(reinterpret_cast<int*>(colmax), (int)sg.live);
+    if (launched()) return CCE_ELAUNCH;
+  }
+  return CCE_OK;
+}
+
+int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, const float* dloss,
+            int64_t N, int64_t D, int64_t V, int32_t ignore_index, const cce_segment* segs,
+            int32_t n_segs, float filter_eps, const int32_t* vocab_perm, uint32_t flags, void* dH,
+            void* dE, void* dE_comp, uint32_t* debug_keep, int64_t debug_rows, void* workspace,
+            size_t workspace_bytes, int32_t* status, void* stream) {
+  if (!sizes_ok(N, D, V)) return CCE_EINVAL;
+  if (flags & ~(CCE_KAHAN_DE | CCE_FP32_GRADS)) return CCE_EINVAL;
+  const bool kahan = flags & CCE_KAHAN_DE;
+  const bool fp32 = flags & CCE_FP32_GRADS;
+  if (kahan && fp32) return CCE_EINVAL;
+  Segs sg;
+  if (int rc = build_segs(E, V, segs, n_segs, sg)) return rc;
+  if (segs == nullptr || n_segs == 0) {
+    sg.s[0].dE = dE;
+    sg.s[0].dE_comp = dE_comp;
+  } else if (dE != nullptr || dE_comp != nullptr) {
+    return CCE_EINVAL;
+  }
+  for (int s = 0; s < sg.n; ++s) {
+    if (!sg.s[s].dE || !aligned16(sg.s[s].dE)) return CCE_EINVAL;
+    if (kahan && (!sg.s[s].dE_comp || !aligned16(sg.s[s].dE_comp))) return CCE_EINVAL;
+  }
+  if (debug_keep && (debug_rows < 0 || debug_rows > N)) return CCE_EINVAL;
+  if (N == 0) return CCE_OK;
+  if (!H || !y || !lse || !dloss || !dH || !status || !aligned16(H) || !aligned16(dH))
+    return CCE_EINVAL;
+  const BwdPlan pl = plan_bwd(N, D, V);
+  if (!workspace || workspace_bytes < pl.total) return CCE_EWORKSPACE;
+  const int sms = device_sms();
+  if (sms <= 0 || !encode_fn()) return CCE_EDEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  int T_v = 0;
+  const SegTable table = dev_table(sg, &T_v);
+  int* inv = vocab_perm ? at<int>(workspace, pl.off_inv) : nullptr;
+  if (vocab_perm) {
+    for (int s = 0; s < sg.n; ++s) {
+      const int n = table.s[s].n, off = table.s[s].live_off;
+      invert_perm_kernel<<<(int)std::min<int64_t>(cdiv(n, 256), sms * 8), 256, 0, st>>>(
+          vocab_perm + off, n, inv + off);
+      if (launched()) return CCE_ELAUNCH;
+    }
+  }
+  CompactParams cp;
+  memset(&cp, 0, sizeof(cp));
+  cp.y = y;
+  cp.N = (int)N;
+  cp.ignore_index = ignore_index;
+  cp.segs = table;
+  cp.idx = at<int>(workspace, pl.off_idx);
+  cp.pos_of_row = at<int>(workspace, pl.off_pos);
+  cp.n_valid = at<int>(workspace, pl.off_nvalid);
+  cp.status = status;
+  cp.lse = lse;
+  cp.dloss = dloss;
+  cp.inv_perm = inv;
+  cp.lse2_c = at<float>(workspace, pl.off_lse2);
+  cp.dloss_c = at<float>(workspace, pl.off_dl);
+  cp.tseg = at<int>(workspace, pl.off_tseg);
+  cp.tpos = at<int>(workspace, pl.off_tpos);
+  __nv_bfloat16* Hc = at<__nv_bfloat16>(workspace, pl.off_hc);
+  if (int rc = run_compaction(cp, H, pl.Npad, D, sms, Hc, st)) return rc;
+  float* dH_acc = at<float>(workspace, pl.off_dh);
+  if (cudaMemsetAsync(dH_acc, 0, (size_t)pl.Npad * D * 4, st) != cudaSuccess) return CCE_ELAUNCH;
+  const int words = (int)cdiv(V, 32);
+  if (debug_keep && debug_rows > 0 &&
+      cudaMemsetAsync(debug_keep, 0, (size_t)debug_rows * words * 4, st) != cudaSuccess)
+    return CCE_ELAUNCH;
+
+  __nv_bfloat16* G = at<__nv_bfloat16>(workspace, pl.off_g);
+  __nv_bfloat16* Ec = at<__nv_bfloat16>(workspace, pl.off_ec);
+  const int Vc = (int)pl.Vc;
+  const int dt = (int)cdiv(D, BN);
+  const int nkbD = (int)cdiv(D, BK);
+  const int mbs = (int)(pl.Npad / BM);
+  const float eps_keep = filter_eps > 0.f ? filter_eps * (1.0f - 1.0f / 256.0f) : 0.f;
+
+  GParams gp;
+  DEParams ep;
+  DHParams hp;
+  memset(&gp, 0, sizeof(gp));
+  memset(&ep, 0, sizeof(ep));
+  memset(&hp, 0, sizeof(hp));
+  if (!make_map(&gp.mapA, Hc, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
+  if (!make_map(&ep.mapA, G, Vc, pl.Npad, Vc, 64, 64)) return CCE_ELAUNCH;
+  if (!make_map(&ep.mapB, Hc, D, pl.Npad, D, 64, 64)) return CCE_ELAUNCH;
+  if (!make_map(&hp.mapA, G, Vc, pl.Npad, Vc, BK, BM)) return CCE_ELAUNCH;
+
+  for (int s = 0; s < sg.n; ++s) {
+    const int ns = table.s[s].n;
+    const int* perm_seg = vocab_perm ? vocab_perm + table.s[s].live_off : nullptr;
+    CUtensorMap segK, segMN;
+    if (!perm_seg) {
+      if (!make_map(&segK, sg.s[s].E, D, ns, D, BK, BN)) return CCE_ELAUNCH;
+      if (!make_map(&segMN, sg.s[s].E, D, ns, D, 64, 64)) return CCE_ELAUNCH;
+    }
+    for (int c0 = 0; c0 < ns; c0 += Vc) {
+      const int cv = std::min(Vc, ns - c0);
+      int row0 = c0;
+      if (perm_seg) {
+        gather_perm_rows_kernel<<<sms * 4, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(sg.s[s].E), perm_seg + c0, cv, (int)D, Ec);
+        if (launched()) return CCE_ELAUNCH;
+        if (!make_map(&segK, Ec, D, cv, D, BK, BN)) return CCE_ELAUNCH;
+        if (!make_map(&segMN, Ec, D, cv, D, 64, 64)) return CCE_ELAUNCH;
+        row0 = 0;
+      }
+      // step 1: G for this chunk
+      gp.mapB = segK;
+      gp.b_row0 = row0;
+      gp.chunk_valid = cv;
+      gp.ct = (int)cdiv(cv, BN);
+      gp.seg = s;
+      gp.c0 = c0;
+      gp.Vc = Vc;
+      gp.nkb = nkbD;
+      gp.n_valid = cp.n_valid;
+      gp.lse2_c = cp.lse2_c;
+      gp.dloss_c = cp.dloss_c;
+      gp.tseg = cp.tseg;
+      gp.tpos = cp.tpos;
+      gp.eps_keep = eps_keep;
+      gp.G = G;
+      gp.debug_keep = debug_keep;
+      gp.debug_rows = (int)debug_rows;
+      gp.words_per_row = words;
+      gp.idx = cp.idx;
+      gp.seg_begin = table.s[s].begin;
+      gp.perm_seg = perm_seg;
+      gp.status = status;
+      if (int rc = launch_tc<GPolicy>(gp, (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct), st))
+        return rc;
+      // step 2: dE rows of this chunk
+      ep.chunk_valid = cv;
+      ep.mt = (int)cdiv(cv, BM);
+      ep.dt = dt;
+      ep.D = (int)D;
+      ep.c0 = c0;
+      ep.perm_seg = perm_seg;
+      ep.dE = sg.s[s].dE;
+      ep.dE_comp = static_cast<__nv_bfloat16*>(sg.s[s].dE_comp);
+      ep.mode = kahan ? 2 : (fp32 ? 1 : 0);
+      ep.n_valid = cp.n_valid;
+      ep.status = status;
+      if (int rc = launch_tc<DEPolicy>(ep, (int)std::min<int64_t>(sms, (int64_t)ep.mt * dt), st))
+        return rc;
+      // step 3: dH += G E_chunk
+      hp.mapB = segMN;
+      hp.b_row0 = row0;
+      hp.nkb = (int)cdiv(cv, BK);
+      hp.dt = dt;
+      hp.D = (int)D;
+      hp.dH_acc = dH_acc;
+      hp.n_valid = cp.n_valid;
+      hp.status = status;
+      if (int rc = launch_tc<DHPolicy>(hp, (int)std::min<int64_t>(sms, (int64_t)mbs * dt), st))
+        return rc;
+    }
+  }
+  dh_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, 8), sms * 8), 256, 0, st>>>(
+      dH_acc, cp.pos_of_row, (int)N, (int)D, dH, fp32 ? 1 : 0);
+  return launched();
+}
+
+
+size_t cce_vocab_sort_workspace_size(int64_t N, int64_t V, int32_t n_segs) {
+  (void)N;
+  if (V <= 0 || V > (int64_t)INT32_MAX - 256 || n_segs < 0 || n_segs > CCE_MAX_SEGMENTS) return 0;
+  return plan_sort(V).total;
+}
+
+int cce_vocab_sort(const float* colmax, const int32_t* y, int64_t N, int64_t V, int32_t ignore_index,
+                   const cce_segment* segs, int32_t n_segs, int32_t* vocab_perm, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  if (V <= 0 || N < 0 || !vocab_perm) return CCE_EINVAL;
+  if (!colmax && !y && N > 0) return CCE_EINVAL;
+  Segs sg;
+  // the classifier pointers are not needed here; accept any non-null marker
+  if (segs == nullptr || n_segs == 0) {
+    sg.n = 1;
+    sg.s[0] = cce_segment{0, V, vocab_perm, nullptr, nullptr};
+    sg.live = V;
+  } else {
+    cce_segment tmp[CCE_MAX_SEGMENTS];
+    if (n_segs < 0 || n_segs > CCE_MAX_SEGMENTS) return CCE_EINVAL;
+    for (int i = 0; i < n_segs; ++i) {
+      tmp[i] = segs[i];
+      tmp[i].E = vocab_perm;
+    }
+    if (int rc = build_segs(nullptr, V, tmp, n_segs, sg)) return rc;
+  }
+  const SortPlan pl = plan_sort(V);
+  if (!workspace || workspace_bytes < pl.total) return CCE_EWORKSPACE;
+  const int sms = device_sms();
+  if (sms <= 0) return CCE_EDEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int T_v = 0;
+  const SegTable table = dev_table(sg, &T_v);
+  float* key = at<float>(workspace, pl.off_key);
+  float* key_out = at<float>(workspace, pl.off_key_out);
+  int* ids = at<int>(workspace, pl.off_ids);
+  void* tmp = at<void>(workspace, pl.off_tmp);
+  if (colmax) {
+    if (cudaMemcpyAsync(key, colmax, sizeof(float) * sg.live, cudaMemcpyDeviceToDevice, st) !=
+        cudaSuccess)
+      return CCE_ELAUNCH;
+  } else {
+    if (cudaMemsetAsync(key, 0, sizeof(float) * sg.live, st) != cudaSuccess) return CCE_ELAUNCH;
+    if (N > 0) {
+      target_hist_kernel<<<sms * 4, 256, 0, st>>>(y, (int)N, ignore_index, table, key);
+      if (launched()) return CCE_ELAUNCH;
+    }
+  }
+  for (int s = 0; s < sg.n; ++s) {
+    const int n = table.s[s].n, off = table.s[s].live_off;
+    iota_kernel<<<(int)std::min<int64_t>(cdiv(n, 256), sms * 8), 256, 0, st>>>(ids + off, n);
+    if (launched()) return CCE_ELAUNCH;
+    size_t need = 0;
+    if (cub::DeviceRadixSort::SortPairsDescending(nullptr, need, key + off, key_out + off, ids + off,
+                                                  vocab_perm + off, n, 0, 32, st) != cudaSuccess)
+      return CCE_ELAUNCH;
+    if (need > pl.tmp_bytes) return CCE_EWORKSPACE;
+    size_t have = pl.tmp_bytes;
+    if (cub::DeviceRadixSort::SortPairsDescending(tmp, have, key + off, key_out + off, ids + off,
+                                                  vocab_perm + off, n, 0, 32, st) != cudaSuccess)
+      return CCE_ELAUNCH;
+  }
+  return CCE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,241 @@
+// Warp-specialised tcgen05 tile engine shared by every tensor-core kernel of
+// the library.
+//
+// One CTA per SM (persistent), 192 threads:
+//   warp 0      one thread issues TMA tile loads into a STAGES-deep ring of
+//               shared-memory stages (A: 128 x 64 bf16, B: 256 x 64 bf16);
+//   warp 1      allocates 512 TMEM columns; one thread issues
+//               tcgen05.mma (M=128, N=256, K=16) into one of two 256-column
+//               fp32 accumulators, so the epilogue of tile t overlaps the
+//               MMAs of tile t+1;
+//   warps 2..5  the epilogue: thread (warp&3)*32+lane owns accumulator row
+//               (TMEM lane) (warp&3)*32+lane and reads it with tcgen05.ld.
+// A policy class supplies the tile order (identical for all roles), the TMA
+// coordinates and the epilogue.  Operands may be K-major (rows of K) or
+// MN-major (rows of M/N) in global memory; both are staged with 128-byte
+// swizzling, which the UMMA descriptors describe.
+#pragma once
+
+#include "cce_ptx.cuh"
+
+namespace cce {
+
+constexpr int BM = 128;   // accumulator rows (TMEM lanes)
+constexpr int BN = 256;   // accumulator columns
+constexpr int BK = 64;    // K per stage: one 128-byte swizzle row of bf16
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 192;
+constexpr int EPI_THREADS = 128;
+constexpr uint32_t TMEM_COLS = 512;
+
+struct Ctl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int consumed;
+  int pad;
+};
+
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + static_cast<int>(sizeof(Ctl)) + 64;
+
+struct Pipe {
+  int stage = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void advance() {
+    if (++stage == STAGES) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+// Per-role state handed to policies.
+struct Engine {
+  Ctl* ctl;
+  uint8_t* smem;  // 1024-byte aligned stage ring
+  uint32_t tmem;
+  int* status;
+  Pipe pipe;
+  int tcount = 0;  // accumulator tiles handled by this role
+  int fills = 0;   // stage fills issued (producer) / consumed (MMA)
+
+  __device__ __forceinline__ volatile int* abort_flag() { return &ctl->abort; }
+
+  // ---- producer: load nkb stages of one tile.  (ax, ay) / (bx, by) are the
+  // tensor-map coordinates of the tile origin; K advances along x for a
+  // K-major operand and along y for an MN-major one.
+  template <bool A_MN, bool B_MN>
+  __device__ __forceinline__ bool produce(const CUtensorMap* mA, const CUtensorMap* mB, int ax,
+                                          int ay, int bx, int by, int nkb) {
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!wait_parity(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u, abort_flag(), status))
+        return false;
+      const uint32_t fb = smem_u32(&ctl->full[pipe.stage]);
+      mbar_arrive_expect_tx(fb, STAGE_BYTES);
+      const uint32_t sa = smem_u32(smem + pipe.stage * STAGE_BYTES);
+      const uint32_t sb = sa + A_BYTES;
+      if (!A_MN) {
+        tma_load_2d(sa, mA, fb, ax + kb * BK, ay);
+      } else {
+        tma_load_2d(sa, mA, fb, ax, ay + kb * BK);
+        tma_load_2d(sa + 8192, mA, fb, ax + 64, ay + kb * BK);
+      }
+      if (!B_MN) {
+        tma_load_2d(sb, mB, fb, bx + kb * BK, by);
+      } else {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_load_2d(sb + b * 8192, mB, fb, bx + b * 64, by + kb * BK);
+      }
+      pipe.advance();
+      ++fills;
+    }
+    return true;
+  }
+
+  // ---- MMA issuer: accumulate one tile over nkb stages into the next
+  // accumulator.  kmask (optional) has bit kb*4+kk set for every K=16 step
+  // that must be issued; cleared bits are skipped (all-zero A slices).  When
+  // a mask skips every step the accumulator is left untouched, so the
+  // policy's epilogue must recognise such a tile from the same mask and
+  // treat it as zero.
+  template <bool A_MN, bool B_MN>
+  __device__ __forceinline__ bool mma(int nkb, const uint32_t* kmask = nullptr) {
+    const int acc = tcount & 1;
+    if (!wait_parity(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u,
+                     abort_flag(), status))
+      return false;
+    tc_fence_after();
+    const uint32_t d = tmem + acc * BN;
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+    uint32_t issued = 0;
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!wait_parity(smem_u32(&ctl->full[pipe.stage]), pipe.phase, abort_flag(), status))
+        return false;
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + pipe.stage * STAGE_BYTES);
+      const uint32_t sb = sa + A_BYTES;
+      const uint32_t bits = kmask ? ((kmask[kb >> 3] >> ((kb & 7) * 4)) & 0xFu) : 0xFu;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        if (!(bits & (1u << kk))) continue;
+        const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                 : smem_desc_sw128(sa + kk * 32, 16, 1024);
+        const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                 : smem_desc_sw128(sb + kk * 32, 16, 1024);
+        umma_bf16(d, ad, bd, idesc, issued);
+        issued = 1;
+      }
+      umma_commit(smem_u32(&ctl->empty[pipe.stage]));
+      pipe.advance();
+      ++fills;
+    }
+    umma_commit(smem_u32(&ctl->tfull[acc]));
+    ++tcount;
+    return true;
+  }
+
+  // ---- epilogue: wait for the next accumulator; returns its TMEM address
+  // for this thread's lane quarter (column 0).
+  __device__ __forceinline__ bool epi_acquire(int quarter, uint32_t& taddr) {
+    const int acc = tcount & 1;
+    if (!wait_parity(smem_u32(&ctl->tfull[acc]), ((uint32_t)tcount >> 1) & 1u, abort_flag(),
+                     status))
+      return false;
+    tc_fence_after();
+    taddr = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
+    return true;
+  }
+  __device__ __forceinline__ void epi_release(int lane) {
+    const int acc = tcount & 1;
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&ctl->tempty[acc]));
+    ++tcount;
+  }
+};
+
+// Bounded wait that ignores the abort flag (used only while draining).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return;
+    if ((it & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+// The kernel body: set-up, role dispatch, drain, TMEM release.
+template <class Policy>
+__global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ typename Policy::Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (base & 1023u)) & 1023u);
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&ctl->full[s]), 1);
+      mbar_init(smem_u32(&ctl->empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&ctl->tfull[a]), 1);
+      mbar_init(smem_u32(&ctl->tempty[a]), EPI_THREADS / 32);
+    }
+    mbar_init(smem_u32(&ctl->drain), 1);
+    ctl->abort = 0;
+    ctl->consumed = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) Policy::prefetch(p);
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  Engine eng;
+  eng.ctl = ctl;
+  eng.smem = smem;
+  eng.tmem = ctl->tmem_base;
+  eng.status = p.status;
+
+  if (warp == 0) {
+    if (lane == 0) Policy::producer(p, eng);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      Policy::mma(p, eng);
+      ctl->consumed = eng.fills;
+      // wait until every tcgen05 op this thread issued has completed
+      umma_commit(smem_u32(&ctl->drain));
+      drain_wait(smem_u32(&ctl->drain), 0);
+    }
+  } else {
+    Policy::epilogue(p, eng, warp & 3, lane);
+  }
+  __syncthreads();
+  if (warp == 0 && lane == 0 && ctl->abort) {
+    // stage fills issued but never consumed (only after an abort): let the
+    // copies land before the CTA exits
+    for (int f = ctl->consumed; f < eng.fills; ++f)
+      drain_wait(smem_u32(&ctl->full[f % STAGES]), (uint32_t)(f / STAGES) & 1u);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(ctl->tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace cce

@@ -1,0 +1,694 @@
+// Kernels of the Cut Cross-Entropy hot path.
+//
+// Sources (web pages, by title and section):
+//   [LM]  "The loss and the mask: Cut Cross-Entropy + FlexAttention (2
+//         papers)", part "Cut Your Losses in Large-Vocabulary Language Models
+//         (CCE)": §Contribution (indexed dot product for the correct-token
+//         logit; blockwise log-sum-exp streamed over vocabulary tiles, logits
+//         never written to global memory; backward skips softmax entries
+//         below bf16 precision; vocabulary sort), §What transfers to us
+//         (valid-row select before the math; two-segment lse by log-add-exp
+//         with a -inf dead gap).
+//   [MAP] "Cut Your Losses in Large-Vocabulary Language Models" (research
+//         map): §Approach (backward recomputes logits blockwise),
+//         §Limitations (thread-safe log-add-exp of partial results; Kahan
+//         summation for the classifier gradient).
+//
+// Forward:  compact_kernel -> gather_rows_kernel -> tc_kernel<FwdPolicy>
+//           (S = H_c E^T tiles in TMEM, online max/sum-exp per row, one
+//           (max, sum) partial per row and vocabulary split) ->
+//           fwd_finalize_kernel (log-add-exp of the partials, correct-token
+//           logit as an fp32 dot product, loss = lse - z_y).
+// Backward: per vocabulary chunk of Vc entries (a bounded slab, never N x V):
+//           tc_kernel<GPolicy> recomputes S and writes
+//           G = dloss * (softmax * keep - onehot) in bf16 with block masks;
+//           tc_kernel<DEPolicy> dE_chunk = G^T H_c (K = rows, on chip);
+//           tc_kernel<DHPolicy> dH_acc += G E_chunk (K = chunk);
+//           then dh_finalize_kernel scatters dH back to the original rows.
+#pragma once
+
+#include <cub/block/block_scan.cuh>
+
+#include "cce_engine.cuh"
+
+namespace cce {
+
+constexpr int MAX_SEGS = 8;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct SegDev {
+  long long begin, end;  // logical ids [begin, end)
+  int n;                 // live rows (end - begin)
+  int tile_off;          // first 256-wide forward tile of this segment
+  int live_off;          // offset in the concatenated live vocabulary
+  int pad;
+  const __nv_bfloat16* E;
+};
+
+struct SegTable {
+  int n_segs;
+  int pad;
+  SegDev s[MAX_SEGS];
+};
+
+__device__ __forceinline__ int segment_of(const SegTable& t, long long y) {
+  for (int s = 0; s < t.n_segs; ++s)
+    if (y >= t.s[s].begin && y < t.s[s].end) return s;
+  return -1;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// =====================================================================
+// Valid-row select ([LM] §What transfers to us): ordered compaction of the
+// rows whose target is not ignore_index.  Single CTA; N int32 reads.
+//   pos_of_row[i] = compact index, -1 for ignored rows, -2 for bad targets.
+// For the backward it also gathers lse (pre-scaled by log2 e), dloss and
+// the target's segment / walk position for each compact row.
+// =====================================================================
+struct CompactParams {
+  const int* y;
+  int N;
+  int ignore_index;
+  SegTable segs;
+  int* idx;
+  int* pos_of_row;
+  int* n_valid;
+  int* status;
+  // backward extras (nullable)
+  const float* lse;
+  const float* dloss;
+  const int* inv_perm;  // [V_live] walk position of each live row, or null
+  float* lse2_c;
+  float* dloss_c;
+  int* tseg;
+  int* tpos;
+};
+
+constexpr int COMPACT_THREADS = 1024;
+
+__device__ __forceinline__ int classify_row(const CompactParams& p, int i, int& seg) {
+  const int y = p.y[i];
+  if (y == p.ignore_index) return 0;
+  seg = segment_of(p.segs, (long long)y);
+  return seg < 0 ? 2 : 1;
+}
+
+__global__ void __launch_bounds__(COMPACT_THREADS) compact_kernel(const CompactParams p) {
+  using Scan = cub::BlockScan<int, COMPACT_THREADS>;
+  __shared__ typename Scan::TempStorage tmp;
+  const int per = (p.N + COMPACT_THREADS - 1) / COMPACT_THREADS;
+  const int lo = threadIdx.x * per;
+  const int hi = min(p.N, lo + per);
+  int cnt = 0;
+  for (int i = lo; i < hi; ++i) {
+    int s;
+    cnt += classify_row(p, i, s) == 1;
+  }
+  int off, total;
+  Scan(tmp).ExclusiveSum(cnt, off, total);
+  bool bad = false;
+  for (int i = lo; i < hi; ++i) {
+    int s = -1;
+    const int st = classify_row(p, i, s);
+    if (st == 1) {
+      p.idx[off] = i;
+      p.pos_of_row[i] = off;
+      if (p.lse2_c) {
+        const int y = p.y[i];
+        const int loc = y - (int)p.segs.s[s].begin;
+        p.lse2_c[off] = p.lse[i] * kLog2e;
+        p.dloss_c[off] = p.dloss[i];
+        p.tseg[off] = s;
+        p.tpos[off] = p.inv_perm ? p.inv_perm[p.segs.s[s].live_off + loc] : loc;
+      }
+      ++off;
+    } else {
+      p.pos_of_row[i] = st == 0 ? -1 : -2;
+      bad |= st == 2;
+    }
+  }
+  if (bad) atomicOr(p.status, kStatusBadTarget);
+  if (threadIdx.x == 0) *p.n_valid = total;
+}
+
+// H_c[j] = H[idx[j]] for j < n_valid, zero rows for n_valid <= j < Npad.
+// One warp per row, 16-byte vectors.  D is a multiple of 8.
+__global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ H, const int* __restrict__ idx,
+                                   const int* __restrict__ n_valid, int Npad, int D,
+                                   __nv_bfloat16* __restrict__ Hc) {
+  const int lane = threadIdx.x & 31;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int nv = *n_valid;
+  const int vec = D >> 3;
+  for (int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; j < Npad; j += nw) {
+    uint4* dst = reinterpret_cast<uint4*>(Hc + (size_t)j * D);
+    if (j < nv) {
+      const uint4* src = reinterpret_cast<const uint4*>(H + (size_t)idx[j] * D);
+      for (int v = lane; v < vec; v += 32) dst[v] = __ldg(src + v);
+    } else {
+      for (int v = lane; v < vec; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+// dst[k] = src[perm[k]] for k < rows (vocabulary rows in walk order).
+__global__ void gather_perm_rows_kernel(const __nv_bfloat16* __restrict__ src,
+                                        const int* __restrict__ perm, int rows, int D,
+                                        __nv_bfloat16* __restrict__ dst) {
+  const int lane = threadIdx.x & 31;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int vec = D >> 3;
+  for (int k = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; k < rows; k += nw) {
+    const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)perm[k] * D);
+    uint4* d = reinterpret_cast<uint4*>(dst + (size_t)k * D);
+    for (int v = lane; v < vec; v += 32) d[v] = __ldg(s + v);
+  }
+}
+
+// =====================================================================
+// Forward tile stream ([LM] §Contribution; [MAP] §Approach).
+// Work item = (row block mb, vocabulary split): tpi consecutive 256-wide
+// vocabulary tiles (tiles never straddle segments).  Items are ordered
+// split-major so the CTAs running at the same time share E tiles through
+// L2.  Each epilogue thread keeps (m, s) of its row in base-2 units:
+//   m = max_j z_j log2 e,  s = sum_j 2^(z_j log2 e - m).
+// =====================================================================
+struct FwdParams {
+  CUtensorMap mapA;            // H_c [Npad, D] bf16, box {64, 128}
+  CUtensorMap mapB[MAX_SEGS];  // E_s [n_s, D] bf16, box {64, 256}
+  SegTable segs;
+  int T_v;     // total vocabulary tiles
+  int tpi;     // tiles per work item
+  int S;       // splits = ceil(T_v / tpi)
+  int Npad;    // partial row stride
+  int nkb;     // ceil(D / 64)
+  const int* n_valid;
+  float2* part;  // [S, Npad] (m, s)
+  int* colmax;   // ordered-int running max per live vocabulary row, or null
+  int* status;
+};
+
+struct FwdPolicy {
+  using Params = FwdParams;
+
+  template <class F>
+  static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
+    const int nv = *p.n_valid;
+    const int num_mb = (nv + BM - 1) / BM;
+    const int num_items = num_mb * p.S;
+    for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
+      const int split = item / num_mb;
+      const int mb = item - split * num_mb;
+      const int t0 = split * p.tpi;
+      const int t1 = min(p.T_v, t0 + p.tpi);
+      int s = 0;
+      for (int t = t0; t < t1; ++t) {
+        while (s + 1 < p.segs.n_segs && t >= p.segs.s[s + 1].tile_off) ++s;
+        if (!f(mb, split, t, s, t == t1 - 1, nv)) return;
+      }
+    }
+  }
+
+  static __device__ void prefetch(const Params& p) {
+    tma_prefetch_map(&p.mapA);
+    for (int s = 0; s < p.segs.n_segs; ++s) tma_prefetch_map(&p.mapB[s]);
+  }
+
+  static __device__ void producer(const Params& p, Engine& eng) {
+    schedule(p, [&](int mb, int, int t, int s, bool, int) {
+      return eng.produce<false, false>(&p.mapA, &p.mapB[s], 0, mb * BM, 0,
+                                       (t - p.segs.s[s].tile_off) * BN, p.nkb);
+    });
+  }
+
+  static __device__ void mma(const Params& p, Engine& eng) {
+    schedule(p, [&](int, int, int, int, bool, int) { return eng.mma<false, false>(p.nkb); });
+  }
+
+  static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
+    const int row = q * 32 + lane;
+    float m2 = -INFINITY, sum = 0.f;
+    schedule(p, [&](int mb, int split, int t, int s, bool last, int nv) {
+      uint32_t taddr;
+      if (!eng.epi_acquire(q, taddr)) return false;
+      const SegDev& sg = p.segs.s[s];
+      const int e0 = (t - sg.tile_off) * BN;
+      const int valid = min(BN, sg.n - e0);
+      const bool row_ok = mb * BM + row < nv;
+      for (int c = 0; c < BN / 32; ++c) {
+        if (c * 32 >= valid) break;  // uniform over the CTA
+        uint32_t r[32];
+        tmem_ld32(taddr + c * 32, r);
+        float cmax = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float v = (c * 32 + j < valid) ? __uint_as_float(r[j]) : -INFINITY;
+          r[j] = __float_as_uint(v);
+          cmax = fmaxf(cmax, v);
+        }
+        if (p.colmax) {
+          int mine = 0;
+          const int neg = f32_to_ordered(-INFINITY);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int key = row_ok ? f32_to_ordered(__uint_as_float(r[j])) : neg;
+            const int red = __reduce_max_sync(0xffffffffu, key);
+            if (lane == j) mine = red;
+          }
+          if (c * 32 + lane < valid) atomicMax(&p.colmax[sg.live_off + e0 + c * 32 + lane], mine);
+        }
+        const float mn = fmaxf(m2, cmax * kLog2e);
+        float acc = sum * ex2_approx(m2 - mn);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc += ex2_approx(fmaf(__uint_as_float(r[j]), kLog2e, -mn));
+        sum = acc;
+        m2 = mn;
+      }
+      eng.epi_release(lane);
+      if (last) {
+        if (row_ok) p.part[(size_t)split * p.Npad + mb * BM + row] = make_float2(m2, sum);
+        m2 = -INFINITY;
+        sum = 0.f;
+      }
+      return true;
+    });
+  }
+};
+
+// log-add-exp of the split partials, the correct-token logit as an indexed
+// dot product in fp32, loss = lse - z_y.  One warp per original row.
+struct FinParams {
+  const __nv_bfloat16* H;
+  const int* y;
+  const int* pos_of_row;
+  const float2* part;
+  SegTable segs;
+  int N, D, S, Npad;
+  float* loss;
+  float* lse;
+};
+
+__global__ void fwd_finalize_kernel(const FinParams p) {
+  const int lane = threadIdx.x & 31;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < p.N; i += nw) {
+    const int j = p.pos_of_row[i];
+    if (j < 0) {
+      if (lane == 0) {
+        const float v = j == -1 ? 0.f : __int_as_float(0x7fc00000);
+        p.loss[i] = v;
+        p.lse[i] = v;
+      }
+      continue;
+    }
+    float M = -INFINITY;
+    for (int s = lane; s < p.S; s += 32) M = fmaxf(M, p.part[(size_t)s * p.Npad + j].x);
+    M = warp_max(M);
+    float acc = 0.f;
+    for (int s = lane; s < p.S; s += 32) {
+      const float2 v = p.part[(size_t)s * p.Npad + j];
+      acc += v.y * ex2_approx(v.x - M);
+    }
+    acc = warp_sum(acc);
+    const int y = p.y[i];
+    const int sg = segment_of(p.segs, (long long)y);
+    const uint4* h = reinterpret_cast<const uint4*>(p.H + (size_t)i * p.D);
+    const uint4* e = reinterpret_cast<const uint4*>(p.segs.s[sg].E +
+                                                    (size_t)(y - p.segs.s[sg].begin) * p.D);
+    float dot = 0.f;
+    for (int v = lane; v < (p.D >> 3); v += 32) {
+      const uint4 a = __ldg(h + v), b = __ldg(e + v);
+      dot = fmaf(bf16lo(a.x), bf16lo(b.x), dot);
+      dot = fmaf(bf16hi(a.x), bf16hi(b.x), dot);
+      dot = fmaf(bf16lo(a.y), bf16lo(b.y), dot);
+      dot = fmaf(bf16hi(a.y), bf16hi(b.y), dot);
+      dot = fmaf(bf16lo(a.z), bf16lo(b.z), dot);
+      dot = fmaf(bf16hi(a.z), bf16hi(b.z), dot);
+      dot = fmaf(bf16lo(a.w), bf16lo(b.w), dot);
+      dot = fmaf(bf16hi(a.w), bf16hi(b.w), dot);
+    }
+    dot = warp_sum(dot);
+    if (lane == 0) {
+      const float l = (M + log2f(acc)) * kLn2;
+      p.lse[i] = l;
+      p.loss[i] = l - dot;
+    }
+  }
+}
+
+__global__ void colmax_init_kernel(int* colmax, int n) {
+  const int neg = f32_to_ordered(-INFINITY);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    colmax[i] = neg;
+}
+__global__ void colmax_final_kernel(int* colmax, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    reinterpret_cast<float*>(colmax)[i] = ordered_to_f32(colmax[i]);
+}
+
+// =====================================================================
+// Backward, step 1: recompute S for a vocabulary chunk and write
+// G = dloss_i * (p_ij * keep_ij - [j == y_i]) in bf16 ([MAP] §Approach:
+// logits recomputed blockwise; [LM] §Contribution: entries below bf16
+// precision carry no gradient).  p_ij = 2^(z_ij log2 e - lse_i log2 e).
+// keep_ij = p_ij >= eps_keep (element granularity).
+// =====================================================================
+struct GParams {
+  CUtensorMap mapA;  // H_c [Npad, D], box {64, 128}
+  CUtensorMap mapB;  // chunk rows of E, K-major, box {64, 256}
+  int b_row0;        // map row of the chunk's first vocabulary entry
+  int chunk_valid;   // vocabulary entries in this chunk
+  int ct;            // 256-wide tiles in the chunk
+  int seg, c0;       // segment and walk position of the chunk start
+  int Vc;            // G row stride (elements)
+  int nkb;
+  const int* n_valid;
+  const float* lse2_c;
+  const float* dloss_c;
+  const int* tseg;
+  const int* tpos;
+  float eps_keep;  // 0: keep everything
+  __nv_bfloat16* G;
+  // optional per-element keep bits of original rows < debug_rows
+  uint32_t* debug_keep;
+  int debug_rows;
+  int words_per_row;
+  const int* idx;
+  long long seg_begin;
+  const int* perm_seg;  // walk position -> local row, or null
+  int* status;
+};
+
+struct GPolicy {
+  using Params = GParams;
+
+  template <class F>
+  static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
+    const int nv = *p.n_valid;
+    const int num_mb = (nv + BM - 1) / BM;
+    const int tiles = num_mb * p.ct;
+    for (int i = blockIdx.x; i < tiles; i += gridDim.x) {
+      const int vt = i / num_mb;
+      if (!f(i - vt * num_mb, vt, nv)) return;
+    }
+  }
+  static __device__ void prefetch(const Params& p) {
+    tma_prefetch_map(&p.mapA);
+    tma_prefetch_map(&p.mapB);
+  }
+  static __device__ void producer(const Params& p, Engine& eng) {
+    schedule(p, [&](int mb, int vt, int) {
+      return eng.produce<false, false>(&p.mapA, &p.mapB, 0, mb * BM, 0, p.b_row0 + vt * BN, p.nkb);
+    });
+  }
+  static __device__ void mma(const Params& p, Engine& eng) {
+    schedule(p, [&](int, int, int) { return eng.mma<false, false>(p.nkb); });
+  }
+  static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
+    const int row = q * 32 + lane;
+    schedule(p, [&](int mb, int vt, int nv) {
+      uint32_t taddr;
+      if (!eng.epi_acquire(q, taddr)) return false;
+      const int jrow = mb * BM + row;
+      const bool ok = jrow < nv;
+      const float lse2 = ok ? p.lse2_c[jrow] : 0.f;
+      const float dl = ok ? p.dloss_c[jrow] : 0.f;
+      const int tcol = (ok && p.tseg[jrow] == p.seg) ? p.tpos[jrow] - p.c0 - vt * BN : -1;
+      const int valid = p.chunk_valid - vt * BN;  // valid columns of this tile
+      __nv_bfloat16* grow = p.G + (size_t)jrow * p.Vc + vt * BN;
+      const bool dbg = p.debug_keep != nullptr && ok && p.idx[jrow] < p.debug_rows;
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(taddr + c * 32, r);
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          float g[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int col = c * 32 + j + u;
+            const float pr = ex2_approx(fmaf(__uint_as_float(r[j + u]), kLog2e, -lse2));
+            const bool keep = pr >= p.eps_keep;
+            float v = keep ? pr : 0.f;
+            v -= (col == tcol) ? 1.f : 0.f;
+            g[u] = (ok && col < valid) ? dl * v : 0.f;
+          }
+          packed[j >> 1] = pack_bf16(g[0], g[1]);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
+        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        dst[2] = make_uint4(packed[8], packed[9], packed[10], packed[11]);
+        dst[3] = make_uint4(packed[12], packed[13], packed[14], packed[15]);
+        if (dbg) {
+          const int orig = p.idx[jrow];
+          for (int j = 0; j < 32; ++j) {
+            const int col = c * 32 + j;
+            if (col >= valid) break;
+            const float pr = ex2_approx(fmaf(__uint_as_float(r[j]), kLog2e, -lse2));
+            if (pr >= p.eps_keep) {
+              const int w = p.c0 + vt * BN + col;
+              const long long lid = p.seg_begin + (p.perm_seg ? p.perm_seg[w] : w);
+              atomicOr(&p.debug_keep[(size_t)orig * p.words_per_row + (lid >> 5)],
+                       1u << (lid & 31));
+            }
+          }
+        }
+      }
+      eng.epi_release(lane);
+      return true;
+    });
+  }
+};
+
+// =====================================================================
+// Backward, step 2: dE_chunk = G^T H_c, K = compact rows, accumulated on
+// chip; each output element written once (bf16, fp32, or Kahan-added into
+// a bf16 sum with a bf16 compensation: [MAP] §Limitations).
+// =====================================================================
+struct DEParams {
+  CUtensorMap mapA;  // G viewed MN-major: [Npad rows, Vc], box {64, 64}
+  CUtensorMap mapB;  // H_c MN-major: [Npad, D], box {64, 64}
+  int chunk_valid;
+  int mt;  // 128-row vocabulary tiles
+  int dt;  // 256-wide D tiles
+  int D;
+  int c0;
+  const int* perm_seg;  // walk position -> local row, or null
+  void* dE;             // segment base
+  __nv_bfloat16* dE_comp;
+  int mode;  // 0 bf16 store, 1 fp32 store, 2 Kahan bf16
+  const int* n_valid;
+  int* status;
+};
+
+struct DEPolicy {
+  using Params = DEParams;
+
+  template <class F>
+  static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
+    const int nkb = (*p.n_valid + BK - 1) / BK;
+    const int tiles = p.mt * p.dt;
+    for (int i = blockIdx.x; i < tiles; i += gridDim.x) {
+      const int vt = i / p.dt;
+      if (!f(vt, i - vt * p.dt, nkb)) return;
+    }
+  }
+  static __device__ void prefetch(const Params& p) {
+    tma_prefetch_map(&p.mapA);
+    tma_prefetch_map(&p.mapB);
+  }
+  static __device__ void producer(const Params& p, Engine& eng) {
+    schedule(p, [&](int vt, int dtile, int nkb) {
+      return eng.produce<true, true>(&p.mapA, &p.mapB, vt * BM, 0, dtile * BN, 0, nkb);
+    });
+  }
+  static __device__ void mma(const Params& p, Engine& eng) {
+    schedule(p, [&](int, int, int nkb) { return nkb == 0 || eng.mma<true, true>(nkb); });
+  }
+  static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
+    const int row = q * 32 + lane;
+    schedule(p, [&](int vt, int dtile, int nkb) {
+      uint32_t taddr = 0;
+      if (nkb > 0 && !eng.epi_acquire(q, taddr)) return false;
+      const int r = vt * BM + row;
+      const bool ok = r < p.chunk_valid;
+      const int w = p.c0 + r;
+      const size_t local = ok ? (size_t)(p.perm_seg ? p.perm_seg[w] : w) : 0;
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = dtile * BN + c * 32;
+        if (col0 >= p.D) break;
+        uint32_t v[32];
+        if (nkb > 0) {
+          tmem_ld32(taddr + c * 32, v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0u;
+        }
+        if (!ok) continue;
+        const size_t off = local * p.D + col0;
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+          if (col0 + g8 * 8 >= p.D) break;
+          const float* f = reinterpret_cast<const float*>(v) + g8 * 8;
+          if (p.mode == 1) {
+            float4* d = reinterpret_cast<float4*>(static_cast<float*>(p.dE) + off + g8 * 8);
+            d[0] = make_float4(f[0], f[1], f[2], f[3]);
+            d[1] = make_float4(f[4], f[5], f[6], f[7]);
+          } else if (p.mode == 0) {
+            uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dE) + off + g8 * 8);
+            *d = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                            pack_bf16(f[6], f[7]));
+          } else {
+            uint4* ds = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dE) + off + g8 * 8);
+            uint4* dc = reinterpret_cast<uint4*>(p.dE_comp + off + g8 * 8);
+            const uint4 s4 = *ds, c4 = *dc;
+            const uint32_t sw[4] = {s4.x, s4.y, s4.z, s4.w};
+            const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
+            uint32_t so[4], co[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              float sv[2] = {bf16lo(sw[k]), bf16hi(sw[k])};
+              float cv[2] = {bf16lo(cw[k]), bf16hi(cw[k])};
+              float tn[2], cn[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const float yv = f[2 * k + u] - cv[u];
+                const float t = __bfloat162float(__float2bfloat16_rn(sv[u] + yv));
+                cn[u] = (t - sv[u]) - yv;
+                tn[u] = t;
+              }
+              so[k] = pack_bf16(tn[0], tn[1]);
+              co[k] = pack_bf16(cn[0], cn[1]);
+            }
+            *ds = make_uint4(so[0], so[1], so[2], so[3]);
+            *dc = make_uint4(co[0], co[1], co[2], co[3]);
+          }
+        }
+      }
+      if (nkb > 0) eng.epi_release(lane);
+      return true;
+    });
+  }
+};
+
+// =====================================================================
+// Backward, step 3: dH_acc[j, :] += G[j, chunk] E_chunk, K = chunk.
+// =====================================================================
+struct DHParams {
+  CUtensorMap mapA;  // G K-major: [Npad, Vc], box {64, 128}
+  CUtensorMap mapB;  // chunk rows of E, MN-major: box {64, 64}
+  int b_row0;
+  int nkb;  // ceil(chunk_valid / 64)
+  int dt;
+  int D;
+  float* dH_acc;  // [Npad, D]
+  const int* n_valid;
+  int* status;
+};
+
+struct DHPolicy {
+  using Params = DHParams;
+
+  template <class F>
+  static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
+    const int nv = *p.n_valid;
+    const int num_mb = (nv + BM - 1) / BM;
+    const int tiles = num_mb * p.dt;
+    for (int i = blockIdx.x; i < tiles; i += gridDim.x) {
+      const int mb = i / p.dt;
+      if (!f(mb, i - mb * p.dt, nv)) return;
+    }
+  }
+  static __device__ void prefetch(const Params& p) {
+    tma_prefetch_map(&p.mapA);
+    tma_prefetch_map(&p.mapB);
+  }
+  static __device__ void producer(const Params& p, Engine& eng) {
+    schedule(p, [&](int mb, int dtile, int) {
+      return eng.produce<false, true>(&p.mapA, &p.mapB, 0, mb * BM, dtile * BN, p.b_row0, p.nkb);
+    });
+  }
+  static __device__ void mma(const Params& p, Engine& eng) {
+    schedule(p, [&](int, int, int) { return eng.mma<false, true>(p.nkb); });
+  }
+  static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
+    const int row = q * 32 + lane;
+    schedule(p, [&](int mb, int dtile, int nv) {
+      uint32_t taddr;
+      if (!eng.epi_acquire(q, taddr)) return false;
+      const int j = mb * BM + row;
+      const bool ok = j < nv;
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = dtile * BN + c * 32;
+        if (col0 >= p.D) break;
+        uint32_t v[32];
+        tmem_ld32(taddr + c * 32, v);
+        if (!ok) continue;
+        float* d = p.dH_acc + (size_t)j * p.D + col0;
+#pragma unroll
+        for (int g4 = 0; g4 < 8; ++g4) {
+          if (col0 + g4 * 4 >= p.D) break;
+          float4 a = *reinterpret_cast<float4*>(d + g4 * 4);
+          a.x += __uint_as_float(v[g4 * 4 + 0]);
+          a.y += __uint_as_float(v[g4 * 4 + 1]);
+          a.z += __uint_as_float(v[g4 * 4 + 2]);
+          a.w += __uint_as_float(v[g4 * 4 + 3]);
+          *reinterpret_cast<float4*>(d + g4 * 4) = a;
+        }
+      }
+      eng.epi_release(lane);
+      return true;
+    });
+  }
+};
+
+// dH[i] = dH_acc[pos_of_row[i]] (bf16 or fp32); 0 for ignored rows, NaN for
+// rows with a bad target.  One warp per row.
+__global__ void dh_finalize_kernel(const float* __restrict__ dH_acc, const int* __restrict__ pos_of_row,
+                                   int N, int D, void* dH, int fp32_out) {
+  const int lane = threadIdx.x & 31;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int vec = D >> 2;
+  for (int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < N; i += nw) {
+    const int j = pos_of_row[i];
+    const float fill = j == -1 ? 0.f : __int_as_float(0x7fc00000);
+    const float4* src = reinterpret_cast<const float4*>(dH_acc + (size_t)(j < 0 ? 0 : j) * D);
+    for (int v = lane; v < vec; v += 32) {
+      const float4 a = j >= 0 ? src[v] : make_float4(fill, fill, fill, fill);
+      if (fp32_out) {
+        reinterpret_cast<float4*>(static_cast<float*>(dH) + (size_t)i * D)[v] = a;
+      } else {
+        reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(dH) + (size_t)i * D)[v] =
+            make_uint2(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w));
+      }
+    }
+  }
+}
+
+// inv[perm[k]] = k for one segment (perm and inv point at the segment's
+// slice of the concatenated live vocabulary; entries are segment-local).
+__global__ void invert_perm_kernel(const int* __restrict__ perm, int n, int* __restrict__ inv) {
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x)
+    inv[perm[k]] = k;
+}
+
+}  // namespace cce

@@ -1,0 +1,108 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/cce.h declares, and rejects bad arguments before any
+device work (no compute call is made here)."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+from linear_cross_entropy_cce_b200 import cce
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "cce.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(cce_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    L = cce.lib()
+    names = _declared()
+    assert set(names) >= set(cce.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.cce_version() >= 10000
+
+
+def test_strerror_covers_codes():
+    L = cce.lib()
+    for c in range(5):
+        assert L.cce_strerror(c)
+    assert b"unknown" in L.cce_strerror(99)
+
+
+def test_workspace_sizes_and_invalid_sizes():
+    L = cce.lib()
+    assert L.cce_fwd_workspace_size(256, 256, 4096, 0) > 0
+    assert L.cce_fwd_workspace_size(256, 250, 4096, 0) == 0      # D % 8 != 0
+    assert L.cce_fwd_workspace_size(-1, 256, 4096, 0) == 0
+    assert L.cce_fwd_workspace_size(256, 256, 0, 0) == 0
+    assert L.cce_fwd_workspace_size(256, 256, 4096, 9) == 0      # too many segments
+    assert L.cce_bwd_workspace_size(256, 256, 4096, 0, 0) > 0
+    assert L.cce_vocab_sort_workspace_size(256, 4096, 0) > 0
+
+
+def test_workspace_is_far_below_materialised_logits():
+    """The page on chunking CE after an OOM prints 12.2 GB for one bf16
+    softmax over 24,576 positions x 248,320 vocabulary; the research-map
+    entry prints 24000 MB of loss memory for Gemma 2 (2B).  libcce's scratch
+    for those shapes stays a small fraction of it (nothing N x V)."""
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "pages_memory.json")))
+    for case in g["cases"]:
+        N, D, V, nseg = case["N"], case["D"], case["V"], case["n_segs"]
+        assert abs(N * V * case["bytes_per_elt"] - case["page_bytes"]) <= case["rel_tol"] * case["page_bytes"]
+        ws = max(cce.fwd_workspace_size(N, D, V, nseg), cce.bwd_workspace_size(N, D, V, nseg))
+        assert ws < 0.05 * case["page_bytes"], (case["name"], ws)
+
+
+def _null_fwd(**kw):
+    L = cce.lib()
+    a = dict(H=16, E=16, y=16, N=4, D=8, V=10, ign=-100, segs=None, nseg=0, loss=16, lse=16,
+             colmax=None, ws=16, wsb=1 << 30, st=16, stream=None)
+    a.update(kw)
+    return L.cce_fwd(a["H"], a["E"], a["y"], a["N"], a["D"], a["V"], a["ign"], a["segs"],
+                     a["nseg"], a["loss"], a["lse"], a["colmax"], a["ws"], a["wsb"], a["st"],
+                     a["stream"])
+
+
+def test_fwd_rejects_bad_arguments_on_host():
+    # None of these reaches the device: validation fails first.
+    assert _null_fwd(D=12) == cce.CCE_EINVAL
+    assert _null_fwd(H=None) == cce.CCE_EINVAL
+    assert _null_fwd(E=None) == cce.CCE_EINVAL
+    assert _null_fwd(H=18) == cce.CCE_EINVAL                    # misaligned
+    assert _null_fwd(ws=None) == cce.CCE_EWORKSPACE
+    assert _null_fwd(wsb=8) == cce.CCE_EWORKSPACE
+    assert _null_fwd(N=0) == cce.CCE_OK                          # nothing to do
+
+
+def test_segment_table_validation():
+    seg = (cce.Segment * 2)()
+    seg[0].vocab_begin, seg[0].vocab_end, seg[0].E = 0, 6, 16
+    seg[1].vocab_begin, seg[1].vocab_end, seg[1].E = 4, 10, 32  # overlaps
+    assert _null_fwd(E=None, segs=seg, nseg=2) == cce.CCE_EINVAL
+    seg[1].vocab_begin = 7
+    seg[1].vocab_end = 11                                       # beyond V
+    assert _null_fwd(E=None, segs=seg, nseg=2) == cce.CCE_EINVAL
+    seg[1].vocab_end = 10
+    assert _null_fwd(E=16, segs=seg, nseg=2) == cce.CCE_EINVAL   # E and segs both given
+    seg[1].E = None
+    assert _null_fwd(E=None, segs=seg, nseg=2) == cce.CCE_EINVAL
+    seg[1].E = 32
+    assert _null_fwd(E=None, segs=seg, nseg=2, ws=None) == cce.CCE_EWORKSPACE
+
+
+def test_bwd_rejects_bad_flags_and_missing_kahan_buffer():
+    L = cce.lib()
+
+    def call(flags=0, dE=16, comp=None):
+        return L.cce_bwd(16, 16, 16, 16, 16, 4, 8, 10, -100, None, 0, 0.0, None, flags,
+                         16, dE, comp, None, 0, 16, 1 << 30, 16, None)
+    assert call(flags=8) == cce.CCE_EINVAL
+    assert call(flags=cce.KAHAN_DE) == cce.CCE_EINVAL           # no compensation buffer
+    assert call(flags=cce.KAHAN_DE | cce.FP32_GRADS, comp=16) == cce.CCE_EINVAL
+    assert call(dE=None) == cce.CCE_EINVAL

@@ -1,0 +1,233 @@
+"""GPU parity: libcce (through its C ABI) against the fp64 oracle.
+
+Sizes here are ones the oracle finishes in seconds while still spanning
+several 128x256 tiles, ragged row/vocabulary/D tails, ignored rows, a
+composite head with a dead gap, filtering, the vocabulary sort and the Kahan
+path.  Tolerances are the acceptance tolerances (tests/_helpers.py).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_cross_entropy_cce_b200 import synthetic as syn
+from _helpers import (EPS_BF16, TOL_GRAD, TOL_GRAD_FILTER, TOL_MEAN_REL, TOL_ROW, normwise,
+                      run_bwd, run_fwd, to_np, upload)
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny": syn.WORKLOADS["tiny"],
+    # ragged everything: N % 128, D % 64 != 0, V % 256 != 0
+    "ragged": syn.Workload("ragged", N=333, D=200, V=1000, logit_std=4.0, ignore_frac=0.15),
+    "gemma_like_small": syn.scaled(syn.WORKLOADS["gemma2_2b_head"], N=700, D=576, V=5000),
+    "phi_like_small": syn.scaled(syn.WORKLOADS["phi35_mini_head"], N=520, D=384, V=3001),
+    "composite_small": syn.scaled(syn.WORKLOADS["composite_two_segment"], N=900, D=256, V=6200,
+                                  segments=((0, 3800), (3954, 6200))),
+    "wide_D": syn.Workload("wide_D", N=260, D=1032, V=2300, logit_std=2.0, ignore_frac=0.0),
+}
+
+
+@pytest.fixture(scope="module")
+def data():
+    return {k: syn.make_inputs(wl, seed=0) for k, wl in CASES.items()}
+
+
+def _fwd_check(x):
+    H, segs, y = upload(x)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    loss, lse = run_fwd(x, H, segs, y, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rl, rs = oracle.forward(x.H, x.segments, x.y, x.wl.V, x.ignore_index)
+    gl, gs = to_np(loss), to_np(lse)
+    assert np.max(np.abs(gl - rl)) <= TOL_ROW, np.max(np.abs(gl - rl))
+    assert np.max(np.abs(gs - rs)) <= TOL_ROW, np.max(np.abs(gs - rs))
+    v = x.valid
+    m_ref = oracle.mean_loss(rl, v)
+    m_got = float(np.sum(gl[v], dtype=np.float64)) / max(1, int(v.sum()))
+    assert abs(m_got - m_ref) <= TOL_MEAN_REL * abs(m_ref)
+    assert np.all(gl[~v] == 0) and np.all(gs[~v] == 0)
+    return H, segs, y, lse
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_forward_matches_oracle(data, case):
+    _fwd_check(data[case])
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_backward_unfiltered_matches_oracle(data, case):
+    x = data[case]
+    H, segs, y, lse = _fwd_check(x)
+    dl = x.dloss_mean()
+    dH, dEs, _ = run_bwd(x, H, segs, y, lse, torch.from_numpy(dl).cuda())
+    torch.cuda.synchronize()
+    rH, rE = oracle.backward(x.H, x.segments, x.y, x.wl.V, dl, x.ignore_index)
+    assert normwise(to_np(dH), rH) <= TOL_GRAD
+    for g, r in zip(dEs, rE):
+        assert normwise(to_np(g), r) <= TOL_GRAD
+    assert np.all(to_np(dH)[~x.valid] == 0)
+
+
+@pytest.mark.parametrize("case", ["gemma_like_small", "phi_like_small", "composite_small", "ragged"])
+def test_backward_filtered_matches_oracle_and_criterion(data, case):
+    x = data[case]
+    H, segs, y, lse = _fwd_check(x)
+    dl = x.dloss_mean()
+    rows = min(64, x.wl.N)
+    dH, dEs, keep = run_bwd(x, H, segs, y, lse, torch.from_numpy(dl).cuda(),
+                            filter_eps=EPS_BF16, debug_rows=rows)
+    torch.cuda.synchronize()
+    rH, rE = oracle.backward(x.H, x.segments, x.y, x.wl.V, dl, x.ignore_index,
+                             filter_eps=EPS_BF16)
+    assert normwise(to_np(dH), rH) <= TOL_GRAD_FILTER
+    for g, r in zip(dEs, rE):
+        assert normwise(to_np(g), r) <= TOL_GRAD_FILTER
+    # every filtered-out entry has oracle softmax < 2^-12; kept ones >= it
+    P = oracle.softmax_rows(x.H, x.segments, x.wl.V, np.arange(rows))
+    bits = keep.cpu().numpy().view(np.uint32)
+    kept = np.unpackbits(bits.view(np.uint8), bitorder="little").reshape(rows, -1)[:, :x.wl.V]
+    live = np.zeros(x.wl.V, bool)
+    for b, e, _ in x.segments:
+        live[b:e] = True
+    valid = x.valid[:rows]
+    dropped = (kept == 0) & live[None, :] & valid[:, None]
+    assert np.all(P[dropped] < EPS_BF16)
+    must_keep = (P >= EPS_BF16 * 1.001) & valid[:, None]
+    assert np.all(kept[must_keep] == 1)
+    assert np.all(kept[~valid] == 0)
+
+
+def test_colmax_matches_oracle(data):
+    x = data["composite_small"]
+    H, segs, y = upload(x)
+    loss, lse, colmax = run_fwd(x, H, segs, y, want_colmax=True)
+    torch.cuda.synchronize()
+    segs64 = [(b, e, oracle.widen_bf16(E)) for b, e, E in x.segments]
+    Z = oracle.logits_rows(oracle.widen_bf16(x.H[x.valid]), segs64, x.wl.V)
+    ref = np.concatenate([Z[:, b:e].max(0) for b, e, _ in x.segments])
+    assert np.max(np.abs(to_np(colmax) - ref)) <= 1e-3
+
+
+@pytest.mark.parametrize("keyed", ["colmax", "targets"])
+def test_vocab_sort_and_permuted_backward(data, keyed):
+    x = data["composite_small"]
+    from linear_cross_entropy_cce_b200 import cce
+    H, segs, y, lse = _fwd_check(x)
+    colmax = run_fwd(x, H, segs, y, want_colmax=True)[2] if keyed == "colmax" else None
+    perm = cce.vocab_sort(colmax, y, x.wl.V, x.ignore_index, segments=segs)
+    torch.cuda.synchronize()
+    p = perm.cpu().numpy()
+    off = 0
+    for b, e, _ in x.segments:
+        n = e - b
+        seg = p[off:off + n]
+        assert np.array_equal(np.sort(seg), np.arange(n))
+        key = (to_np(colmax)[off:off + n] if colmax is not None else
+               np.bincount(x.y[(x.y >= b) & (x.y < e)] - b, minlength=n).astype(np.float64))
+        k = key[seg]
+        assert np.all(k[:-1] >= k[1:])
+        ties = k[:-1] == k[1:]
+        assert np.all(seg[:-1][ties] < seg[1:][ties])
+        off += n
+    dl = x.dloss_mean()
+    dH, dEs, _ = run_bwd(x, H, segs, y, lse, torch.from_numpy(dl).cuda(), vocab_perm=perm,
+                         filter_eps=EPS_BF16)
+    rH, rE = oracle.backward(x.H, x.segments, x.y, x.wl.V, dl, x.ignore_index,
+                             filter_eps=EPS_BF16)
+    assert normwise(to_np(dH), rH) <= TOL_GRAD_FILTER
+    for g, r in zip(dEs, rE):
+        assert normwise(to_np(g), r) <= TOL_GRAD_FILTER
+
+
+def test_kahan_accumulation_is_deterministic_and_accurate():
+    from linear_cross_entropy_cce_b200 import cce
+    wl = syn.Workload("k", N=300, D=128, V=1500, logit_std=2.0, ignore_frac=0.1)
+    xs = [syn.make_inputs(wl, seed=s) for s in range(4)]
+    E = xs[0].segments  # same head for every micro-batch
+    finals = []
+    for rep in range(2):
+        Ssum = torch.zeros((wl.V, wl.D), dtype=torch.bfloat16, device="cuda")
+        C = torch.zeros_like(Ssum)
+        for x in xs:
+            H = cce.bf16_from_bits(x.H, "cuda")
+            Et = cce.bf16_from_bits(E[0][2], "cuda")
+            y = torch.from_numpy(x.y).cuda()
+            loss, lse = cce.fwd(H, Et, y)
+            dl = torch.from_numpy(x.dloss_mean()).cuda()
+            cce.bwd(H, Et, y, lse, dl, kahan=True, dE_out=Ssum, dE_comp=C)
+        torch.cuda.synchronize()
+        finals.append(Ssum.clone())
+    assert torch.equal(finals[0], finals[1])
+    parts = [oracle.backward(x.H, E, x.y, wl.V, x.dloss_mean(), -100)[1][0] for x in xs]
+    ref = oracle.kahan_reference(parts)
+    got = to_np(finals[0]) - to_np(C)  # s - c is the compensated value
+    assert normwise(to_np(finals[0]), ref) <= TOL_GRAD
+    assert normwise(got, ref) <= TOL_GRAD
+
+
+def test_fp32_grads(data):
+    x = data["ragged"]
+    H, segs, y, lse = _fwd_check(x)
+    dl = x.dloss_mean()
+    dH, dEs, _ = run_bwd(x, H, segs, y, lse, torch.from_numpy(dl).cuda(), fp32_grads=True)
+    assert dH.dtype == torch.float32 and dEs[0].dtype == torch.float32
+    rH, rE = oracle.backward(x.H, x.segments, x.y, x.wl.V, dl, x.ignore_index)
+    assert normwise(to_np(dH), rH) <= TOL_GRAD / 2
+    assert normwise(to_np(dEs[0]), rE[0]) <= TOL_GRAD / 2
+
+
+def test_zero_head_gives_lnV():
+    from linear_cross_entropy_cce_b200 import cce
+    N, D, V = 300, 64, 5000
+    H = torch.randn(N, D, device="cuda").to(torch.bfloat16)
+    E = torch.zeros(V, D, device="cuda", dtype=torch.bfloat16)
+    y = torch.randint(0, V, (N,), device="cuda", dtype=torch.int32)
+    loss, lse = cce.fwd(H, E, y)
+    assert torch.max(torch.abs(loss - math.log(V))).item() <= 1e-5
+    assert torch.max(torch.abs(lse - math.log(V))).item() <= 1e-5
+
+
+def test_bad_targets_set_status_and_nan():
+    from linear_cross_entropy_cce_b200 import cce
+    N, D, V = 200, 64, 700
+    H = torch.randn(N, D, device="cuda").to(torch.bfloat16)
+    EA = (torch.randn(300, D, device="cuda") * 0.1).to(torch.bfloat16)
+    EB = (torch.randn(350, D, device="cuda") * 0.1).to(torch.bfloat16)
+    segs = [(0, 300, EA), (350, 700, EB)]
+    y = torch.randint(0, 300, (N,), device="cuda", dtype=torch.int32)
+    y[3] = 320      # in the gap
+    y[7] = 700      # out of range
+    y[9] = -100     # ignored
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    loss, lse = cce.fwd(H, None, y, segments=segs, V=V, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & cce.STATUS_BADTARGET
+    l = loss.cpu().numpy()
+    assert math.isnan(l[3]) and math.isnan(l[7]) and l[9] == 0
+    assert np.isfinite(np.delete(l, [3, 7])).all()
+    dl = torch.full((N,), 1.0 / N, device="cuda")
+    st.zero_()
+    dH, dEs, _ = cce.bwd(H, None, y, lse, dl, segments=segs, V=V, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & cce.STATUS_BADTARGET
+    d = dH.float().cpu().numpy()
+    assert np.isnan(d[3]).all() and np.isnan(d[7]).all() and (d[9] == 0).all()
+    assert np.isfinite(np.delete(d, [3, 7], axis=0)).all()
+    assert all(torch.isfinite(g.float()).all() for g in dEs)
+
+
+def test_all_rows_ignored():
+    from linear_cross_entropy_cce_b200 import cce
+    N, D, V = 130, 64, 600
+    H = torch.randn(N, D, device="cuda").to(torch.bfloat16)
+    E = torch.randn(V, D, device="cuda").to(torch.bfloat16)
+    y = torch.full((N,), -100, device="cuda", dtype=torch.int32)
+    loss, lse = cce.fwd(H, E, y)
+    dH, dE, _ = cce.bwd(H, E, y, lse, torch.zeros(N, device="cuda"))
+    torch.cuda.synchronize()
+    assert (loss == 0).all() and (lse == 0).all()
+    assert (dH.float() == 0).all() and (dE.float() == 0).all()
