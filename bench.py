@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Fused classifier matmul + cross-entropy, forward+backward, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = the whole hot path on one batch of synthetic input, inputs already
+resident in HBM: cce_fwd (loss, lse, and the colmax statistic when the
+vocabulary sort is on) -> cce_vocab_sort (when on) -> cce_bwd (dH, dE).
+Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one process per GPU)
+every rank runs its own batch (weak scaling, no collective on the data path);
+the time is the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle on a bounded row sample of the
+same workload on the host cores (the only other place this file runs the
+oracle is the cpu_baseline leg of the default arm).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_cross_entropy_cce_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "fused CE fwd+bwd tokens/s and % of B200 bf16 tensor peak; peak MB"
+UNIT = "tokens/s"
+EPS_BF16 = 2.0 ** -12
+# per workload: (gradient filter on, vocabulary sort on)
+MODES = {
+    "tiny": (False, False),
+    "gemma2_2b_head": (True, True),
+    "llama3_8b_head": (False, False),
+    "phi35_mini_head": (True, False),
+    "composite_two_segment": (True, False),
+}
+L2_BYTES = 126 * 2 ** 20
+
+
+def peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0,
+                "fallback": True}
+
+
+def host_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ------------------------------------------------------------------ oracle
+def oracle_sample(x, seconds: float, max_rows: int = 2048):
+    """Time the fp64 oracle (forward + backward) on a row sample; returns
+    (rows/s, rows, seconds, description)."""
+    import oracle
+    segs64 = [(b, e, oracle.widen_bf16(E)) for b, e, E in x.segments]
+    valid = np.nonzero(x.valid)[0]
+    dl = x.dloss_mean()
+
+    def run(rows):
+        Hs, ys, ds = x.H[rows], x.y[rows], dl[rows]
+        t = time.perf_counter()
+        oracle.forward(Hs, segs64, ys, x.wl.V, x.ignore_index)
+        oracle.backward(Hs, segs64, ys, x.wl.V, ds, x.ignore_index,
+                        filter_eps=EPS_BF16 if MODES.get(x.wl.name, (False,))[0] else 0.0)
+        return time.perf_counter() - t
+
+    r0 = valid[:8]
+    t0 = run(r0)
+    R = int(min(max_rows, len(valid), max(8, seconds / max(t0, 1e-6) * len(r0))))
+    R = max(8, (R // 8) * 8)
+    rows = valid[np.linspace(0, len(valid) - 1, R).astype(np.int64)]
+    t = run(rows)
+    desc = (f"fp64 numpy oracle, forward+backward over {R} valid rows of {x.wl.name} "
+            f"(N={x.wl.N}, D={x.wl.D}, V={x.wl.V}); full vocabulary and full dE per slice")
+    return R / t, R, t, desc
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.p = None
+        return self
+
+    def __exit__(self, *a):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.out = self.p.communicate(timeout=10)[0]
+            except Exception:
+                self.p.kill()
+                self.out = ""
+
+    def summary(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "out", "").splitlines():
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9 or (self.uuid and f[0] != self.uuid):
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="gemma2_2b_head", choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--filter", choices=["on", "off", "default"], default="default")
+    ap.add_argument("--sort", choices=["on", "off", "default"], default="default")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = syn.WORKLOADS[a.workload]
+    filt, sort = MODES[wl.name]
+    if a.filter != "default":
+        filt = a.filter == "on"
+    if a.sort != "default":
+        sort = a.sort == "on"
+    eps = EPS_BF16 if filt else 0.0
+
+    if a.impl == "reference":
+        return reference_arm(a, wl, world, rank, filt)
+
+    import torch
+    import torch.distributed as dist
+    from linear_cross_entropy_cce_b200 import cce
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    x = syn.make_inputs(wl, seed=rank)
+    H = cce.bf16_from_bits(x.H, dev)
+    segs = [(b, e, cce.bf16_from_bits(E, dev)) for b, e, E in x.segments]
+    single = len(segs) == 1 and segs[0][0] == 0 and segs[0][1] == wl.V
+    y = torch.from_numpy(x.y).to(dev)
+    dloss = torch.from_numpy(x.dloss_mean()).to(dev)
+    N, D, V = wl.N, wl.D, wl.V
+    nseg = 0 if single else len(segs)
+    n_valid, v_live = x.n_valid, wl.v_live
+    ws_f = torch.empty(cce.fwd_workspace_size(N, D, V, nseg), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(cce.bwd_workspace_size(N, D, V, nseg), dtype=torch.uint8, device=dev)
+    ws_s = torch.empty(cce.vocab_sort_workspace_size(N, V, nseg), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    input_bytes = H.numel() * 2 + sum(s[2].numel() * 2 for s in segs) + y.numel() * 4
+
+    def step(Hd=H, segd=segs, yd=y):
+        kw = dict(workspace=ws_f, status=status)
+        if single:
+            out = cce.fwd(Hd, segd[0][2], yd, x.ignore_index, want_colmax=sort, **kw)
+        else:
+            out = cce.fwd(Hd, None, yd, x.ignore_index, segments=segd, V=V, want_colmax=sort, **kw)
+        loss, lse = out[0], out[1]
+        perm = None
+        if sort:
+            perm = cce.vocab_sort(out[2], yd, V, x.ignore_index,
+                                  segments=None if single else segd, workspace=ws_s)
+        kw = dict(filter_eps=eps, vocab_perm=perm, workspace=ws_b, status=status)
+        if single:
+            dH, dE, _ = cce.bwd(Hd, segd[0][2], yd, lse, dloss, x.ignore_index, **kw)
+        else:
+            dH, dE, _ = cce.bwd(Hd, None, yd, lse, dloss, x.ignore_index, segments=segd, V=V, **kw)
+        return loss, dH, dE
+
+    def fwd_only():
+        if single:
+            return cce.fwd(H, segs[0][2], y, x.ignore_index, workspace=ws_f, status=status)
+        return cce.fwd(H, None, y, x.ignore_index, segments=segs, V=V, workspace=ws_f,
+                       status=status)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(fn, k):
+        barrier()
+        torch.cuda.synchronize(dev)
+        s = torch.cuda.current_stream(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(k):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ms = e0.elapsed_time(e1) / k
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise SystemExit(f"device status {int(status.item())} during warm-up")
+
+    uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", ""))
+    uuid = uuid if uuid.startswith("GPU-") or not uuid else "GPU-" + uuid
+    l0 = cce.launch_count()
+    with ClockSampler(uuid) as clk:
+        ms_step = timed(step, a.steps)
+    launches = cce.launch_count() - l0
+    clocks = clk.summary()
+
+    # forward alone (context), then a per-kernel-class timing pass
+    for _ in range(3):
+        fwd_only()
+    ms_fwd = timed(fwd_only, a.steps)
+    cce.timing_enable(0b11111)
+    ms_prof = timed(step, a.steps)
+    per_class = cce.timing_read()
+    cce.timing_enable(0)
+
+    # peak memory of one step beyond the resident inputs and workspaces
+    torch.cuda.synchronize(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    step()
+    torch.cuda.synchronize(dev)
+    peak_extra = torch.cuda.max_memory_allocated(dev) - base
+    ws_bytes = ws_f.numel() + ws_b.numel() + ws_s.numel()
+
+    # end to end through the public API from pinned host buffers
+    e2e = None
+    if not a.no_e2e:
+        hH = torch.from_numpy(x.H.view(np.int16)).pin_memory()
+        hE = [torch.from_numpy(E.view(np.int16)).pin_memory() for _, _, E in x.segments]
+        hy = torch.from_numpy(x.y).pin_memory()
+        hloss = torch.empty(N, dtype=torch.float32).pin_memory()
+        dH_ = torch.empty_like(H)
+        Ed_ = [torch.empty_like(s[2]) for s in segs]
+        dy_ = torch.empty_like(y)
+
+        def e2e_step():
+            dH_.view(torch.int16).copy_(hH, non_blocking=True)
+            for d, h in zip(Ed_, hE):
+                d.view(torch.int16).copy_(h, non_blocking=True)
+            dy_.copy_(hy, non_blocking=True)
+            segd = [(b, e, d) for (b, e, _), d in zip(segs, Ed_)]
+            loss, _, _ = step(dH_, segd, dy_)
+            hloss.copy_(loss, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        ms_e2e = timed(e2e_step, a.steps)
+        h2d = hH.numel() * 2 + sum(h.numel() * 2 for h in hE) + hy.numel() * 4
+        e2e = {"value": round(N * world / (ms_e2e / 1e3), 1), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(N * 4),
+               "ms_per_step": round(ms_e2e, 3)}
+
+    P = peaks()
+    flops_fwd = 2.0 * n_valid * D * v_live
+    flops_step = 8.0 * n_valid * D * v_live
+    class_flops = {"fwd_tile_stream": flops_fwd, "bwd_g_producer": flops_fwd,
+                   "bwd_dE_contraction": flops_fwd, "bwd_dH_contraction": flops_fwd}
+    dom = max(class_flops, key=lambda k: per_class[k][0])
+    dom_ms, dom_n = per_class[dom]
+    achieved = class_flops[dom] * a.steps / (dom_ms / 1e3) / 1e12 if dom_ms > 0 else None
+    peak_sus = float(P.get("bf16_tflops_sustained", P.get("bf16_tflops")))
+    peak_burst = float(P["bf16_tflops"])
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1) if achieved else None,
+                "peak": peak_sus, "unit": "TFLOP/s",
+                "frac": round(achieved / peak_sus, 4) if achieved else None,
+                "peak_kind": "sustained bf16 (measured, cuBLAS) - kernel timed inside the step",
+                "traffic": None,
+                "launches_per_step": dom_n // max(1, a.steps),
+                "avg_launch_ms": round(dom_ms / max(1, dom_n), 4)}
+    step_tflops = flops_step / (ms_step / 1e3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        rps, R, t, desc = oracle_sample(x, a.cpu_seconds)
+        cpu = {"value": round(rps, 3), "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+               "sample": desc, "seconds": round(t, 2)}
+
+    out = {
+        "metric": METRIC, "value": round(N * world / (ms_step / 1e3), 1), "unit": UNIT,
+        "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; shapes and value recipe of the workload; no dataset or trained weights)",
+        "config": {"workload": wl.name, "N": N, "N_valid": n_valid, "D": D, "V": V,
+                   "V_live": v_live, "segments": [list(s) for s in wl.segs()],
+                   "logit_std": wl.logit_std, "filter_eps": eps, "vocab_sort": sort,
+                   "global_batch_tokens": N * world, "parallelism": f"dp{world} (independent batches)",
+                   "l2": f"inputs larger than L2 (E = {sum(s[2].numel() for s in segs) * 2 / 2**20:.0f} MiB > 126 MiB)",
+                   "tokens_per_s_valid_rows": round(n_valid * world / (ms_step / 1e3), 1)},
+        "tensor_peak_frac": {"of_measured_burst": round(step_tflops / peak_burst, 4),
+                             "of_measured_sustained": round(step_tflops / peak_sus, 4),
+                             "of_spec_2250": round(step_tflops / 2250.0, 4),
+                             "tflops_unfiltered_8NDV": round(step_tflops, 1)},
+        "fwd_ms": round(ms_fwd, 3), "fwd_bwd_ms": round(ms_step, 3),
+        "peak_mb": round((peak_extra + ws_bytes) / 2 ** 20, 1),
+        "peak_mb_detail": {"workspaces_mb": round(ws_bytes / 2 ** 20, 1),
+                           "step_allocations_mb": round(peak_extra / 2 ** 20, 1),
+                           "inputs_mb": round(input_bytes / 2 ** 20, 1),
+                           "materialised_logits_bf16_mb": round(N * V * 2 / 2 ** 20, 1)},
+        "roofline": roofline,
+        "per_kernel_ms_per_step": {k: round(v[0] / a.steps, 3) for k, v in per_class.items()},
+        "profiled_ms_per_step": round(ms_prof, 3),
+        "gpu_launches": int(launches),
+        "gpu_launches_per_step": int(launches // max(1, a.steps)),
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def reference_arm(a, wl, world, rank, filt):
+    """The fp64 CPU oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    x = syn.make_inputs(wl, seed=0)
+    per_step = max(2.0, 120.0 / max(1, a.steps + a.warmup))
+    times, R = [], 0
+    for i in range(a.warmup + a.steps):
+        rps, R, t, desc = oracle_sample(x, per_step)
+        if i >= a.warmup:
+            times.append(R / rps)
+    ms = 1e3 * float(np.mean(times))
+    v = R / (ms / 1e3)
+    out = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": UNIT,
+           "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms, 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": wl.name, "N": wl.N, "D": wl.D, "V": wl.V,
+                                            "rows_per_step": R},
+           "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": host_cores(),
+                            "kind": "oracle", "sample": desc},
+           "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -180,6 +180,25 @@ int cce_vocab_sort(const float* colmax, const int32_t* y, int64_t N, int64_t V,
                    int32_t* vocab_perm, void* workspace, size_t workspace_bytes,
                    void* stream);
 
+/*
+ * Diagnostics (not needed for computing anything).
+ *
+ * cce_launch_count: number of kernels libcce has enqueued in this process
+ * since it was loaded (every entry point counts its launches).
+ *
+ * cce_timing_enable: while class_mask != 0, each launch of a selected kernel
+ * class is bracketed by two CUDA events recorded on the stream the kernel is
+ * launched on.  Classes: bit 0 forward tile stream, bit 1 backward G
+ * producer, bit 2 backward dE contraction, bit 3 backward dH contraction,
+ * bit 4 every other kernel.  cce_timing_read synchronises on the recorded
+ * events, writes per class the summed milliseconds and the number of timed
+ * launches (arrays of n_classes <= 5 entries, host memory), and clears the
+ * record.  Not thread-safe.  Returns CCE_OK or CCE_EINVAL/CCE_ELAUNCH.
+ */
+uint64_t cce_launch_count(void);
+int cce_timing_enable(uint32_t class_mask);
+int cce_timing_read(float* ms, int64_t* launches, int32_t n_classes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,7 +23,10 @@ MAX_SEGMENTS = 8
 
 EXPORTS = ("cce_version", "cce_strerror", "cce_fwd_workspace_size", "cce_fwd",
            "cce_bwd_workspace_size", "cce_bwd", "cce_vocab_sort_workspace_size",
-           "cce_vocab_sort")
+           "cce_vocab_sort", "cce_launch_count", "cce_timing_enable", "cce_timing_read")
+# kernel classes for cce_timing_enable / cce_timing_read
+KC_FWD, KC_G, KC_DE, KC_DH, KC_AUX = 0, 1, 2, 3, 4
+KC_NAMES = ("fwd_tile_stream", "bwd_g_producer", "bwd_dE_contraction", "bwd_dH_contraction", "aux")
 
 
 class CCEError(RuntimeError):
@@ -66,6 +69,11 @@ def lib() -> ctypes.CDLL:
     L.cce_vocab_sort_workspace_size.argtypes = [i64, i64, i32]
     L.cce_vocab_sort.restype = ctypes.c_int
     L.cce_vocab_sort.argtypes = [vp, vp, i64, i64, i32, ctypes.POINTER(Segment), i32, vp, vp, sz, vp]
+    L.cce_launch_count.restype = ctypes.c_uint64
+    L.cce_timing_enable.restype = ctypes.c_int
+    L.cce_timing_enable.argtypes = [u32]
+    L.cce_timing_read.restype = ctypes.c_int
+    L.cce_timing_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int64), i32]
     _lib = L
     return L
 
@@ -214,6 +222,23 @@ def vocab_sort(colmax: Optional[torch.Tensor], y: torch.Tensor, V: int, ignore_i
                               _ptr(perm), _ptr(ws), ws.numel(), _stream_ptr(dev))
     _check(rc, "cce_vocab_sort")
     return perm
+
+
+def launch_count() -> int:
+    """Kernels libcce has enqueued in this process."""
+    return int(lib().cce_launch_count())
+
+
+def timing_enable(class_mask: int):
+    _check(lib().cce_timing_enable(class_mask), "cce_timing_enable")
+
+
+def timing_read():
+    """{class name: (summed ms, timed launches)}; clears the record."""
+    ms = (ctypes.c_float * 5)()
+    n = (ctypes.c_int64 * 5)()
+    _check(lib().cce_timing_read(ms, n, 5), "cce_timing_read")
+    return {KC_NAMES[i]: (float(ms[i]), int(n[i])) for i in range(5)}
 
 
 def bf16_from_bits(bits, device) -> torch.Tensor:

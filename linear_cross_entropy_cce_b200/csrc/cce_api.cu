@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
+#include <vector>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -184,16 +186,58 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V) {
   return p;
 }
 
+// ---------------------------------------------------------- diagnostics
+enum KernelClass { KC_FWD = 0, KC_G = 1, KC_DE = 2, KC_DH = 3, KC_AUX = 4, KC_N = 5 };
+
+std::atomic<uint64_t> g_launches{0};
+
+struct Timing {
+  uint32_t mask = 0;
+  std::vector<cudaEvent_t> pool;  // reused across enable cycles
+  size_t used = 0;
+  std::vector<std::pair<int, size_t>> rec;  // (class, index of the start event)
+} g_timing;
+
+cudaEvent_t timing_event() {
+  if (g_timing.used == g_timing.pool.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    g_timing.pool.push_back(e);
+  }
+  return g_timing.pool[g_timing.used++];
+}
+
+// Records the start event of a timed launch; returns the record slot or -1.
+long timing_begin(int cls, cudaStream_t st) {
+  if (!(g_timing.mask & (1u << cls))) return -1;
+  const size_t i = g_timing.used;
+  cudaEvent_t a = timing_event();
+  if (!a || !timing_event()) return -1;
+  cudaEventRecord(a, st);
+  g_timing.rec.emplace_back(cls, i);
+  return (long)i;
+}
+void timing_end(long slot, cudaStream_t st) {
+  if (slot >= 0) cudaEventRecord(g_timing.pool[slot + 1], st);
+}
+
 template <class Policy>
-int launch_tc(const typename Policy::Params& prm, int grid, cudaStream_t st) {
+int launch_tc(const typename Policy::Params& prm, int grid, cudaStream_t st, int cls) {
   auto k = tc_kernel<Policy>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
     return CCE_ELAUNCH;
+  const long slot = timing_begin(cls, st);
   k<<<grid, THREADS, SMEM_BYTES, st>>>(prm);
+  timing_end(slot, st);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? CCE_OK : CCE_ELAUNCH;
 }
 
-int launched() { return cudaGetLastError() == cudaSuccess ? CCE_OK : CCE_ELAUNCH; }
+// Called right after every other kernel launch: counts it and checks it.
+int launched() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? CCE_OK : CCE_ELAUNCH;
+}
 
 template <class T>
 T* at(void* ws, size_t off) {
@@ -321,7 +365,7 @@ int cce_fwd(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D
   fp.colmax = reinterpret_cast<int*>(colmax);
   fp.status = status;
   const int64_t items = (pl.Npad / BM) * fp.S;
-  if (int rc = launch_tc<FwdPolicy>(fp, (int)std::min<int64_t>(sms, items), st)) return rc;
+  if (int rc = launch_tc<FwdPolicy>(fp, (int)std::min<int64_t>(sms, items), st, KC_FWD)) return rc;
 
   FinParams fin;
   fin.H = static_cast<const __nv_bfloat16*>(H);
@@ -474,7 +518,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       gp.seg_begin = table.s[s].begin;
       gp.perm_seg = perm_seg;
       gp.status = status;
-      if (int rc = launch_tc<GPolicy>(gp, (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct), st))
+      if (int rc = launch_tc<GPolicy>(gp, (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct), st, KC_G))
         return rc;
       // step 2: dE rows of this chunk
       ep.chunk_valid = cv;
@@ -488,7 +532,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       ep.mode = kahan ? 2 : (fp32 ? 1 : 0);
       ep.n_valid = cp.n_valid;
       ep.status = status;
-      if (int rc = launch_tc<DEPolicy>(ep, (int)std::min<int64_t>(sms, (int64_t)ep.mt * dt), st))
+      if (int rc = launch_tc<DEPolicy>(ep, (int)std::min<int64_t>(sms, (int64_t)ep.mt * dt), st, KC_DE))
         return rc;
       // step 3: dH += G E_chunk
       hp.mapB = segMN;
@@ -499,7 +543,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       hp.dH_acc = dH_acc;
       hp.n_valid = cp.n_valid;
       hp.status = status;
-      if (int rc = launch_tc<DHPolicy>(hp, (int)std::min<int64_t>(sms, (int64_t)mbs * dt), st))
+      if (int rc = launch_tc<DHPolicy>(hp, (int)std::min<int64_t>(sms, (int64_t)mbs * dt), st, KC_DH))
         return rc;
     }
   }
@@ -570,8 +614,41 @@ int cce_vocab_sort(const float* colmax, const int32_t* y, int64_t N, int64_t V, 
     if (cub::DeviceRadixSort::SortPairsDescending(tmp, have, key + off, key_out + off, ids + off,
                                                   vocab_perm + off, n, 0, 32, st) != cudaSuccess)
       return CCE_ELAUNCH;
+    if (launched()) return CCE_ELAUNCH;  // counted as one (a short sequence of cub kernels)
   }
   return CCE_OK;
+}
+
+uint64_t cce_launch_count(void) { return g_launches.load(); }
+
+int cce_timing_enable(uint32_t class_mask) {
+  if (class_mask >= (1u << KC_N)) return CCE_EINVAL;
+  g_timing.mask = class_mask;
+  return CCE_OK;
+}
+
+int cce_timing_read(float* ms, int64_t* launches, int32_t n_classes) {
+  if (!ms || !launches || n_classes < 0 || n_classes > KC_N) return CCE_EINVAL;
+  for (int c = 0; c < n_classes; ++c) {
+    ms[c] = 0.f;
+    launches[c] = 0;
+  }
+  int rc = CCE_OK;
+  for (const auto& r : g_timing.rec) {
+    float t = 0.f;
+    if (cudaEventSynchronize(g_timing.pool[r.second + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&t, g_timing.pool[r.second], g_timing.pool[r.second + 1]) != cudaSuccess) {
+      rc = CCE_ELAUNCH;
+      continue;
+    }
+    if (r.first < n_classes) {
+      ms[r.first] += t;
+      launches[r.first] += 1;
+    }
+  }
+  g_timing.rec.clear();
+  g_timing.used = 0;
+  return rc;
 }
 
 }  // extern "C"
