@@ -181,6 +181,34 @@ int cce_vocab_sort(const float* colmax, const int32_t* y, int64_t N, int64_t V,
                    void* stream);
 
 /*
+ * Forward without a caller-provided workspace and without any device
+ * allocation (the pages describe no such entry point; it has no counterpart
+ * in the paper).  Meant for callers that cannot call cudaMalloc: code running
+ * inside a host framework that owns all device memory and offers no
+ * allocation hook (plugin interfaces of inference engines, C or Fortran
+ * programs linking libcce without a device allocator), or code that must not
+ * trigger the implicit device synchronisation an allocation can cause.
+ *
+ * Arguments and results are those of cce_fwd; the scratch the forward needs
+ * lives in a fixed array of CCE_NOALLOC_SCRATCH_BYTES inside the library's
+ * device image, which every GPU that loads libcce holds until the process
+ * exits.  Returns CCE_EWORKSPACE when cce_fwd_workspace_size(N, D, V, n_segs)
+ * exceeds that size (e.g. N = 4096, D = 2048, V = 128k fits; N = 8192,
+ * D = 2304 does not).  The first call on each device looks up the array's
+ * device address with that device current; make that first call before any
+ * stream capture.  All calls on a device share the one array and the
+ * forward overwrites every scratch byte it reads, so nothing needs clearing
+ * between calls, but calls whose work overlaps on the GPU (other streams,
+ * other host threads) race on it: serialise them.
+ */
+#define CCE_NOALLOC_SCRATCH_BYTES (32u << 20)
+int cce_fwd_noalloc(const void* H, const void* E, const int32_t* y,
+                    int64_t N, int64_t D, int64_t V, int32_t ignore_index,
+                    const cce_segment* segs, int32_t n_segs,
+                    float* loss, float* lse, float* colmax,
+                    int32_t* status, void* stream);
+
+/*
  * Diagnostics (not needed for computing anything).
  *
  * cce_launch_count: number of kernels libcce has enqueued in this process

@@ -12,7 +12,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libcce.so")
-SOURCES = ["cce_api.cu"]
+SOURCES = ["cce_api.cu", "cce_noalloc.cu"]
 HEADERS = ["cce_ptx.cuh", "cce_engine.cuh", "cce_kernels.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
