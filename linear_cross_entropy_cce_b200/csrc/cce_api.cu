@@ -159,7 +159,9 @@ FwdPlan plan_fwd(int64_t N, int64_t D, int64_t V, int32_t n_segs) {
 struct BwdPlan {
   int64_t Npad, Vc;
   size_t off_nvalid, off_idx, off_pos, off_lse2, off_dl, off_tseg, off_tpos, off_inv, off_hc,
-      off_dh, off_g, off_ec, total;
+      off_dh, off_g, off_ec, off_masks, total;
+  int dh_words, de_words;
+  size_t mask_bytes;
 };
 
 BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V) {
@@ -182,6 +184,10 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V) {
   p.off_dh = o; o += align_up((size_t)p.Npad * D * 4);
   p.off_g = o; o += align_up((size_t)p.Npad * p.Vc * 2);
   p.off_ec = o; o += align_up((size_t)p.Vc * D * 2);
+  p.dh_words = (int)cdiv(p.Vc, 512);
+  p.de_words = (int)cdiv(p.Npad, 512);
+  p.mask_bytes = sizeof(uint32_t) * ((size_t)(p.Npad / BM) * p.dh_words + (size_t)(p.Vc / BM) * p.de_words);
+  p.off_masks = o; o += align_up(p.mask_bytes);
   p.total = o;
   return p;
 }
@@ -458,6 +464,8 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
     return CCE_ELAUNCH;
 
   __nv_bfloat16* G = at<__nv_bfloat16>(workspace, pl.off_g);
+  uint32_t* dh_mask = at<uint32_t>(workspace, pl.off_masks);
+  uint32_t* de_mask = dh_mask + (size_t)(pl.Npad / BM) * pl.dh_words;
   __nv_bfloat16* Ec = at<__nv_bfloat16>(workspace, pl.off_ec);
   const int Vc = (int)pl.Vc;
   const int dt = (int)cdiv(D, BN);
@@ -495,7 +503,12 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
         if (!make_map(&segMN, Ec, D, cv, D, 64, 64)) return CCE_ELAUNCH;
         row0 = 0;
       }
-      // step 1: G for this chunk
+      // step 1: G for this chunk, with its zero-slice masks
+      if (cudaMemsetAsync(dh_mask, 0, pl.mask_bytes, st) != cudaSuccess) return CCE_ELAUNCH;
+      gp.dh_mask = dh_mask;
+      gp.dh_words = pl.dh_words;
+      gp.de_mask = de_mask;
+      gp.de_words = pl.de_words;
       gp.mapB = segK;
       gp.b_row0 = row0;
       gp.chunk_valid = cv;
@@ -530,6 +543,8 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       ep.dE = sg.s[s].dE;
       ep.dE_comp = static_cast<__nv_bfloat16*>(sg.s[s].dE_comp);
       ep.mode = kahan ? 2 : (fp32 ? 1 : 0);
+      ep.mask = de_mask;
+      ep.mwords = pl.de_words;
       ep.n_valid = cp.n_valid;
       ep.status = status;
       if (int rc = launch_tc<DEPolicy>(ep, (int)std::min<int64_t>(sms, (int64_t)ep.mt * dt), st, KC_DE))
@@ -541,6 +556,8 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       hp.dt = dt;
       hp.D = (int)D;
       hp.dH_acc = dH_acc;
+      hp.mask = dh_mask;
+      hp.mwords = pl.dh_words;
       hp.n_valid = cp.n_valid;
       hp.status = status;
       if (int rc = launch_tc<DHPolicy>(hp, (int)std::min<int64_t>(sms, (int64_t)mbs * dt), st, KC_DH))

@@ -56,6 +56,32 @@ struct Pipe {
   }
 };
 
+// Sequential reader of a K-step mask: bit (kb & 7) * 4 + kk of word kb >> 3
+// is set when the K=16 step kk of stage kb must be issued.  The next word is
+// fetched one word ahead so the single MMA-issuing thread rarely waits on it.
+// A null mask means every step is issued.
+struct MaskCursor {
+  const uint32_t* p;
+  uint32_t cur, nxt;
+  int nwords;
+  __device__ __forceinline__ void init(const uint32_t* m, int nkb) {
+    p = m;
+    nwords = (nkb + 7) >> 3;
+    cur = (m && nwords > 0) ? __ldg(m) : 0xFFFFFFFFu;
+    nxt = (m && nwords > 1) ? __ldg(m + 1) : 0u;
+  }
+  // must be called for kb = 0, 1, 2, ... in order
+  __device__ __forceinline__ uint32_t bits(int kb) {
+    if (!p) return 0xFu;
+    if (kb > 0 && (kb & 7) == 0) {
+      cur = nxt;
+      const int w = (kb >> 3) + 1;
+      nxt = w < nwords ? __ldg(p + w) : 0u;
+    }
+    return (cur >> ((kb & 7) * 4)) & 0xFu;
+  }
+};
+
 // Per-role state handed to policies.
 struct Engine {
   Ctl* ctl;
@@ -70,11 +96,16 @@ struct Engine {
 
   // ---- producer: load nkb stages of one tile.  (ax, ay) / (bx, by) are the
   // tensor-map coordinates of the tile origin; K advances along x for a
-  // K-major operand and along y for an MN-major one.
+  // K-major operand and along y for an MN-major one.  With a K-step mask
+  // (see mma()), stages whose four K=16 steps are all masked are not loaded.
   template <bool A_MN, bool B_MN>
   __device__ __forceinline__ bool produce(const CUtensorMap* mA, const CUtensorMap* mB, int ax,
-                                          int ay, int bx, int by, int nkb) {
+                                          int ay, int bx, int by, int nkb,
+                                          const uint32_t* kmask = nullptr) {
+    MaskCursor mc;
+    mc.init(kmask, nkb);
     for (int kb = 0; kb < nkb; ++kb) {
+      if (!mc.bits(kb)) continue;
       if (!wait_parity(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u, abort_flag(), status))
         return false;
       const uint32_t fb = smem_u32(&ctl->full[pipe.stage]);
@@ -115,13 +146,16 @@ struct Engine {
     const uint32_t d = tmem + acc * BN;
     constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
     uint32_t issued = 0;
+    MaskCursor mc;
+    mc.init(kmask, nkb);
     for (int kb = 0; kb < nkb; ++kb) {
+      const uint32_t bits = mc.bits(kb);
+      if (!bits) continue;  // the producer skipped this stage too
       if (!wait_parity(smem_u32(&ctl->full[pipe.stage]), pipe.phase, abort_flag(), status))
         return false;
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + pipe.stage * STAGE_BYTES);
       const uint32_t sb = sa + A_BYTES;
-      const uint32_t bits = kmask ? ((kmask[kb >> 3] >> ((kb & 7) * 4)) & 0xFu) : 0xFu;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         if (!(bits & (1u << kk))) continue;

@@ -387,6 +387,15 @@ struct GParams {
   const int* tpos;
   float eps_keep;  // 0: keep everything
   __nv_bfloat16* G;
+  // Zero-slice masks for the two contractions (zeroed before this launch):
+  //   dh_mask[mb * dh_words + g / 32] bit g % 32: some row of row block mb
+  //     has a non-zero G entry in chunk columns 16g .. 16g+15;
+  //   de_mask[vb * de_words + r / 32] bit r % 32: some entry of compact rows
+  //     16r .. 16r+15 is non-zero in chunk columns 128vb .. 128vb+127.
+  uint32_t* dh_mask;
+  int dh_words;
+  uint32_t* de_mask;
+  int de_words;
   // optional per-element keep bits of original rows < debug_rows
   uint32_t* debug_keep;
   int debug_rows;
@@ -435,10 +444,12 @@ struct GPolicy {
       const int valid = p.chunk_valid - vt * BN;  // valid columns of this tile
       __nv_bfloat16* grow = p.G + (size_t)jrow * p.Vc + vt * BN;
       const bool dbg = p.debug_keep != nullptr && ok && p.idx[jrow] < p.debug_rows;
+      uint32_t half_nz = 0;  // bit h: this row has a non-zero in tile columns 128h..128h+127
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(taddr + c * 32, r);
         uint32_t packed[16];
+        bool nz[2] = {false, false};
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           float g[2];
@@ -452,12 +463,22 @@ struct GPolicy {
             g[u] = (ok && col < valid) ? dl * v : 0.f;
           }
           packed[j >> 1] = pack_bf16(g[0], g[1]);
+          nz[j >> 4] |= (packed[j >> 1] & 0x7FFF7FFFu) != 0u;  // non-zero after rounding
         }
         uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
         dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
         dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         dst[2] = make_uint4(packed[8], packed[9], packed[10], packed[11]);
         dst[3] = make_uint4(packed[12], packed[13], packed[14], packed[15]);
+        // warp vote: which 16-column slices of this chunk hold any non-zero
+        const uint32_t b0 = __ballot_sync(0xffffffffu, nz[0]);
+        const uint32_t b1 = __ballot_sync(0xffffffffu, nz[1]);
+        if (lane == 0 && (b0 | b1)) {
+          const int g = vt * (BN / 16) + c * 2;
+          atomicOr(&p.dh_mask[mb * p.dh_words + (g >> 5)],
+                   ((b0 ? 1u : 0u) | (b1 ? 2u : 0u)) << (g & 31));
+        }
+        half_nz |= (nz[0] || nz[1]) ? (1u << (c >> 2)) : 0u;
         if (dbg) {
           const int orig = p.idx[jrow];
           for (int j = 0; j < 32; ++j) {
@@ -471,6 +492,16 @@ struct GPolicy {
                        1u << (lid & 31));
             }
           }
+        }
+      }
+      // warp vote per 16-row group for the dE contraction's K slices
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t b = __ballot_sync(0xffffffffu, (half_nz >> h) & 1u);
+        if (lane == 0 && b) {
+          const int g = mb * (BM / 16) + q * 2;
+          atomicOr(&p.de_mask[(vt * 2 + h) * p.de_words + (g >> 5)],
+                   (((b & 0xFFFFu) ? 1u : 0u) | ((b >> 16) ? 2u : 0u)) << (g & 31));
         }
       }
       eng.epi_release(lane);
@@ -496,9 +527,19 @@ struct DEParams {
   void* dE;             // segment base
   __nv_bfloat16* dE_comp;
   int mode;  // 0 bf16 store, 1 fp32 store, 2 Kahan bf16
+  const uint32_t* mask;  // de_mask of the G producer (K-step mask per vocabulary block)
+  int mwords;
   const int* n_valid;
   int* status;
 };
+
+// True when no K step of a masked tile is issued (the tile is exactly zero).
+__device__ __forceinline__ bool mask_empty(const uint32_t* m, int nkb) {
+  if (!m) return false;
+  uint32_t any = 0;
+  for (int w = 0; w < ((nkb + 7) >> 3); ++w) any |= __ldg(m + w);
+  return any == 0;
+}
 
 struct DEPolicy {
   using Params = DEParams;
@@ -518,17 +559,21 @@ struct DEPolicy {
   }
   static __device__ void producer(const Params& p, Engine& eng) {
     schedule(p, [&](int vt, int dtile, int nkb) {
-      return eng.produce<true, true>(&p.mapA, &p.mapB, vt * BM, 0, dtile * BN, 0, nkb);
+      return eng.produce<true, true>(&p.mapA, &p.mapB, vt * BM, 0, dtile * BN, 0, nkb,
+                                     p.mask + vt * p.mwords);
     });
   }
   static __device__ void mma(const Params& p, Engine& eng) {
-    schedule(p, [&](int, int, int nkb) { return nkb == 0 || eng.mma<true, true>(nkb); });
+    schedule(p, [&](int vt, int, int nkb) {
+      return nkb == 0 || eng.mma<true, true>(nkb, p.mask + vt * p.mwords);
+    });
   }
   static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
     const int row = q * 32 + lane;
     schedule(p, [&](int vt, int dtile, int nkb) {
       uint32_t taddr = 0;
       if (nkb > 0 && !eng.epi_acquire(q, taddr)) return false;
+      const bool zero = nkb == 0 || mask_empty(p.mask + vt * p.mwords, nkb);
       const int r = vt * BM + row;
       const bool ok = r < p.chunk_valid;
       const int w = p.c0 + r;
@@ -537,7 +582,7 @@ struct DEPolicy {
         const int col0 = dtile * BN + c * 32;
         if (col0 >= p.D) break;
         uint32_t v[32];
-        if (nkb > 0) {
+        if (!zero) {
           tmem_ld32(taddr + c * 32, v);
         } else {
 #pragma unroll
@@ -601,6 +646,8 @@ struct DHParams {
   int dt;
   int D;
   float* dH_acc;  // [Npad, D]
+  const uint32_t* mask;  // dh_mask of the G producer (K-step mask per row block)
+  int mwords;
   const int* n_valid;
   int* status;
 };
@@ -624,11 +671,12 @@ struct DHPolicy {
   }
   static __device__ void producer(const Params& p, Engine& eng) {
     schedule(p, [&](int mb, int dtile, int) {
-      return eng.produce<false, true>(&p.mapA, &p.mapB, 0, mb * BM, dtile * BN, p.b_row0, p.nkb);
+      return eng.produce<false, true>(&p.mapA, &p.mapB, 0, mb * BM, dtile * BN, p.b_row0, p.nkb,
+                                      p.mask + mb * p.mwords);
     });
   }
   static __device__ void mma(const Params& p, Engine& eng) {
-    schedule(p, [&](int, int, int) { return eng.mma<false, true>(p.nkb); });
+    schedule(p, [&](int mb, int, int) { return eng.mma<false, true>(p.nkb, p.mask + mb * p.mwords); });
   }
   static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
     const int row = q * 32 + lane;
@@ -637,9 +685,10 @@ struct DHPolicy {
       if (!eng.epi_acquire(q, taddr)) return false;
       const int j = mb * BM + row;
       const bool ok = j < nv;
+      const bool zero = mask_empty(p.mask + mb * p.mwords, p.nkb);  // nothing to add
       for (int c = 0; c < BN / 32; ++c) {
         const int col0 = dtile * BN + c * 32;
-        if (col0 >= p.D) break;
+        if (col0 >= p.D || zero) break;
         uint32_t v[32];
         tmem_ld32(taddr + c * 32, v);
         if (!ok) continue;

@@ -27,6 +27,9 @@ CASES = {
     "composite_small": syn.scaled(syn.WORKLOADS["composite_two_segment"], N=900, D=256, V=6200,
                                   segments=((0, 3800), (3954, 6200))),
     "wide_D": syn.Workload("wide_D", N=260, D=1032, V=2300, logit_std=2.0, ignore_frac=0.0),
+    # logit std 40: after filtering nearly every 16-wide slice of G is zero,
+    # so most tensor-core steps and whole tiles are skipped
+    "peaky": syn.Workload("peaky", N=400, D=320, V=9000, logit_std=40.0, ignore_frac=0.05),
 }
 
 
@@ -72,7 +75,8 @@ def test_backward_unfiltered_matches_oracle(data, case):
     assert np.all(to_np(dH)[~x.valid] == 0)
 
 
-@pytest.mark.parametrize("case", ["gemma_like_small", "phi_like_small", "composite_small", "ragged"])
+@pytest.mark.parametrize("case", ["gemma_like_small", "phi_like_small", "composite_small", "ragged",
+                                  "peaky"])
 def test_backward_filtered_matches_oracle_and_criterion(data, case):
     x = data[case]
     H, segs, y, lse = _fwd_check(x)
