@@ -49,17 +49,21 @@ EncodeTiledFn encode_fn() {
 
 // 2-D bf16 tensor map over a row-major [rows, cols] matrix with the given row
 // stride (elements), 128-byte swizzle, zero fill out of bounds.
-bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld,
-              uint32_t box_cols, uint32_t box_rows) {
+bool make_map_t(CUtensorMap* m, CUtensorMapDataType dt, uint64_t esize, const void* base,
+                uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_cols, uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {ld * 2};
+  cuuint64_t strides[1] = {ld * esize};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld,
+              uint32_t box_cols, uint32_t box_rows) {
+  return make_map_t(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, cols, rows, ld, box_cols, box_rows);
 }
 
 int device_sms() {
@@ -230,10 +234,12 @@ void timing_end(long slot, cudaStream_t st) {
 template <class Policy>
 int launch_tc(const typename Policy::Params& prm, int grid, cudaStream_t st, int cls) {
   auto k = tc_kernel<Policy>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+  constexpr int smem = smem_bytes<Policy>();
+  static_assert(smem <= 232448, "shared memory per CTA exceeds 227 KB");
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return CCE_ELAUNCH;
   const long slot = timing_begin(cls, st);
-  k<<<grid, THREADS, SMEM_BYTES, st>>>(prm);
+  k<<<grid, THREADS, smem, st>>>(prm);
   timing_end(slot, st);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? CCE_OK : CCE_ELAUNCH;
@@ -483,6 +489,8 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   if (!make_map(&ep.mapA, G, Vc, pl.Npad, Vc, 64, 64)) return CCE_ELAUNCH;
   if (!make_map(&ep.mapB, Hc, D, pl.Npad, D, 64, 64)) return CCE_ELAUNCH;
   if (!make_map(&hp.mapA, G, Vc, pl.Npad, Vc, BK, BM)) return CCE_ELAUNCH;
+  if (!make_map_t(&hp.mapC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dH_acc, D, pl.Npad, D, 32, 32))
+    return CCE_ELAUNCH;
 
   for (int s = 0; s < sg.n; ++s) {
     const int ns = table.s[s].n;

@@ -43,7 +43,13 @@ struct Ctl {
   int pad;
 };
 
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + static_cast<int>(sizeof(Ctl)) + 64;
+// Dynamic shared memory of a policy's kernel: the stage ring, the policy's
+// own 1024-aligned epilogue buffer (Policy::EXTRA_SMEM bytes) and the control
+// block, plus alignment slack.
+template <class Policy>
+constexpr int smem_bytes() {
+  return STAGES * STAGE_BYTES + Policy::EXTRA_SMEM + static_cast<int>(sizeof(Ctl)) + 1024 + 64;
+}
 
 struct Pipe {
   int stage = 0;
@@ -85,7 +91,8 @@ struct MaskCursor {
 // Per-role state handed to policies.
 struct Engine {
   Ctl* ctl;
-  uint8_t* smem;  // 1024-byte aligned stage ring
+  uint8_t* smem;   // 1024-byte aligned stage ring
+  uint8_t* extra;  // 1024-byte aligned policy epilogue buffer
   uint32_t tmem;
   int* status;
   Pipe pipe;
@@ -211,7 +218,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (base & 1023u)) & 1023u);
-  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* extra = smem + STAGES * STAGE_BYTES;
+  Ctl* ctl = reinterpret_cast<Ctl*>(extra + Policy::EXTRA_SMEM);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -241,6 +249,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
   Engine eng;
   eng.ctl = ctl;
   eng.smem = smem;
+  eng.extra = extra;
   eng.tmem = ctl->tmem_base;
   eng.status = p.status;
 

@@ -208,6 +208,7 @@ struct FwdParams {
 
 struct FwdPolicy {
   using Params = FwdParams;
+  static constexpr int EXTRA_SMEM = 0;
 
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
@@ -408,6 +409,7 @@ struct GParams {
 
 struct GPolicy {
   using Params = GParams;
+  static constexpr int EXTRA_SMEM = 0;
 
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
@@ -543,6 +545,7 @@ __device__ __forceinline__ bool mask_empty(const uint32_t* m, int nkb) {
 
 struct DEPolicy {
   using Params = DEParams;
+  static constexpr int EXTRA_SMEM = 0;
 
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
@@ -641,6 +644,7 @@ struct DEPolicy {
 struct DHParams {
   CUtensorMap mapA;  // G K-major: [Npad, Vc], box {64, 128}
   CUtensorMap mapB;  // chunk rows of E, MN-major: box {64, 64}
+  CUtensorMap mapC;  // dH_acc fp32 [Npad, D], box {32, 32}, 128-byte swizzle
   int b_row0;
   int nkb;  // ceil(chunk_valid / 64)
   int dt;
@@ -654,6 +658,8 @@ struct DHParams {
 
 struct DHPolicy {
   using Params = DHParams;
+  // per epilogue warp: two 32 x 32 fp32 staging tiles for the TMA reduce-add
+  static constexpr int EXTRA_SMEM = 4 * 2 * 4096;
 
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
@@ -668,6 +674,7 @@ struct DHPolicy {
   static __device__ void prefetch(const Params& p) {
     tma_prefetch_map(&p.mapA);
     tma_prefetch_map(&p.mapB);
+    tma_prefetch_map(&p.mapC);
   }
   static __device__ void producer(const Params& p, Engine& eng) {
     schedule(p, [&](int mb, int dtile, int) {
@@ -678,35 +685,47 @@ struct DHPolicy {
   static __device__ void mma(const Params& p, Engine& eng) {
     schedule(p, [&](int mb, int, int) { return eng.mma<false, true>(p.nkb, p.mask + mb * p.mwords); });
   }
+  // Each warp adds its 32 accumulator rows into dH_acc 32 columns at a time:
+  // tcgen05.ld -> swizzled staging tile in shared memory -> TMA reduce-add
+  // (performed in L2), double-buffered so the next chunk is staged while the
+  // previous reduction still reads shared memory.  Rows past n_valid hold
+  // zeros (their G rows are zero), columns past D are clipped by the map.
   static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
-    const int row = q * 32 + lane;
-    schedule(p, [&](int mb, int dtile, int nv) {
+    uint8_t* stage = eng.extra + q * 2 * 4096;
+    const uint32_t st0 = smem_u32(stage);
+    int nbuf = 0;
+    schedule(p, [&](int mb, int dtile, int) {
       uint32_t taddr;
       if (!eng.epi_acquire(q, taddr)) return false;
-      const int j = mb * BM + row;
-      const bool ok = j < nv;
       const bool zero = mask_empty(p.mask + mb * p.mwords, p.nkb);  // nothing to add
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < BN / 32 && !zero; ++c) {
         const int col0 = dtile * BN + c * 32;
-        if (col0 >= p.D || zero) break;
+        if (col0 >= p.D) break;
         uint32_t v[32];
         tmem_ld32(taddr + c * 32, v);
-        if (!ok) continue;
-        float* d = p.dH_acc + (size_t)j * p.D + col0;
+        const int b = nbuf & 1;
+        if (lane == 0) bulk_wait_read<1>();  // the reduction that used buffer b is done reading
+        __syncwarp();
+        uint8_t* row = stage + b * 4096 + lane * 128;
 #pragma unroll
-        for (int g4 = 0; g4 < 8; ++g4) {
-          if (col0 + g4 * 4 >= p.D) break;
-          float4 a = *reinterpret_cast<float4*>(d + g4 * 4);
-          a.x += __uint_as_float(v[g4 * 4 + 0]);
-          a.y += __uint_as_float(v[g4 * 4 + 1]);
-          a.z += __uint_as_float(v[g4 * 4 + 2]);
-          a.w += __uint_as_float(v[g4 * 4 + 3]);
-          *reinterpret_cast<float4*>(d + g4 * 4) = a;
+        for (int k = 0; k < 8; ++k) {
+          float4 f = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                 __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+          *reinterpret_cast<float4*>(row + ((k ^ (lane & 7)) << 4)) = f;  // 128-byte swizzle
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_2d(&p.mapC, st0 + b * 4096, col0, mb * BM + q * 32);
+          bulk_commit();
+        }
+        ++nbuf;
       }
       eng.epi_release(lane);
       return true;
     });
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 };
 
