@@ -21,7 +21,9 @@ using namespace cce;
 namespace {
 
 constexpr int kPlanSMs = 148;            // SM count the workspace plan assumes
-constexpr size_t kGBudgetBytes = 64ull << 20;  // bf16 G slab per vocabulary chunk
+constexpr size_t kGBudgetBytes = 64ull << 20;   // preferred bf16 G slab (about L2-sized)
+constexpr size_t kGCapBytes = 512ull << 20;     // never more than this for the slab
+constexpr int64_t kDeWaves = 4;                 // dE tiles per chunk >= this many waves
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
@@ -171,9 +173,15 @@ struct BwdPlan {
 BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V) {
   BwdPlan p;
   p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
-  int64_t vc = (int64_t)(kGBudgetBytes / (2 * (size_t)p.Npad)) / BN * BN;
-  p.Vc = std::max<int64_t>(BN, std::min<int64_t>(8192, vc));
-  p.Vc = std::min<int64_t>(p.Vc, cdiv(V, BN) * BN);
+  // Vocabulary chunk width: an L2-sized slab, widened so that the dE
+  // contraction of one chunk ((Vc / 128) x (D / 256) tiles) fills at least
+  // kDeWaves waves of the SMs, within the slab cap.
+  const int64_t dt = cdiv(D, BN);
+  int64_t vc = (int64_t)(kGBudgetBytes / (2 * (size_t)p.Npad));
+  vc = std::max<int64_t>(vc, cdiv(kDeWaves * kPlanSMs * BM, dt));
+  vc = std::min<int64_t>(vc, (int64_t)(kGCapBytes / (2 * (size_t)p.Npad)));
+  vc = std::min<int64_t>(16384, vc) / BN * BN;
+  p.Vc = std::max<int64_t>(BN, std::min<int64_t>(vc, cdiv(V, BN) * BN));
   const size_t n4 = sizeof(int) * (size_t)std::max<int64_t>(N, 1);
   size_t o = 0;
   p.off_nvalid = o; o += align_up(16);
@@ -500,8 +508,11 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       if (!make_map(&segK, sg.s[s].E, D, ns, D, BK, BN)) return CCE_ELAUNCH;
       if (!make_map(&segMN, sg.s[s].E, D, ns, D, 64, 64)) return CCE_ELAUNCH;
     }
-    for (int c0 = 0; c0 < ns; c0 += Vc) {
-      const int cv = std::min(Vc, ns - c0);
+    // equal chunks (multiples of 256) so the last one is not a sliver
+    const int nch = (int)cdiv(ns, Vc);
+    const int cw = (int)std::min<int64_t>(Vc, cdiv(cdiv(ns, nch), BN) * BN);
+    for (int c0 = 0; c0 < ns; c0 += cw) {
+      const int cv = std::min(cw, ns - c0);
       int row0 = c0;
       if (perm_seg) {
         gather_perm_rows_kernel<<<sms * 4, 256, 0, st>>>(

