@@ -536,11 +536,12 @@ struct DEParams {
 };
 
 // True when no K step of a masked tile is issued (the tile is exactly zero).
-__device__ __forceinline__ bool mask_empty(const uint32_t* m, int nkb) {
+// Warp-parallel: one round of loads; every lane of the warp must call it.
+__device__ __forceinline__ bool mask_empty(const uint32_t* m, int nkb, int lane) {
   if (!m) return false;
   uint32_t any = 0;
-  for (int w = 0; w < ((nkb + 7) >> 3); ++w) any |= __ldg(m + w);
-  return any == 0;
+  for (int w = lane; w < ((nkb + 7) >> 3); w += 32) any |= __ldg(m + w);
+  return __all_sync(0xffffffffu, any == 0u);
 }
 
 struct DEPolicy {
@@ -574,9 +575,9 @@ struct DEPolicy {
   static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
     const int row = q * 32 + lane;
     schedule(p, [&](int vt, int dtile, int nkb) {
+      const bool zero = nkb == 0 || mask_empty(p.mask + vt * p.mwords, nkb, lane);
       uint32_t taddr = 0;
       if (nkb > 0 && !eng.epi_acquire(q, taddr)) return false;
-      const bool zero = nkb == 0 || mask_empty(p.mask + vt * p.mwords, nkb);
       const int r = vt * BM + row;
       const bool ok = r < p.chunk_valid;
       const int w = p.c0 + r;
@@ -695,9 +696,9 @@ struct DHPolicy {
     const uint32_t st0 = smem_u32(stage);
     int nbuf = 0;
     schedule(p, [&](int mb, int dtile, int) {
+      const bool zero = mask_empty(p.mask + mb * p.mwords, p.nkb, lane);  // nothing to add
       uint32_t taddr;
       if (!eng.epi_acquire(q, taddr)) return false;
-      const bool zero = mask_empty(p.mask + mb * p.mwords, p.nkb);  // nothing to add
       for (int c = 0; c < BN / 32 && !zero; ++c) {
         const int col0 = dtile * BN + c * 32;
         if (col0 >= p.D) break;
