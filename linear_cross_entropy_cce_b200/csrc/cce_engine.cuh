@@ -41,7 +41,12 @@ struct Ctl {
   int abort;
   int consumed;
   int pad;
+  // Stage records of the masked path, written by the producer before it
+  // arrives on full[s] and read by the MMA issuer after waiting on it:
+  // bits 0..3 = K=16 steps to issue, REC_LAST = last stage of its tile.
+  uint32_t rec[STAGES];
 };
+constexpr uint32_t REC_LAST = 1u << 4;
 
 // Dynamic shared memory of a policy's kernel: the stage ring, the policy's
 // own 1024-aligned epilogue buffer (Policy::EXTRA_SMEM bytes) and the control
@@ -176,6 +181,101 @@ struct Engine {
       umma_commit(smem_u32(&ctl->empty[pipe.stage]));
       pipe.advance();
       ++fills;
+    }
+    umma_commit(smem_u32(&ctl->tfull[acc]));
+    ++tcount;
+    return true;
+  }
+
+  // ---- masked producer (lane 0): like produce() with a K-step mask, but the
+  // MMA issuer never reads the mask: each loaded stage carries a record (its
+  // non-zero K steps, and REC_LAST on the tile's last loaded stage).  A stage
+  // is announced (record + arrive) only once the next non-zero stage is found
+  // or the tile ends, so REC_LAST is known; a tile with no non-zero stage
+  // still sends one empty REC_LAST stage.
+  template <bool A_MN, bool B_MN>
+  __device__ __forceinline__ bool produce_rec(const CUtensorMap* mA, const CUtensorMap* mB, int ax,
+                                              int ay, int bx, int by, int nkb,
+                                              const uint32_t* kmask) {
+    MaskCursor mc;
+    mc.init(kmask, nkb);
+    int pend = -1;         // stage announced last (awaiting its record)
+    uint32_t pend_bits = 0;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const uint32_t bits = mc.bits(kb);
+      if (!bits) continue;
+      if (!wait_parity(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u, abort_flag(), status))
+        return false;
+      const uint32_t fb = smem_u32(&ctl->full[pipe.stage]);
+      mbar_expect_tx(fb, STAGE_BYTES);
+      const uint32_t sa = smem_u32(smem + pipe.stage * STAGE_BYTES);
+      const uint32_t sb = sa + A_BYTES;
+      if (!A_MN) {
+        tma_load_2d(sa, mA, fb, ax + kb * BK, ay);
+      } else {
+        tma_load_2d(sa, mA, fb, ax, ay + kb * BK);
+        tma_load_2d(sa + 8192, mA, fb, ax + 64, ay + kb * BK);
+      }
+      if (!B_MN) {
+        tma_load_2d(sb, mB, fb, bx + kb * BK, by);
+      } else {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_load_2d(sb + b * 8192, mB, fb, bx + b * 64, by + kb * BK);
+      }
+      if (pend >= 0) {  // the previous stage was not the last one
+        ctl->rec[pend] = pend_bits;
+        mbar_arrive(smem_u32(&ctl->full[pend]));
+      }
+      pend = pipe.stage;
+      pend_bits = bits;
+      pipe.advance();
+      ++fills;
+    }
+    if (pend < 0) {  // nothing to load: one empty stage ends the tile
+      if (!wait_parity(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u, abort_flag(), status))
+        return false;
+      pend = pipe.stage;
+      pend_bits = 0;
+      pipe.advance();
+      ++fills;
+    }
+    ctl->rec[pend] = pend_bits | REC_LAST;
+    mbar_arrive(smem_u32(&ctl->full[pend]));
+    return true;
+  }
+
+  // ---- masked MMA issuer: consumes the producer's records until REC_LAST.
+  template <bool A_MN, bool B_MN>
+  __device__ __forceinline__ bool mma_rec() {
+    const int acc = tcount & 1;
+    if (!wait_parity(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u,
+                     abort_flag(), status))
+      return false;
+    tc_fence_after();
+    const uint32_t d = tmem + acc * BN;
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+    constexpr uint32_t a_step = A_MN ? 2048 : 32;  // bytes per K=16 step
+    constexpr uint32_t b_step = B_MN ? 2048 : 32;
+    const uint64_t ad0 = A_MN ? smem_desc_sw128(smem_u32(smem), 8192, 1024)
+                              : smem_desc_sw128(smem_u32(smem), 16, 1024);
+    const uint64_t bd0 = B_MN ? smem_desc_sw128(smem_u32(smem) + A_BYTES, 8192, 1024)
+                              : smem_desc_sw128(smem_u32(smem) + A_BYTES, 16, 1024);
+    uint32_t issued = 0;
+    for (;;) {
+      if (!wait_parity(smem_u32(&ctl->full[pipe.stage]), pipe.phase, abort_flag(), status))
+        return false;
+      const uint32_t rec = *reinterpret_cast<volatile uint32_t*>(&ctl->rec[pipe.stage]);
+      const uint64_t so = (uint64_t)((pipe.stage * STAGE_BYTES) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        if (!(rec & (1u << kk))) continue;
+        umma_bf16(d, ad0 + so + kk * (a_step >> 4), bd0 + so + kk * (b_step >> 4), idesc, issued);
+        issued = 1;
+      }
+      umma_commit(smem_u32(&ctl->empty[pipe.stage]));
+      pipe.advance();
+      ++fills;
+      if (rec & REC_LAST) break;
     }
     umma_commit(smem_u32(&ctl->tfull[acc]));
     ++tcount;

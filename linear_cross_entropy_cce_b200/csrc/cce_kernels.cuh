@@ -563,13 +563,13 @@ struct DEPolicy {
   }
   static __device__ void producer(const Params& p, Engine& eng) {
     schedule(p, [&](int vt, int dtile, int nkb) {
-      return eng.produce<true, true>(&p.mapA, &p.mapB, vt * BM, 0, dtile * BN, 0, nkb,
-                                     p.mask + vt * p.mwords);
+      return eng.produce_rec<true, true>(&p.mapA, &p.mapB, vt * BM, 0, dtile * BN, 0, nkb,
+                                         p.mask + vt * p.mwords);
     });
   }
   static __device__ void mma(const Params& p, Engine& eng) {
     schedule(p, [&](int vt, int, int nkb) {
-      return nkb == 0 || eng.mma<true, true>(nkb, p.mask + vt * p.mwords);
+      return nkb == 0 || eng.mma_rec<true, true>();
     });
   }
   static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
@@ -679,12 +679,12 @@ struct DHPolicy {
   }
   static __device__ void producer(const Params& p, Engine& eng) {
     schedule(p, [&](int mb, int dtile, int) {
-      return eng.produce<false, true>(&p.mapA, &p.mapB, 0, mb * BM, dtile * BN, p.b_row0, p.nkb,
-                                      p.mask + mb * p.mwords);
+      return eng.produce_rec<false, true>(&p.mapA, &p.mapB, 0, mb * BM, dtile * BN, p.b_row0,
+                                          p.nkb, p.mask + mb * p.mwords);
     });
   }
   static __device__ void mma(const Params& p, Engine& eng) {
-    schedule(p, [&](int mb, int, int) { return eng.mma<false, true>(p.nkb, p.mask + mb * p.mwords); });
+    schedule(p, [&](int, int, int) { return eng.mma_rec<false, true>(); });
   }
   // Each warp adds its 32 accumulator rows into dH_acc 32 columns at a time:
   // tcgen05.ld -> swizzled staging tile in shared memory -> TMA reduce-add
