@@ -13,7 +13,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libcce.so")
 SOURCES = ["cce_api.cu", "cce_noalloc.cu"]
-HEADERS = ["cce_ptx.cuh", "cce_engine.cuh", "cce_kernels.cuh"]
+HEADERS = ["cce_ptx.cuh", "cce_engine.cuh", "cce_kernels.cuh", "cce_sparse.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 

@@ -168,6 +168,9 @@ struct BwdPlan {
       off_dh, off_g, off_ec, off_masks, total;
   int dh_words, de_words;
   size_t mask_bytes;
+  // sparse backward (filtered gradients)
+  int64_t nch_max, cap;
+  size_t off_nzcnt, off_lists, off_colc, off_csorted, off_rowc, off_rsorted;
 };
 
 BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V) {
@@ -200,6 +203,15 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V) {
   p.de_words = (int)cdiv(p.Npad, 512);
   p.mask_bytes = sizeof(uint32_t) * ((size_t)(p.Npad / BM) * p.dh_words + (size_t)(p.Vc / BM) * p.de_words);
   p.off_masks = o; o += align_up(p.mask_bytes);
+  // sparse path: per chunk a list of up to `cap` non-zeros (density 1/2048)
+  p.nch_max = cdiv(V, p.Vc) + CCE_MAX_SEGMENTS;
+  p.cap = std::max<int64_t>(4096, p.Npad * p.Vc / 2048);
+  p.off_nzcnt = o; o += align_up(sizeof(int) * (size_t)p.nch_max);
+  p.off_lists = o; o += align_up(sizeof(NzEntry) * (size_t)p.nch_max * p.cap);
+  p.off_colc = o; o += align_up(sizeof(int) * 3 * (size_t)(p.Vc + 1));
+  p.off_csorted = o; o += align_up(sizeof(int2) * (size_t)p.cap);
+  p.off_rowc = o; o += align_up(sizeof(int) * 3 * (size_t)(p.Npad + 1));
+  p.off_rsorted = o; o += align_up(sizeof(int2) * (size_t)p.nch_max * p.cap);
   p.total = o;
   return p;
 }
@@ -486,6 +498,27 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   const int nkbD = (int)cdiv(D, BK);
   const int mbs = (int)(pl.Npad / BM);
   const float eps_keep = filter_eps > 0.f ? filter_eps * (1.0f - 1.0f / 256.0f) : 0.f;
+  // Sparse contractions for filtered gradients (chunks with at most `cap`
+  // non-zeros; the Kahan path stays on the deterministic dense route).
+  bool sparse = filter_eps > 0.f && !kahan;
+  for (int s = 0; s < sg.n; ++s) sparse = sparse && table.s[s].n < (1 << 29);
+  const int cap = (int)pl.cap;
+  int* nz_cnt = at<int>(workspace, pl.off_nzcnt);
+  NzEntry* lists = at<NzEntry>(workspace, pl.off_lists);
+  int* col_cnt = at<int>(workspace, pl.off_colc);
+  int* col_ptr = col_cnt + (pl.Vc + 1);
+  int* col_cur = col_ptr + (pl.Vc + 1);
+  int2* csorted = at<int2>(workspace, pl.off_csorted);
+  int* row_cnt = at<int>(workspace, pl.off_rowc);
+  int* row_ptr = row_cnt + (pl.Npad + 1);
+  int* row_cur = row_ptr + (pl.Npad + 1);
+  int2* rsorted = at<int2>(workspace, pl.off_rsorted);
+  if (sparse && cudaMemsetAsync(nz_cnt, 0, sizeof(int) * pl.nch_max, st) != cudaSuccess)
+    return CCE_ELAUNCH;
+  ChunkMap cmap;
+  memset(&cmap, 0, sizeof(cmap));
+  cmap.n_segs = sg.n;
+  int chunk = 0;  // global chunk index
 
   GParams gp;
   DEParams ep;
@@ -511,7 +544,9 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
     // equal chunks (multiples of 256) so the last one is not a sliver
     const int nch = (int)cdiv(ns, Vc);
     const int cw = (int)std::min<int64_t>(Vc, cdiv(cdiv(ns, nch), BN) * BN);
-    for (int c0 = 0; c0 < ns; c0 += cw) {
+    cmap.chunk_begin[s] = chunk;
+    cmap.width[s] = cw;
+    for (int c0 = 0; c0 < ns; c0 += cw, ++chunk) {
       const int cv = std::min(cw, ns - c0);
       int row0 = c0;
       if (perm_seg) {
@@ -550,9 +585,41 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       gp.seg_begin = table.s[s].begin;
       gp.perm_seg = perm_seg;
       gp.status = status;
+      gp.nz_list = sparse ? lists + (size_t)chunk * cap : nullptr;
+      gp.nz_cnt = nz_cnt + chunk;
+      gp.nz_cap = cap;
+      gp.col_cnt = col_cnt;
+      if (sparse && cudaMemsetAsync(col_cnt, 0, sizeof(int) * (size_t)cv, st) != cudaSuccess)
+        return CCE_ELAUNCH;
       if (int rc = launch_tc<GPolicy>(gp, (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct), st, KC_G))
         return rc;
-      // step 2: dE rows of this chunk
+      // step 2: dE rows of this chunk (sparse gathers, or the dense contraction)
+      if (sparse) {
+        sparse_col_scan_kernel<<<1, SCAN_THREADS, 0, st>>>(nz_cnt + chunk, cap, col_cnt, cv, col_ptr,
+                                                           col_cur);
+        if (launched()) return CCE_ELAUNCH;
+        sparse_col_scatter_kernel<<<sms * 2, 256, 0, st>>>(nz_cnt + chunk, cap,
+                                                          lists + (size_t)chunk * cap, col_cur, csorted);
+        if (launched()) return CCE_ELAUNCH;
+        SparseDEParams sp;
+        sp.nz_cnt = nz_cnt + chunk;
+        sp.cap = cap;
+        sp.col_ptr = col_ptr;
+        sp.sorted = csorted;
+        sp.Hc = Hc;
+        sp.D = (int)D;
+        sp.cv = cv;
+        sp.c0 = c0;
+        sp.perm_seg = perm_seg;
+        sp.dE = sg.s[s].dE;
+        sp.dE_comp = nullptr;
+        sp.mode = fp32 ? 1 : 0;
+        const int64_t warps = (int64_t)cv * cdiv(D, 256);
+        sparse_de_kernel<<<(int)std::min<int64_t>(sms * 16, cdiv(warps, 8)), 256, 0, st>>>(sp);
+        if (launched()) return CCE_ELAUNCH;
+      }
+      ep.nz_cnt = sparse ? nz_cnt + chunk : nullptr;
+      ep.nz_cap = cap;
       ep.chunk_valid = cv;
       ep.mt = (int)cdiv(cv, BM);
       ep.dt = dt;
@@ -575,6 +642,8 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       hp.dt = dt;
       hp.D = (int)D;
       hp.dH_acc = dH_acc;
+      hp.nz_cnt = sparse ? nz_cnt + chunk : nullptr;
+      hp.nz_cap = cap;
       hp.mask = dh_mask;
       hp.mwords = pl.dh_words;
       hp.n_valid = cp.n_valid;
@@ -583,8 +652,38 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
         return rc;
     }
   }
-  dh_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, 8), sms * 8), 256, 0, st>>>(
-      dH_acc, cp.pos_of_row, (int)N, (int)D, dH, fp32 ? 1 : 0);
+  // sparse chunks' dH contributions: row lists over every chunk
+  if (sparse) {
+    if (cudaMemsetAsync(row_cnt, 0, sizeof(int) * (size_t)pl.Npad, st) != cudaSuccess)
+      return CCE_ELAUNCH;
+    SparseRowsParams rp;
+    rp.nz_cnt = nz_cnt;
+    rp.nch = chunk;
+    rp.cap = cap;
+    rp.lists = lists;
+    rp.row_cnt = row_cnt;
+    rp.row_cur = row_cur;
+    rp.rsorted = rsorted;
+    rp.cmap = cmap;
+    sparse_row_count_kernel<<<sms * 4, 256, 0, st>>>(rp);
+    if (launched()) return CCE_ELAUNCH;
+    sparse_row_scan_kernel<<<1, SCAN_THREADS, 0, st>>>(row_cnt, (int)pl.Npad, row_ptr, row_cur);
+    if (launched()) return CCE_ELAUNCH;
+    sparse_row_scatter_kernel<<<sms * 4, 256, 0, st>>>(rp);
+    if (launched()) return CCE_ELAUNCH;
+  }
+  DHFinParams fp_;
+  fp_.dH_acc = dH_acc;
+  fp_.pos_of_row = cp.pos_of_row;
+  fp_.N = (int)N;
+  fp_.D = (int)D;
+  fp_.dH = dH;
+  fp_.fp32_out = fp32 ? 1 : 0;
+  fp_.row_ptr = sparse ? row_ptr : nullptr;
+  fp_.rsorted = rsorted;
+  fp_.segs = table;
+  fp_.vocab_perm = vocab_perm;
+  dh_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, 8), sms * 8), 256, 0, st>>>(fp_);
   return launched();
 }
 

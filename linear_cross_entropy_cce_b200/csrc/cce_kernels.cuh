@@ -30,6 +30,7 @@
 #include <cub/block/block_scan.cuh>
 
 #include "cce_engine.cuh"
+#include "cce_sparse.cuh"
 
 namespace cce {
 
@@ -58,12 +59,6 @@ __device__ __forceinline__ int segment_of(const SegTable& t, long long y) {
   return -1;
 }
 
-__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -397,6 +392,11 @@ struct GParams {
   int dh_words;
   uint32_t* de_mask;
   int de_words;
+  // sparse list of this chunk's non-zeros (null: not collected)
+  NzEntry* nz_list;
+  int* nz_cnt;   // entries emitted (may exceed nz_cap: the chunk is then dense)
+  int nz_cap;
+  int* col_cnt;  // per chunk column: entries (zeroed before this launch)
   // optional per-element keep bits of original rows < debug_rows
   uint32_t* debug_keep;
   int debug_rows;
@@ -435,6 +435,7 @@ struct GPolicy {
   }
   static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
     const int row = q * 32 + lane;
+    bool emit = true;  // this warp still lists non-zeros (warp-uniform)
     schedule(p, [&](int mb, int vt, int nv) {
       uint32_t taddr;
       if (!eng.epi_acquire(q, taddr)) return false;
@@ -452,6 +453,7 @@ struct GPolicy {
         tmem_ld32(taddr + c * 32, r);
         uint32_t packed[16];
         bool nz[2] = {false, false};
+        uint32_t nzb = 0;  // bit j: fp32 G of column c*32+j is non-zero
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           float g[2];
@@ -466,6 +468,42 @@ struct GPolicy {
           }
           packed[j >> 1] = pack_bf16(g[0], g[1]);
           nz[j >> 4] |= (packed[j >> 1] & 0x7FFF7FFFu) != 0u;  // non-zero after rounding
+          nzb |= (g[0] != 0.f ? 1u : 0u) << j;
+          nzb |= (g[1] != 0.f ? 1u : 0u) << (j + 1);
+        }
+        if (p.nz_list && emit) {
+          // warp-aggregated reservation of this chunk's non-zeros in the list
+          const int cnt = __popc(nzb);
+          int incl = cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+          }
+          const int total = __shfl_sync(0xffffffffu, incl, 31);
+          if (total > 0) {
+            int base = 0;
+            if (lane == 0) base = atomicAdd(p.nz_cnt, total);
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (base + total > p.nz_cap) emit = false;  // the chunk goes dense: stop listing
+            int pos = base + incl - cnt;
+            if (nzb) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (!((nzb >> j) & 1u)) continue;
+                // the same arithmetic as above, so the same value
+                const int col = c * 32 + j;
+                const float pr = ex2_approx(fmaf(__uint_as_float(r[j]), kLog2e, -lse2));
+                float v = pr >= p.eps_keep ? pr : 0.f;
+                v -= (col == tcol) ? 1.f : 0.f;
+                if (pos < p.nz_cap) {
+                  p.nz_list[pos] = NzEntry{jrow, vt * BN + col, dl * v, 0};
+                  atomicAdd(&p.col_cnt[vt * BN + col], 1);
+                }
+                ++pos;
+              }
+            }
+          }
         }
         uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
         dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
@@ -529,6 +567,8 @@ struct DEParams {
   void* dE;             // segment base
   __nv_bfloat16* dE_comp;
   int mode;  // 0 bf16 store, 1 fp32 store, 2 Kahan bf16
+  const int* nz_cnt;  // chunk handled by the sparse path when *nz_cnt <= nz_cap
+  int nz_cap;
   const uint32_t* mask;  // de_mask of the G producer (K-step mask per vocabulary block)
   int mwords;
   const int* n_valid;
@@ -551,7 +591,7 @@ struct DEPolicy {
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
     const int nkb = (*p.n_valid + BK - 1) / BK;
-    const int tiles = p.mt * p.dt;
+    const int tiles = (p.nz_cnt && *p.nz_cnt <= p.nz_cap) ? 0 : p.mt * p.dt;
     for (int i = blockIdx.x; i < tiles; i += gridDim.x) {
       const int vt = i / p.dt;
       if (!f(vt, i - vt * p.dt, nkb)) return;
@@ -651,6 +691,8 @@ struct DHParams {
   int dt;
   int D;
   float* dH_acc;  // [Npad, D]
+  const int* nz_cnt;  // chunk handled by the sparse path when *nz_cnt <= nz_cap
+  int nz_cap;
   const uint32_t* mask;  // dh_mask of the G producer (K-step mask per row block)
   int mwords;
   const int* n_valid;
@@ -666,7 +708,7 @@ struct DHPolicy {
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
     const int nv = *p.n_valid;
     const int num_mb = (nv + BM - 1) / BM;
-    const int tiles = num_mb * p.dt;
+    const int tiles = (p.nz_cnt && *p.nz_cnt <= p.nz_cap) ? 0 : num_mb * p.dt;
     for (int i = blockIdx.x; i < tiles; i += gridDim.x) {
       const int mb = i / p.dt;
       if (!f(mb, i - mb * p.dt, nv)) return;
@@ -730,24 +772,62 @@ struct DHPolicy {
   }
 };
 
-// dH[i] = dH_acc[pos_of_row[i]] (bf16 or fp32); 0 for ignored rows, NaN for
-// rows with a bad target.  One warp per row.
-__global__ void dh_finalize_kernel(const float* __restrict__ dH_acc, const int* __restrict__ pos_of_row,
-                                   int N, int D, void* dH, int fp32_out) {
+// dH[i] = dH_acc[pos_of_row[i]] + (sparse chunks) sum_j G_ij e_j, in bf16 or
+// fp32; 0 for ignored rows, NaN for rows with a bad target.  One warp per
+// row; lane owns 8 consecutive columns of each 256-wide slice of D.
+struct DHFinParams {
+  const float* dH_acc;
+  const int* pos_of_row;
+  int N, D;
+  void* dH;
+  int fp32_out;
+  const int* row_ptr;    // null: no sparse chunks
+  const int2* rsorted;   // (segment << 29 | walk position, g)
+  SegTable segs;
+  const int* vocab_perm; // concatenated per-segment permutations, or null
+};
+
+__global__ void dh_finalize_kernel(const DHFinParams p) {
   const int lane = threadIdx.x & 31;
   const int nw = (gridDim.x * blockDim.x) >> 5;
-  const int vec = D >> 2;
-  for (int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < N; i += nw) {
-    const int j = pos_of_row[i];
+  for (int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < p.N; i += nw) {
+    const int j = p.pos_of_row[i];
     const float fill = j == -1 ? 0.f : __int_as_float(0x7fc00000);
-    const float4* src = reinterpret_cast<const float4*>(dH_acc + (size_t)(j < 0 ? 0 : j) * D);
-    for (int v = lane; v < vec; v += 32) {
-      const float4 a = j >= 0 ? src[v] : make_float4(fill, fill, fill, fill);
-      if (fp32_out) {
-        reinterpret_cast<float4*>(static_cast<float*>(dH) + (size_t)i * D)[v] = a;
+    const int e0 = (j >= 0 && p.row_ptr) ? p.row_ptr[j] : 0;
+    const int e1 = (j >= 0 && p.row_ptr) ? p.row_ptr[j + 1] : 0;
+    for (int d0 = lane * 8; d0 < p.D; d0 += 256) {
+      float a[8];
+      if (j >= 0) {
+        const float4* src = reinterpret_cast<const float4*>(p.dH_acc + (size_t)j * p.D + d0);
+        const float4 u = src[0], v = src[1];
+        a[0] = u.x; a[1] = u.y; a[2] = u.z; a[3] = u.w;
+        a[4] = v.x; a[5] = v.y; a[6] = v.z; a[7] = v.w;
+        for (int e = e0; e < e1; ++e) {
+          const int2 t = p.rsorted[e];
+          const float g = __int_as_float(t.y);
+          const int s = (int)((unsigned)t.x >> 29), w = t.x & ((1 << 29) - 1);
+          const int loc = p.vocab_perm ? p.vocab_perm[p.segs.s[s].live_off + w] : w;
+          const uint4 h = __ldg(reinterpret_cast<const uint4*>(p.segs.s[s].E + (size_t)loc * p.D + d0));
+          a[0] = fmaf(g, bf16lo(h.x), a[0]);
+          a[1] = fmaf(g, bf16hi(h.x), a[1]);
+          a[2] = fmaf(g, bf16lo(h.y), a[2]);
+          a[3] = fmaf(g, bf16hi(h.y), a[3]);
+          a[4] = fmaf(g, bf16lo(h.z), a[4]);
+          a[5] = fmaf(g, bf16hi(h.z), a[5]);
+          a[6] = fmaf(g, bf16lo(h.w), a[6]);
+          a[7] = fmaf(g, bf16hi(h.w), a[7]);
+        }
       } else {
-        reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(dH) + (size_t)i * D)[v] =
-            make_uint2(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w));
+        for (int k = 0; k < 8; ++k) a[k] = fill;
+      }
+      if (p.fp32_out) {
+        float4* d = reinterpret_cast<float4*>(static_cast<float*>(p.dH) + (size_t)i * p.D + d0);
+        d[0] = make_float4(a[0], a[1], a[2], a[3]);
+        d[1] = make_float4(a[4], a[5], a[6], a[7]);
+      } else {
+        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dH) + (size_t)i * p.D + d0) =
+            make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]),
+                       pack_bf16(a[6], a[7]));
       }
     }
   }

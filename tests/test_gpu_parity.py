@@ -30,6 +30,11 @@ CASES = {
     # logit std 40: after filtering nearly every 16-wide slice of G is zero,
     # so most tensor-core steps and whole tiles are skipped
     "peaky": syn.Workload("peaky", N=400, D=320, V=9000, logit_std=40.0, ignore_frac=0.05),
+    # filtered G below 1/2048 density: the sparse (CUDA-core) contractions run
+    "sparse_g": syn.Workload("sparse_g", N=900, D=264, V=30000, logit_std=16.0, ignore_frac=0.1),
+    "sparse_g_segments": syn.Workload("sparse_g_segments", N=700, D=192, V=26000, logit_std=16.0,
+                                      ignore_frac=0.3, segments=((0, 15000), (15500, 26000)),
+                                      segment_mix=(0.7, 0.3)),
 }
 
 
@@ -76,7 +81,7 @@ def test_backward_unfiltered_matches_oracle(data, case):
 
 
 @pytest.mark.parametrize("case", ["gemma_like_small", "phi_like_small", "composite_small", "ragged",
-                                  "peaky"])
+                                  "peaky", "sparse_g", "sparse_g_segments"])
 def test_backward_filtered_matches_oracle_and_criterion(data, case):
     x = data[case]
     H, segs, y, lse = _fwd_check(x)
