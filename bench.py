@@ -53,6 +53,28 @@ def peaks():
                 "fallback": True}
 
 
+def src_hash16():
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "linear_cross_entropy_cce_b200", "csrc", "*.cu*")))
+    for f in files + [os.path.join(ROOT, "include", "cce.h")]:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu record, or None
+    when the CUDA sources changed since it was captured."""
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "roofline_traffic.json")))
+    except Exception:
+        return None
+    if rec.get("csrc_sha256_16") != src_hash16():
+        return None
+    return rec.get("per_launch_dram_bytes", {}).get(kernel)
+
+
 def host_cores():
     try:
         from threadpoolctl import threadpool_info
@@ -317,7 +339,9 @@ def main():
                 "peak": peak_sus, "unit": "TFLOP/s",
                 "frac": round(achieved / peak_sus, 4) if achieved else None,
                 "peak_kind": "sustained bf16 (measured, cuBLAS) - kernel timed inside the step",
-                "traffic": None,
+                "traffic": recorded_traffic(dom) if wl.name == "gemma2_2b_head" else None,
+                "traffic_note": "DRAM bytes of one launch of this kernel from the committed ncu capture "
+                                "(profiles/roofline_traffic.json, cold cache); null if the sources changed",
                 "launches_per_step": dom_n // max(1, a.steps),
                 "avg_launch_ms": round(dom_ms / max(1, dom_n), 4)}
     step_tflops = flops_step / (ms_step / 1e3) / 1e12
@@ -351,6 +375,8 @@ def main():
                            "materialised_logits_bf16_mb": round(N * V * 2 / 2 ** 20, 1)},
         "roofline": roofline,
         "per_kernel_ms_per_step": {k: round(v[0] / a.steps, 3) for k, v in per_class.items()},
+        "other_kernels_ms_per_step": round(ms_prof - sum(v[0] for k, v in per_class.items()
+                                                         if k != "aux") / a.steps, 3),
         "profiled_ms_per_step": round(ms_prof, 3),
         "gpu_launches": int(launches),
         "gpu_launches_per_step": int(launches // max(1, a.steps)),
