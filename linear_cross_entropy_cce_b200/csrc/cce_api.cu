@@ -206,7 +206,7 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V) {
   // sparse path: per chunk a list of up to `cap` non-zeros (density 1/2048)
   p.nch_max = cdiv(V, p.Vc) + CCE_MAX_SEGMENTS;
   p.cap = std::max<int64_t>(4096, p.Npad * p.Vc / 2048);
-  p.off_nzcnt = o; o += align_up(sizeof(int) * (size_t)p.nch_max);
+  p.off_nzcnt = o; o += align_up(sizeof(int) * 2 * (size_t)p.nch_max);  // counts + slab flags
   p.off_lists = o; o += align_up(sizeof(NzEntry) * (size_t)p.nch_max * p.cap);
   p.off_colc = o; o += align_up(sizeof(int) * 3 * (size_t)(p.Vc + 1));
   p.off_csorted = o; o += align_up(sizeof(int2) * (size_t)p.cap);
@@ -513,7 +513,8 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   int* row_ptr = row_cnt + (pl.Npad + 1);
   int* row_cur = row_ptr + (pl.Npad + 1);
   int2* rsorted = at<int2>(workspace, pl.off_rsorted);
-  if (sparse && cudaMemsetAsync(nz_cnt, 0, sizeof(int) * pl.nch_max, st) != cudaSuccess)
+  int* slab_flag = nz_cnt + pl.nch_max;
+  if (sparse && cudaMemsetAsync(nz_cnt, 0, sizeof(int) * 2 * pl.nch_max, st) != cudaSuccess)
     return CCE_ELAUNCH;
   ChunkMap cmap;
   memset(&cmap, 0, sizeof(cmap));
@@ -577,6 +578,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       gp.tseg = cp.tseg;
       gp.tpos = cp.tpos;
       gp.eps_keep = eps_keep;
+      gp.l2eps = eps_keep > 0.f ? log2f(eps_keep) : -INFINITY;
       gp.G = G;
       gp.debug_keep = debug_keep;
       gp.debug_rows = (int)debug_rows;
@@ -589,10 +591,18 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       gp.nz_cnt = nz_cnt + chunk;
       gp.nz_cap = cap;
       gp.col_cnt = col_cnt;
+      gp.prev_nz_cnt = chunk > 0 ? nz_cnt + chunk - 1 : nullptr;
+      gp.slab_flag = slab_flag + chunk;
+      gp.repair = 0;
       if (sparse && cudaMemsetAsync(col_cnt, 0, sizeof(int) * (size_t)cv, st) != cudaSuccess)
         return CCE_ELAUNCH;
       if (int rc = launch_tc<GPolicy>(gp, (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct), st, KC_G))
         return rc;
+      if (sparse) {  // recompute with the dense fallback if the chunk was mispredicted
+        gp.repair = 1;
+        if (int rc = launch_tc<GPolicy>(gp, (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct), st, KC_G))
+          return rc;
+      }
       // step 2: dE rows of this chunk (sparse gathers, or the dense contraction)
       if (sparse) {
         sparse_col_scan_kernel<<<1, SCAN_THREADS, 0, st>>>(nz_cnt + chunk, cap, col_cnt, cv, col_ptr,

@@ -382,6 +382,7 @@ struct GParams {
   const int* tseg;
   const int* tpos;
   float eps_keep;  // 0: keep everything
+  float l2eps;     // log2(eps_keep) (-inf when 0): keep_ij = z_ij log2 e - lse_i log2 e >= l2eps
   __nv_bfloat16* G;
   // Zero-slice masks for the two contractions (zeroed before this launch):
   //   dh_mask[mb * dh_words + g / 32] bit g % 32: some row of row block mb
@@ -397,6 +398,14 @@ struct GParams {
   int* nz_cnt;   // entries emitted (may exceed nz_cap: the chunk is then dense)
   int nz_cap;
   int* col_cnt;  // per chunk column: entries (zeroed before this launch)
+  // With a list, the bf16 slab and the masks (the dense fallback) are
+  // written only when this chunk is predicted dense: the first chunk, or a
+  // chunk after one that overflowed its list.  A mispredicted chunk is
+  // recomputed by a second launch with `repair` set, which runs only when
+  // the chunk overflowed and its slab was not written.
+  const int* prev_nz_cnt;  // previous chunk's count, or null
+  int* slab_flag;          // set when this chunk's slab has been written
+  int repair;
   // optional per-element keep bits of original rows < debug_rows
   uint32_t* debug_keep;
   int debug_rows;
@@ -411,11 +420,21 @@ struct GPolicy {
   using Params = GParams;
   static constexpr int EXTRA_SMEM = 0;
 
+  // Whether this launch writes the dense fallback (slab + masks), and
+  // whether it runs at all (a repair launch usually has nothing to do).
+  static __device__ __forceinline__ bool writes_slab(const Params& p) {
+    if (!p.nz_list || p.repair) return true;
+    return p.prev_nz_cnt == nullptr || *p.prev_nz_cnt > p.nz_cap;
+  }
+  static __device__ __forceinline__ bool active(const Params& p) {
+    return !p.repair || (*p.nz_cnt > p.nz_cap && *p.slab_flag == 0);
+  }
+
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
     const int nv = *p.n_valid;
     const int num_mb = (nv + BM - 1) / BM;
-    const int tiles = num_mb * p.ct;
+    const int tiles = active(p) ? num_mb * p.ct : 0;
     for (int i = blockIdx.x; i < tiles; i += gridDim.x) {
       const int vt = i / num_mb;
       if (!f(i - vt * num_mb, vt, nv)) return;
@@ -435,7 +454,10 @@ struct GPolicy {
   }
   static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
     const int row = q * 32 + lane;
-    bool emit = true;  // this warp still lists non-zeros (warp-uniform)
+    const bool slab = writes_slab(p);
+    bool emit = p.nz_list != nullptr && !p.repair;  // this warp still lists non-zeros
+    if (slab && p.slab_flag && !p.repair && blockIdx.x == 0 && threadIdx.x == 64)
+      *p.slab_flag = 1;
     schedule(p, [&](int mb, int vt, int nv) {
       uint32_t taddr;
       if (!eng.epi_acquire(q, taddr)) return false;
@@ -451,27 +473,49 @@ struct GPolicy {
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(taddr + c * 32, r);
-        uint32_t packed[16];
-        bool nz[2] = {false, false};
-        uint32_t nzb = 0;  // bit j: fp32 G of column c*32+j is non-zero
+        // keep bits: softmax part retained (p >= eps, decided in base-2 log
+        // space), then the non-zero set including the target's one-hot term
+        uint32_t kb = 0;
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          float g[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = c * 32 + j + u;
-            const float pr = ex2_approx(fmaf(__uint_as_float(r[j + u]), kLog2e, -lse2));
-            const bool keep = pr >= p.eps_keep;
-            float v = keep ? pr : 0.f;
-            v -= (col == tcol) ? 1.f : 0.f;
-            g[u] = (ok && col < valid) ? dl * v : 0.f;
-          }
-          packed[j >> 1] = pack_bf16(g[0], g[1]);
-          nz[j >> 4] |= (packed[j >> 1] & 0x7FFF7FFFu) != 0u;  // non-zero after rounding
-          nzb |= (g[0] != 0.f ? 1u : 0u) << j;
-          nzb |= (g[1] != 0.f ? 1u : 0u) << (j + 1);
+        for (int j = 0; j < 32; ++j) {
+          const float z2 = fmaf(__uint_as_float(r[j]), kLog2e, -lse2);
+          r[j] = __float_as_uint(z2);
+          kb |= (z2 >= p.l2eps ? 1u : 0u) << j;
         }
-        if (p.nz_list && emit) {
+        const int nvc = min(32, max(0, valid - c * 32));  // valid columns in this 32-chunk
+        const uint32_t cm = (ok && dl != 0.f) ? (nvc == 32 ? 0xFFFFFFFFu : ((1u << nvc) - 1u)) : 0u;
+        kb &= cm;
+        const int tj = tcol - c * 32;
+        const uint32_t tb = (tj >= 0 && tj < 32) ? (cm & (1u << tj)) : 0u;
+        const uint32_t nzb = kb | tb;  // entries of G that are non-zero
+        if (slab) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            float g[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const float v = ((kb >> (j + u)) & 1u) ? ex2_approx(__uint_as_float(r[j + u])) : 0.f;
+              g[u] = dl * (v - (((tb >> (j + u)) & 1u) ? 1.f : 0.f));
+            }
+            packed[j >> 1] = pack_bf16(g[0], g[1]);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
+          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          dst[2] = make_uint4(packed[8], packed[9], packed[10], packed[11]);
+          dst[3] = make_uint4(packed[12], packed[13], packed[14], packed[15]);
+          // warp vote: which 16-column slices of this chunk hold any non-zero
+          const uint32_t b0 = __ballot_sync(0xffffffffu, (nzb & 0xFFFFu) != 0u);
+          const uint32_t b1 = __ballot_sync(0xffffffffu, (nzb >> 16) != 0u);
+          if (lane == 0 && (b0 | b1)) {
+            const int g = vt * (BN / 16) + c * 2;
+            atomicOr(&p.dh_mask[mb * p.dh_words + (g >> 5)],
+                     ((b0 ? 1u : 0u) | (b1 ? 2u : 0u)) << (g & 31));
+          }
+          half_nz |= nzb ? (1u << (c >> 2)) : 0u;
+        }
+        if (emit) {
           // warp-aggregated reservation of this chunk's non-zeros in the list
           const int cnt = __popc(nzb);
           int incl = cnt;
@@ -491,57 +535,37 @@ struct GPolicy {
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
                 if (!((nzb >> j) & 1u)) continue;
-                // the same arithmetic as above, so the same value
-                const int col = c * 32 + j;
-                const float pr = ex2_approx(fmaf(__uint_as_float(r[j]), kLog2e, -lse2));
-                float v = pr >= p.eps_keep ? pr : 0.f;
-                v -= (col == tcol) ? 1.f : 0.f;
+                const float v = ((kb >> j) & 1u) ? ex2_approx(__uint_as_float(r[j])) : 0.f;
+                const float g = dl * (v - (((tb >> j) & 1u) ? 1.f : 0.f));
                 if (pos < p.nz_cap) {
-                  p.nz_list[pos] = NzEntry{jrow, vt * BN + col, dl * v, 0};
-                  atomicAdd(&p.col_cnt[vt * BN + col], 1);
+                  p.nz_list[pos] = NzEntry{jrow, vt * BN + c * 32 + j, g, 0};
+                  atomicAdd(&p.col_cnt[vt * BN + c * 32 + j], 1);
                 }
                 ++pos;
               }
             }
           }
         }
-        uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
-        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-        dst[2] = make_uint4(packed[8], packed[9], packed[10], packed[11]);
-        dst[3] = make_uint4(packed[12], packed[13], packed[14], packed[15]);
-        // warp vote: which 16-column slices of this chunk hold any non-zero
-        const uint32_t b0 = __ballot_sync(0xffffffffu, nz[0]);
-        const uint32_t b1 = __ballot_sync(0xffffffffu, nz[1]);
-        if (lane == 0 && (b0 | b1)) {
-          const int g = vt * (BN / 16) + c * 2;
-          atomicOr(&p.dh_mask[mb * p.dh_words + (g >> 5)],
-                   ((b0 ? 1u : 0u) | (b1 ? 2u : 0u)) << (g & 31));
-        }
-        half_nz |= (nz[0] || nz[1]) ? (1u << (c >> 2)) : 0u;
-        if (dbg) {
+        if (dbg && kb) {
           const int orig = p.idx[jrow];
           for (int j = 0; j < 32; ++j) {
-            const int col = c * 32 + j;
-            if (col >= valid) break;
-            const float pr = ex2_approx(fmaf(__uint_as_float(r[j]), kLog2e, -lse2));
-            if (pr >= p.eps_keep) {
-              const int w = p.c0 + vt * BN + col;
-              const long long lid = p.seg_begin + (p.perm_seg ? p.perm_seg[w] : w);
-              atomicOr(&p.debug_keep[(size_t)orig * p.words_per_row + (lid >> 5)],
-                       1u << (lid & 31));
-            }
+            if (!((kb >> j) & 1u)) continue;
+            const int w = p.c0 + vt * BN + c * 32 + j;
+            const long long lid = p.seg_begin + (p.perm_seg ? p.perm_seg[w] : w);
+            atomicOr(&p.debug_keep[(size_t)orig * p.words_per_row + (lid >> 5)], 1u << (lid & 31));
           }
         }
       }
-      // warp vote per 16-row group for the dE contraction's K slices
+      if (slab) {
+        // warp vote per 16-row group for the dE contraction's K slices
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t b = __ballot_sync(0xffffffffu, (half_nz >> h) & 1u);
-        if (lane == 0 && b) {
-          const int g = mb * (BM / 16) + q * 2;
-          atomicOr(&p.de_mask[(vt * 2 + h) * p.de_words + (g >> 5)],
-                   (((b & 0xFFFFu) ? 1u : 0u) | ((b >> 16) ? 2u : 0u)) << (g & 31));
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t b = __ballot_sync(0xffffffffu, (half_nz >> h) & 1u);
+          if (lane == 0 && b) {
+            const int g = mb * (BM / 16) + q * 2;
+            atomicOr(&p.de_mask[(vt * 2 + h) * p.de_words + (g >> 5)],
+                     (((b & 0xFFFFu) ? 1u : 0u) | ((b >> 16) ? 2u : 0u)) << (g & 31));
+          }
         }
       }
       eng.epi_release(lane);
