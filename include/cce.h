@@ -218,10 +218,12 @@ int cce_fwd_noalloc(const void* H, const void* E, const int32_t* y,
  * class is bracketed by two CUDA events recorded on the stream the kernel is
  * launched on.  Classes: bit 0 forward tile stream, bit 1 backward G
  * producer, bit 2 backward dE contraction, bit 3 backward dH contraction,
- * bit 4 every other kernel.  cce_timing_read synchronises on the recorded
- * events, writes per class the summed milliseconds and the number of timed
- * launches (arrays of n_classes <= 5 entries, host memory), and clears the
- * record.  Not thread-safe.  Returns CCE_OK or CCE_EINVAL/CCE_ELAUNCH.
+ * bit 4 row compaction, gathers and finalize passes, bit 5 the sparse
+ * gradient kernels (list sorts, gathers, dH finalize).  cce_timing_read
+ * synchronises on the recorded events, writes per class the summed
+ * milliseconds and the number of timed launches (arrays of n_classes <= 6
+ * entries, host memory), and clears the record.  Not thread-safe.  Returns
+ * CCE_OK or CCE_EINVAL/CCE_ELAUNCH.
  */
 uint64_t cce_launch_count(void);
 int cce_timing_enable(uint32_t class_mask);

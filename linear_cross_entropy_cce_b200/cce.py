@@ -25,8 +25,9 @@ EXPORTS = ("cce_version", "cce_strerror", "cce_fwd_workspace_size", "cce_fwd",
            "cce_bwd_workspace_size", "cce_bwd", "cce_vocab_sort_workspace_size",
            "cce_vocab_sort", "cce_launch_count", "cce_timing_enable", "cce_timing_read")
 # kernel classes for cce_timing_enable / cce_timing_read
-KC_FWD, KC_G, KC_DE, KC_DH, KC_AUX = 0, 1, 2, 3, 4
-KC_NAMES = ("fwd_tile_stream", "bwd_g_producer", "bwd_dE_contraction", "bwd_dH_contraction", "aux")
+KC_FWD, KC_G, KC_DE, KC_DH, KC_AUX, KC_SPARSE = 0, 1, 2, 3, 4, 5
+KC_NAMES = ("fwd_tile_stream", "bwd_g_producer", "bwd_dE_contraction", "bwd_dH_contraction", "aux",
+            "bwd_sparse")
 
 
 class CCEError(RuntimeError):
@@ -235,10 +236,10 @@ def timing_enable(class_mask: int):
 
 def timing_read():
     """{class name: (summed ms, timed launches)}; clears the record."""
-    ms = (ctypes.c_float * 5)()
-    n = (ctypes.c_int64 * 5)()
-    _check(lib().cce_timing_read(ms, n, 5), "cce_timing_read")
-    return {KC_NAMES[i]: (float(ms[i]), int(n[i])) for i in range(5)}
+    ms = (ctypes.c_float * 6)()
+    n = (ctypes.c_int64 * 6)()
+    _check(lib().cce_timing_read(ms, n, 6), "cce_timing_read")
+    return {KC_NAMES[i]: (float(ms[i]), int(n[i])) for i in range(6)}
 
 
 def bf16_from_bits(bits, device) -> torch.Tensor:

@@ -217,7 +217,7 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V) {
 }
 
 // ---------------------------------------------------------- diagnostics
-enum KernelClass { KC_FWD = 0, KC_G = 1, KC_DE = 2, KC_DH = 3, KC_AUX = 4, KC_N = 5 };
+enum KernelClass { KC_FWD = 0, KC_G = 1, KC_DE = 2, KC_DH = 3, KC_AUX = 4, KC_SPARSE = 5, KC_N = 6 };
 
 std::atomic<uint64_t> g_launches{0};
 
@@ -265,6 +265,15 @@ int launch_tc(const typename Policy::Params& prm, int grid, cudaStream_t st, int
   return cudaGetLastError() == cudaSuccess ? CCE_OK : CCE_ELAUNCH;
 }
 
+// Brackets a plain kernel launch of class `cls` with timing events (when
+// that class is being timed); use as  { TimedLaunch t(cls, st); k<<<..>>>(); }
+struct TimedLaunch {
+  long slot;
+  cudaStream_t st;
+  TimedLaunch(int cls, cudaStream_t s) : slot(timing_begin(cls, s)), st(s) {}
+  ~TimedLaunch() { timing_end(slot, st); }
+};
+
 // Called right after every other kernel launch: counts it and checks it.
 int launched() {
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -279,10 +288,16 @@ T* at(void* ws, size_t off) {
 // Compaction + H_c gather shared by forward and backward.
 int run_compaction(const CompactParams& cp, const void* H, int64_t Npad, int64_t D, int sms,
                    __nv_bfloat16* Hc, cudaStream_t st) {
-  compact_kernel<<<1, COMPACT_THREADS, 0, st>>>(cp);
+  {
+    TimedLaunch tl_(KC_AUX, st);
+    compact_kernel<<<1, COMPACT_THREADS, 0, st>>>(cp);
+  }
   if (launched() != CCE_OK) return CCE_ELAUNCH;
-  gather_rows_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(H), cp.idx,
-                                              cp.n_valid, (int)Npad, (int)D, Hc);
+  {
+    TimedLaunch tl_(KC_AUX, st);
+    gather_rows_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(H), cp.idx,
+                                                cp.n_valid, (int)Npad, (int)D, Hc);
+  }
   return launched();
 }
 
@@ -411,7 +426,10 @@ int cce_fwd(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D
   fin.Npad = fp.Npad;
   fin.loss = loss;
   fin.lse = lse;
-  fwd_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, 8), sms * 8), 256, 0, st>>>(fin);
+  {
+    TimedLaunch tl_(KC_AUX, st);
+    fwd_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, 8), sms * 8), 256, 0, st>>>(fin);
+  }
   if (launched()) return CCE_ELAUNCH;
   if (colmax) {
     colmax_final_kernel<<<sms, 256, 0, st>>>(reinterpret_cast<int*>(colmax), (int)sg.live);
@@ -458,8 +476,11 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   if (vocab_perm) {
     for (int s = 0; s < sg.n; ++s) {
       const int n = table.s[s].n, off = table.s[s].live_off;
-      invert_perm_kernel<<<(int)std::min<int64_t>(cdiv(n, 256), sms * 8), 256, 0, st>>>(
-          vocab_perm + off, n, inv + off);
+      {
+        TimedLaunch tl_(KC_AUX, st);
+        invert_perm_kernel<<<(int)std::min<int64_t>(cdiv(n, 256), sms * 8), 256, 0, st>>>(
+            vocab_perm + off, n, inv + off);
+      }
       if (launched()) return CCE_ELAUNCH;
     }
   }
@@ -551,8 +572,11 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       const int cv = std::min(cw, ns - c0);
       int row0 = c0;
       if (perm_seg) {
-        gather_perm_rows_kernel<<<sms * 4, 256, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(sg.s[s].E), perm_seg + c0, cv, (int)D, Ec);
+        {
+          TimedLaunch tl_(KC_AUX, st);
+          gather_perm_rows_kernel<<<sms * 4, 256, 0, st>>>(
+              static_cast<const __nv_bfloat16*>(sg.s[s].E), perm_seg + c0, cv, (int)D, Ec);
+        }
         if (launched()) return CCE_ELAUNCH;
         if (!make_map(&segK, Ec, D, cv, D, BK, BN)) return CCE_ELAUNCH;
         if (!make_map(&segMN, Ec, D, cv, D, 64, 64)) return CCE_ELAUNCH;
@@ -605,11 +629,12 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       }
       // step 2: dE rows of this chunk (sparse gathers, or the dense contraction)
       if (sparse) {
-        sparse_col_scan_kernel<<<1, SCAN_THREADS, 0, st>>>(nz_cnt + chunk, cap, col_cnt, cv, col_ptr,
-                                                           col_cur);
-        if (launched()) return CCE_ELAUNCH;
-        sparse_col_scatter_kernel<<<sms * 2, 256, 0, st>>>(nz_cnt + chunk, cap,
-                                                          lists + (size_t)chunk * cap, col_cur, csorted);
+        {
+          TimedLaunch tl_(KC_SPARSE, st);
+          sparse_col_sort_kernel<<<1, SCAN_THREADS, 0, st>>>(nz_cnt + chunk, cap, col_cnt, cv, col_ptr,
+                                                             col_cur, lists + (size_t)chunk * cap,
+                                                             csorted);
+        }
         if (launched()) return CCE_ELAUNCH;
         SparseDEParams sp;
         sp.nz_cnt = nz_cnt + chunk;
@@ -625,7 +650,10 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
         sp.dE_comp = nullptr;
         sp.mode = fp32 ? 1 : 0;
         const int64_t warps = (int64_t)cv * cdiv(D, 256);
-        sparse_de_kernel<<<(int)std::min<int64_t>(sms * 16, cdiv(warps, 8)), 256, 0, st>>>(sp);
+        {
+          TimedLaunch tl_(KC_SPARSE, st);
+          sparse_de_kernel<<<(int)std::min<int64_t>(sms * 16, cdiv(warps, 8)), 256, 0, st>>>(sp);
+        }
         if (launched()) return CCE_ELAUNCH;
       }
       ep.nz_cnt = sparse ? nz_cnt + chunk : nullptr;
@@ -675,11 +703,20 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
     rp.row_cur = row_cur;
     rp.rsorted = rsorted;
     rp.cmap = cmap;
-    sparse_row_count_kernel<<<sms * 4, 256, 0, st>>>(rp);
+    {
+      TimedLaunch tl_(KC_SPARSE, st);
+      sparse_row_count_kernel<<<sms * 4, 256, 0, st>>>(rp);
+    }
     if (launched()) return CCE_ELAUNCH;
-    sparse_row_scan_kernel<<<1, SCAN_THREADS, 0, st>>>(row_cnt, (int)pl.Npad, row_ptr, row_cur);
+    {
+      TimedLaunch tl_(KC_SPARSE, st);
+      sparse_row_scan_kernel<<<1, SCAN_THREADS, 0, st>>>(row_cnt, (int)pl.Npad, row_ptr, row_cur);
+    }
     if (launched()) return CCE_ELAUNCH;
-    sparse_row_scatter_kernel<<<sms * 4, 256, 0, st>>>(rp);
+    {
+      TimedLaunch tl_(KC_SPARSE, st);
+      sparse_row_scatter_kernel<<<sms * 4, 256, 0, st>>>(rp);
+    }
     if (launched()) return CCE_ELAUNCH;
   }
   DHFinParams fp_;
@@ -693,7 +730,10 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   fp_.rsorted = rsorted;
   fp_.segs = table;
   fp_.vocab_perm = vocab_perm;
-  dh_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, 8), sms * 8), 256, 0, st>>>(fp_);
+  {
+    TimedLaunch tl_(KC_SPARSE, st);
+    dh_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, 8), sms * 8), 256, 0, st>>>(fp_);
+  }
   return launched();
 }
 

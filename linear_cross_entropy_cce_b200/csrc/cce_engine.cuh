@@ -322,6 +322,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
   Ctl* ctl = reinterpret_cast<Ctl*>(extra + Policy::EXTRA_SMEM);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (!Policy::active(p)) return;  // nothing to do in this launch: skip all set-up
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {

@@ -204,6 +204,7 @@ struct FwdParams {
 struct FwdPolicy {
   using Params = FwdParams;
   static constexpr int EXTRA_SMEM = 0;
+  static __device__ __forceinline__ bool active(const Params&) { return true; }
 
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
@@ -611,6 +612,10 @@ __device__ __forceinline__ bool mask_empty(const uint32_t* m, int nkb, int lane)
 struct DEPolicy {
   using Params = DEParams;
   static constexpr int EXTRA_SMEM = 0;
+  // a chunk taken by the sparse route has no dense work
+  static __device__ __forceinline__ bool active(const Params& p) {
+    return !(p.nz_cnt && *p.nz_cnt <= p.nz_cap);
+  }
 
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
@@ -725,6 +730,9 @@ struct DHParams {
 
 struct DHPolicy {
   using Params = DHParams;
+  static __device__ __forceinline__ bool active(const Params& p) {
+    return !(p.nz_cnt && *p.nz_cnt <= p.nz_cap);
+  }
   // per epilogue warp: two 32 x 32 fp32 staging tiles for the TMA reduce-add
   static constexpr int EXTRA_SMEM = 4 * 2 * 4096;
 
@@ -819,28 +827,30 @@ __global__ void dh_finalize_kernel(const DHFinParams p) {
     const float fill = j == -1 ? 0.f : __int_as_float(0x7fc00000);
     const int e0 = (j >= 0 && p.row_ptr) ? p.row_ptr[j] : 0;
     const int e1 = (j >= 0 && p.row_ptr) ? p.row_ptr[j + 1] : 0;
-    for (int d0 = lane * 8; d0 < p.D; d0 += 256) {
-      float a[8];
+    for (int d0base = 0; d0base < p.D; d0base += 256) {
+      const int d0 = d0base + lane * 8;
+      float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // sparse chunks: g * e_j for the row's entries, staged 32 at a time in
+      // the lanes (E row pointer, g) and gathered 4 deep
+      for (int eb = e0; eb < e1; eb += 32) {
+        const int n = min(32, e1 - eb);
+        const __nv_bfloat16* myrow = p.segs.s[0].E;
+        float myg = 0.f;
+        if (lane < n) {
+          const int2 t = p.rsorted[eb + lane];
+          const int s = (int)((unsigned)t.x >> 29), w = t.x & ((1 << 29) - 1);
+          const int loc = p.vocab_perm ? p.vocab_perm[p.segs.s[s].live_off + w] : w;
+          myrow = p.segs.s[s].E + (size_t)loc * p.D;
+          myg = __int_as_float(t.y);
+        }
+        gather_rows_fma(a, myrow, myg, n, d0 < p.D ? d0 : 0);
+      }
+      if (d0 >= p.D) continue;
       if (j >= 0) {
         const float4* src = reinterpret_cast<const float4*>(p.dH_acc + (size_t)j * p.D + d0);
         const float4 u = src[0], v = src[1];
-        a[0] = u.x; a[1] = u.y; a[2] = u.z; a[3] = u.w;
-        a[4] = v.x; a[5] = v.y; a[6] = v.z; a[7] = v.w;
-        for (int e = e0; e < e1; ++e) {
-          const int2 t = p.rsorted[e];
-          const float g = __int_as_float(t.y);
-          const int s = (int)((unsigned)t.x >> 29), w = t.x & ((1 << 29) - 1);
-          const int loc = p.vocab_perm ? p.vocab_perm[p.segs.s[s].live_off + w] : w;
-          const uint4 h = __ldg(reinterpret_cast<const uint4*>(p.segs.s[s].E + (size_t)loc * p.D + d0));
-          a[0] = fmaf(g, bf16lo(h.x), a[0]);
-          a[1] = fmaf(g, bf16hi(h.x), a[1]);
-          a[2] = fmaf(g, bf16lo(h.y), a[2]);
-          a[3] = fmaf(g, bf16hi(h.y), a[3]);
-          a[4] = fmaf(g, bf16lo(h.z), a[4]);
-          a[5] = fmaf(g, bf16hi(h.z), a[5]);
-          a[6] = fmaf(g, bf16lo(h.w), a[6]);
-          a[7] = fmaf(g, bf16hi(h.w), a[7]);
-        }
+        a[0] += u.x; a[1] += u.y; a[2] += u.z; a[3] += u.w;
+        a[4] += v.x; a[5] += v.y; a[6] += v.z; a[7] += v.w;
       } else {
         for (int k = 0; k < 8; ++k) a[k] = fill;
       }
