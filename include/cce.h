@@ -59,6 +59,7 @@ extern "C" {
 /* cce_bwd flags. */
 #define CCE_KAHAN_DE 1u   /* dE += grad with a bf16 Kahan compensation buffer  */
 #define CCE_FP32_GRADS 2u /* dH and dE are written as fp32 instead of bf16     */
+#define CCE_FULL_DE 4u    /* filter only dH; the classifier gradient dE is full */
 
 #define CCE_MAX_SEGMENTS 8
 
@@ -139,7 +140,13 @@ size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs,
  *            backward walks the vocabulary in that order so that surviving
  *            blocks cluster; results do not depend on it beyond rounding.
  *            NULL = identity.
- *   flags    CCE_KAHAN_DE | CCE_FP32_GRADS.
+ *   flags    CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE.  CCE_FULL_DE keeps
+ *            the classifier gradient dE unfiltered while dH uses the filtered
+ *            softmax (the "FullC" variant of "Cut Your Losses in
+ *            Large-Vocabulary Language Models", research-map entry, §Key
+ *            results / §Limitations); vocabulary chunks too dense for the
+ *            sparse dH route then contribute their full (unfiltered)
+ *            gradient to dH as well.
  *   dH       [N, D] output (bf16, or fp32 with CCE_FP32_GRADS).
  *   dE       [V, D] output when segs == NULL (else per-segment dE).  Written
  *            (overwritten) unless CCE_KAHAN_DE, in which case the new

@@ -1,0 +1,84 @@
+"""torch.autograd drop-in over libcce: the role of the pip package's loss
+function ("The loss and the mask ...", part "Cut Your Losses in
+Large-Vocabulary Language Models (CCE)": code on PyPI as a drop-in loss).
+
+    loss = linear_cross_entropy(H, E, y)                 # mean over valid rows
+    loss.backward()                                      # dH, dE via cce_bwd
+
+The forward runs cce_fwd and keeps lse; the backward turns the upstream
+gradient of the reduction into the per-row dloss and runs cce_bwd.  The
+reduction over rows (mean / sum) is a single torch reduction of the per-row
+losses; every other step runs in libcce's kernels.
+"""
+from __future__ import annotations
+
+from typing import Optional, Sequence
+
+import torch
+
+from . import cce
+
+
+class _LinearCrossEntropy(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, H, E, y, ignore_index, filter_eps, full_de, vocab_sort, segments_meta, *seg_E):
+        segments = [(b, e, t) for (b, e), t in zip(segments_meta, seg_E)] if segments_meta else None
+        V = segments_meta[-1][1] if segments_meta else None
+        if vocab_sort:
+            loss, lse, colmax = cce.fwd(H, E, y, ignore_index, segments=segments, V=V,
+                                        want_colmax=True)
+            perm = cce.vocab_sort(colmax, y, V if segments else E.shape[0], ignore_index,
+                                  segments=segments)
+        else:
+            loss, lse = cce.fwd(H, E, y, ignore_index, segments=segments, V=V)
+            perm = None
+        ctx.save_for_backward(H, E if E is not None else torch.empty(0), y, lse,
+                              perm if perm is not None else torch.empty(0), *seg_E)
+        ctx.meta = (ignore_index, filter_eps, full_de, segments_meta, E is not None, perm is not None)
+        return loss
+
+    @staticmethod
+    def backward(ctx, grad_loss):
+        H, E, y, lse, perm, *seg_E = ctx.saved_tensors
+        ignore_index, filter_eps, full_de, segments_meta, has_E, has_perm = ctx.meta
+        segments = [(b, e, t) for (b, e), t in zip(segments_meta, seg_E)] if segments_meta else None
+        V = segments_meta[-1][1] if segments_meta else None
+        dloss = grad_loss.contiguous().to(torch.float32)
+        dH, dE, _ = cce.bwd(H, E if has_E else None, y, lse, dloss, ignore_index, segments=segments,
+                            V=V, filter_eps=filter_eps, vocab_perm=perm if has_perm else None,
+                            full_de=full_de)
+        dH = dH.to(H.dtype)
+        if segments:
+            return (dH, None, None, None, None, None, None, None, *[g.to(t.dtype) for g, t in zip(dE, seg_E)])
+        return (dH, dE.to(E.dtype), None, None, None, None, None, None)
+
+
+def linear_cross_entropy(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor,
+                         ignore_index: int = -100, reduction: str = "mean",
+                         filter_eps: float = 2.0 ** -12, full_de: bool = False,
+                         vocab_sort: bool = False,
+                         segments: Optional[Sequence] = None) -> torch.Tensor:
+    """Cross-entropy of the logits H @ E^T (never materialised) against y.
+
+    H [N, D] bf16, E [V, D] bf16 (or `segments` = [(begin, end, E_s), ...] for
+    a composite head with dead gaps), y [N] int32 (int64 is converted).
+    reduction: "mean" over rows whose target is not ignore_index, "sum", or
+    "none" (per-row losses, ignored rows 0).  filter_eps <= 0 disables the
+    gradient filter; full_de keeps the classifier gradient unfiltered;
+    vocab_sort walks the vocabulary in descending max-logit order in the
+    backward.
+    """
+    if y.dtype != torch.int32:
+        y = y.to(torch.int32)
+    meta = tuple((int(b), int(e)) for b, e, _ in segments) if segments else ()
+    seg_E = tuple(t for _, _, t in segments) if segments else ()
+    per_row = _LinearCrossEntropy.apply(H, E, y, ignore_index, float(filter_eps), bool(full_de),
+                                        bool(vocab_sort), meta, *seg_E)
+    if reduction == "none":
+        return per_row
+    if reduction == "sum":
+        return per_row.sum()
+    if reduction == "mean":
+        n_valid = (y != ignore_index).sum()
+        return per_row.sum() / n_valid
+    raise ValueError(f"unknown reduction {reduction!r}")

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libcce.so")
 
 CCE_OK, CCE_EINVAL, CCE_EWORKSPACE, CCE_ELAUNCH, CCE_EDEVICE = 0, 1, 2, 3, 4
 STATUS_BADTARGET, STATUS_TIMEOUT = 1, 2
-KAHAN_DE, FP32_GRADS = 1, 2
+KAHAN_DE, FP32_GRADS, FULL_DE = 1, 2, 4
 MAX_SEGMENTS = 8
 
 EXPORTS = ("cce_version", "cce_strerror", "cce_fwd_workspace_size", "cce_fwd",
@@ -166,7 +166,7 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
         dloss: torch.Tensor, ignore_index: int = -100,
         segments: Optional[Sequence[SegSpec]] = None, V: Optional[int] = None,
         filter_eps: float = 0.0, vocab_perm: Optional[torch.Tensor] = None,
-        kahan: bool = False, fp32_grads: bool = False,
+        kahan: bool = False, fp32_grads: bool = False, full_de: bool = False,
         dE_out=None, dE_comp=None, debug_rows: int = 0,
         workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
     """Gradients (dH, dE) of sum_i dloss_i loss_i.  See cce_bwd.
@@ -195,7 +195,7 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
     if kahan:
         comps = list(dE_comp) if isinstance(dE_comp, (list, tuple)) else [dE_comp]
     dH = torch.empty((N, D), dtype=gdt, device=dev)
-    flags = (KAHAN_DE if kahan else 0) | (FP32_GRADS if fp32_grads else 0)
+    flags = (KAHAN_DE if kahan else 0) | (FP32_GRADS if fp32_grads else 0) | (FULL_DE if full_de else 0)
     words = (V + 31) // 32
     dbg = torch.empty((debug_rows, words), dtype=torch.int32, device=dev) if debug_rows > 0 else None
     segarr, nseg = _seg_array(segments, dEs if segments else None, comps if segments else None)

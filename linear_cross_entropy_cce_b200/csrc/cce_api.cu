@@ -444,7 +444,8 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
             void* dE, void* dE_comp, uint32_t* debug_keep, int64_t debug_rows, void* workspace,
             size_t workspace_bytes, int32_t* status, void* stream) {
   if (!sizes_ok(N, D, V)) return CCE_EINVAL;
-  if (flags & ~(CCE_KAHAN_DE | CCE_FP32_GRADS)) return CCE_EINVAL;
+  if (flags & ~(CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE)) return CCE_EINVAL;
+  const bool full_de = flags & CCE_FULL_DE;
   const bool kahan = flags & CCE_KAHAN_DE;
   const bool fp32 = flags & CCE_FP32_GRADS;
   if (kahan && fp32) return CCE_EINVAL;
@@ -521,8 +522,11 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   const float eps_keep = filter_eps > 0.f ? filter_eps * (1.0f - 1.0f / 256.0f) : 0.f;
   // Sparse contractions for filtered gradients (chunks with at most `cap`
   // non-zeros; the Kahan path stays on the deterministic dense route).
+  // dH may take the sparse route whenever filtering is on; dE only when it is
+  // filtered too (not CCE_FULL_DE).
   bool sparse = filter_eps > 0.f && !kahan;
   for (int s = 0; s < sg.n; ++s) sparse = sparse && table.s[s].n < (1 << 29);
+  const bool sparse_de = sparse && !full_de;
   const int cap = (int)pl.cap;
   int* nz_cnt = at<int>(workspace, pl.off_nzcnt);
   NzEntry* lists = at<NzEntry>(workspace, pl.off_lists);
@@ -618,17 +622,19 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       gp.prev_nz_cnt = chunk > 0 ? nz_cnt + chunk - 1 : nullptr;
       gp.slab_flag = slab_flag + chunk;
       gp.repair = 0;
+      gp.always_slab = full_de ? 1 : 0;
+      gp.slab_unfiltered = full_de ? 1 : 0;
       if (sparse && cudaMemsetAsync(col_cnt, 0, sizeof(int) * (size_t)cv, st) != cudaSuccess)
         return CCE_ELAUNCH;
       if (int rc = launch_tc<GPolicy>(gp, (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct), st, KC_G))
         return rc;
-      if (sparse) {  // recompute with the dense fallback if the chunk was mispredicted
+      if (sparse && !full_de) {  // recompute with the dense fallback if the chunk was mispredicted
         gp.repair = 1;
         if (int rc = launch_tc<GPolicy>(gp, (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct), st, KC_G))
           return rc;
       }
       // step 2: dE rows of this chunk (sparse gathers, or the dense contraction)
-      if (sparse) {
+      if (sparse_de) {
         {
           TimedLaunch tl_(KC_SPARSE, st);
           sparse_col_sort_kernel<<<1, SCAN_THREADS, 0, st>>>(nz_cnt + chunk, cap, col_cnt, cv, col_ptr,
@@ -656,7 +662,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
         }
         if (launched()) return CCE_ELAUNCH;
       }
-      ep.nz_cnt = sparse ? nz_cnt + chunk : nullptr;
+      ep.nz_cnt = sparse_de ? nz_cnt + chunk : nullptr;
       ep.nz_cap = cap;
       ep.chunk_valid = cv;
       ep.mt = (int)cdiv(cv, BM);

@@ -407,6 +407,8 @@ struct GParams {
   const int* prev_nz_cnt;  // previous chunk's count, or null
   int* slab_flag;          // set when this chunk's slab has been written
   int repair;
+  int always_slab;      // write the slab for every chunk (dE always dense)
+  int slab_unfiltered;  // the slab holds the unfiltered G (full classifier gradient)
   // optional per-element keep bits of original rows < debug_rows
   uint32_t* debug_keep;
   int debug_rows;
@@ -424,7 +426,7 @@ struct GPolicy {
   // Whether this launch writes the dense fallback (slab + masks), and
   // whether it runs at all (a repair launch usually has nothing to do).
   static __device__ __forceinline__ bool writes_slab(const Params& p) {
-    if (!p.nz_list || p.repair) return true;
+    if (!p.nz_list || p.repair || p.always_slab) return true;
     return p.prev_nz_cnt == nullptr || *p.prev_nz_cnt > p.nz_cap;
   }
   static __device__ __forceinline__ bool active(const Params& p) {
@@ -490,13 +492,15 @@ struct GPolicy {
         const uint32_t tb = (tj >= 0 && tj < 32) ? (cm & (1u << tj)) : 0u;
         const uint32_t nzb = kb | tb;  // entries of G that are non-zero
         if (slab) {
+          const uint32_t ks = p.slab_unfiltered ? cm : kb;  // softmax entries the slab keeps
+          const uint32_t nzs = ks | tb;
           uint32_t packed[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
             float g[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-              const float v = ((kb >> (j + u)) & 1u) ? ex2_approx(__uint_as_float(r[j + u])) : 0.f;
+              const float v = ((ks >> (j + u)) & 1u) ? ex2_approx(__uint_as_float(r[j + u])) : 0.f;
               g[u] = dl * (v - (((tb >> (j + u)) & 1u) ? 1.f : 0.f));
             }
             packed[j >> 1] = pack_bf16(g[0], g[1]);
@@ -507,14 +511,14 @@ struct GPolicy {
           dst[2] = make_uint4(packed[8], packed[9], packed[10], packed[11]);
           dst[3] = make_uint4(packed[12], packed[13], packed[14], packed[15]);
           // warp vote: which 16-column slices of this chunk hold any non-zero
-          const uint32_t b0 = __ballot_sync(0xffffffffu, (nzb & 0xFFFFu) != 0u);
-          const uint32_t b1 = __ballot_sync(0xffffffffu, (nzb >> 16) != 0u);
+          const uint32_t b0 = __ballot_sync(0xffffffffu, (nzs & 0xFFFFu) != 0u);
+          const uint32_t b1 = __ballot_sync(0xffffffffu, (nzs >> 16) != 0u);
           if (lane == 0 && (b0 | b1)) {
             const int g = vt * (BN / 16) + c * 2;
             atomicOr(&p.dh_mask[mb * p.dh_words + (g >> 5)],
                      ((b0 ? 1u : 0u) | (b1 ? 2u : 0u)) << (g & 31));
           }
-          half_nz |= nzb ? (1u << (c >> 2)) : 0u;
+          half_nz |= nzs ? (1u << (c >> 2)) : 0u;
         }
         if (emit) {
           // warp-aggregated reservation of this chunk's non-zeros in the list

@@ -150,13 +150,15 @@ def dlogits(Z: np.ndarray, lse: np.ndarray, y_rows: np.ndarray,
 
 
 def backward(H, segments, y, V: int, dloss, ignore_index: int = -100,
-             filter_eps: float = 0.0, slice_rows: int = SLICE_ROWS):
+             filter_eps: float = 0.0, slice_rows: int = SLICE_ROWS, filter_dE: bool = True):
     """Exact gradients of sum_i dloss_i * loss_i w.r.t. H and each E segment.
 
     Returns (dH[N, D] fp64, [dE_s[n_s, D] fp64 per segment]).  Ignored rows
     get a zero dH row and contribute nothing to dE.  [LM] §Contribution,
     [MAP] §Approach (the method recomputes these blockwise; the oracle just
-    forms them slice by slice).
+    forms them slice by slice).  filter_dE=False keeps the classifier
+    gradient unfiltered while dH is filtered: the "FullC" variant of [MAP]
+    §Key results / §Limitations (full classifier gradient).
     """
     segs64 = _segments_f64(segments)
     y = np.asarray(y, dtype=np.int64)
@@ -173,12 +175,13 @@ def backward(H, segments, y, V: int, dloss, ignore_index: int = -100,
         r = r[g]
         H64 = as_f64(H[r])
         Z = logits_rows(H64, segs64, V)
-        G = dlogits(Z, logsumexp_rows(Z), y[r], dloss[r], filter_eps)
+        lse = logsumexp_rows(Z)
+        G = dlogits(Z, lse, y[r], dloss[r], filter_eps)
+        GE = G if filter_dE else dlogits(Z, lse, y[r], dloss[r], 0.0)
         acc = np.zeros((r.shape[0], D))
         for k, (begin, end, E64) in enumerate(segs64):
-            Gs = G[:, begin:end]
-            acc += Gs @ E64
-            dE[k] += Gs.T @ H64
+            acc += G[:, begin:end] @ E64
+            dE[k] += GE[:, begin:end].T @ H64
         dH[r] = acc
     dH[bad] = np.nan
     return dH, dE

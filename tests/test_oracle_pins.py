@@ -303,3 +303,17 @@ def test_dE_columns_match_backward():
     got = oracle.dE_columns(x.H, x.segments, x.y, 50, dl, cols, IGN, filter_eps=1e-3, slice_rows=9)
     ref = np.stack([dE[0][0], dE[0][19], dE[1][0], dE[1][23]])
     assert np.allclose(got, ref, rtol=1e-12, atol=1e-16)
+
+
+def test_full_classifier_gradient_variant():
+    """filter_dE=False ("FullC"): dE equals the unfiltered dE, dH the filtered
+    dH; and the filter does change both on this peaky case (so the variant is
+    not vacuous)."""
+    x = _small(N=40, D=16, V=200, std=10.0, ignore=0.1)
+    dl = x.dloss_mean()
+    eps = 2.0 ** -12
+    fH, fE = oracle.backward(x.H, x.segments, x.y, 200, dl, IGN, filter_eps=eps)
+    uH, uE = oracle.backward(x.H, x.segments, x.y, 200, dl, IGN)
+    cH, cE = oracle.backward(x.H, x.segments, x.y, 200, dl, IGN, filter_eps=eps, filter_dE=False)
+    assert np.array_equal(cH, fH) and np.array_equal(cE[0], uE[0])
+    assert not np.allclose(fE[0], uE[0], rtol=1e-9, atol=0) and not np.allclose(fH, uH, rtol=1e-9, atol=0)
