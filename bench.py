@@ -163,6 +163,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------- multi-rank
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest `value` over all ranks (one all-reduce of one float); the
+    value itself when there is a single rank."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def tokens_per_s(tokens_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (ms / 1e3)
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -258,12 +276,7 @@ def main():
         e1.record(s)
         torch.cuda.synchronize(dev)
         barrier()
-        ms = e0.elapsed_time(e1) / k
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(e0.elapsed_time(e1) / k, world, dev)
 
     for _ in range(a.warmup):
         step()
@@ -321,7 +334,7 @@ def main():
             e2e_step()
         ms_e2e = timed(e2e_step, a.steps)
         h2d = hH.numel() * 2 + sum(h.numel() * 2 for h in hE) + hy.numel() * 4
-        e2e = {"value": round(N * world / (ms_e2e / 1e3), 1), "unit": UNIT,
+        e2e = {"value": round(tokens_per_s(N, world, ms_e2e), 1), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(N * 4),
                "ms_per_step": round(ms_e2e, 3)}
 
@@ -353,7 +366,7 @@ def main():
                "sample": desc, "seconds": round(t, 2)}
 
     out = {
-        "metric": METRIC, "value": round(N * world / (ms_step / 1e3), 1), "unit": UNIT,
+        "metric": METRIC, "value": round(tokens_per_s(N, world, ms_step), 1), "unit": UNIT,
         "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_step, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; shapes and value recipe of the workload; no dataset or trained weights)",
