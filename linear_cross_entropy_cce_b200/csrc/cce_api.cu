@@ -165,7 +165,7 @@ FwdPlan plan_fwd(int64_t N, int64_t D, int64_t V, int32_t n_segs) {
 struct BwdPlan {
   int64_t Npad, Vc;
   size_t off_nvalid, off_idx, off_pos, off_lse2, off_dl, off_tseg, off_tpos, off_inv, off_hc,
-      off_dh, off_g, off_ec, off_masks, total;
+      off_dh, off_g, off_ec, off_gfull, off_masks, total;
   int dh_words, de_words;
   size_t mask_bytes;
   // sparse backward (filtered gradients)
@@ -173,7 +173,7 @@ struct BwdPlan {
   size_t off_nzcnt, off_lists, off_colc, off_csorted, off_rowc, off_rsorted;
 };
 
-BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V) {
+BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags) {
   BwdPlan p;
   p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
   // Vocabulary chunk width: an L2-sized slab, widened so that the dE
@@ -199,6 +199,8 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V) {
   p.off_dh = o; o += align_up((size_t)p.Npad * D * 4);
   p.off_g = o; o += align_up((size_t)p.Npad * p.Vc * 2);
   p.off_ec = o; o += align_up((size_t)p.Vc * D * 2);
+  // CCE_FULL_DE: a second slab with the unfiltered G, read by dE only
+  p.off_gfull = o; o += (flags & CCE_FULL_DE) ? align_up((size_t)p.Npad * p.Vc * 2) : 0;
   p.dh_words = (int)cdiv(p.Vc, 512);
   p.de_words = (int)cdiv(p.Npad, 512);
   p.mask_bytes = sizeof(uint32_t) * ((size_t)(p.Npad / BM) * p.dh_words + (size_t)(p.Vc / BM) * p.de_words);
@@ -357,9 +359,8 @@ size_t cce_fwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs) {
 }
 
 size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs, uint32_t flags) {
-  (void)flags;
   if (!sizes_ok(N, D, V) || n_segs < 0 || n_segs > CCE_MAX_SEGMENTS) return 0;
-  return plan_bwd(N, D, V).total;
+  return plan_bwd(N, D, V, flags).total;
 }
 
 int cce_fwd(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D, int64_t V,
@@ -465,7 +466,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   if (N == 0) return CCE_OK;
   if (!H || !y || !lse || !dloss || !dH || !status || !aligned16(H) || !aligned16(dH))
     return CCE_EINVAL;
-  const BwdPlan pl = plan_bwd(N, D, V);
+  const BwdPlan pl = plan_bwd(N, D, V, flags);
   if (!workspace || workspace_bytes < pl.total) return CCE_EWORKSPACE;
   const int sms = device_sms();
   if (sms <= 0 || !encode_fn()) return CCE_EDEVICE;
@@ -512,6 +513,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
     return CCE_ELAUNCH;
 
   __nv_bfloat16* G = at<__nv_bfloat16>(workspace, pl.off_g);
+  __nv_bfloat16* G_full = full_de ? at<__nv_bfloat16>(workspace, pl.off_gfull) : nullptr;
   uint32_t* dh_mask = at<uint32_t>(workspace, pl.off_masks);
   uint32_t* de_mask = dh_mask + (size_t)(pl.Npad / BM) * pl.dh_words;
   __nv_bfloat16* Ec = at<__nv_bfloat16>(workspace, pl.off_ec);
@@ -553,7 +555,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   memset(&ep, 0, sizeof(ep));
   memset(&hp, 0, sizeof(hp));
   if (!make_map(&gp.mapA, Hc, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
-  if (!make_map(&ep.mapA, G, Vc, pl.Npad, Vc, 64, 64)) return CCE_ELAUNCH;
+  if (!make_map(&ep.mapA, full_de ? G_full : G, Vc, pl.Npad, Vc, 64, 64)) return CCE_ELAUNCH;
   if (!make_map(&ep.mapB, Hc, D, pl.Npad, D, 64, 64)) return CCE_ELAUNCH;
   if (!make_map(&hp.mapA, G, Vc, pl.Npad, Vc, BK, BM)) return CCE_ELAUNCH;
   if (!make_map_t(&hp.mapC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dH_acc, D, pl.Npad, D, 32, 32))
@@ -622,15 +624,17 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       gp.prev_nz_cnt = chunk > 0 ? nz_cnt + chunk - 1 : nullptr;
       gp.slab_flag = slab_flag + chunk;
       gp.repair = 0;
-      gp.always_slab = full_de ? 1 : 0;
-      gp.slab_unfiltered = full_de ? 1 : 0;
+      gp.G_full = G_full;
       if (sparse && cudaMemsetAsync(col_cnt, 0, sizeof(int) * (size_t)cv, st) != cudaSuccess)
         return CCE_ELAUNCH;
-      if (int rc = launch_tc<GPolicy>(gp, (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct), st, KC_G))
+      const int g_grid = (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct);
+      if (int rc = full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
+                           : launch_tc<GPolicy>(gp, g_grid, st, KC_G))
         return rc;
-      if (sparse && !full_de) {  // recompute with the dense fallback if the chunk was mispredicted
+      if (sparse) {  // recompute with the dense fallback if the chunk was mispredicted
         gp.repair = 1;
-        if (int rc = launch_tc<GPolicy>(gp, (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct), st, KC_G))
+        if (int rc = full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
+                             : launch_tc<GPolicy>(gp, g_grid, st, KC_G))
           return rc;
       }
       // step 2: dE rows of this chunk (sparse gathers, or the dense contraction)

@@ -407,8 +407,12 @@ struct GParams {
   const int* prev_nz_cnt;  // previous chunk's count, or null
   int* slab_flag;          // set when this chunk's slab has been written
   int repair;
-  int always_slab;      // write the slab for every chunk (dE always dense)
-  int slab_unfiltered;  // the slab holds the unfiltered G (full classifier gradient)
+  // Full classifier gradient (CCE_FULL_DE, GPolicyT<true> only): the
+  // unfiltered G of every chunk goes to G_full, which only the dE
+  // contraction reads, and de_mask follows G_full; G keeps the filtered
+  // values that dH reads.  Written by the first launch of a chunk, not by
+  // its repair.
+  __nv_bfloat16* G_full;
   // optional per-element keep bits of original rows < debug_rows
   uint32_t* debug_keep;
   int debug_rows;
@@ -419,14 +423,15 @@ struct GParams {
   int* status;
 };
 
-struct GPolicy {
+template <bool FULL>
+struct GPolicyT {
   using Params = GParams;
   static constexpr int EXTRA_SMEM = 0;
 
   // Whether this launch writes the dense fallback (slab + masks), and
   // whether it runs at all (a repair launch usually has nothing to do).
   static __device__ __forceinline__ bool writes_slab(const Params& p) {
-    if (!p.nz_list || p.repair || p.always_slab) return true;
+    if (!p.nz_list || p.repair) return true;
     return p.prev_nz_cnt == nullptr || *p.prev_nz_cnt > p.nz_cap;
   }
   static __device__ __forceinline__ bool active(const Params& p) {
@@ -458,6 +463,8 @@ struct GPolicy {
   static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
     const int row = q * 32 + lane;
     const bool slab = writes_slab(p);
+    const bool full = FULL && !p.repair;        // this launch writes G_full
+    const bool de_bits = FULL ? full : slab;    // ... and the dE contraction's masks
     bool emit = p.nz_list != nullptr && !p.repair;  // this warp still lists non-zeros
     if (slab && p.slab_flag && !p.repair && blockIdx.x == 0 && threadIdx.x == 64)
       *p.slab_flag = 1;
@@ -471,6 +478,7 @@ struct GPolicy {
       const int tcol = (ok && p.tseg[jrow] == p.seg) ? p.tpos[jrow] - p.c0 - vt * BN : -1;
       const int valid = p.chunk_valid - vt * BN;  // valid columns of this tile
       __nv_bfloat16* grow = p.G + (size_t)jrow * p.Vc + vt * BN;
+      __nv_bfloat16* frow = FULL ? p.G_full + (size_t)jrow * p.Vc + vt * BN : nullptr;
       const bool dbg = p.debug_keep != nullptr && ok && p.idx[jrow] < p.debug_rows;
       uint32_t half_nz = 0;  // bit h: this row has a non-zero in tile columns 128h..128h+127
       for (int c = 0; c < BN / 32; ++c) {
@@ -491,34 +499,48 @@ struct GPolicy {
         const int tj = tcol - c * 32;
         const uint32_t tb = (tj >= 0 && tj < 32) ? (cm & (1u << tj)) : 0u;
         const uint32_t nzb = kb | tb;  // entries of G that are non-zero
-        if (slab) {
-          const uint32_t ks = p.slab_unfiltered ? cm : kb;  // softmax entries the slab keeps
-          const uint32_t nzs = ks | tb;
-          uint32_t packed[16];
+        if (slab || full) {
+          // softmax entries evaluated: the kept ones, or all valid ones for G_full
+          const uint32_t ks = full ? cm : kb;
+          uint32_t pk[16], pf[FULL ? 16 : 1];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            float g[2];
+            float gk[2], gf[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
+              const float t = ((tb >> (j + u)) & 1u) ? 1.f : 0.f;
               const float v = ((ks >> (j + u)) & 1u) ? ex2_approx(__uint_as_float(r[j + u])) : 0.f;
-              g[u] = dl * (v - (((tb >> (j + u)) & 1u) ? 1.f : 0.f));
+              gf[u] = dl * (v - t);
+              gk[u] = ((kb >> (j + u)) & 1u) ? gf[u] : (t != 0.f ? -dl : 0.f);
             }
-            packed[j >> 1] = pack_bf16(g[0], g[1]);
+            pk[j >> 1] = pack_bf16(gk[0], gk[1]);
+            if constexpr (FULL) pf[j >> 1] = pack_bf16(gf[0], gf[1]);
           }
-          uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
-          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-          dst[2] = make_uint4(packed[8], packed[9], packed[10], packed[11]);
-          dst[3] = make_uint4(packed[12], packed[13], packed[14], packed[15]);
-          // warp vote: which 16-column slices of this chunk hold any non-zero
-          const uint32_t b0 = __ballot_sync(0xffffffffu, (nzs & 0xFFFFu) != 0u);
-          const uint32_t b1 = __ballot_sync(0xffffffffu, (nzs >> 16) != 0u);
-          if (lane == 0 && (b0 | b1)) {
-            const int g = vt * (BN / 16) + c * 2;
-            atomicOr(&p.dh_mask[mb * p.dh_words + (g >> 5)],
-                     ((b0 ? 1u : 0u) | (b1 ? 2u : 0u)) << (g & 31));
+          if (slab) {
+            uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+            dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+            // warp vote: which 16-column slices of this chunk hold any non-zero
+            const uint32_t b0 = __ballot_sync(0xffffffffu, (nzb & 0xFFFFu) != 0u);
+            const uint32_t b1 = __ballot_sync(0xffffffffu, (nzb >> 16) != 0u);
+            if (lane == 0 && (b0 | b1)) {
+              const int g = vt * (BN / 16) + c * 2;
+              atomicOr(&p.dh_mask[mb * p.dh_words + (g >> 5)],
+                       ((b0 ? 1u : 0u) | (b1 ? 2u : 0u)) << (g & 31));
+            }
           }
-          half_nz |= nzs ? (1u << (c >> 2)) : 0u;
+          if constexpr (FULL) {
+            if (full) {
+              uint4* dst = reinterpret_cast<uint4*>(frow + c * 32);
+              dst[0] = make_uint4(pf[0], pf[1], pf[2], pf[3]);
+              dst[1] = make_uint4(pf[4], pf[5], pf[6], pf[7]);
+              dst[2] = make_uint4(pf[8], pf[9], pf[10], pf[11]);
+              dst[3] = make_uint4(pf[12], pf[13], pf[14], pf[15]);
+            }
+          }
+          half_nz |= (de_bits && (full ? (cm | tb) : nzb)) ? (1u << (c >> 2)) : 0u;
         }
         if (emit) {
           // warp-aggregated reservation of this chunk's non-zeros in the list
@@ -561,7 +583,7 @@ struct GPolicy {
           }
         }
       }
-      if (slab) {
+      if (de_bits) {
         // warp vote per 16-row group for the dE contraction's K slices
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -578,6 +600,9 @@ struct GPolicy {
     });
   }
 };
+
+using GPolicy = GPolicyT<false>;
+using GPolicyFull = GPolicyT<true>;
 
 // =====================================================================
 // Backward, step 2: dE_chunk = G^T H_c, K = compact rows, accumulated on

@@ -43,6 +43,10 @@ def test_workspace_sizes_and_invalid_sizes():
     assert L.cce_fwd_workspace_size(256, 256, 0, 0) == 0
     assert L.cce_fwd_workspace_size(256, 256, 4096, 9) == 0      # too many segments
     assert L.cce_bwd_workspace_size(256, 256, 4096, 0, 0) > 0
+    # CCE_FULL_DE adds one more bf16 slab of G (the full one, read by dE only)
+    plain, full = L.cce_bwd_workspace_size(256, 256, 4096, 0, 0), L.cce_bwd_workspace_size(256, 256, 4096, 0, 4)
+    assert full - plain >= 256 * 4096 * 2
+    assert L.cce_bwd_workspace_size(256, 256, 4096, 0, 1) == plain   # Kahan needs no scratch
     assert L.cce_vocab_sort_workspace_size(256, 4096, 0) > 0
 
 

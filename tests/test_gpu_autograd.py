@@ -69,16 +69,56 @@ def test_full_classifier_gradient(std):
     wl = syn.Workload("fullc", N=700, D=256, V=24000, logit_std=std, ignore_frac=0.1)
     x = syn.make_inputs(wl, seed=5)
     H, segs, y = upload(x)
-    loss, lse = cce.fwd(H, segs[0][2], y)
+    E = segs[0][2]
+    loss, lse = cce.fwd(H, E, y)
     dl = x.dloss_mean()
-    dH, dE, _ = cce.bwd(H, segs[0][2], y, lse, torch.from_numpy(dl).cuda(), filter_eps=EPS_BF16,
-                        full_de=True)
+    dlt = torch.from_numpy(dl).cuda()
+    dH, dE, _ = cce.bwd(H, E, y, lse, dlt, filter_eps=EPS_BF16, full_de=True)
+    dH_f, _, _ = cce.bwd(H, E, y, lse, dlt, filter_eps=EPS_BF16)   # both filtered
+    _, dE_u, _ = cce.bwd(H, E, y, lse, dlt, filter_eps=0.0)        # both full
     torch.cuda.synchronize()
     rH, rE = oracle.backward(x.H, x.segments, x.y, wl.V, dl, x.ignore_index, filter_eps=EPS_BF16,
                              filter_dE=False)
-    uH, _ = oracle.backward(x.H, x.segments, x.y, wl.V, dl, x.ignore_index)
-    # dE is the full (unfiltered) classifier gradient
+    # dE is the full classifier gradient: the filter-off result, bit for bit
+    assert torch.equal(dE.view(torch.int16), dE_u.view(torch.int16))
     assert normwise(to_np(dE), rE[0]) <= TOL_GRAD
-    # dH is the filtered one; chunks too dense for the sparse route give the
-    # full dH instead, which is within the same tolerance of either
-    assert min(normwise(to_np(dH), rH), normwise(to_np(dH), uH)) <= TOL_GRAD_FILTER
+    # dH is the filtered input gradient, in dense and sparse-route chunks alike;
+    # it takes the same G entries as the default filtered path
+    assert normwise(to_np(dH), rH) <= TOL_GRAD_FILTER
+    assert normwise(to_np(dH), to_np(dH_f).astype(np.float64)) <= 2e-3
+
+
+def test_full_classifier_gradient_with_kahan():
+    """FullC combined with Kahan accumulation of dE over micro-batches: the
+    Kahan path runs every chunk on the dense route, so dH comes from the
+    filtered slab and dE from the full one."""
+    from linear_cross_entropy_cce_b200 import cce
+    wl = syn.Workload("fullck", N=400, D=128, V=5000, logit_std=5.0, ignore_frac=0.1)
+    xs = [syn.make_inputs(wl, seed=s) for s in range(3)]
+    Eh = xs[0].segments
+    Et = cce.bf16_from_bits(Eh[0][2], "cuda")
+    out = {}
+    for full in (True, False):
+        S = torch.zeros((wl.V, wl.D), dtype=torch.bfloat16, device="cuda")
+        C = torch.zeros_like(S)
+        dHs = []
+        for x in xs:
+            H = cce.bf16_from_bits(x.H, "cuda")
+            y = torch.from_numpy(x.y).cuda()
+            _, lse = cce.fwd(H, Et, y)
+            dl = torch.from_numpy(x.dloss_mean()).cuda()
+            eps = EPS_BF16 if full else 0.0
+            dH, _, _ = cce.bwd(H, Et, y, lse, dl, filter_eps=eps, kahan=True, full_de=full,
+                               dE_out=S, dE_comp=C)
+            dHs.append(dH)
+        torch.cuda.synchronize()
+        out[full] = (S, C, dHs)
+    S, C, dHs = out[True]
+    # the full dE parts are the filter-off parts, so the Kahan state matches bit for bit
+    assert torch.equal(S, out[False][0]) and torch.equal(C, out[False][1])
+    parts = [oracle.backward(x.H, Eh, x.y, wl.V, x.dloss_mean(), -100)[1][0] for x in xs]
+    assert normwise(to_np(S) - to_np(C), oracle.kahan_reference(parts)) <= TOL_GRAD
+    for x, dH in zip(xs, dHs):
+        rH, _ = oracle.backward(x.H, Eh, x.y, wl.V, x.dloss_mean(), -100, filter_eps=EPS_BF16,
+                                filter_dE=False)
+        assert normwise(to_np(dH), rH) <= TOL_GRAD_FILTER
