@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include <cub/device/device_radix_sort.cuh>
+#include <cub/device/device_scan.cuh>
 
 #include "../../include/cce.h"
 #include "cce_kernels.cuh"
@@ -170,7 +171,7 @@ struct BwdPlan {
   size_t mask_bytes;
   // sparse backward (filtered gradients)
   int64_t nch_max, cap;
-  size_t off_nzcnt, off_lists, off_colc, off_csorted, off_rowc, off_rsorted;
+  size_t off_nzcnt, off_lists, off_colc, off_csorted, off_rowc, off_rsorted, off_scan, scan_bytes;
 };
 
 BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags) {
@@ -210,10 +211,13 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags) {
   p.cap = std::max<int64_t>(4096, p.Npad * p.Vc / 2048);
   p.off_nzcnt = o; o += align_up(sizeof(int) * 2 * (size_t)p.nch_max);  // counts + slab flags
   p.off_lists = o; o += align_up(sizeof(NzEntry) * (size_t)p.nch_max * p.cap);
-  p.off_colc = o; o += align_up(sizeof(int) * 3 * (size_t)(p.Vc + 1));
-  p.off_csorted = o; o += align_up(sizeof(int2) * (size_t)p.cap);
-  p.off_rowc = o; o += align_up(sizeof(int) * 3 * (size_t)(p.Npad + 1));
+  p.off_colc = o; o += align_up(sizeof(int) * 2 * (size_t)(V + 1));  // counts, offsets
+  p.off_csorted = o; o += align_up(sizeof(int2) * (size_t)p.nch_max * p.cap);
+  p.off_rowc = o; o += align_up(sizeof(int) * 2 * (size_t)(p.Npad + 1));
   p.off_rsorted = o; o += align_up(sizeof(int2) * (size_t)p.nch_max * p.cap);
+  // generous bound on cub's single-pass scan scratch (checked again at run time)
+  p.scan_bytes = align_up(sizeof(int) * (size_t)(std::max<int64_t>(V, p.Npad) + 1) / 8 + (1u << 20));
+  p.off_scan = o; o += p.scan_bytes;
   p.total = o;
   return p;
 }
@@ -532,13 +536,12 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   const int cap = (int)pl.cap;
   int* nz_cnt = at<int>(workspace, pl.off_nzcnt);
   NzEntry* lists = at<NzEntry>(workspace, pl.off_lists);
+  const int64_t v_live = sg.live;
   int* col_cnt = at<int>(workspace, pl.off_colc);
-  int* col_ptr = col_cnt + (pl.Vc + 1);
-  int* col_cur = col_ptr + (pl.Vc + 1);
+  int* col_ptr = col_cnt + (v_live + 1);
   int2* csorted = at<int2>(workspace, pl.off_csorted);
   int* row_cnt = at<int>(workspace, pl.off_rowc);
   int* row_ptr = row_cnt + (pl.Npad + 1);
-  int* row_cur = row_ptr + (pl.Npad + 1);
   int2* rsorted = at<int2>(workspace, pl.off_rsorted);
   int* slab_flag = nz_cnt + pl.nch_max;
   if (sparse && cudaMemsetAsync(nz_cnt, 0, sizeof(int) * 2 * pl.nch_max, st) != cudaSuccess)
@@ -546,6 +549,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   ChunkMap cmap;
   memset(&cmap, 0, sizeof(cmap));
   cmap.n_segs = sg.n;
+  for (int s = 0; s < sg.n; ++s) cmap.live_off[s] = table.s[s].live_off;
   int chunk = 0;  // global chunk index
 
   GParams gp;
@@ -620,13 +624,10 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       gp.nz_list = sparse ? lists + (size_t)chunk * cap : nullptr;
       gp.nz_cnt = nz_cnt + chunk;
       gp.nz_cap = cap;
-      gp.col_cnt = col_cnt;
       gp.prev_nz_cnt = chunk > 0 ? nz_cnt + chunk - 1 : nullptr;
       gp.slab_flag = slab_flag + chunk;
       gp.repair = 0;
       gp.G_full = G_full;
-      if (sparse && cudaMemsetAsync(col_cnt, 0, sizeof(int) * (size_t)cv, st) != cudaSuccess)
-        return CCE_ELAUNCH;
       const int g_grid = (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct);
       if (int rc = full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
                            : launch_tc<GPolicy>(gp, g_grid, st, KC_G))
@@ -637,35 +638,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
                              : launch_tc<GPolicy>(gp, g_grid, st, KC_G))
           return rc;
       }
-      // step 2: dE rows of this chunk (sparse gathers, or the dense contraction)
-      if (sparse_de) {
-        {
-          TimedLaunch tl_(KC_SPARSE, st);
-          sparse_col_sort_kernel<<<1, SCAN_THREADS, 0, st>>>(nz_cnt + chunk, cap, col_cnt, cv, col_ptr,
-                                                             col_cur, lists + (size_t)chunk * cap,
-                                                             csorted);
-        }
-        if (launched()) return CCE_ELAUNCH;
-        SparseDEParams sp;
-        sp.nz_cnt = nz_cnt + chunk;
-        sp.cap = cap;
-        sp.col_ptr = col_ptr;
-        sp.sorted = csorted;
-        sp.Hc = Hc;
-        sp.D = (int)D;
-        sp.cv = cv;
-        sp.c0 = c0;
-        sp.perm_seg = perm_seg;
-        sp.dE = sg.s[s].dE;
-        sp.dE_comp = nullptr;
-        sp.mode = fp32 ? 1 : 0;
-        const int64_t warps = (int64_t)cv * cdiv(D, 256);
-        {
-          TimedLaunch tl_(KC_SPARSE, st);
-          sparse_de_kernel<<<(int)std::min<int64_t>(sms * 16, cdiv(warps, 8)), 256, 0, st>>>(sp);
-        }
-        if (launched()) return CCE_ELAUNCH;
-      }
+      // step 2: dE rows of this chunk (chunks on the sparse route: after the loop)
       ep.nz_cnt = sparse_de ? nz_cnt + chunk : nullptr;
       ep.nz_cap = cap;
       ep.chunk_valid = cv;
@@ -700,49 +673,95 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
         return rc;
     }
   }
-  // sparse chunks' dH contributions: row lists over every chunk
+  // sparse chunks: lists -> CSR by column (dE) and by row (dH), then the gathers
+  const int gthreads = gather_threads(D);
+  const int gblocks = sms * std::max(1, 2048 / gthreads);
   if (sparse) {
-    if (cudaMemsetAsync(row_cnt, 0, sizeof(int) * (size_t)pl.Npad, st) != cudaSuccess)
+    if (cudaMemsetAsync(row_cnt, 0, sizeof(int) * (size_t)(pl.Npad + 1), st) != cudaSuccess ||
+        (sparse_de && cudaMemsetAsync(col_cnt, 0, sizeof(int) * (size_t)(v_live + 1), st) != cudaSuccess))
       return CCE_ELAUNCH;
-    SparseRowsParams rp;
-    rp.nz_cnt = nz_cnt;
-    rp.nch = chunk;
-    rp.cap = cap;
-    rp.lists = lists;
-    rp.row_cnt = row_cnt;
-    rp.row_cur = row_cur;
-    rp.rsorted = rsorted;
-    rp.cmap = cmap;
+    SparseListParams lp;
+    lp.nz_cnt = nz_cnt;
+    lp.nch = chunk;
+    lp.cap = cap;
+    lp.lists = lists;
+    lp.cmap = cmap;
+    lp.col_cnt = sparse_de ? col_cnt : nullptr;
+    lp.col_ptr = col_ptr;
+    lp.csorted = csorted;
+    lp.row_cnt = row_cnt;
+    lp.row_ptr = row_ptr;
+    lp.rsorted = rsorted;
+    const dim3 lgrid((unsigned)std::min<int64_t>(cdiv(cap, 256), std::max(1, 4 * sms / chunk)), chunk);
     {
       TimedLaunch tl_(KC_SPARSE, st);
-      sparse_row_count_kernel<<<sms * 4, 256, 0, st>>>(rp);
+      sparse_count_kernel<<<lgrid, 256, 0, st>>>(lp);
     }
     if (launched()) return CCE_ELAUNCH;
+    void* scan_tmp = at<void>(workspace, pl.off_scan);
+    for (int pass = 0; pass < 2; ++pass) {
+      if (pass == 0 && !sparse_de) continue;
+      int* cnt = pass == 0 ? col_cnt : row_cnt;
+      int* ptr = pass == 0 ? col_ptr : row_ptr;
+      const int n = (int)(pass == 0 ? v_live + 1 : pl.Npad + 1);
+      size_t need = 0;
+      if (cub::DeviceScan::ExclusiveSum(nullptr, need, cnt, ptr, n, st) != cudaSuccess ||
+          need > pl.scan_bytes)
+        return CCE_ELAUNCH;
+      TimedLaunch tl_(KC_SPARSE, st);
+      if (cub::DeviceScan::ExclusiveSum(scan_tmp, need, cnt, ptr, n, st) != cudaSuccess)
+        return CCE_ELAUNCH;
+    }
     {
       TimedLaunch tl_(KC_SPARSE, st);
-      sparse_row_scan_kernel<<<1, SCAN_THREADS, 0, st>>>(row_cnt, (int)pl.Npad, row_ptr, row_cur);
+      sparse_scatter_kernel<<<lgrid, 256, 0, st>>>(lp);
     }
     if (launched()) return CCE_ELAUNCH;
-    {
-      TimedLaunch tl_(KC_SPARSE, st);
-      sparse_row_scatter_kernel<<<sms * 4, 256, 0, st>>>(rp);
+    if (sparse_de) {
+      SparseDEParams dp;
+      memset(&dp, 0, sizeof(dp));
+      dp.col_ptr = col_ptr;
+      dp.csorted = csorted;
+      dp.Hc = Hc;
+      dp.v_live = v_live;
+      dp.D = (int)D;
+      dp.range = GATHER_RANGE;
+      dp.nz_cnt = nz_cnt;
+      dp.cap = cap;
+      dp.cmap = cmap;
+      dp.vocab_perm = vocab_perm;
+      for (int s = 0; s < sg.n; ++s) dp.dE[s] = sg.s[s].dE;
+      dp.fp32_out = fp32 ? 1 : 0;
+      {
+        TimedLaunch tl_(KC_SPARSE, st);
+        sparse_de_kernel<<<(int)std::min<int64_t>(cdiv(v_live, GATHER_RANGE), gblocks), gthreads, 0,
+                           st>>>(dp);
+      }
+      if (launched()) return CCE_ELAUNCH;
     }
-    if (launched()) return CCE_ELAUNCH;
   }
-  DHFinParams fp_;
-  fp_.dH_acc = dH_acc;
-  fp_.pos_of_row = cp.pos_of_row;
-  fp_.N = (int)N;
-  fp_.D = (int)D;
-  fp_.dH = dH;
-  fp_.fp32_out = fp32 ? 1 : 0;
-  fp_.row_ptr = sparse ? row_ptr : nullptr;
-  fp_.rsorted = rsorted;
-  fp_.segs = table;
-  fp_.vocab_perm = vocab_perm;
+  SparseDHParams hq;
+  memset(&hq, 0, sizeof(hq));
+  hq.dH_acc = dH_acc;
+  hq.pos_of_row = cp.pos_of_row;
+  hq.N = N;
+  hq.D = (int)D;
+  hq.range = 4;
+  hq.dH = dH;
+  hq.fp32_out = fp32 ? 1 : 0;
+  hq.row_ptr = sparse ? row_ptr : nullptr;
+  hq.rsorted = rsorted;
+  hq.nz_cnt = sparse ? nz_cnt : nullptr;
+  hq.nch = chunk;
+  hq.cap = cap;
+  for (int s = 0; s < sg.n; ++s) {
+    hq.E[s] = table.s[s].E;
+    hq.live_off[s] = table.s[s].live_off;
+  }
+  hq.vocab_perm = vocab_perm;
   {
     TimedLaunch tl_(KC_SPARSE, st);
-    dh_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, 8), sms * 8), 256, 0, st>>>(fp_);
+    dh_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, hq.range), gblocks), gthreads, 0, st>>>(hq);
   }
   return launched();
 }

@@ -24,7 +24,9 @@
 //           G = dloss * (softmax * keep - onehot) in bf16 with block masks;
 //           tc_kernel<DEPolicy> dE_chunk = G^T H_c (K = rows, on chip);
 //           tc_kernel<DHPolicy> dH_acc += G E_chunk (K = chunk);
-//           then dh_finalize_kernel scatters dH back to the original rows.
+//           chunks sparse enough skip the last two for the list gathers of
+//           cce_sparse.cuh, which run once after all chunks; its
+//           dh_finalize_kernel scatters dH back to the original rows.
 #pragma once
 
 #include <cub/block/block_scan.cuh>
@@ -398,7 +400,6 @@ struct GParams {
   NzEntry* nz_list;
   int* nz_cnt;   // entries emitted (may exceed nz_cap: the chunk is then dense)
   int nz_cap;
-  int* col_cnt;  // per chunk column: entries (zeroed before this launch)
   // With a list, the bf16 slab and the masks (the dense fallback) are
   // written only when this chunk is predicted dense: the first chunk, or a
   // chunk after one that overflowed its list.  A mispredicted chunk is
@@ -564,10 +565,7 @@ struct GPolicyT {
                 if (!((nzb >> j) & 1u)) continue;
                 const float v = ((kb >> j) & 1u) ? ex2_approx(__uint_as_float(r[j])) : 0.f;
                 const float g = dl * (v - (((tb >> j) & 1u) ? 1.f : 0.f));
-                if (pos < p.nz_cap) {
-                  p.nz_list[pos] = NzEntry{jrow, vt * BN + c * 32 + j, g, 0};
-                  atomicAdd(&p.col_cnt[vt * BN + c * 32 + j], 1);
-                }
+                if (pos < p.nz_cap) p.nz_list[pos] = NzEntry{jrow, vt * BN + c * 32 + j, g, 0};
                 ++pos;
               }
             }
@@ -832,69 +830,6 @@ struct DHPolicy {
     __syncwarp();
   }
 };
-
-// dH[i] = dH_acc[pos_of_row[i]] + (sparse chunks) sum_j G_ij e_j, in bf16 or
-// fp32; 0 for ignored rows, NaN for rows with a bad target.  One warp per
-// row; lane owns 8 consecutive columns of each 256-wide slice of D.
-struct DHFinParams {
-  const float* dH_acc;
-  const int* pos_of_row;
-  int N, D;
-  void* dH;
-  int fp32_out;
-  const int* row_ptr;    // null: no sparse chunks
-  const int2* rsorted;   // (segment << 29 | walk position, g)
-  SegTable segs;
-  const int* vocab_perm; // concatenated per-segment permutations, or null
-};
-
-__global__ void dh_finalize_kernel(const DHFinParams p) {
-  const int lane = threadIdx.x & 31;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
-  for (int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < p.N; i += nw) {
-    const int j = p.pos_of_row[i];
-    const float fill = j == -1 ? 0.f : __int_as_float(0x7fc00000);
-    const int e0 = (j >= 0 && p.row_ptr) ? p.row_ptr[j] : 0;
-    const int e1 = (j >= 0 && p.row_ptr) ? p.row_ptr[j + 1] : 0;
-    for (int d0base = 0; d0base < p.D; d0base += 256) {
-      const int d0 = d0base + lane * 8;
-      float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      // sparse chunks: g * e_j for the row's entries, staged 32 at a time in
-      // the lanes (E row pointer, g) and gathered 4 deep
-      for (int eb = e0; eb < e1; eb += 32) {
-        const int n = min(32, e1 - eb);
-        const __nv_bfloat16* myrow = p.segs.s[0].E;
-        float myg = 0.f;
-        if (lane < n) {
-          const int2 t = p.rsorted[eb + lane];
-          const int s = (int)((unsigned)t.x >> 29), w = t.x & ((1 << 29) - 1);
-          const int loc = p.vocab_perm ? p.vocab_perm[p.segs.s[s].live_off + w] : w;
-          myrow = p.segs.s[s].E + (size_t)loc * p.D;
-          myg = __int_as_float(t.y);
-        }
-        gather_rows_fma(a, myrow, myg, n, d0 < p.D ? d0 : 0);
-      }
-      if (d0 >= p.D) continue;
-      if (j >= 0) {
-        const float4* src = reinterpret_cast<const float4*>(p.dH_acc + (size_t)j * p.D + d0);
-        const float4 u = src[0], v = src[1];
-        a[0] += u.x; a[1] += u.y; a[2] += u.z; a[3] += u.w;
-        a[4] += v.x; a[5] += v.y; a[6] += v.z; a[7] += v.w;
-      } else {
-        for (int k = 0; k < 8; ++k) a[k] = fill;
-      }
-      if (p.fp32_out) {
-        float4* d = reinterpret_cast<float4*>(static_cast<float*>(p.dH) + (size_t)i * p.D + d0);
-        d[0] = make_float4(a[0], a[1], a[2], a[3]);
-        d[1] = make_float4(a[4], a[5], a[6], a[7]);
-      } else {
-        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dH) + (size_t)i * p.D + d0) =
-            make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]),
-                       pack_bf16(a[6], a[7]));
-      }
-    }
-  }
-}
 
 // inv[perm[k]] = k for one segment (perm and inv point at the segment's
 // slice of the concatenated live vocabulary; entries are segment-local).
