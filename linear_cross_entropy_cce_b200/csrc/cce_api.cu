@@ -205,7 +205,8 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags) {
   p.dh_words = (int)cdiv(p.Vc, 512);
   p.de_words = (int)cdiv(p.Npad, 512);
   p.mask_bytes = sizeof(uint32_t) * ((size_t)(p.Npad / BM) * p.dh_words + (size_t)(p.Vc / BM) * p.de_words);
-  p.off_masks = o; o += align_up(p.mask_bytes);
+  // two mask buffers: chunk c uses buffer c % 2 and its G launch clears the other
+  p.off_masks = o; o += 2 * align_up(p.mask_bytes);
   // sparse path: per chunk a list of up to `cap` non-zeros (density 1/2048)
   p.nch_max = cdiv(V, p.Vc) + CCE_MAX_SEGMENTS;
   p.cap = std::max<int64_t>(4096, p.Npad * p.Vc / 2048);
@@ -518,8 +519,9 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
 
   __nv_bfloat16* G = at<__nv_bfloat16>(workspace, pl.off_g);
   __nv_bfloat16* G_full = full_de ? at<__nv_bfloat16>(workspace, pl.off_gfull) : nullptr;
-  uint32_t* dh_mask = at<uint32_t>(workspace, pl.off_masks);
-  uint32_t* de_mask = dh_mask + (size_t)(pl.Npad / BM) * pl.dh_words;
+  uint32_t* masks = at<uint32_t>(workspace, pl.off_masks);
+  const size_t mask_stride = align_up(pl.mask_bytes) / sizeof(uint32_t);
+  if (cudaMemsetAsync(masks, 0, 2 * align_up(pl.mask_bytes), st) != cudaSuccess) return CCE_ELAUNCH;
   __nv_bfloat16* Ec = at<__nv_bfloat16>(workspace, pl.off_ec);
   const int Vc = (int)pl.Vc;
   const int dt = (int)cdiv(D, BN);
@@ -593,7 +595,10 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
         row0 = 0;
       }
       // step 1: G for this chunk, with its zero-slice masks
-      if (cudaMemsetAsync(dh_mask, 0, pl.mask_bytes, st) != cudaSuccess) return CCE_ELAUNCH;
+      uint32_t* dh_mask = masks + (size_t)(chunk & 1) * mask_stride;
+      uint32_t* de_mask = dh_mask + (size_t)(pl.Npad / BM) * pl.dh_words;
+      gp.mask_clear = masks + (size_t)((chunk + 1) & 1) * mask_stride;
+      gp.mask_clear_words = (int)(pl.mask_bytes / sizeof(uint32_t));
       gp.dh_mask = dh_mask;
       gp.dh_words = pl.dh_words;
       gp.de_mask = de_mask;
@@ -718,50 +723,57 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
     }
     if (launched()) return CCE_ELAUNCH;
     if (sparse_de) {
-      SparseDEParams dp;
-      memset(&dp, 0, sizeof(dp));
-      dp.col_ptr = col_ptr;
-      dp.csorted = csorted;
-      dp.Hc = Hc;
-      dp.v_live = v_live;
-      dp.D = (int)D;
-      dp.range = GATHER_RANGE;
-      dp.nz_cnt = nz_cnt;
-      dp.cap = cap;
-      dp.cmap = cmap;
-      dp.vocab_perm = vocab_perm;
-      for (int s = 0; s < sg.n; ++s) dp.dE[s] = sg.s[s].dE;
-      dp.fp32_out = fp32 ? 1 : 0;
+      DERows dr;
+      memset(&dr, 0, sizeof(dr));
+      dr.ptr = col_ptr;
+      dr.ent = csorted;
+      dr.Hc = Hc;
+      dr.v_live = v_live;
+      dr.D = (int)D;
+      dr.range = gather_range(v_live, gblocks);
+      dr.nz_cnt = nz_cnt;
+      dr.cap = cap;
+      dr.cmap = cmap;
+      dr.vocab_perm = vocab_perm;
+      for (int s = 0; s < sg.n; ++s) dr.dE[s] = sg.s[s].dE;
+      dr.fp32_out = fp32 ? 1 : 0;
       {
         TimedLaunch tl_(KC_SPARSE, st);
-        sparse_de_kernel<<<(int)std::min<int64_t>(cdiv(v_live, GATHER_RANGE), gblocks), gthreads, 0,
-                           st>>>(dp);
+        csr_rows_kernel<DERows><<<(int)std::min<int64_t>(cdiv(v_live, dr.range), gblocks), gthreads, 0,
+                                  st>>>(dr);
       }
       if (launched()) return CCE_ELAUNCH;
     }
   }
-  SparseDHParams hq;
-  memset(&hq, 0, sizeof(hq));
-  hq.dH_acc = dH_acc;
-  hq.pos_of_row = cp.pos_of_row;
-  hq.N = N;
-  hq.D = (int)D;
-  hq.range = 4;
-  hq.dH = dH;
-  hq.fp32_out = fp32 ? 1 : 0;
-  hq.row_ptr = sparse ? row_ptr : nullptr;
-  hq.rsorted = rsorted;
-  hq.nz_cnt = sparse ? nz_cnt : nullptr;
-  hq.nch = chunk;
-  hq.cap = cap;
+  DHRows hr;
+  memset(&hr, 0, sizeof(hr));
+  hr.ptr = sparse ? row_ptr : nullptr;
+  hr.ent = rsorted;
+  hr.n_valid = cp.n_valid;
+  hr.idx = cp.idx;
+  hr.dH_acc = dH_acc;
+  hr.nz_cnt = sparse ? nz_cnt : nullptr;
+  hr.nch = chunk;
+  hr.cap = cap;
+  hr.D = (int)D;
+  hr.range = gather_range(pl.Npad, gblocks);
+  hr.dH = dH;
+  hr.fp32_out = fp32 ? 1 : 0;
   for (int s = 0; s < sg.n; ++s) {
-    hq.E[s] = table.s[s].E;
-    hq.live_off[s] = table.s[s].live_off;
+    hr.E[s] = table.s[s].E;
+    hr.live_off[s] = table.s[s].live_off;
   }
-  hq.vocab_perm = vocab_perm;
+  hr.vocab_perm = vocab_perm;
   {
     TimedLaunch tl_(KC_SPARSE, st);
-    dh_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, hq.range), gblocks), gthreads, 0, st>>>(hq);
+    csr_rows_kernel<DHRows><<<(int)std::min<int64_t>(cdiv(pl.Npad, hr.range), gblocks), gthreads, 0,
+                              st>>>(hr);
+  }
+  if (launched()) return CCE_ELAUNCH;
+  {
+    TimedLaunch tl_(KC_SPARSE, st);
+    dh_fill_kernel<<<(int)std::min<int64_t>(cdiv(N * (D / 8), 256), sms * 8), 256, 0, st>>>(
+        cp.pos_of_row, N, (int)D, dH, fp32 ? 1 : 0);
   }
   return launched();
 }

@@ -25,8 +25,8 @@
 //           tc_kernel<DEPolicy> dE_chunk = G^T H_c (K = rows, on chip);
 //           tc_kernel<DHPolicy> dH_acc += G E_chunk (K = chunk);
 //           chunks sparse enough skip the last two for the list gathers of
-//           cce_sparse.cuh, which run once after all chunks; its
-//           dh_finalize_kernel scatters dH back to the original rows.
+//           cce_sparse.cuh, which run once after all chunks and write dH
+//           back to the original rows.
 #pragma once
 
 #include <cub/block/block_scan.cuh>
@@ -396,6 +396,10 @@ struct GParams {
   int dh_words;
   uint32_t* de_mask;
   int de_words;
+  // The other mask buffer, cleared by the first launch of this chunk for the
+  // next chunk (its last readers, the previous chunk's contractions, are done).
+  uint32_t* mask_clear;
+  int mask_clear_words;
   // sparse list of this chunk's non-zeros (null: not collected)
   NzEntry* nz_list;
   int* nz_cnt;   // entries emitted (may exceed nz_cap: the chunk is then dense)
@@ -469,6 +473,10 @@ struct GPolicyT {
     bool emit = p.nz_list != nullptr && !p.repair;  // this warp still lists non-zeros
     if (slab && p.slab_flag && !p.repair && blockIdx.x == 0 && threadIdx.x == 64)
       *p.slab_flag = 1;
+    if (!p.repair && p.mask_clear)
+      for (int i = blockIdx.x * EPI_THREADS + q * 32 + lane; i < p.mask_clear_words;
+           i += gridDim.x * EPI_THREADS)
+        p.mask_clear[i] = 0u;
     schedule(p, [&](int mb, int vt, int nv) {
       uint32_t taddr;
       if (!eng.epi_acquire(q, taddr)) return false;

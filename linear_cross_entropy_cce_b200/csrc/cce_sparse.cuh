@@ -17,15 +17,16 @@
 //   sparse_count_kernel    entries per column (global walk position) and row
 //   (exclusive scans)      column and row offsets (CSR)
 //   sparse_scatter_kernel  entries into column order and into row order
-//   sparse_de_kernel       each dE row of a sparse chunk: zero, or the
-//                          gather over its column list
-//   dh_finalize_kernel     each dH row: the dense accumulator plus the
-//                          gather over its row list
-// A block owns one output row at a time, its threads 8 consecutive elements
-// of D each; the row's list is staged in shared memory and its source rows
-// are read 8 deep.  Entries of one row or column are summed in an order set
-// by atomics, so these sums are not bitwise reproducible run to run.
+//   csr_rows_kernel<DERows>  each dE row of a sparse chunk: the gather over
+//                            its column list (zero when empty)
+//   csr_rows_kernel<DHRows>  each valid dH row: the dense accumulator plus
+//                            the gather over its row list; dh_fill_kernel
+//                            writes the other rows
+// Entries of one row or column are summed in an order set by atomics, so
+// these sums are not bitwise reproducible run to run.
 #pragma once
+
+#include <type_traits>
 
 #include "cce_ptx.cuh"
 
@@ -108,13 +109,13 @@ __global__ void sparse_scatter_kernel(const SparseListParams p) {
 
 // ---- CSR x dense rows ----------------------------------------------------------
 constexpr int GATHER_STAGE = 512;  // list entries staged in shared memory at once
-constexpr int GATHER_RANGE = 64;   // output rows whose offsets are loaded together
-constexpr int GATHER_MAX_THREADS = 1024;
+constexpr int GATHER_RANGE = 64;   // most output rows one block takes at a time
+constexpr int GATHER_MAX_THREADS = 512;
 
 struct GatherSrc {
   const __nv_bfloat16* src;
   float g;
-  int pad;
+  int row;  // output row within the block's range
 };
 
 // Adds g * (8 bf16 in h) into acc.
@@ -129,35 +130,6 @@ __device__ __forceinline__ void fma8(float (&acc)[8], float g, const uint4 h) {
   acc[7] = fmaf(g, bf16hi(h.w), acc[7]);
 }
 
-// acc += sum over list entries [e0, e1) of g * src[d .. d+8).  Every thread of
-// the block calls this with the same e0, e1 (it synchronises the block); a
-// thread whose d lies past D passes active = false and only helps staging.
-template <class SrcOf>
-__device__ __forceinline__ void csr_accumulate(float (&acc)[8], int e0, int e1,
-                                               const int2* __restrict__ ent, SrcOf&& src_of,
-                                               int d, bool active, GatherSrc* stage) {
-  for (int wb = e0; wb < e1; wb += GATHER_STAGE) {
-    const int n = min(GATHER_STAGE, e1 - wb);
-    __syncthreads();  // the previous window is no longer read
-    for (int k = threadIdx.x; k < n; k += blockDim.x) {
-      const int2 v = ent[wb + k];
-      stage[k] = GatherSrc{src_of(v.x), __int_as_float(v.y), 0};
-    }
-    __syncthreads();
-    if (!active) continue;
-    int k = 0;
-    for (; k + 8 <= n; k += 8) {
-      uint4 h[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) h[u] = __ldg(reinterpret_cast<const uint4*>(stage[k + u].src + d));
-#pragma unroll
-      for (int u = 0; u < 8; ++u) fma8(acc, stage[k + u].g, h[u]);
-    }
-    for (; k < n; ++k)
-      fma8(acc, stage[k].g, __ldg(reinterpret_cast<const uint4*>(stage[k].src + d)));
-  }
-}
-
 __device__ __forceinline__ void store_row8(void* row, int d, const float (&a)[8], int fp32_out) {
   if (fp32_out) {
     float4* o = reinterpret_cast<float4*>(static_cast<float*>(row) + d);
@@ -170,12 +142,24 @@ __device__ __forceinline__ void store_row8(void* row, int d, const float (&a)[8]
   }
 }
 
+// Rows of a CSR matrix times dense bf16 source rows, one output row each:
+//   out_r = addend_r + sum_{e in [ptr[r], ptr[r+1])} g_e * src(key_e).
+// A block takes `range` consecutive rows: their list entries are contiguous,
+// so it stages them (window by window) with each entry's row and walks them
+// in one flat pass, 8 source loads in flight across row boundaries; a row is
+// stored when the walk passes it, empty rows included.  Each thread owns 8
+// consecutive elements of D (a slice of blockDim * 8 at a time).
+//
+// R supplies: rows() (count), ptr, ent, src(key), out(row) (null: not
+// written here), addend(row) (null: 0), fp32_out, D, range.  For DHRows the
+// addend (dH_acc) is read only when some chunk took the dense route.
+
 // dE rows of the chunks taken by the sparse route, indexed by global walk
-// position w (segment s, w - live_off[s] within it): zero where the column
-// list is empty.  Rows of dense chunks are left to the dense contraction.
-struct SparseDEParams {
-  const int* col_ptr;  // [V_live + 1]
-  const int2* csorted;
+// position w (segment s, w - live_off[s] within it).  Rows of dense chunks are
+// left to the dense contraction.
+struct DERows {
+  const int* ptr;  // [V_live + 1]
+  const int2* ent; // (compact row, g)
   const __nv_bfloat16* Hc;  // [Npad, D]
   long long v_live;
   int D, range;
@@ -185,118 +169,178 @@ struct SparseDEParams {
   const int* vocab_perm;  // concatenated per-segment permutations, or null
   void* dE[SP_MAX_SEGS];
   int fp32_out;
+
+  __device__ long long rows() const { return v_live; }
+  __device__ const __nv_bfloat16* src(int key) const { return Hc + (size_t)key * D; }
+  __device__ void* out(long long r) const {
+    const int w = (int)r;
+    int s = 0;
+    while (s + 1 < cmap.n_segs && w >= cmap.live_off[s + 1]) ++s;
+    const int wl = w - cmap.live_off[s];
+    if (nz_cnt[cmap.chunk_begin[s] + wl / cmap.width[s]] > cap) return nullptr;
+    const size_t row = (size_t)(vocab_perm ? vocab_perm[w] : wl);
+    return fp32_out ? (void*)(static_cast<float*>(dE[s]) + row * D)
+                    : (void*)(static_cast<__nv_bfloat16*>(dE[s]) + row * D);
+  }
+  __device__ const float* addend(long long) const { return nullptr; }
 };
 
-__global__ void __launch_bounds__(GATHER_MAX_THREADS) sparse_de_kernel(const SparseDEParams p) {
+// dH rows of the valid (compact) rows j: dH_acc row j (when some chunk took
+// the dense route) plus the row list over E rows, written to original row
+// idx[j].  Ignored and bad-target rows are written by dh_fill_kernel.
+struct DHRows {
+  const int* ptr;   // [Npad + 1]; null: no row lists (every chunk dense)
+  const int2* ent;  // (segment << 29 | walk position in segment, g)
+  const int* n_valid;
+  const int* idx;   // compact -> original row
+  const float* dH_acc;  // [Npad, D]; read only when some chunk took the dense route
+  const int* nz_cnt;  // [nch]; null: every chunk took the dense route
+  int nch, cap;
+  int D, range;
+  void* dH;
+  int fp32_out;
+  const __nv_bfloat16* E[SP_MAX_SEGS];
+  int live_off[SP_MAX_SEGS];
+  const int* vocab_perm;
+
+  __device__ long long rows() const { return *n_valid; }
+  __device__ const __nv_bfloat16* src(int key) const {
+    const int s = (int)((unsigned)key >> 29), w = key & ((1 << 29) - 1);
+    const int loc = vocab_perm ? vocab_perm[live_off[s] + w] : w;
+    return E[s] + (size_t)loc * D;
+  }
+  __device__ void* out(long long j) const {
+    const size_t i = (size_t)idx[j];
+    return fp32_out ? (void*)(static_cast<float*>(dH) + i * D)
+                    : (void*)(static_cast<__nv_bfloat16*>(dH) + i * D);
+  }
+  __device__ const float* addend(long long j) const { return dH_acc + (size_t)j * D; }
+};
+
+template <class R>
+__global__ void __launch_bounds__(GATHER_MAX_THREADS, 1) csr_rows_kernel(const R p) {
   __shared__ int sp[GATHER_RANGE + 1];
-  __shared__ void* dst[GATHER_RANGE];  // null: written by the dense route
+  __shared__ void* dst[GATHER_RANGE];
+  __shared__ const float* add[GATHER_RANGE];
   __shared__ GatherSrc stage[GATHER_STAGE];
+  bool use_add = true;
+  if constexpr (std::is_same<R, DHRows>::value) {
+    // dH_acc holds anything only if some chunk took the dense route
+    __shared__ int dense_any;
+    if (threadIdx.x == 0) dense_any = p.nz_cnt ? 0 : 1;
+    __syncthreads();
+    if (p.nz_cnt)
+      for (int c = threadIdx.x; c < p.nch; c += blockDim.x)
+        if (p.nz_cnt[c] > p.cap) dense_any = 1;
+    __syncthreads();
+    use_add = dense_any != 0;
+  }
+  const long long nrows = p.rows();
   const long long step = (long long)gridDim.x * p.range;
-  for (long long r0 = (long long)blockIdx.x * p.range; r0 < p.v_live; r0 += step) {
-    const int nr = (int)min((long long)p.range, p.v_live - r0);
-    __syncthreads();  // the previous range's offsets are no longer read
+  for (long long r0 = (long long)blockIdx.x * p.range; r0 < nrows; r0 += step) {
+    const int nr = (int)min((long long)p.range, nrows - r0);
+    __syncthreads();  // the previous range is no longer read
     for (int k = threadIdx.x; k <= nr; k += blockDim.x) {
-      sp[k] = p.col_ptr[r0 + k];
+      sp[k] = p.ptr ? p.ptr[r0 + k] : 0;
       if (k < nr) {
-        const int w = (int)(r0 + k);
-        int s = 0;
-        while (s + 1 < p.cmap.n_segs && w >= p.cmap.live_off[s + 1]) ++s;
-        const int wl = w - p.cmap.live_off[s];
-        void* d = nullptr;
-        if (p.nz_cnt[p.cmap.chunk_begin[s] + wl / p.cmap.width[s]] <= p.cap) {
-          const size_t row = (size_t)(p.vocab_perm ? p.vocab_perm[w] : wl);
-          d = p.fp32_out ? (void*)(static_cast<float*>(p.dE[s]) + row * p.D)
-                         : (void*)(static_cast<__nv_bfloat16*>(p.dE[s]) + row * p.D);
-        }
-        dst[k] = d;
+        dst[k] = p.out(r0 + k);
+        add[k] = use_add ? p.addend(r0 + k) : nullptr;
       }
     }
     __syncthreads();
-    for (int r = 0; r < nr; ++r) {
-      void* out = dst[r];
-      if (!out) continue;
-      const int e0 = sp[r], e1 = sp[r + 1];
-      for (int db = 0; db < p.D; db += blockDim.x * 8) {
-        const int d = db + threadIdx.x * 8;
-        float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        csr_accumulate(a, e0, e1, p.csorted,
-                       [&](int row) { return p.Hc + (size_t)row * p.D; }, d, d < p.D, stage);
-        if (d < p.D) store_row8(out, d, a, p.fp32_out);
+    const int E0 = sp[0], E1 = sp[nr];
+    for (int db = 0; db < p.D; db += blockDim.x * 8) {
+      const int d = db + threadIdx.x * 8;
+      const bool act = d < p.D;
+      int cur = 0;  // row being accumulated
+      float a[8];
+      auto start = [&](int r) {
+        const float* ad = add[r];
+        if (ad && act) {
+          const float4 u = *reinterpret_cast<const float4*>(ad + d);
+          const float4 v = *reinterpret_cast<const float4*>(ad + d + 4);
+          a[0] = u.x; a[1] = u.y; a[2] = u.z; a[3] = u.w;
+          a[4] = v.x; a[5] = v.y; a[6] = v.z; a[7] = v.w;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) a[k] = 0.f;
+        }
+      };
+      auto finish = [&](int r) {
+        if (act && dst[r]) store_row8(dst[r], d, a, p.fp32_out);
+      };
+      start(0);
+      for (int wb = E0; wb < E1; wb += GATHER_STAGE) {
+        const int n = min(GATHER_STAGE, E1 - wb);
+        __syncthreads();  // the previous window is no longer read
+        for (int k = threadIdx.x; k < n; k += blockDim.x) {
+          const int e = wb + k;
+          int lo = 0, hi = nr;  // the row r with sp[r] <= e < sp[r + 1]
+          while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (sp[mid] <= e) lo = mid; else hi = mid;
+          }
+          const int2 v = p.ent[e];
+          stage[k] = GatherSrc{p.src(v.x), __int_as_float(v.y), lo};
+        }
+        __syncthreads();
+        if (!act) continue;
+        int k = 0;
+        for (; k + 8 <= n; k += 8) {
+          uint4 h[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) h[u] = __ldg(reinterpret_cast<const uint4*>(stage[k + u].src + d));
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int r = stage[k + u].row;
+            while (cur < r) {
+              finish(cur);
+              start(++cur);
+            }
+            fma8(a, stage[k + u].g, h[u]);
+          }
+        }
+        for (; k < n; ++k) {
+          const int r = stage[k].row;
+          while (cur < r) {
+            finish(cur);
+            start(++cur);
+          }
+          fma8(a, stage[k].g, __ldg(reinterpret_cast<const uint4*>(stage[k].src + d)));
+        }
+      }
+      // the rows after the last entry (all of them if the range has none)
+      for (;;) {
+        finish(cur);
+        if (++cur >= nr) break;
+        start(cur);
       }
     }
   }
 }
 
-// dH[i] = dH_acc[pos_of_row[i]] + (sparse chunks) sum_j G_ij e_j, in bf16 or
-// fp32; 0 for ignored rows, NaN for rows with a bad target.  dH_acc is read
-// only when some chunk took the dense route.
-struct SparseDHParams {
-  const float* dH_acc;    // [Npad, D]
-  const int* pos_of_row;  // original row -> compact row; -1 ignored, < -1 bad target
-  long long N;
-  int D, range;
-  void* dH;
-  int fp32_out;
-  const int* row_ptr;  // [Npad + 1]; null: no row lists
-  const int2* rsorted;
-  const int* nz_cnt;   // [nch]; null: every chunk took the dense route
-  int nch, cap;
-  const __nv_bfloat16* E[SP_MAX_SEGS];
-  int live_off[SP_MAX_SEGS];
-  const int* vocab_perm;  // concatenated per-segment permutations, or null
-};
-
-__global__ void __launch_bounds__(GATHER_MAX_THREADS) dh_finalize_kernel(const SparseDHParams p) {
-  __shared__ int pj[GATHER_RANGE];
-  __shared__ int pe[GATHER_RANGE][2];
-  __shared__ GatherSrc stage[GATHER_STAGE];
-  __shared__ int dense_any;
-  if (threadIdx.x == 0) dense_any = p.nz_cnt ? 0 : 1;
-  __syncthreads();
-  if (p.nz_cnt)
-    for (int c = threadIdx.x; c < p.nch; c += blockDim.x)
-      if (p.nz_cnt[c] > p.cap) dense_any = 1;
-  __syncthreads();
-  const bool use_acc = dense_any != 0;
-  auto src_of = [&](int key) {
-    const int s = (int)((unsigned)key >> 29), w = key & ((1 << 29) - 1);
-    const int loc = p.vocab_perm ? p.vocab_perm[p.live_off[s] + w] : w;
-    return p.E[s] + (size_t)loc * p.D;
-  };
-  const long long step = (long long)gridDim.x * p.range;
-  for (long long r0 = (long long)blockIdx.x * p.range; r0 < p.N; r0 += step) {
-    const int nr = (int)min((long long)p.range, p.N - r0);
-    __syncthreads();
-    for (int k = threadIdx.x; k < nr; k += blockDim.x) {
-      const int j = p.pos_of_row[r0 + k];
-      pj[k] = j;
-      pe[k][0] = (j >= 0 && p.row_ptr) ? p.row_ptr[j] : 0;
-      pe[k][1] = (j >= 0 && p.row_ptr) ? p.row_ptr[j + 1] : 0;
-    }
-    __syncthreads();
-    for (int r = 0; r < nr; ++r) {
-      const int j = pj[r];
-      void* out = p.fp32_out ? (void*)(static_cast<float*>(p.dH) + (size_t)(r0 + r) * p.D)
-                             : (void*)(static_cast<__nv_bfloat16*>(p.dH) + (size_t)(r0 + r) * p.D);
-      for (int db = 0; db < p.D; db += blockDim.x * 8) {
-        const int d = db + threadIdx.x * 8;
-        const bool act = d < p.D;
-        float a[8];
-        if (j >= 0 && use_acc && act) {
-          const float4* src = reinterpret_cast<const float4*>(p.dH_acc + (size_t)j * p.D + d);
-          const float4 u = src[0], v = src[1];
-          a[0] = u.x; a[1] = u.y; a[2] = u.z; a[3] = u.w;
-          a[4] = v.x; a[5] = v.y; a[6] = v.z; a[7] = v.w;
-        } else {
-          const float fill = j >= 0 || j == -1 ? 0.f : __int_as_float(0x7fc00000);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) a[k] = fill;
-        }
-        if (j >= 0) csr_accumulate(a, pe[r][0], pe[r][1], p.rsorted, src_of, d, act, stage);
-        if (act) store_row8(out, d, a, p.fp32_out);
-      }
-    }
+// dH rows without a compact row: 0 for ignored rows, NaN for bad targets.
+__global__ void dh_fill_kernel(const int* __restrict__ pos_of_row, long long N, int D, void* dH,
+                               int fp32_out) {
+  const int per_row = D / 8;
+  const long long total = N * per_row;
+  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < total;
+       t += (long long)gridDim.x * blockDim.x) {
+    const long long i = t / per_row;
+    const int j = pos_of_row[i];
+    if (j >= 0) continue;
+    const float f = j == -1 ? 0.f : __int_as_float(0x7fc00000);
+    const float a[8] = {f, f, f, f, f, f, f, f};
+    void* row = fp32_out ? (void*)(static_cast<float*>(dH) + i * D)
+                         : (void*)(static_cast<__nv_bfloat16*>(dH) + i * D);
+    store_row8(row, (int)(t - i * per_row) * 8, a, fp32_out);
   }
+}
+
+// Rows per block range: enough ranges for every block, at most GATHER_RANGE.
+inline int gather_range(long long rows, int blocks) {
+  const long long r = rows / (blocks > 0 ? blocks : 1);
+  return (int)(r < 4 ? 4 : (r > GATHER_RANGE ? GATHER_RANGE : r));
 }
 
 // Threads per block for the gathers: 8 elements of D each, whole warps.
