@@ -248,7 +248,8 @@ def main():
         if sort:
             perm = cce.vocab_sort(out[2], yd, V, x.ignore_index,
                                   segments=None if single else segd, workspace=ws_s)
-        kw = dict(filter_eps=eps, vocab_perm=perm, workspace=ws_b, status=status)
+        kw = dict(filter_eps=eps, vocab_perm=perm, colmax=out[2] if sort else None,
+                  workspace=ws_b, status=status)
         if single:
             dH, dE, _ = cce.bwd(Hd, segd[0][2], yd, lse, dloss, x.ignore_index, **kw)
         else:

@@ -140,13 +140,23 @@ size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs,
  *            backward walks the vocabulary in that order so that surviving
  *            blocks cluster; results do not depend on it beyond rounding.
  *            NULL = identity.
+ *   colmax   optional [V_live] fp32, the colmax output of cce_fwd on the
+ *            same H, E, y and segments (a bound on every logit of each
+ *            vocabulary row).  With filtering on (and without
+ *            CCE_FULL_DE) a 128-row x 256-column tile of the backward whose
+ *            bound  max colmax - min lse  over the tile lies below
+ *            ln(filter_eps) by a margin is not recomputed: every softmax
+ *            entry in it would be filtered, so only its one-hot entries are
+ *            written: the block skip of the first page's §Contribution
+ *            and of the research-map entry's §Approach, taken exactly.  The
+ *            skip never changes which entries are kept.  A colmax that is not such a bound
+ *            drops gradient entries.  NULL = no tile skip.
  *   flags    CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE.  CCE_FULL_DE keeps
  *            the classifier gradient dE unfiltered while dH uses the filtered
  *            softmax (the "FullC" variant of "Cut Your Losses in
  *            Large-Vocabulary Language Models", research-map entry, §Key
- *            results / §Limitations); vocabulary chunks too dense for the
- *            sparse dH route then contribute their full (unfiltered)
- *            gradient to dH as well.
+ *            results / §Limitations), in every vocabulary chunk; it needs
+ *            one more bf16 slab of workspace (see cce_bwd_workspace_size).
  *   dH       [N, D] output (bf16, or fp32 with CCE_FP32_GRADS).
  *   dE       [V, D] output when segs == NULL (else per-segment dE).  Written
  *            (overwritten) unless CCE_KAHAN_DE, in which case the new
@@ -165,7 +175,8 @@ int cce_bwd(const void* H, const void* E, const int32_t* y,
             const float* lse, const float* dloss,
             int64_t N, int64_t D, int64_t V, int32_t ignore_index,
             const cce_segment* segs, int32_t n_segs,
-            float filter_eps, const int32_t* vocab_perm, uint32_t flags,
+            float filter_eps, const int32_t* vocab_perm, const float* colmax,
+            uint32_t flags,
             void* dH, void* dE, void* dE_comp,
             uint32_t* debug_keep, int64_t debug_rows,
             void* workspace, size_t workspace_bytes,

@@ -31,22 +31,23 @@ class _LinearCrossEntropy(torch.autograd.Function):
                                   segments=segments)
         else:
             loss, lse = cce.fwd(H, E, y, ignore_index, segments=segments, V=V)
-            perm = None
+            perm = colmax = None
         ctx.save_for_backward(H, E if E is not None else torch.empty(0), y, lse,
-                              perm if perm is not None else torch.empty(0), *seg_E)
+                              perm if perm is not None else torch.empty(0),
+                              colmax if colmax is not None else torch.empty(0), *seg_E)
         ctx.meta = (ignore_index, filter_eps, full_de, segments_meta, E is not None, perm is not None)
         return loss
 
     @staticmethod
     def backward(ctx, grad_loss):
-        H, E, y, lse, perm, *seg_E = ctx.saved_tensors
+        H, E, y, lse, perm, colmax, *seg_E = ctx.saved_tensors
         ignore_index, filter_eps, full_de, segments_meta, has_E, has_perm = ctx.meta
         segments = [(b, e, t) for (b, e), t in zip(segments_meta, seg_E)] if segments_meta else None
         V = segments_meta[-1][1] if segments_meta else None
         dloss = grad_loss.contiguous().to(torch.float32)
         dH, dE, _ = cce.bwd(H, E if has_E else None, y, lse, dloss, ignore_index, segments=segments,
                             V=V, filter_eps=filter_eps, vocab_perm=perm if has_perm else None,
-                            full_de=full_de)
+                            colmax=colmax if has_perm else None, full_de=full_de)
         dH = dH.to(H.dtype)
         if segments:
             return (dH, None, None, None, None, None, None, None, *[g.to(t.dtype) for g, t in zip(dE, seg_E)])
@@ -66,7 +67,8 @@ def linear_cross_entropy(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Te
     "none" (per-row losses, ignored rows 0).  filter_eps <= 0 disables the
     gradient filter; full_de keeps the classifier gradient unfiltered;
     vocab_sort walks the vocabulary in descending max-logit order in the
-    backward.
+    backward and, with the filter on, skips the tiles whose every softmax
+    entry the forward's column maxima bound below filter_eps.
     """
     if y.dtype != torch.int32:
         y = y.to(torch.int32)

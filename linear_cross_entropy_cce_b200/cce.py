@@ -65,7 +65,7 @@ def lib() -> ctypes.CDLL:
     L.cce_bwd_workspace_size.argtypes = [i64, i64, i64, i32, u32]
     L.cce_bwd.restype = ctypes.c_int
     L.cce_bwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, ctypes.POINTER(Segment), i32,
-                          fp, vp, u32, vp, vp, vp, vp, i64, vp, sz, vp, vp]
+                          fp, vp, vp, u32, vp, vp, vp, vp, i64, vp, sz, vp, vp]
     L.cce_vocab_sort_workspace_size.restype = sz
     L.cce_vocab_sort_workspace_size.argtypes = [i64, i64, i32]
     L.cce_vocab_sort.restype = ctypes.c_int
@@ -166,18 +166,19 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
         dloss: torch.Tensor, ignore_index: int = -100,
         segments: Optional[Sequence[SegSpec]] = None, V: Optional[int] = None,
         filter_eps: float = 0.0, vocab_perm: Optional[torch.Tensor] = None,
-        kahan: bool = False, fp32_grads: bool = False, full_de: bool = False,
+        colmax: Optional[torch.Tensor] = None, kahan: bool = False, fp32_grads: bool = False, full_de: bool = False,
         dE_out=None, dE_comp=None, debug_rows: int = 0,
         workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
     """Gradients (dH, dE) of sum_i dloss_i loss_i.  See cce_bwd.
 
     dE is one tensor for a single head, a list (one per segment) otherwise.
     With kahan=True, dE_out and dE_comp (bf16, same shape(s)) are required
-    and updated in place.  Returns (dH, dE, debug_keep or None).
+    and updated in place.  colmax (the forward's, same inputs) enables the
+    exact tile skip when filtering.  Returns (dH, dE, debug_keep or None).
     """
     N, D = H.shape
     dev = H.device
-    _require_cuda(H, E, y, lse, dloss, vocab_perm)
+    _require_cuda(H, E, y, lse, dloss, vocab_perm, colmax)
     gdt = torch.float32 if fp32_grads else torch.bfloat16
     if segments:
         V = V if V is not None else int(segments[-1][1])
@@ -203,7 +204,7 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
     st = status if status is not None else torch.zeros(1, dtype=torch.int32, device=dev)
     rc = lib().cce_bwd(_ptr(H), _ptr(E) if not segments else None, _ptr(y), _ptr(lse), _ptr(dloss),
                        N, D, V, ignore_index, segarr, nseg, float(filter_eps), _ptr(vocab_perm),
-                       flags, _ptr(dH), None if segments else dEs[0].data_ptr(),
+                       _ptr(colmax), flags, _ptr(dH), None if segments else dEs[0].data_ptr(),
                        None if (segments or not kahan) else comps[0].data_ptr(),
                        _ptr(dbg), debug_rows, _ptr(ws), ws.numel(), _ptr(st), _stream_ptr(dev))
     _check(rc, "cce_bwd")

@@ -172,6 +172,7 @@ struct BwdPlan {
   // sparse backward (filtered gradients)
   int64_t nch_max, cap;
   size_t off_nzcnt, off_lists, off_colc, off_csorted, off_rowc, off_rsorted, off_scan, scan_bytes;
+  size_t off_tcmax, off_blkmin;  // tile-skip bounds
 };
 
 BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags) {
@@ -219,6 +220,8 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags) {
   // generous bound on cub's single-pass scan scratch (checked again at run time)
   p.scan_bytes = align_up(sizeof(int) * (size_t)(std::max<int64_t>(V, p.Npad) + 1) / 8 + (1u << 20));
   p.off_scan = o; o += p.scan_bytes;
+  p.off_tcmax = o; o += align_up(sizeof(float) * (size_t)(cdiv(V, BN) + CCE_MAX_SEGMENTS));
+  p.off_blkmin = o; o += align_up(sizeof(float) * (size_t)(p.Npad / BM));
   p.total = o;
   return p;
 }
@@ -446,7 +449,8 @@ int cce_fwd(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D
 
 int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, const float* dloss,
             int64_t N, int64_t D, int64_t V, int32_t ignore_index, const cce_segment* segs,
-            int32_t n_segs, float filter_eps, const int32_t* vocab_perm, uint32_t flags, void* dH,
+            int32_t n_segs, float filter_eps, const int32_t* vocab_perm, const float* colmax,
+            uint32_t flags, void* dH,
             void* dE, void* dE_comp, uint32_t* debug_keep, int64_t debug_rows, void* workspace,
             size_t workspace_bytes, int32_t* status, void* stream) {
   if (!sizes_ok(N, D, V)) return CCE_EINVAL;
@@ -532,6 +536,38 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   // non-zeros; the Kahan path stays on the deterministic dense route).
   // dH may take the sparse route whenever filtering is on; dE only when it is
   // filtered too (not CCE_FULL_DE).
+  // exact tile skip from the forward's column maxima (not for FullC, whose
+  // dE needs every entry)
+  const bool tile_skip = colmax != nullptr && filter_eps > 0.f && !full_de;
+  float* tile_cmax2 = at<float>(workspace, pl.off_tcmax);
+  float* blk_lse2min = at<float>(workspace, pl.off_blkmin);
+  int tile_off[CCE_MAX_SEGMENTS + 1];
+  tile_off[0] = 0;
+  for (int s = 0; s < sg.n; ++s) tile_off[s + 1] = tile_off[s] + (int)cdiv(table.s[s].n, BN);
+  if (tile_skip) {
+    SkipBoundParams bp;
+    memset(&bp, 0, sizeof(bp));
+    bp.colmax = colmax;
+    bp.vocab_perm = vocab_perm;
+    bp.n_segs = sg.n;
+    for (int s = 0; s < sg.n; ++s) {
+      bp.live_off[s] = table.s[s].live_off;
+      bp.n[s] = table.s[s].n;
+    }
+    for (int s = 0; s <= sg.n; ++s) bp.tile_off[s] = tile_off[s];
+    bp.tile_cmax2 = tile_cmax2;
+    bp.lse2_c = cp.lse2_c;
+    bp.dloss_c = cp.dloss_c;
+    bp.n_valid = cp.n_valid;
+    bp.n_blk = (int)(pl.Npad / BM);
+    bp.blk_lse2min = blk_lse2min;
+    const int64_t warps = tile_off[sg.n] + bp.n_blk;
+    {
+      TimedLaunch tl_(KC_AUX, st);
+      skip_bounds_kernel<<<(int)std::min<int64_t>(cdiv(warps, 8), sms * 8), 256, 0, st>>>(bp);
+    }
+    if (launched()) return CCE_ELAUNCH;
+  }
   bool sparse = filter_eps > 0.f && !kahan;
   for (int s = 0; s < sg.n; ++s) sparse = sparse && table.s[s].n < (1 << 29);
   const bool sparse_de = sparse && !full_de;
@@ -633,6 +669,9 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       gp.slab_flag = slab_flag + chunk;
       gp.repair = 0;
       gp.G_full = G_full;
+      gp.tile_cmax2 = tile_skip ? tile_cmax2 + tile_off[s] + c0 / BN : nullptr;
+      gp.blk_lse2min = blk_lse2min;
+      gp.skip_l2 = gp.l2eps - 1.0f / 16.0f;  // margin over fp32 differences of the two logits
       const int g_grid = (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct);
       if (int rc = full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
                            : launch_tc<GPolicy>(gp, g_grid, st, KC_G))

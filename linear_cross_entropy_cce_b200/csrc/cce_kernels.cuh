@@ -396,6 +396,14 @@ struct GParams {
   int dh_words;
   uint32_t* de_mask;
   int de_words;
+  // Exact tile skip: tile (mb, vt) is not recomputed when
+  //   tile_cmax2[vt] - blk_lse2min[mb] < skip_l2,
+  // the largest log2 softmax any of its entries can reach (from the
+  // forward's column maxima) staying below the keep threshold by a margin;
+  // only its one-hot entries are written.  tile_cmax2 null: no skip.
+  const float* tile_cmax2;   // per 256-wide tile of this chunk: max colmax * log2 e
+  const float* blk_lse2min;  // per 128-row block: min lse * log2 e (rows with dloss != 0)
+  float skip_l2;
   // The other mask buffer, cleared by the first launch of this chunk for the
   // next chunk (its last readers, the previous chunk's contractions, are done).
   uint32_t* mask_clear;
@@ -442,6 +450,9 @@ struct GPolicyT {
   static __device__ __forceinline__ bool active(const Params& p) {
     return !p.repair || (*p.nz_cnt > p.nz_cap && *p.slab_flag == 0);
   }
+  static __device__ __forceinline__ bool skip(const Params& p, int mb, int vt) {
+    return p.tile_cmax2 != nullptr && p.tile_cmax2[vt] - p.blk_lse2min[mb] < p.skip_l2;
+  }
 
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
@@ -459,11 +470,15 @@ struct GPolicyT {
   }
   static __device__ void producer(const Params& p, Engine& eng) {
     schedule(p, [&](int mb, int vt, int) {
+      if (skip(p, mb, vt)) return true;
       return eng.produce<false, false>(&p.mapA, &p.mapB, 0, mb * BM, 0, p.b_row0 + vt * BN, p.nkb);
     });
   }
   static __device__ void mma(const Params& p, Engine& eng) {
-    schedule(p, [&](int, int, int) { return eng.mma<false, false>(p.nkb); });
+    schedule(p, [&](int mb, int vt, int) {
+      if (skip(p, mb, vt)) return true;
+      return eng.mma<false, false>(p.nkb);
+    });
   }
   static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
     const int row = q * 32 + lane;
@@ -478,8 +493,10 @@ struct GPolicyT {
            i += gridDim.x * EPI_THREADS)
         p.mask_clear[i] = 0u;
     schedule(p, [&](int mb, int vt, int nv) {
-      uint32_t taddr;
-      if (!eng.epi_acquire(q, taddr)) return false;
+      // a skipped tile has no accumulator: no softmax entry is kept in it
+      const bool sk = skip(p, mb, vt);
+      uint32_t taddr = 0;
+      if (!sk && !eng.epi_acquire(q, taddr)) return false;
       const int jrow = mb * BM + row;
       const bool ok = jrow < nv;
       const float lse2 = ok ? p.lse2_c[jrow] : 0.f;
@@ -492,15 +509,20 @@ struct GPolicyT {
       uint32_t half_nz = 0;  // bit h: this row has a non-zero in tile columns 128h..128h+127
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(taddr + c * 32, r);
         // keep bits: softmax part retained (p >= eps, decided in base-2 log
         // space), then the non-zero set including the target's one-hot term
         uint32_t kb = 0;
+        if (sk) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float z2 = fmaf(__uint_as_float(r[j]), kLog2e, -lse2);
-          r[j] = __float_as_uint(z2);
-          kb |= (z2 >= p.l2eps ? 1u : 0u) << j;
+          for (int j = 0; j < 32; ++j) r[j] = 0u;
+        } else {
+          tmem_ld32(taddr + c * 32, r);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float z2 = fmaf(__uint_as_float(r[j]), kLog2e, -lse2);
+            r[j] = __float_as_uint(z2);
+            kb |= (z2 >= p.l2eps ? 1u : 0u) << j;
+          }
         }
         const int nvc = min(32, max(0, valid - c * 32));  // valid columns in this 32-chunk
         const uint32_t cm = (ok && dl != 0.f) ? (nvc == 32 ? 0xFFFFFFFFu : ((1u << nvc) - 1u)) : 0u;
@@ -601,7 +623,7 @@ struct GPolicyT {
           }
         }
       }
-      eng.epi_release(lane);
+      if (!sk) eng.epi_release(lane);
       return true;
     });
   }
@@ -838,6 +860,56 @@ struct DHPolicy {
     __syncwarp();
   }
 };
+
+// Bounds for the exact tile skip of the G producer.  One warp per output:
+//   tile_cmax2[tile_off[s] + t] = log2 e * max colmax over walk positions
+//     256t .. 256t+255 of segment s (through the vocabulary permutation);
+//   blk_lse2min[b] = min lse * log2 e over the valid compact rows of block b
+//     with a non-zero dloss (+inf if none).
+struct SkipBoundParams {
+  const float* colmax;     // [V_live], segment order
+  const int* vocab_perm;   // concatenated per-segment permutations, or null
+  int n_segs;
+  int live_off[MAX_SEGS], n[MAX_SEGS], tile_off[MAX_SEGS + 1];
+  float* tile_cmax2;
+  const float* lse2_c;
+  const float* dloss_c;
+  const int* n_valid;
+  int n_blk;
+  float* blk_lse2min;
+};
+
+__global__ void skip_bounds_kernel(const SkipBoundParams p) {
+  const int lane = threadIdx.x & 31;
+  const int n_tiles = p.tile_off[p.n_segs];
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < n_tiles + p.n_blk; w += nw) {
+    if (w < n_tiles) {
+      int s = 0;
+      while (s + 1 < p.n_segs && w >= p.tile_off[s + 1]) ++s;
+      const int t = w - p.tile_off[s];
+      float m = -INFINITY;
+      for (int k = lane; k < BN; k += 32) {
+        const int wl = t * BN + k;
+        if (wl >= p.n[s]) break;
+        const int v = p.vocab_perm ? p.vocab_perm[p.live_off[s] + wl] : wl;
+        m = fmaxf(m, p.colmax[p.live_off[s] + v]);
+      }
+      m = warp_max(m);
+      if (lane == 0) p.tile_cmax2[w] = m * kLog2e;
+    } else {
+      const int b = w - n_tiles;
+      const int nv = *p.n_valid;
+      float m = INFINITY;
+      for (int k = lane; k < BM; k += 32) {
+        const int j = b * BM + k;
+        if (j < nv && p.dloss_c[j] != 0.f) m = fminf(m, p.lse2_c[j]);
+      }
+      m = -warp_max(-m);
+      if (lane == 0) p.blk_lse2min[b] = m;
+    }
+  }
+}
 
 // inv[perm[k]] = k for one segment (perm and inv point at the segment's
 // slice of the concatenated live vocabulary; entries are segment-local).
