@@ -191,6 +191,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--filter", choices=["on", "off", "default"], default="default")
     ap.add_argument("--sort", choices=["on", "off", "default"], default="default")
+    ap.add_argument("--kahan", action="store_true",
+                    help="accumulate dE across steps with the Kahan-compensated bf16 path")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -236,6 +238,11 @@ def main():
     ws_s = torch.empty(cce.vocab_sort_workspace_size(N, V, nseg), dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     input_bytes = H.numel() * 2 + sum(s[2].numel() * 2 for s in segs) + y.numel() * 4
+    kahan_kw = {}
+    if a.kahan:  # running bf16 sum and compensation, kept across steps
+        S = [torch.zeros_like(t) for _, _, t in segs]
+        C = [torch.zeros_like(t) for _, _, t in segs]
+        kahan_kw = dict(kahan=True, dE_out=S[0] if single else S, dE_comp=C[0] if single else C)
 
     def step(Hd=H, segd=segs, yd=y):
         kw = dict(workspace=ws_f, status=status)
@@ -249,7 +256,7 @@ def main():
             perm = cce.vocab_sort(out[2], yd, V, x.ignore_index,
                                   segments=None if single else segd, workspace=ws_s)
         kw = dict(filter_eps=eps, vocab_perm=perm, colmax=out[2] if sort else None,
-                  workspace=ws_b, status=status)
+                  workspace=ws_b, status=status, **kahan_kw)
         if single:
             dH, dE, _ = cce.bwd(Hd, segd[0][2], yd, lse, dloss, x.ignore_index, **kw)
         else:
@@ -374,6 +381,7 @@ def main():
         "config": {"workload": wl.name, "N": N, "N_valid": n_valid, "D": D, "V": V,
                    "V_live": v_live, "segments": [list(s) for s in wl.segs()],
                    "logit_std": wl.logit_std, "filter_eps": eps, "vocab_sort": sort,
+                   "kahan_dE": bool(a.kahan),
                    "global_batch_tokens": N * world, "parallelism": f"dp{world} (independent batches)",
                    "l2": f"inputs larger than L2 (E = {sum(s[2].numel() for s in segs) * 2 / 2**20:.0f} MiB > 126 MiB)",
                    "tokens_per_s_valid_rows": round(n_valid * world / (ms_step / 1e3), 1)},
