@@ -60,6 +60,7 @@ extern "C" {
 #define CCE_KAHAN_DE 1u   /* dE += grad with a bf16 Kahan compensation buffer  */
 #define CCE_FP32_GRADS 2u /* dH and dE are written as fp32 instead of bf16     */
 #define CCE_FULL_DE 4u    /* filter only dH; the classifier gradient dE is full */
+#define CCE_VOCAB_SHARD 8u /* E is one rank's vocabulary shard (see cce_fwd_shard) */
 
 #define CCE_MAX_SEGMENTS 8
 
@@ -119,6 +120,34 @@ int cce_fwd(const void* H, const void* E, const int32_t* y,
             void* workspace, size_t workspace_bytes,
             int32_t* status, void* stream);
 
+/*
+ * Forward over one vocabulary shard (vocabulary-parallel cross-entropy).
+ * The live vocabulary given by E / segs is this rank's part of a vocabulary
+ * of V ids split across ranks.  Per row it writes
+ *   lse_part  the log-sum-exp over this shard's ids,
+ *   zy_part   the correct-token logit <h_i, e_{y_i}> if this shard holds
+ *             y_i, else 0.
+ * Combining the ranks is plain arithmetic: lse = log-add-exp of lse_part
+ * over ranks, z_y = sum of zy_part, loss = lse - z_y ("Cut Your Losses in
+ * Large-Vocabulary Language Models", first page §Contribution: the loss
+ * needs only the indexed logit and the log-sum-exp, and the log-sum-exp
+ * composes blockwise; research-map entry §Limitations: log-add-exp of
+ * partial results).  A target in [0, V) outside the shard is not an error
+ * here; targets outside [0, V) set CCE_STATUS_BADTARGET and give NaN.
+ * Ignored rows give 0 in both outputs.  Other arguments, the workspace
+ * (cce_fwd_workspace_size) and errors as for cce_fwd.
+ * The backward of a shard is cce_bwd with CCE_VOCAB_SHARD, the combined lse
+ * and the same shard: it returns this shard's dE rows (complete) and this
+ * shard's share of dH (to be summed over ranks); a target outside the shard
+ * adds no one-hot term.
+ */
+int cce_fwd_shard(const void* H, const void* E, const int32_t* y,
+                  int64_t N, int64_t D, int64_t V, int32_t ignore_index,
+                  const cce_segment* segs, int32_t n_segs,
+                  float* lse_part, float* zy_part, float* colmax,
+                  void* workspace, size_t workspace_bytes,
+                  int32_t* status, void* stream);
+
 /* Workspace bytes cce_bwd needs (0 on invalid sizes). */
 size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs,
                               uint32_t flags);
@@ -151,7 +180,9 @@ size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs,
  *            and of the research-map entry's §Approach, taken exactly.  The
  *            skip never changes which entries are kept.  A colmax that is not such a bound
  *            drops gradient entries.  NULL = no tile skip.
- *   flags    CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE.  CCE_FULL_DE keeps
+ *   flags    CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE | CCE_VOCAB_SHARD
+ *            (the backward of cce_fwd_shard: lse is the combined one, dH this
+ *            shard's share).  CCE_FULL_DE keeps
  *            the classifier gradient dE unfiltered while dH uses the filtered
  *            softmax (the "FullC" variant of "Cut Your Losses in
  *            Large-Vocabulary Language Models", research-map entry, §Key

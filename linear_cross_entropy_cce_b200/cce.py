@@ -18,10 +18,10 @@ LIB_PATH = os.path.join(_PKG, "libcce.so")
 
 CCE_OK, CCE_EINVAL, CCE_EWORKSPACE, CCE_ELAUNCH, CCE_EDEVICE = 0, 1, 2, 3, 4
 STATUS_BADTARGET, STATUS_TIMEOUT = 1, 2
-KAHAN_DE, FP32_GRADS, FULL_DE = 1, 2, 4
+KAHAN_DE, FP32_GRADS, FULL_DE, VOCAB_SHARD = 1, 2, 4, 8
 MAX_SEGMENTS = 8
 
-EXPORTS = ("cce_version", "cce_strerror", "cce_fwd_workspace_size", "cce_fwd",
+EXPORTS = ("cce_version", "cce_strerror", "cce_fwd_workspace_size", "cce_fwd", "cce_fwd_shard",
            "cce_bwd_workspace_size", "cce_bwd", "cce_vocab_sort_workspace_size",
            "cce_vocab_sort", "cce_launch_count", "cce_timing_enable", "cce_timing_read")
 # kernel classes for cce_timing_enable / cce_timing_read
@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
     L.cce_fwd.restype = ctypes.c_int
     L.cce_fwd.argtypes = [vp, vp, vp, i64, i64, i64, i32, ctypes.POINTER(Segment), i32,
                           vp, vp, vp, vp, sz, vp, vp]
+    L.cce_fwd_shard.restype = ctypes.c_int
+    L.cce_fwd_shard.argtypes = L.cce_fwd.argtypes
     L.cce_bwd_workspace_size.restype = sz
     L.cce_bwd_workspace_size.argtypes = [i64, i64, i64, i32, u32]
     L.cce_bwd.restype = ctypes.c_int
@@ -136,8 +138,12 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.
 def fwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, ignore_index: int = -100,
         segments: Optional[Sequence[SegSpec]] = None, V: Optional[int] = None,
         want_colmax: bool = False, workspace: Optional[torch.Tensor] = None,
-        status: Optional[torch.Tensor] = None):
-    """Per-row (loss, lse) fp32; optional colmax [V_live].  See cce_fwd."""
+        status: Optional[torch.Tensor] = None, shard: bool = False):
+    """Per-row (loss, lse) fp32; optional colmax [V_live].  See cce_fwd.
+
+    shard=True runs cce_fwd_shard instead and returns (zy_part, lse_part)
+    in place of (loss, lse): the correct-token logit when this shard holds
+    the target (else 0) and the log-sum-exp over this shard."""
     N, D = H.shape
     if segments:
         V = V if V is not None else int(segments[-1][1])
@@ -153,10 +159,11 @@ def fwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, ignore_inde
     segarr, nseg = _seg_array(segments)
     ws = _workspace(fwd_workspace_size(N, D, V, nseg), dev, workspace)
     st = status if status is not None else torch.zeros(1, dtype=torch.int32, device=dev)
-    rc = lib().cce_fwd(_ptr(H), _ptr(E) if not segments else None, _ptr(y), N, D, V, ignore_index,
-                       segarr, nseg, _ptr(loss), _ptr(lse), _ptr(colmax), _ptr(ws),
-                       ws.numel(), _ptr(st), _stream_ptr(dev))
-    _check(rc, "cce_fwd")
+    fn = lib().cce_fwd_shard if shard else lib().cce_fwd
+    rc = fn(_ptr(H), _ptr(E) if not segments else None, _ptr(y), N, D, V, ignore_index,
+            segarr, nseg, _ptr(lse) if shard else _ptr(loss), _ptr(loss) if shard else _ptr(lse),
+            _ptr(colmax), _ptr(ws), ws.numel(), _ptr(st), _stream_ptr(dev))
+    _check(rc, "cce_fwd_shard" if shard else "cce_fwd")
     if want_colmax:
         return loss, lse, colmax
     return loss, lse
@@ -166,7 +173,7 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
         dloss: torch.Tensor, ignore_index: int = -100,
         segments: Optional[Sequence[SegSpec]] = None, V: Optional[int] = None,
         filter_eps: float = 0.0, vocab_perm: Optional[torch.Tensor] = None,
-        colmax: Optional[torch.Tensor] = None, kahan: bool = False, fp32_grads: bool = False, full_de: bool = False,
+        colmax: Optional[torch.Tensor] = None, kahan: bool = False, shard: bool = False, fp32_grads: bool = False, full_de: bool = False,
         dE_out=None, dE_comp=None, debug_rows: int = 0,
         workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
     """Gradients (dH, dE) of sum_i dloss_i loss_i.  See cce_bwd.
@@ -196,7 +203,8 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
     if kahan:
         comps = list(dE_comp) if isinstance(dE_comp, (list, tuple)) else [dE_comp]
     dH = torch.empty((N, D), dtype=gdt, device=dev)
-    flags = (KAHAN_DE if kahan else 0) | (FP32_GRADS if fp32_grads else 0) | (FULL_DE if full_de else 0)
+    flags = ((KAHAN_DE if kahan else 0) | (FP32_GRADS if fp32_grads else 0) |
+             (FULL_DE if full_de else 0) | (VOCAB_SHARD if shard else 0))
     words = (V + 31) // 32
     dbg = torch.empty((debug_rows, words), dtype=torch.int32, device=dev) if debug_rows > 0 else None
     segarr, nseg = _seg_array(segments, dEs if segments else None, comps if segments else None)

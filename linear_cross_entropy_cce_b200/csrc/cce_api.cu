@@ -371,9 +371,15 @@ size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs, u
   return plan_bwd(N, D, V, flags).total;
 }
 
-int cce_fwd(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D, int64_t V,
-            int32_t ignore_index, const cce_segment* segs, int32_t n_segs, float* loss, float* lse,
-            float* colmax, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+}  // extern "C"
+
+namespace {
+// The forward of cce_fwd and of cce_fwd_shard (shard: `loss` receives the
+// correct-token logit, 0 for targets another shard owns).
+int fwd_impl(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D, int64_t V,
+             int32_t ignore_index, const cce_segment* segs, int32_t n_segs, float* loss, float* lse,
+             float* colmax, void* workspace, size_t workspace_bytes, int32_t* status, void* stream,
+             bool shard) {
   if (!sizes_ok(N, D, V)) return CCE_EINVAL;
   Segs sg;
   if (int rc = build_segs(E, V, segs, n_segs, sg)) return rc;
@@ -397,6 +403,8 @@ int cce_fwd(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D
   cp.pos_of_row = at<int>(workspace, pl.off_pos);
   cp.n_valid = at<int>(workspace, pl.off_nvalid);
   cp.status = status;
+  cp.shard = shard ? 1 : 0;
+  cp.V = V;
   __nv_bfloat16* Hc = at<__nv_bfloat16>(workspace, pl.off_hc);
   if (int rc = run_compaction(cp, H, pl.Npad, D, sms, Hc, st)) return rc;
 
@@ -435,6 +443,7 @@ int cce_fwd(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D
   fin.Npad = fp.Npad;
   fin.loss = loss;
   fin.lse = lse;
+  fin.shard = shard ? 1 : 0;
   {
     TimedLaunch tl_(KC_AUX, st);
     fwd_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, 8), sms * 8), 256, 0, st>>>(fin);
@@ -446,6 +455,24 @@ int cce_fwd(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D
   }
   return CCE_OK;
 }
+}  // namespace
+
+extern "C" {
+
+int cce_fwd(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D, int64_t V,
+            int32_t ignore_index, const cce_segment* segs, int32_t n_segs, float* loss, float* lse,
+            float* colmax, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  return fwd_impl(H, E, y, N, D, V, ignore_index, segs, n_segs, loss, lse, colmax, workspace,
+                  workspace_bytes, status, stream, false);
+}
+
+int cce_fwd_shard(const void* H, const void* E, const int32_t* y, int64_t N, int64_t D, int64_t V,
+                  int32_t ignore_index, const cce_segment* segs, int32_t n_segs, float* lse_part,
+                  float* zy_part, float* colmax, void* workspace, size_t workspace_bytes,
+                  int32_t* status, void* stream) {
+  return fwd_impl(H, E, y, N, D, V, ignore_index, segs, n_segs, zy_part, lse_part, colmax,
+                  workspace, workspace_bytes, status, stream, true);
+}
 
 int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, const float* dloss,
             int64_t N, int64_t D, int64_t V, int32_t ignore_index, const cce_segment* segs,
@@ -454,7 +481,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
             void* dE, void* dE_comp, uint32_t* debug_keep, int64_t debug_rows, void* workspace,
             size_t workspace_bytes, int32_t* status, void* stream) {
   if (!sizes_ok(N, D, V)) return CCE_EINVAL;
-  if (flags & ~(CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE)) return CCE_EINVAL;
+  if (flags & ~(CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE | CCE_VOCAB_SHARD)) return CCE_EINVAL;
   const bool full_de = flags & CCE_FULL_DE;
   const bool kahan = flags & CCE_KAHAN_DE;
   const bool fp32 = flags & CCE_FP32_GRADS;
@@ -505,6 +532,8 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   cp.pos_of_row = at<int>(workspace, pl.off_pos);
   cp.n_valid = at<int>(workspace, pl.off_nvalid);
   cp.status = status;
+  cp.shard = (flags & CCE_VOCAB_SHARD) ? 1 : 0;
+  cp.V = V;
   cp.lse = lse;
   cp.dloss = dloss;
   cp.inv_perm = inv;

@@ -89,6 +89,11 @@ struct CompactParams {
   int* pos_of_row;
   int* n_valid;
   int* status;
+  // Vocabulary shard: the live vocabulary is this rank's part of a larger
+  // one, so a target in [0, V) outside it is a valid row without a one-hot
+  // term here (another shard owns it); only targets outside [0, V) are bad.
+  int shard;
+  long long V;
   // backward extras (nullable)
   const float* lse;
   const float* dloss;
@@ -101,11 +106,14 @@ struct CompactParams {
 
 constexpr int COMPACT_THREADS = 1024;
 
+// 0 ignored, 1 valid with its target here, 2 bad target, 3 valid with its
+// target in another vocabulary shard.
 __device__ __forceinline__ int classify_row(const CompactParams& p, int i, int& seg) {
   const int y = p.y[i];
   if (y == p.ignore_index) return 0;
   seg = segment_of(p.segs, (long long)y);
-  return seg < 0 ? 2 : 1;
+  if (seg >= 0) return 1;
+  return (p.shard && y >= 0 && (long long)y < p.V) ? 3 : 2;
 }
 
 __global__ void __launch_bounds__(COMPACT_THREADS) compact_kernel(const CompactParams p) {
@@ -117,7 +125,8 @@ __global__ void __launch_bounds__(COMPACT_THREADS) compact_kernel(const CompactP
   int cnt = 0;
   for (int i = lo; i < hi; ++i) {
     int s;
-    cnt += classify_row(p, i, s) == 1;
+    const int st = classify_row(p, i, s);
+    cnt += st == 1 || st == 3;
   }
   int off, total;
   Scan(tmp).ExclusiveSum(cnt, off, total);
@@ -125,16 +134,20 @@ __global__ void __launch_bounds__(COMPACT_THREADS) compact_kernel(const CompactP
   for (int i = lo; i < hi; ++i) {
     int s = -1;
     const int st = classify_row(p, i, s);
-    if (st == 1) {
+    if (st == 1 || st == 3) {
       p.idx[off] = i;
       p.pos_of_row[i] = off;
       if (p.lse2_c) {
-        const int y = p.y[i];
-        const int loc = y - (int)p.segs.s[s].begin;
         p.lse2_c[off] = p.lse[i] * kLog2e;
         p.dloss_c[off] = p.dloss[i];
-        p.tseg[off] = s;
-        p.tpos[off] = p.inv_perm ? p.inv_perm[p.segs.s[s].live_off + loc] : loc;
+        if (st == 1) {
+          const int loc = p.y[i] - (int)p.segs.s[s].begin;
+          p.tseg[off] = s;
+          p.tpos[off] = p.inv_perm ? p.inv_perm[p.segs.s[s].live_off + loc] : loc;
+        } else {
+          p.tseg[off] = -1;  // no one-hot term in this shard
+          p.tpos[off] = -1;
+        }
       }
       ++off;
     } else {
@@ -301,8 +314,9 @@ struct FinParams {
   const float2* part;
   SegTable segs;
   int N, D, S, Npad;
-  float* loss;
-  float* lse;
+  float* loss;  // shard mode: the correct-token logit (0 if another shard owns the target)
+  float* lse;   // shard mode: the log-sum-exp over this shard's vocabulary
+  int shard;
 };
 
 __global__ void fwd_finalize_kernel(const FinParams p) {
@@ -328,12 +342,12 @@ __global__ void fwd_finalize_kernel(const FinParams p) {
     }
     acc = warp_sum(acc);
     const int y = p.y[i];
-    const int sg = segment_of(p.segs, (long long)y);
+    const int sg = segment_of(p.segs, (long long)y);  // < 0 only for another shard's target
     const uint4* h = reinterpret_cast<const uint4*>(p.H + (size_t)i * p.D);
-    const uint4* e = reinterpret_cast<const uint4*>(p.segs.s[sg].E +
-                                                    (size_t)(y - p.segs.s[sg].begin) * p.D);
+    const uint4* e = reinterpret_cast<const uint4*>(
+        sg >= 0 ? p.segs.s[sg].E + (size_t)(y - p.segs.s[sg].begin) * p.D : p.H);
     float dot = 0.f;
-    for (int v = lane; v < (p.D >> 3); v += 32) {
+    for (int v = lane; sg >= 0 && v < (p.D >> 3); v += 32) {
       const uint4 a = __ldg(h + v), b = __ldg(e + v);
       dot = fmaf(bf16lo(a.x), bf16lo(b.x), dot);
       dot = fmaf(bf16hi(a.x), bf16hi(b.x), dot);
@@ -348,7 +362,7 @@ __global__ void fwd_finalize_kernel(const FinParams p) {
     if (lane == 0) {
       const float l = (M + log2f(acc)) * kLn2;
       p.lse[i] = l;
-      p.loss[i] = l - dot;
+      p.loss[i] = p.shard ? dot : l - dot;
     }
   }
 }

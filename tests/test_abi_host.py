@@ -108,7 +108,7 @@ def test_bwd_rejects_bad_flags_and_missing_kahan_buffer():
     def call(flags=0, dE=16, comp=None):
         return L.cce_bwd(16, 16, 16, 16, 16, 4, 8, 10, -100, None, 0, 0.0, None, None, flags,
                          16, dE, comp, None, 0, 16, 1 << 30, 16, None)
-    assert call(flags=8) == cce.CCE_EINVAL
+    assert call(flags=16) == cce.CCE_EINVAL                      # unknown flag bit
     assert call(flags=cce.KAHAN_DE) == cce.CCE_EINVAL           # no compensation buffer
     assert call(flags=cce.KAHAN_DE | cce.FP32_GRADS, comp=16) == cce.CCE_EINVAL
     assert call(dE=None) == cce.CCE_EINVAL
