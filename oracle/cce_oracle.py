@@ -13,7 +13,9 @@ Sources (web pages, cited by title and section):
   [MAP] "Cut Your Losses in Large-Vocabulary Language Models" (research-map
         entry): §Approach, §Key results, §Limitations.
   [DE]  "The Defensive Edit: Chunking Cross-Entropy Loss After an OOM Wake-Up
-        Call": §The Trade-Off Analysis / §Assumptions (Assumption 2).
+        Call": §The OOM: A 12.2 GB Softmax Wall (the soft KL between a
+        student and a teacher softmax, computed in position chunks),
+        §The Trade-Off Analysis / §Assumptions (Assumption 2).
 
 What it computes.  The cross-entropy of row i is the log-sum-exp of its logits
 minus its correct-token logit, the logits being plain dot products
@@ -241,3 +243,66 @@ def kahan_reference(parts: Sequence[np.ndarray]) -> np.ndarray:
     for p in parts:
         acc += p
     return acc
+
+
+# ---------------------------------------------------------------------------
+# Soft-target KL ([DE] §The OOM: the KL divergence between the student and the
+# teacher softmax over the whole vocabulary, computed in position chunks).
+# Readings where the page is silent (each also listed in the design doc):
+#   * direction KL(p_t || p_s): the teacher distribution is the target;
+#   * temperature 1, no bias; p_s = softmax(H_s E_s^T), p_t = softmax(H_t E_t^T)
+#     (E_s and E_t may be the same head);
+#   * the teacher is a constant: gradients flow to H_s and E_s only, and
+#     d KL_i / d z_s,ij = p_s,ij - p_t,ij;
+#   * rows with row_mask == 0 have KL = 0 and no gradient;
+#   * the gradient filter drops entry (i, j) when both p_s,ij and p_t,ij are
+#     below filter_eps (its gradient is then below filter_eps in magnitude).
+
+def _kl_rows(Hs, Es64, Ht, Et64, r):
+    Zs = as_f64(Hs[r]) @ Es64.T
+    Zt = as_f64(Ht[r]) @ Et64.T
+    ls = logsumexp_rows(Zs)
+    lt = logsumexp_rows(Zt)
+    return Zs - ls[:, None], Zt - lt[:, None], ls, lt
+
+
+def kl_forward(Hs, Es, Ht, Et, row_mask=None, slice_rows: int = SLICE_ROWS):
+    """Per row (KL(p_t || p_s), lse_s, lse_t), fp64; masked rows give zeros."""
+    N = Hs.shape[0]
+    mask = np.ones(N, bool) if row_mask is None else np.asarray(row_mask) != 0
+    Es64, Et64 = as_f64(Es), as_f64(Et)
+    kl, ls_o, lt_o = np.zeros(N), np.zeros(N), np.zeros(N)
+    for s in range(0, N, slice_rows):
+        r = np.arange(s, min(N, s + slice_rows))
+        r = r[mask[r]]
+        if r.shape[0] == 0:
+            continue
+        log_ps, log_pt, ls, lt = _kl_rows(Hs, Es64, Ht, Et64, r)
+        kl[r] = np.sum(np.exp(log_pt) * (log_pt - log_ps), axis=1)
+        ls_o[r], lt_o[r] = ls, lt
+    return kl, ls_o, lt_o
+
+
+def kl_backward(Hs, Es, Ht, Et, dloss, row_mask=None, filter_eps: float = 0.0,
+                slice_rows: int = SLICE_ROWS):
+    """Gradients of sum_i dloss_i KL_i w.r.t. H_s and E_s (fp64)."""
+    N, D = Hs.shape
+    mask = np.ones(N, bool) if row_mask is None else np.asarray(row_mask) != 0
+    Es64, Et64 = as_f64(Es), as_f64(Et)
+    dloss = np.asarray(dloss, dtype=np.float64)
+    dH = np.zeros((N, D))
+    dE = np.zeros_like(Es64)
+    for s in range(0, N, slice_rows):
+        r = np.arange(s, min(N, s + slice_rows))
+        r = r[mask[r]]
+        if r.shape[0] == 0:
+            continue
+        log_ps, log_pt, _, _ = _kl_rows(Hs, Es64, Ht, Et64, r)
+        Ps, Pt = np.exp(log_ps), np.exp(log_pt)
+        G = Ps - Pt
+        if filter_eps > 0.0:
+            G = np.where((Ps < filter_eps) & (Pt < filter_eps), 0.0, G)
+        G *= dloss[r][:, None]
+        dH[r] = G @ Es64
+        dE += G.T @ as_f64(Hs[r])
+    return dH, dE

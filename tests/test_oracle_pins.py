@@ -317,3 +317,104 @@ def test_full_classifier_gradient_variant():
     cH, cE = oracle.backward(x.H, x.segments, x.y, 200, dl, IGN, filter_eps=eps, filter_dE=False)
     assert np.array_equal(cH, fH) and np.array_equal(cE[0], uE[0])
     assert not np.allclose(fE[0], uE[0], rtol=1e-9, atol=0) and not np.allclose(fH, uH, rtol=1e-9, atol=0)
+
+
+# ------------------------------------------------------------- soft-target KL
+def _kl_inputs(N=29, D=16, V=61, seed=3, std_s=2.0, std_t=3.0, shared=False):
+    rng = np.random.default_rng(seed)
+    Hs = rng.standard_normal((N, D))
+    Ht = rng.standard_normal((N, D))
+    Es = rng.standard_normal((V, D)) * std_s / math.sqrt(D)
+    Et = Es if shared else rng.standard_normal((V, D)) * std_t / math.sqrt(D)
+    return Hs, Es, Ht, Et
+
+
+def test_kl_matches_torch_kl_div_fp64():
+    """torch.nn.functional.kl_div (log targets) on the materialised logits,
+    fp64, is an independent implementation of KL(p_t || p_s)."""
+    Hs, Es, Ht, Et = _kl_inputs()
+    mask = np.ones(len(Hs), np.int32)
+    mask[[2, 11]] = 0
+    kl, ls, lt = oracle.kl_forward(Hs, Es, Ht, Et, mask)
+    zs = torch.from_numpy(Hs @ Es.T)
+    zt = torch.from_numpy(Ht @ Et.T)
+    ref = torch.nn.functional.kl_div(torch.log_softmax(zs, -1), torch.log_softmax(zt, -1),
+                                     reduction="none", log_target=True).sum(-1).numpy()
+    on = mask != 0
+    assert np.allclose(kl[on], ref[on], rtol=1e-12, atol=1e-14)
+    assert np.all(kl[~on] == 0) and np.all(ls[~on] == 0) and np.all(kl[on] >= 0)
+    assert np.allclose(ls[on], torch.logsumexp(zs, -1).numpy()[on], rtol=1e-14)
+    assert np.allclose(lt[on], torch.logsumexp(zt, -1).numpy()[on], rtol=1e-14)
+
+
+def test_kl_two_classes_is_bernoulli_kl():
+    """V = 2: KL between Bernoulli(q) and Bernoulli(p) in closed form, with
+    p = sigmoid of the logit difference."""
+    rng = np.random.default_rng(4)
+    Hs, Ht = rng.standard_normal((9, 3)), rng.standard_normal((9, 3))
+    Es, Et = rng.standard_normal((2, 3)), rng.standard_normal((2, 3))
+    kl, _, _ = oracle.kl_forward(Hs, Es, Ht, Et)
+    ps = 1.0 / (1.0 + np.exp(-(Hs @ (Es[0] - Es[1]))))
+    pt = 1.0 / (1.0 + np.exp(-(Ht @ (Et[0] - Et[1]))))
+    ref = pt * np.log(pt / ps) + (1 - pt) * np.log((1 - pt) / (1 - ps))
+    assert np.allclose(kl, ref, rtol=1e-10, atol=1e-15)
+
+
+def test_kl_of_identical_models_is_zero_with_zero_gradient():
+    Hs, Es, _, _ = _kl_inputs(shared=True)
+    kl, _, _ = oracle.kl_forward(Hs, Es, Hs, Es)
+    dH, dE = oracle.kl_backward(Hs, Es, Hs, Es, np.ones(len(Hs)))
+    assert np.all(kl == 0) and np.all(dH == 0) and np.all(dE == 0)
+
+
+def test_kl_gradient_central_differences_and_torch_autograd():
+    """d(sum_i dloss_i KL_i)/dH_s and /dE_s: central differences on a tiny
+    case, and torch autograd through kl_div with the teacher detached."""
+    Hs, Es, Ht, Et = _kl_inputs(N=3, D=4, V=6, seed=8)
+    dl = np.array([0.9, -0.4, 1.7])
+    dH, dE = oracle.kl_backward(Hs, Es, Ht, Et, dl)
+
+    def f(Hx, Ex):
+        return float(np.dot(dl, oracle.kl_forward(Hx, Ex, Ht, Et)[0]))
+
+    h = 1e-6
+    for arr, grad in ((Hs, dH), (Es, dE)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            old = arr[idx]
+            arr[idx] = old + h
+            fp = f(Hs, Es)
+            arr[idx] = old - h
+            fm = f(Hs, Es)
+            arr[idx] = old
+            num[idx] = (fp - fm) / (2 * h)
+        assert np.linalg.norm(num - grad) / np.linalg.norm(grad) <= 1e-7
+    Hs, Es, Ht, Et = _kl_inputs(N=17, D=8, V=40, seed=9)
+    dl = np.linspace(-1, 2, 17)
+    dH, dE = oracle.kl_backward(Hs, Es, Ht, Et, dl)
+    tH = torch.tensor(Hs, requires_grad=True)
+    tE = torch.tensor(Es, requires_grad=True)
+    zt = torch.from_numpy(Ht @ Et.T)
+    kl = torch.nn.functional.kl_div(torch.log_softmax(tH @ tE.T, -1), torch.log_softmax(zt, -1),
+                                    reduction="none", log_target=True).sum(-1)
+    (kl * torch.from_numpy(dl)).sum().backward()
+    assert np.allclose(tH.grad.numpy(), dH, rtol=1e-10, atol=1e-13)
+    assert np.allclose(tE.grad.numpy(), dE, rtol=1e-10, atol=1e-13)
+
+
+def test_kl_filter_drops_only_entries_small_in_both():
+    """With the filter, dH_s is G E_s where G keeps p_s - p_t unless both are
+    below eps: checked against the explicit rule on materialised softmaxes."""
+    Hs, Es, Ht, Et = _kl_inputs(N=21, D=12, V=300, seed=10, std_s=6.0, std_t=6.0)
+    eps = 2.0 ** -12
+    dl = np.full(21, 0.5)
+    dH, dE = oracle.kl_backward(Hs, Es, Ht, Et, dl, filter_eps=eps)
+    uH, _ = oracle.kl_backward(Hs, Es, Ht, Et, dl)
+    Ps = torch.softmax(torch.from_numpy(Hs @ Es.T), -1).numpy()
+    Pt = torch.softmax(torch.from_numpy(Ht @ Et.T), -1).numpy()
+    drop = (Ps < eps) & (Pt < eps)
+    assert drop.any() and (~drop).any()
+    G = np.where(drop, 0.0, Ps - Pt) * 0.5
+    assert np.allclose(dH, G @ Es, rtol=1e-10, atol=1e-15)
+    assert np.allclose(dE, G.T @ Hs, rtol=1e-10, atol=1e-15)
+    assert not np.allclose(dH, uH, rtol=1e-12, atol=0)
