@@ -213,6 +213,49 @@ int cce_bwd(const void* H, const void* E, const int32_t* y,
             void* workspace, size_t workspace_bytes,
             int32_t* status, void* stream);
 
+/*
+ * Soft-target KL divergence, never materialising either softmax ("The
+ * Defensive Edit: Chunking Cross-Entropy Loss After an OOM Wake-Up Call",
+ * §The OOM: A 12.2 GB Softmax Wall, where the soft KL between a student and a
+ * teacher softmax over the vocabulary is the loss that needed chunking).
+ * Per row i, with z_s = H_s E_s^T and z_t = H_t E_t^T (temperature 1; E_s and
+ * E_t may be the same pointer):
+ *   kl[i] = sum_j p_t,ij (log p_t,ij - log p_s,ij),  p = softmax(z).
+ *   Hs, Ht   [N, D] bf16 student / teacher rows.
+ *   Es, Et   [V, D] bf16 student / teacher classifiers.
+ *   row_mask optional [N] int32: rows with 0 are skipped (kl = lse = 0,
+ *            zero gradient); NULL = every row.
+ *   kl, lse_s, lse_t  [N] fp32 outputs (the two log-sum-exps feed the
+ *            backward).
+ * Workspace and errors as for cce_fwd.
+ */
+size_t cce_kl_fwd_workspace_size(int64_t N, int64_t D, int64_t V);
+int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
+               const int32_t* row_mask, int64_t N, int64_t D, int64_t V,
+               float* kl, float* lse_s, float* lse_t,
+               void* workspace, size_t workspace_bytes,
+               int32_t* status, void* stream);
+
+/*
+ * Backward of sum_i dloss_i kl_i with the teacher held constant: the
+ * gradients w.r.t. the student only, from G = dloss (p_s - p_t) through the
+ * same dE / dH contractions as cce_bwd:
+ *   dH = G E_s  ([N, D]),  dE = G^T H_s  ([V, D]).
+ *   lse_s, lse_t  the forward's outputs for the same inputs.
+ *   filter_eps  drops entry (i, j) when both p_s,ij and p_t,ij are below it
+ *            (its gradient is then smaller than filter_eps); <= 0 = off.
+ *   flags    CCE_FP32_GRADS and/or CCE_KAHAN_DE (with dE_comp) as for
+ *            cce_bwd; CCE_FULL_DE and CCE_VOCAB_SHARD are rejected.
+ * Workspace: cce_kl_bwd_workspace_size(); errors as for cce_bwd.
+ */
+size_t cce_kl_bwd_workspace_size(int64_t N, int64_t D, int64_t V, uint32_t flags);
+int cce_kl_bwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
+               const int32_t* row_mask, const float* lse_s, const float* lse_t,
+               const float* dloss, int64_t N, int64_t D, int64_t V,
+               float filter_eps, uint32_t flags, void* dH, void* dE, void* dE_comp,
+               void* workspace, size_t workspace_bytes,
+               int32_t* status, void* stream);
+
 /* Workspace bytes cce_vocab_sort needs. */
 size_t cce_vocab_sort_workspace_size(int64_t N, int64_t V, int32_t n_segs);
 

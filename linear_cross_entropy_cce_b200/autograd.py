@@ -84,3 +84,43 @@ def linear_cross_entropy(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Te
         n_valid = (y != ignore_index).sum()
         return per_row.sum() / n_valid
     raise ValueError(f"unknown reduction {reduction!r}")
+
+
+class _SoftTargetKL(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, Hs, Es, Ht, Et, row_mask, filter_eps):
+        kl, lse_s, lse_t = cce.kl_fwd(Hs, Es, Ht, Et, row_mask)
+        ctx.save_for_backward(Hs, Es, Ht, Et, lse_s, lse_t,
+                              row_mask if row_mask is not None else torch.empty(0))
+        ctx.meta = (filter_eps, row_mask is not None)
+        return kl
+
+    @staticmethod
+    def backward(ctx, grad_kl):
+        Hs, Es, Ht, Et, lse_s, lse_t, row_mask = ctx.saved_tensors
+        filter_eps, has_mask = ctx.meta
+        dH, dE = cce.kl_bwd(Hs, Es, Ht, Et, lse_s, lse_t, grad_kl.contiguous().to(torch.float32),
+                            row_mask if has_mask else None, filter_eps=filter_eps)
+        return dH.to(Hs.dtype), dE.to(Es.dtype), None, None, None, None
+
+
+def soft_target_kl(Hs: torch.Tensor, Es: torch.Tensor, Ht: torch.Tensor, Et: torch.Tensor,
+                   row_mask: Optional[torch.Tensor] = None, reduction: str = "mean",
+                   filter_eps: float = 2.0 ** -12) -> torch.Tensor:
+    """KL(p_teacher || p_student) per row with p = softmax(H E^T), never
+    materialising either softmax.  The teacher (Ht, Et) is a constant target:
+    gradients flow to Hs and Es only (pass the same tensor as Es and Et for a
+    shared head; only its student use is differentiated).  row_mask [N]
+    (nonzero = counted row) is optional; "mean" averages over counted rows.
+    filter_eps drops gradient entries where both probabilities are below it."""
+    if row_mask is not None and row_mask.dtype != torch.int32:
+        row_mask = row_mask.to(torch.int32)
+    per_row = _SoftTargetKL.apply(Hs, Es, Ht.detach(), Et.detach(), row_mask, float(filter_eps))
+    if reduction == "none":
+        return per_row
+    if reduction == "sum":
+        return per_row.sum()
+    if reduction == "mean":
+        n = Hs.shape[0] if row_mask is None else int((row_mask != 0).sum())
+        return per_row.sum() / n
+    raise ValueError(f"unknown reduction {reduction!r}")

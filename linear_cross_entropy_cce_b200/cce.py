@@ -23,7 +23,8 @@ MAX_SEGMENTS = 8
 
 EXPORTS = ("cce_version", "cce_strerror", "cce_fwd_workspace_size", "cce_fwd", "cce_fwd_shard",
            "cce_bwd_workspace_size", "cce_bwd", "cce_vocab_sort_workspace_size",
-           "cce_vocab_sort", "cce_launch_count", "cce_timing_enable", "cce_timing_read")
+           "cce_vocab_sort", "cce_launch_count", "cce_timing_enable", "cce_timing_read",
+           "cce_kl_fwd_workspace_size", "cce_kl_fwd", "cce_kl_bwd_workspace_size", "cce_kl_bwd")
 # kernel classes for cce_timing_enable / cce_timing_read
 KC_FWD, KC_G, KC_DE, KC_DH, KC_AUX, KC_SPARSE = 0, 1, 2, 3, 4, 5
 KC_NAMES = ("fwd_tile_stream", "bwd_g_producer", "bwd_dE_contraction", "bwd_dH_contraction", "aux",
@@ -63,6 +64,15 @@ def lib() -> ctypes.CDLL:
                           vp, vp, vp, vp, sz, vp, vp]
     L.cce_fwd_shard.restype = ctypes.c_int
     L.cce_fwd_shard.argtypes = L.cce_fwd.argtypes
+    L.cce_kl_fwd_workspace_size.restype = sz
+    L.cce_kl_fwd_workspace_size.argtypes = [i64, i64, i64]
+    L.cce_kl_fwd.restype = ctypes.c_int
+    L.cce_kl_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp, sz, vp, vp]
+    L.cce_kl_bwd_workspace_size.restype = sz
+    L.cce_kl_bwd_workspace_size.argtypes = [i64, i64, i64, u32]
+    L.cce_kl_bwd.restype = ctypes.c_int
+    L.cce_kl_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, fp, u32, vp, vp, vp,
+                             vp, sz, vp, vp]
     L.cce_bwd_workspace_size.restype = sz
     L.cce_bwd_workspace_size.argtypes = [i64, i64, i64, i32, u32]
     L.cce_bwd.restype = ctypes.c_int
@@ -256,3 +266,49 @@ def bf16_from_bits(bits, device) -> torch.Tensor:
     import numpy as np
     t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
     return t.to(device).view(torch.bfloat16)
+
+
+def kl_fwd(Hs: torch.Tensor, Es: torch.Tensor, Ht: torch.Tensor, Et: torch.Tensor,
+           row_mask: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+           status: Optional[torch.Tensor] = None):
+    """Per-row (KL(p_t || p_s), lse_s, lse_t) fp32.  See cce_kl_fwd."""
+    N, D = Hs.shape
+    V = int(Es.shape[0])
+    _require_cuda(Hs, Es, Ht, Et, row_mask)
+    dev = Hs.device
+    kl = torch.empty(N, dtype=torch.float32, device=dev)
+    ls = torch.empty(N, dtype=torch.float32, device=dev)
+    lt = torch.empty(N, dtype=torch.float32, device=dev)
+    ws = _workspace(int(lib().cce_kl_fwd_workspace_size(N, D, V)), dev, workspace)
+    st = status if status is not None else torch.zeros(1, dtype=torch.int32, device=dev)
+    rc = lib().cce_kl_fwd(_ptr(Hs), _ptr(Es), _ptr(Ht), _ptr(Et), _ptr(row_mask), N, D, V,
+                          _ptr(kl), _ptr(ls), _ptr(lt), _ptr(ws), ws.numel(), _ptr(st),
+                          _stream_ptr(dev))
+    _check(rc, "cce_kl_fwd")
+    return kl, ls, lt
+
+
+def kl_bwd(Hs: torch.Tensor, Es: torch.Tensor, Ht: torch.Tensor, Et: torch.Tensor,
+           lse_s: torch.Tensor, lse_t: torch.Tensor, dloss: torch.Tensor,
+           row_mask: Optional[torch.Tensor] = None, filter_eps: float = 0.0,
+           fp32_grads: bool = False, kahan: bool = False, dE_out=None, dE_comp=None,
+           workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
+    """Student gradients (dH, dE) of sum_i dloss_i KL_i.  See cce_kl_bwd."""
+    N, D = Hs.shape
+    V = int(Es.shape[0])
+    _require_cuda(Hs, Es, Ht, Et, lse_s, lse_t, dloss, row_mask)
+    dev = Hs.device
+    gdt = torch.float32 if fp32_grads else torch.bfloat16
+    if kahan and (dE_out is None or dE_comp is None):
+        raise CCEError("kahan accumulation needs dE_out and dE_comp")
+    dE = dE_out if dE_out is not None else torch.empty((V, D), dtype=gdt, device=dev)
+    dH = torch.empty((N, D), dtype=gdt, device=dev)
+    flags = (KAHAN_DE if kahan else 0) | (FP32_GRADS if fp32_grads else 0)
+    ws = _workspace(int(lib().cce_kl_bwd_workspace_size(N, D, V, flags)), dev, workspace)
+    st = status if status is not None else torch.zeros(1, dtype=torch.int32, device=dev)
+    rc = lib().cce_kl_bwd(_ptr(Hs), _ptr(Es), _ptr(Ht), _ptr(Et), _ptr(row_mask), _ptr(lse_s),
+                          _ptr(lse_t), _ptr(dloss), N, D, V, float(filter_eps), flags, _ptr(dH),
+                          _ptr(dE), _ptr(dE_comp) if kahan else None, _ptr(ws), ws.numel(),
+                          _ptr(st), _stream_ptr(dev))
+    _check(rc, "cce_kl_bwd")
+    return dH, dE

@@ -16,6 +16,7 @@
 
 #include "../../include/cce.h"
 #include "cce_kernels.cuh"
+#include "cce_kl.cuh"
 
 using namespace cce;
 
@@ -162,6 +163,31 @@ FwdPlan plan_fwd(int64_t N, int64_t D, int64_t V, int32_t n_segs) {
   return p;
 }
 
+// ------------------------------------------------------ soft-target KL plan
+struct KLFwdPlan {
+  int64_t Npad;
+  int T_v, tpi, S;
+  size_t off_nvalid, off_idx, off_pos, off_hs, off_ht, off_part, total;
+};
+
+KLFwdPlan plan_kl_fwd(int64_t N, int64_t D, int64_t V) {
+  KLFwdPlan p;
+  p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
+  p.T_v = (int)cdiv(V, BN);
+  const int64_t num_mb = p.Npad / BM;
+  p.tpi = (int)std::min<int64_t>(16, std::max<int64_t>(2, num_mb * p.T_v / (kPlanSMs * 24)));
+  p.S = (int)cdiv(p.T_v, p.tpi);
+  size_t o = 0;
+  p.off_nvalid = o; o += align_up(16);
+  p.off_idx = o; o += align_up(sizeof(int) * (size_t)std::max<int64_t>(N, 1));
+  p.off_pos = o; o += align_up(sizeof(int) * (size_t)std::max<int64_t>(N, 1));
+  p.off_hs = o; o += align_up((size_t)p.Npad * D * 2);
+  p.off_ht = o; o += align_up((size_t)p.Npad * D * 2);
+  p.off_part = o; o += align_up((size_t)p.S * 5 * p.Npad * sizeof(float));
+  p.total = o;
+  return p;
+}
+
 // ----------------------------------------------------------- backward plan
 struct BwdPlan {
   int64_t Npad, Vc;
@@ -173,9 +199,10 @@ struct BwdPlan {
   int64_t nch_max, cap;
   size_t off_nzcnt, off_lists, off_colc, off_csorted, off_rowc, off_rsorted, off_scan, scan_bytes;
   size_t off_tcmax, off_blkmin;  // tile-skip bounds
+  size_t off_htc, off_lt2;       // soft-target KL: teacher rows and lse
 };
 
-BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags) {
+BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = false) {
   BwdPlan p;
   p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
   // Vocabulary chunk width: an L2-sized slab, widened so that the dE
@@ -222,6 +249,8 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags) {
   p.off_scan = o; o += p.scan_bytes;
   p.off_tcmax = o; o += align_up(sizeof(float) * (size_t)(cdiv(V, BN) + CCE_MAX_SEGMENTS));
   p.off_blkmin = o; o += align_up(sizeof(float) * (size_t)(p.Npad / BM));
+  p.off_htc = o; o += kl ? align_up((size_t)p.Npad * D * 2) : 0;
+  p.off_lt2 = o; o += kl ? align_up(sizeof(float) * (size_t)std::max<int64_t>(N, 1)) : 0;
   p.total = o;
   return p;
 }
@@ -474,14 +503,27 @@ int cce_fwd_shard(const void* H, const void* E, const int32_t* y, int64_t N, int
                   workspace, workspace_bytes, status, stream, true);
 }
 
-int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, const float* dloss,
+}  // extern "C"
+
+namespace {
+// Soft-target KL extras of the shared backward: the teacher's rows, head and
+// lse.  With them, y is only a row mask (0 = dropped row, or NULL) and G is
+// dloss (p_s - p_t) on the student (H, E).
+struct KLArgs {
+  const void* Ht;
+  const void* Et;
+  const float* lse_t;
+};
+
+int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, const float* dloss,
             int64_t N, int64_t D, int64_t V, int32_t ignore_index, const cce_segment* segs,
             int32_t n_segs, float filter_eps, const int32_t* vocab_perm, const float* colmax,
             uint32_t flags, void* dH,
             void* dE, void* dE_comp, uint32_t* debug_keep, int64_t debug_rows, void* workspace,
-            size_t workspace_bytes, int32_t* status, void* stream) {
+            size_t workspace_bytes, int32_t* status, void* stream, const KLArgs* kl) {
   if (!sizes_ok(N, D, V)) return CCE_EINVAL;
   if (flags & ~(CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE | CCE_VOCAB_SHARD)) return CCE_EINVAL;
+  if (kl && (flags & (CCE_FULL_DE | CCE_VOCAB_SHARD))) return CCE_EINVAL;
   const bool full_de = flags & CCE_FULL_DE;
   const bool kahan = flags & CCE_KAHAN_DE;
   const bool fp32 = flags & CCE_FP32_GRADS;
@@ -500,9 +542,11 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   }
   if (debug_keep && (debug_rows < 0 || debug_rows > N)) return CCE_EINVAL;
   if (N == 0) return CCE_OK;
-  if (!H || !y || !lse || !dloss || !dH || !status || !aligned16(H) || !aligned16(dH))
+  if (!H || (!y && !kl) || !lse || !dloss || !dH || !status || !aligned16(H) || !aligned16(dH))
     return CCE_EINVAL;
-  const BwdPlan pl = plan_bwd(N, D, V, flags);
+  if (kl && (!kl->Ht || !kl->Et || !kl->lse_t || !aligned16(kl->Ht) || !aligned16(kl->Et)))
+    return CCE_EINVAL;
+  const BwdPlan pl = plan_bwd(N, D, V, flags, kl != nullptr);
   if (!workspace || workspace_bytes < pl.total) return CCE_EWORKSPACE;
   const int sms = device_sms();
   if (sms <= 0 || !encode_fn()) return CCE_EDEVICE;
@@ -541,8 +585,23 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   cp.dloss_c = at<float>(workspace, pl.off_dl);
   cp.tseg = at<int>(workspace, pl.off_tseg);
   cp.tpos = at<int>(workspace, pl.off_tpos);
+  if (kl) {
+    cp.no_target = 1;
+    cp.ignore_index = 0;
+    cp.lse_t = kl->lse_t;
+    cp.lt2_c = at<float>(workspace, pl.off_lt2);
+  }
   __nv_bfloat16* Hc = at<__nv_bfloat16>(workspace, pl.off_hc);
   if (int rc = run_compaction(cp, H, pl.Npad, D, sms, Hc, st)) return rc;
+  __nv_bfloat16* Ht_c = kl ? at<__nv_bfloat16>(workspace, pl.off_htc) : nullptr;
+  if (kl) {
+    {
+      TimedLaunch tl_(KC_AUX, st);
+      gather_rows_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(kl->Ht), cp.idx,
+                                                  cp.n_valid, (int)pl.Npad, (int)D, Ht_c);
+    }
+    if (launched()) return CCE_ELAUNCH;
+  }
   float* dH_acc = at<float>(workspace, pl.off_dh);
   if (cudaMemsetAsync(dH_acc, 0, (size_t)pl.Npad * D * 4, st) != cudaSuccess) return CCE_ELAUNCH;
   const int words = (int)cdiv(V, 32);
@@ -567,7 +626,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   // filtered too (not CCE_FULL_DE).
   // exact tile skip from the forward's column maxima (not for FullC, whose
   // dE needs every entry)
-  const bool tile_skip = colmax != nullptr && filter_eps > 0.f && !full_de;
+  const bool tile_skip = colmax != nullptr && filter_eps > 0.f && !full_de && !kl;
   float* tile_cmax2 = at<float>(workspace, pl.off_tcmax);
   float* blk_lse2min = at<float>(workspace, pl.off_blkmin);
   int tile_off[CCE_MAX_SEGMENTS + 1];
@@ -626,6 +685,11 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
   memset(&ep, 0, sizeof(ep));
   memset(&hp, 0, sizeof(hp));
   if (!make_map(&gp.mapA, Hc, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
+  if (kl) {
+    if (!make_map(&gp.mapA2, Ht_c, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
+    if (!make_map(&gp.mapB2, kl->Et, D, V, D, BK, BN)) return CCE_ELAUNCH;
+    gp.lt2_c = cp.lt2_c;
+  }
   if (!make_map(&ep.mapA, full_de ? G_full : G, Vc, pl.Npad, Vc, 64, 64)) return CCE_ELAUNCH;
   if (!make_map(&ep.mapB, Hc, D, pl.Npad, D, 64, 64)) return CCE_ELAUNCH;
   if (!make_map(&hp.mapA, G, Vc, pl.Npad, Vc, BK, BM)) return CCE_ELAUNCH;
@@ -702,13 +766,15 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
       gp.blk_lse2min = blk_lse2min;
       gp.skip_l2 = gp.l2eps - 1.0f / 16.0f;  // margin over fp32 differences of the two logits
       const int g_grid = (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct);
-      if (int rc = full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
-                           : launch_tc<GPolicy>(gp, g_grid, st, KC_G))
+      if (int rc = kl ? launch_tc<GPolicyKL>(gp, g_grid, st, KC_G)
+                      : full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
+                                : launch_tc<GPolicy>(gp, g_grid, st, KC_G))
         return rc;
       if (sparse) {  // recompute with the dense fallback if the chunk was mispredicted
         gp.repair = 1;
-        if (int rc = full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
-                             : launch_tc<GPolicy>(gp, g_grid, st, KC_G))
+        if (int rc = kl ? launch_tc<GPolicyKL>(gp, g_grid, st, KC_G)
+                        : full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
+                                  : launch_tc<GPolicy>(gp, g_grid, st, KC_G))
           return rc;
       }
       // step 2: dE rows of this chunk (chunks on the sparse route: after the loop)
@@ -844,6 +910,112 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
         cp.pos_of_row, N, (int)D, dH, fp32 ? 1 : 0);
   }
   return launched();
+}
+
+}  // namespace
+
+extern "C" {
+
+int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, const float* dloss,
+            int64_t N, int64_t D, int64_t V, int32_t ignore_index, const cce_segment* segs,
+            int32_t n_segs, float filter_eps, const int32_t* vocab_perm, const float* colmax,
+            uint32_t flags, void* dH, void* dE, void* dE_comp, uint32_t* debug_keep,
+            int64_t debug_rows, void* workspace, size_t workspace_bytes, int32_t* status,
+            void* stream) {
+  return bwd_impl(H, E, y, lse, dloss, N, D, V, ignore_index, segs, n_segs, filter_eps, vocab_perm,
+                  colmax, flags, dH, dE, dE_comp, debug_keep, debug_rows, workspace,
+                  workspace_bytes, status, stream, nullptr);
+}
+
+// ------------------------------------------------------------ soft-target KL
+size_t cce_kl_fwd_workspace_size(int64_t N, int64_t D, int64_t V) {
+  if (!sizes_ok(N, D, V)) return 0;
+  return plan_kl_fwd(N, D, V).total;
+}
+
+int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
+               const int32_t* row_mask, int64_t N, int64_t D, int64_t V, float* kl, float* lse_s,
+               float* lse_t, void* workspace, size_t workspace_bytes, int32_t* status,
+               void* stream) {
+  if (!sizes_ok(N, D, V)) return CCE_EINVAL;
+  if (N == 0) return CCE_OK;
+  if (!Hs || !Es || !Ht || !Et || !kl || !lse_s || !lse_t || !status || !aligned16(Hs) ||
+      !aligned16(Es) || !aligned16(Ht) || !aligned16(Et))
+    return CCE_EINVAL;
+  const KLFwdPlan pl = plan_kl_fwd(N, D, V);
+  if (!workspace || workspace_bytes < pl.total) return CCE_EWORKSPACE;
+  const int sms = device_sms();
+  if (sms <= 0 || !encode_fn()) return CCE_EDEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  CompactParams cp;
+  memset(&cp, 0, sizeof(cp));
+  cp.y = row_mask;
+  cp.N = (int)N;
+  cp.ignore_index = 0;
+  cp.no_target = 1;
+  cp.idx = at<int>(workspace, pl.off_idx);
+  cp.pos_of_row = at<int>(workspace, pl.off_pos);
+  cp.n_valid = at<int>(workspace, pl.off_nvalid);
+  cp.status = status;
+  __nv_bfloat16* Hs_c = at<__nv_bfloat16>(workspace, pl.off_hs);
+  __nv_bfloat16* Ht_c = at<__nv_bfloat16>(workspace, pl.off_ht);
+  if (int rc = run_compaction(cp, Hs, pl.Npad, D, sms, Hs_c, st)) return rc;
+  {
+    TimedLaunch tl_(KC_AUX, st);
+    gather_rows_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(Ht), cp.idx,
+                                                cp.n_valid, (int)pl.Npad, (int)D, Ht_c);
+  }
+  if (launched()) return CCE_ELAUNCH;
+
+  KLFwdParams kp;
+  memset(&kp, 0, sizeof(kp));
+  if (!make_map(&kp.mapAs, Hs_c, D, pl.Npad, D, BK, BM) ||
+      !make_map(&kp.mapAt, Ht_c, D, pl.Npad, D, BK, BM) ||
+      !make_map(&kp.mapBs, Es, D, V, D, BK, BN) || !make_map(&kp.mapBt, Et, D, V, D, BK, BN))
+    return CCE_ELAUNCH;
+  kp.V = (int)V;
+  kp.T_v = pl.T_v;
+  kp.tpi = pl.tpi;
+  kp.S = pl.S;
+  kp.Npad = (int)pl.Npad;
+  kp.nkb = (int)cdiv(D, BK);
+  kp.n_valid = cp.n_valid;
+  kp.part = at<float>(workspace, pl.off_part);
+  kp.status = status;
+  const int64_t items = (pl.Npad / BM) * pl.S;
+  if (int rc = launch_tc<KLFwdPolicy>(kp, (int)std::min<int64_t>(sms, items), st, KC_FWD))
+    return rc;
+  KLFinParams fin;
+  fin.pos_of_row = cp.pos_of_row;
+  fin.part = kp.part;
+  fin.N = (int)N;
+  fin.S = pl.S;
+  fin.Npad = (int)pl.Npad;
+  fin.kl = kl;
+  fin.lse_s = lse_s;
+  fin.lse_t = lse_t;
+  {
+    TimedLaunch tl_(KC_AUX, st);
+    kl_finalize_kernel<<<(int)std::min<int64_t>(cdiv(N, 8), sms * 8), 256, 0, st>>>(fin);
+  }
+  return launched();
+}
+
+size_t cce_kl_bwd_workspace_size(int64_t N, int64_t D, int64_t V, uint32_t flags) {
+  if (!sizes_ok(N, D, V)) return 0;
+  return plan_bwd(N, D, V, flags, true).total;
+}
+
+int cce_kl_bwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
+               const int32_t* row_mask, const float* lse_s, const float* lse_t,
+               const float* dloss, int64_t N, int64_t D, int64_t V, float filter_eps,
+               uint32_t flags, void* dH, void* dE, void* dE_comp, void* workspace,
+               size_t workspace_bytes, int32_t* status, void* stream) {
+  const KLArgs a{Ht, Et, lse_t};
+  return bwd_impl(Hs, Es, row_mask, lse_s, dloss, N, D, V, 0, nullptr, 0, filter_eps, nullptr,
+                  nullptr, flags, dH, dE, dE_comp, nullptr, 0, workspace, workspace_bytes, status,
+                  stream, &a);
 }
 
 

@@ -300,6 +300,27 @@ struct Engine {
     if (lane == 0) mbar_arrive(smem_u32(&ctl->tempty[acc]));
     ++tcount;
   }
+  // ---- epilogue over a pair of tiles (t, t+1) held at once, one in each
+  // accumulator (used when a work unit computes two products of the same
+  // shape, e.g. teacher and student logits).  The MMA of the next pair waits
+  // until both are released, so the pair's epilogue does not overlap it.
+  __device__ __forceinline__ bool epi_acquire2(int quarter, uint32_t& ta, uint32_t& tb) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int t = tcount + k;
+      if (!wait_parity(smem_u32(&ctl->tfull[t & 1]), ((uint32_t)t >> 1) & 1u, abort_flag(), status))
+        return false;
+    }
+    tc_fence_after();
+    const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
+    ta = tmem + (tcount & 1) * BN + lanes;
+    tb = tmem + ((tcount + 1) & 1) * BN + lanes;
+    return true;
+  }
+  __device__ __forceinline__ void epi_release2(int lane) {
+    epi_release(lane);
+    epi_release(lane);
+  }
 };
 
 // Bounded wait that ignores the abort flag (used only while draining).

@@ -94,6 +94,10 @@ struct CompactParams {
   // term here (another shard owns it); only targets outside [0, V) are bad.
   int shard;
   long long V;
+  // No targets (soft-target KL): y, if given, is only a row mask (rows with
+  // y == ignore_index are dropped), and every other row is valid without a
+  // one-hot term.
+  int no_target;
   // backward extras (nullable)
   const float* lse;
   const float* dloss;
@@ -102,6 +106,8 @@ struct CompactParams {
   float* dloss_c;
   int* tseg;
   int* tpos;
+  const float* lse_t;  // teacher lse (KL), or null
+  float* lt2_c;
 };
 
 constexpr int COMPACT_THREADS = 1024;
@@ -109,8 +115,10 @@ constexpr int COMPACT_THREADS = 1024;
 // 0 ignored, 1 valid with its target here, 2 bad target, 3 valid with its
 // target in another vocabulary shard.
 __device__ __forceinline__ int classify_row(const CompactParams& p, int i, int& seg) {
+  if (p.y == nullptr) return 3;
   const int y = p.y[i];
   if (y == p.ignore_index) return 0;
+  if (p.no_target) return 3;
   seg = segment_of(p.segs, (long long)y);
   if (seg >= 0) return 1;
   return (p.shard && y >= 0 && (long long)y < p.V) ? 3 : 2;
@@ -140,6 +148,7 @@ __global__ void __launch_bounds__(COMPACT_THREADS) compact_kernel(const CompactP
       if (p.lse2_c) {
         p.lse2_c[off] = p.lse[i] * kLog2e;
         p.dloss_c[off] = p.dloss[i];
+        if (p.lt2_c) p.lt2_c[off] = p.lse_t[i] * kLog2e;
         if (st == 1) {
           const int loc = p.y[i] - (int)p.segs.s[s].begin;
           p.tseg[off] = s;
@@ -440,6 +449,12 @@ struct GParams {
   // values that dH reads.  Written by the first launch of a chunk, not by
   // its repair.
   __nv_bfloat16* G_full;
+  // Soft-target KL (GPolicyT<false, true> only): the teacher's rows and
+  // classifier, and its lse * log2 e per compact row.  G = dloss (p_s - p_t),
+  // an entry kept when either probability reaches the threshold.
+  CUtensorMap mapA2;  // H_t,c [Npad, D], box {64, 128}
+  CUtensorMap mapB2;  // E_t rows, K-major, box {64, 256}
+  const float* lt2_c;
   // optional per-element keep bits of original rows < debug_rows
   uint32_t* debug_keep;
   int debug_rows;
@@ -450,7 +465,7 @@ struct GParams {
   int* status;
 };
 
-template <bool FULL>
+template <bool FULL, bool KL = false>
 struct GPolicyT {
   using Params = GParams;
   static constexpr int EXTRA_SMEM = 0;
@@ -485,12 +500,20 @@ struct GPolicyT {
   static __device__ void producer(const Params& p, Engine& eng) {
     schedule(p, [&](int mb, int vt, int) {
       if (skip(p, mb, vt)) return true;
+      if constexpr (KL) {  // teacher tile first: it lands in the even accumulator
+        if (!eng.produce<false, false>(&p.mapA2, &p.mapB2, 0, mb * BM, 0, p.b_row0 + vt * BN,
+                                       p.nkb))
+          return false;
+      }
       return eng.produce<false, false>(&p.mapA, &p.mapB, 0, mb * BM, 0, p.b_row0 + vt * BN, p.nkb);
     });
   }
   static __device__ void mma(const Params& p, Engine& eng) {
     schedule(p, [&](int mb, int vt, int) {
       if (skip(p, mb, vt)) return true;
+      if constexpr (KL) {
+        if (!eng.mma<false, false>(p.nkb)) return false;
+      }
       return eng.mma<false, false>(p.nkb);
     });
   }
@@ -509,11 +532,18 @@ struct GPolicyT {
     schedule(p, [&](int mb, int vt, int nv) {
       // a skipped tile has no accumulator: no softmax entry is kept in it
       const bool sk = skip(p, mb, vt);
-      uint32_t taddr = 0;
-      if (!sk && !eng.epi_acquire(q, taddr)) return false;
+      uint32_t taddr = 0, tteach = 0;
+      if (!sk) {
+        if constexpr (KL) {
+          if (!eng.epi_acquire2(q, tteach, taddr)) return false;
+        } else {
+          if (!eng.epi_acquire(q, taddr)) return false;
+        }
+      }
       const int jrow = mb * BM + row;
       const bool ok = jrow < nv;
       const float lse2 = ok ? p.lse2_c[jrow] : 0.f;
+      const float lt2 = (KL && ok) ? p.lt2_c[jrow] : 0.f;
       const float dl = ok ? p.dloss_c[jrow] : 0.f;
       const int tcol = (ok && p.tseg[jrow] == p.seg) ? p.tpos[jrow] - p.c0 - vt * BN : -1;
       const int valid = p.chunk_valid - vt * BN;  // valid columns of this tile
@@ -523,21 +553,37 @@ struct GPolicyT {
       uint32_t half_nz = 0;  // bit h: this row has a non-zero in tile columns 128h..128h+127
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
+        uint32_t rt[KL ? 32 : 1];  // teacher log2 softmax (KL)
         // keep bits: softmax part retained (p >= eps, decided in base-2 log
-        // space), then the non-zero set including the target's one-hot term
+        // space; for KL either distribution's), then the non-zero set
+        // including the target's one-hot term
         uint32_t kb = 0;
         if (sk) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = 0u;
         } else {
           tmem_ld32(taddr + c * 32, r);
+          if constexpr (KL) tmem_ld32(tteach + c * 32, rt);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float z2 = fmaf(__uint_as_float(r[j]), kLog2e, -lse2);
             r[j] = __float_as_uint(z2);
-            kb |= (z2 >= p.l2eps ? 1u : 0u) << j;
+            bool keep = z2 >= p.l2eps;
+            if constexpr (KL) {
+              const float t2 = fmaf(__uint_as_float(rt[j]), kLog2e, -lt2);
+              rt[j] = __float_as_uint(t2);
+              keep = keep || t2 >= p.l2eps;
+            }
+            kb |= (keep ? 1u : 0u) << j;
           }
         }
+        // softmax part of G at column j (before dloss): p_ij, or p_s - p_t
+        auto pval = [&](int j) {
+          if constexpr (KL)
+            return ex2_approx(__uint_as_float(r[j])) - ex2_approx(__uint_as_float(rt[j]));
+          else
+            return ex2_approx(__uint_as_float(r[j]));
+        };
         const int nvc = min(32, max(0, valid - c * 32));  // valid columns in this 32-chunk
         const uint32_t cm = (ok && dl != 0.f) ? (nvc == 32 ? 0xFFFFFFFFu : ((1u << nvc) - 1u)) : 0u;
         kb &= cm;
@@ -554,7 +600,7 @@ struct GPolicyT {
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
               const float t = ((tb >> (j + u)) & 1u) ? 1.f : 0.f;
-              const float v = ((ks >> (j + u)) & 1u) ? ex2_approx(__uint_as_float(r[j + u])) : 0.f;
+              const float v = ((ks >> (j + u)) & 1u) ? pval(j + u) : 0.f;
               gf[u] = dl * (v - t);
               gk[u] = ((kb >> (j + u)) & 1u) ? gf[u] : (t != 0.f ? -dl : 0.f);
             }
@@ -607,7 +653,7 @@ struct GPolicyT {
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
                 if (!((nzb >> j) & 1u)) continue;
-                const float v = ((kb >> j) & 1u) ? ex2_approx(__uint_as_float(r[j])) : 0.f;
+                const float v = ((kb >> j) & 1u) ? pval(j) : 0.f;
                 const float g = dl * (v - (((tb >> j) & 1u) ? 1.f : 0.f));
                 if (pos < p.nz_cap) p.nz_list[pos] = NzEntry{jrow, vt * BN + c * 32 + j, g, 0};
                 ++pos;
@@ -637,7 +683,12 @@ struct GPolicyT {
           }
         }
       }
-      if (!sk) eng.epi_release(lane);
+      if (!sk) {
+        if constexpr (KL)
+          eng.epi_release2(lane);
+        else
+          eng.epi_release(lane);
+      }
       return true;
     });
   }
@@ -645,6 +696,7 @@ struct GPolicyT {
 
 using GPolicy = GPolicyT<false>;
 using GPolicyFull = GPolicyT<true>;
+using GPolicyKL = GPolicyT<false, true>;
 
 // =====================================================================
 // Backward, step 2: dE_chunk = G^T H_c, K = compact rows, accumulated on

@@ -1,0 +1,197 @@
+// Soft-target KL divergence without materialised logits.
+//
+// "The Defensive Edit: Chunking Cross-Entropy Loss After an OOM Wake-Up
+// Call", §The OOM: A 12.2 GB Softmax Wall: a soft KL term between a student
+// and a teacher softmax over a 248k vocabulary needs two [positions, V]
+// softmaxes, which the page then computes in position chunks.  Here neither
+// is ever written: per row
+//   KL_i = sum_j p_t,ij (log p_t,ij - log p_s,ij)
+//        = A_i - lse_t,i + lse_s,i,   A_i = sum_j p_t,ij (z_t,ij - z_s,ij),
+// with z_s = H_s E_s^T, z_t = H_t E_t^T (the same head may serve both).
+// The forward streams vocabulary tiles like the cross-entropy forward (the
+// log-sum-exp composed blockwise, "Cut Your Losses in Large-Vocabulary
+// Language Models", first page §Contribution), each tile as a pair of
+// accumulators, teacher then student: per row an online (max, sum) for each
+// softmax plus the teacher-weighted sum of z_t - z_s, rescaled with the
+// teacher's running max.  The backward (teacher constant) is
+// G = dloss (p_s - p_t), produced by GPolicyKL and contracted by the
+// cross-entropy path's dE/dH kernels.
+#pragma once
+
+#include "cce_kernels.cuh"
+
+namespace cce {
+
+struct KLFwdParams {
+  CUtensorMap mapAs, mapAt;  // H_s,c / H_t,c [Npad, D], box {64, 128}
+  CUtensorMap mapBs, mapBt;  // E_s / E_t [V, D], box {64, 256}
+  int V;
+  int T_v;   // vocabulary tiles
+  int tpi;   // tiles per work item
+  int S;     // splits
+  int Npad;  // partial row stride
+  int nkb;
+  const int* n_valid;
+  float* part;  // [S][5][Npad]: m_t (log2), s_t, w, m_s (log2), s_s
+  int* status;
+};
+
+struct KLFwdPolicy {
+  using Params = KLFwdParams;
+  static constexpr int EXTRA_SMEM = 0;
+  static __device__ __forceinline__ bool active(const Params&) { return true; }
+
+  template <class F>
+  static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
+    const int nv = *p.n_valid;
+    const int num_mb = (nv + BM - 1) / BM;
+    const int num_items = num_mb * p.S;
+    for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
+      const int split = item / num_mb;
+      const int mb = item - split * num_mb;
+      const int t0 = split * p.tpi;
+      const int t1 = min(p.T_v, t0 + p.tpi);
+      for (int t = t0; t < t1; ++t)
+        if (!f(mb, split, t, t == t1 - 1, nv)) return;
+    }
+  }
+
+  static __device__ void prefetch(const Params& p) {
+    tma_prefetch_map(&p.mapAs);
+    tma_prefetch_map(&p.mapAt);
+    tma_prefetch_map(&p.mapBs);
+    tma_prefetch_map(&p.mapBt);
+  }
+
+  static __device__ void producer(const Params& p, Engine& eng) {
+    schedule(p, [&](int mb, int, int t, bool, int) {
+      return eng.produce<false, false>(&p.mapAt, &p.mapBt, 0, mb * BM, 0, t * BN, p.nkb) &&
+             eng.produce<false, false>(&p.mapAs, &p.mapBs, 0, mb * BM, 0, t * BN, p.nkb);
+    });
+  }
+
+  static __device__ void mma(const Params& p, Engine& eng) {
+    schedule(p, [&](int, int, int, bool, int) {
+      return eng.mma<false, false>(p.nkb) && eng.mma<false, false>(p.nkb);
+    });
+  }
+
+  static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
+    const int row = q * 32 + lane;
+    float mt = -INFINITY, st = 0.f, w = 0.f;  // teacher (log2 max, sum, weighted z_t - z_s)
+    float ms = -INFINITY, ss = 0.f;           // student
+    schedule(p, [&](int mb, int split, int t, bool last, int nv) {
+      uint32_t ta, tb;
+      if (!eng.epi_acquire2(q, ta, tb)) return false;
+      const int valid = min(BN, p.V - t * BN);
+      const bool row_ok = mb * BM + row < nv;
+      for (int c = 0; c < BN / 32; ++c) {
+        if (c * 32 >= valid) break;  // uniform over the CTA
+        const int nvc = min(32, valid - c * 32);
+        uint32_t rt[32], rs[32];
+        tmem_ld32(ta + c * 32, rt);
+        tmem_ld32(tb + c * 32, rs);
+        float cmt = -INFINITY, cms = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (j < nvc) {
+            cmt = fmaxf(cmt, __uint_as_float(rt[j]));
+            cms = fmaxf(cms, __uint_as_float(rs[j]));
+          }
+        }
+        const float nt = fmaxf(mt, cmt * kLog2e);
+        const float sct = ex2_approx(mt - nt);
+        float at = st * sct, aw = w * sct;
+        const float ns = fmaxf(ms, cms * kLog2e);
+        float as = ss * ex2_approx(ms - ns);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (j < nvc) {
+            const float zt = __uint_as_float(rt[j]), zs = __uint_as_float(rs[j]);
+            const float e = ex2_approx(fmaf(zt, kLog2e, -nt));
+            at += e;
+            aw = fmaf(e, zt - zs, aw);
+            as += ex2_approx(fmaf(zs, kLog2e, -ns));
+          }
+        }
+        mt = nt;
+        st = at;
+        w = aw;
+        ms = ns;
+        ss = as;
+      }
+      eng.epi_release2(lane);
+      if (last) {
+        if (row_ok) {
+          float* o = p.part + (size_t)split * 5 * p.Npad + mb * BM + row;
+          o[0] = mt;
+          o[(size_t)p.Npad] = st;
+          o[(size_t)2 * p.Npad] = w;
+          o[(size_t)3 * p.Npad] = ms;
+          o[(size_t)4 * p.Npad] = ss;
+        }
+        mt = -INFINITY;
+        st = 0.f;
+        w = 0.f;
+        ms = -INFINITY;
+        ss = 0.f;
+      }
+      return true;
+    });
+  }
+};
+
+// Splits combined per row (one warp per original row): KL = A - lse_t +
+// lse_s with A = w / s_t after both are rescaled to the teacher's overall
+// max.  Masked rows give 0 in all three outputs.
+struct KLFinParams {
+  const int* pos_of_row;
+  const float* part;
+  int N, S, Npad;
+  float* kl;
+  float* lse_s;
+  float* lse_t;
+};
+
+__global__ void kl_finalize_kernel(const KLFinParams p) {
+  const int lane = threadIdx.x & 31;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < p.N; i += nw) {
+    const int j = p.pos_of_row[i];
+    if (j < 0) {
+      if (lane == 0) {
+        p.kl[i] = 0.f;
+        p.lse_s[i] = 0.f;
+        p.lse_t[i] = 0.f;
+      }
+      continue;
+    }
+    auto at = [&](int s, int k) { return p.part[((size_t)s * 5 + k) * p.Npad + j]; };
+    float Mt = -INFINITY, Ms = -INFINITY;
+    for (int s = lane; s < p.S; s += 32) {
+      Mt = fmaxf(Mt, at(s, 0));
+      Ms = fmaxf(Ms, at(s, 3));
+    }
+    Mt = warp_max(Mt);
+    Ms = warp_max(Ms);
+    float St = 0.f, W = 0.f, Ss = 0.f;
+    for (int s = lane; s < p.S; s += 32) {
+      const float ft = ex2_approx(at(s, 0) - Mt);
+      St = fmaf(at(s, 1), ft, St);
+      W = fmaf(at(s, 2), ft, W);
+      Ss = fmaf(at(s, 4), ex2_approx(at(s, 3) - Ms), Ss);
+    }
+    St = warp_sum(St);
+    W = warp_sum(W);
+    Ss = warp_sum(Ss);
+    if (lane == 0) {
+      const float lt = (Mt + log2f(St)) * kLn2;
+      const float ls = (Ms + log2f(Ss)) * kLn2;
+      p.lse_t[i] = lt;
+      p.lse_s[i] = ls;
+      p.kl[i] = W / St - lt + ls;
+    }
+  }
+}
+
+}  // namespace cce

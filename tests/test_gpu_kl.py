@@ -1,0 +1,100 @@
+"""Soft-target KL (cce_kl_fwd / cce_kl_bwd) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_cross_entropy_cce_b200 import synthetic as syn
+from _helpers import EPS_BF16, TOL_GRAD, TOL_GRAD_FILTER, TOL_ROW, normwise, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _kl_case(N, D, V, std_s, std_t, shared, seed, masked):
+    """Student and teacher rows from two seeded synthetic draws of the same
+    shapes (H ~ N(0, 1), E scaled to the logit std); optionally one head."""
+    xs = syn.make_inputs(syn.Workload("kls", N=N, D=D, V=V, logit_std=std_s, ignore_frac=0.0),
+                         seed=seed)
+    xt = syn.make_inputs(syn.Workload("klt", N=N, D=D, V=V, logit_std=std_t, ignore_frac=0.0),
+                         seed=seed + 100)
+    Es = xs.segments[0][2]
+    Et = Es if shared else xt.segments[0][2]
+    mask = None
+    if masked:
+        mask = (np.random.default_rng(seed).random(N) > 0.2).astype(np.int32)
+    return xs.H, Es, xt.H, Et, mask
+
+
+def _up(a):
+    from linear_cross_entropy_cce_b200 import cce
+    return cce.bf16_from_bits(a, "cuda")
+
+
+CASES = {
+    "separate_heads": dict(N=333, D=200, V=5000, std_s=3.0, std_t=4.0, shared=False, seed=1, masked=True),
+    "shared_head": dict(N=300, D=256, V=7001, std_s=2.0, std_t=2.0, shared=True, seed=2, masked=False),
+    # peaky distributions: after filtering the sparse (CUDA-core) route runs
+    "sparse": dict(N=700, D=192, V=30000, std_s=14.0, std_t=14.0, shared=True, seed=3, masked=True),
+}
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+@pytest.mark.parametrize("eps", [0.0, EPS_BF16])
+def test_kl_matches_oracle(case, eps):
+    from linear_cross_entropy_cce_b200 import cce
+    Hs, Es, Ht, Et, mask = _kl_case(**CASES[case])
+    tm = torch.from_numpy(mask).cuda() if mask is not None else None
+    Hs_d, Es_d, Ht_d = _up(Hs), _up(Es), _up(Ht)
+    Et_d = Es_d if CASES[case]["shared"] else _up(Et)
+    kl, ls, lt = cce.kl_fwd(Hs_d, Es_d, Ht_d, Et_d, tm)
+    N = Hs.shape[0]
+    dl = np.linspace(0.2, 1.0, N) / N
+    dH, dE = cce.kl_bwd(Hs_d, Es_d, Ht_d, Et_d, ls, lt, torch.from_numpy(dl).float().cuda(), tm,
+                        filter_eps=eps)
+    torch.cuda.synchronize()
+    rk, rls, rlt = oracle.kl_forward(Hs, Es, Ht, Et, mask)
+    assert np.max(np.abs(to_np(kl) - rk)) <= TOL_ROW
+    assert np.max(np.abs(to_np(ls) - rls)) <= TOL_ROW
+    assert np.max(np.abs(to_np(lt) - rlt)) <= TOL_ROW
+    rH, rE = oracle.kl_backward(Hs, Es, Ht, Et, dl, mask, filter_eps=eps)
+    tol = TOL_GRAD_FILTER if eps > 0 else TOL_GRAD
+    assert normwise(to_np(dH), rH) <= tol
+    assert normwise(to_np(dE), rE) <= tol
+    if mask is not None:
+        off = mask == 0
+        assert np.all(to_np(kl)[off] == 0) and np.all(to_np(dH)[off] == 0)
+
+
+def test_kl_of_identical_models_is_exactly_zero():
+    """Teacher = student: the two tiles of every pair are the same products,
+    so KL, dH and dE come out exactly 0."""
+    from linear_cross_entropy_cce_b200 import cce
+    Hs, Es, _, _, _ = _kl_case(N=260, D=128, V=3000, std_s=5.0, std_t=5.0, shared=True, seed=4,
+                               masked=False)
+    H, E = _up(Hs), _up(Es)
+    kl, ls, lt = cce.kl_fwd(H, E, H, E)
+    dH, dE = cce.kl_bwd(H, E, H, E, ls, lt, torch.full((260,), 0.5, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(ls, lt)
+    assert torch.all(kl == 0) and torch.all(dH == 0) and torch.all(dE == 0)
+
+
+def test_soft_target_kl_autograd():
+    from linear_cross_entropy_cce_b200.autograd import soft_target_kl
+    Hs, Es, Ht, Et, mask = _kl_case(**CASES["separate_heads"])
+    Hl = _up(Hs).requires_grad_(True)
+    El = _up(Es).requires_grad_(True)
+    tm = torch.from_numpy(mask).cuda()
+    loss = soft_target_kl(Hl, El, _up(Ht), _up(Et), row_mask=tm, filter_eps=0.0)
+    loss.backward()
+    torch.cuda.synchronize()
+    rk, _, _ = oracle.kl_forward(Hs, Es, Ht, Et, mask)
+    n = int((mask != 0).sum())
+    ref = math.fsum(rk.tolist()) / n
+    assert abs(loss.item() - ref) <= 1e-4 * abs(ref)
+    dl = np.where(mask != 0, 1.0 / n, 0.0)
+    rH, rE = oracle.kl_backward(Hs, Es, Ht, Et, dl, mask)
+    assert normwise(to_np(Hl.grad), rH) <= TOL_GRAD
+    assert normwise(to_np(El.grad), rE) <= TOL_GRAD
