@@ -191,6 +191,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--filter", choices=["on", "off", "default"], default="default")
     ap.add_argument("--sort", choices=["on", "off", "default"], default="default")
+    ap.add_argument("--loss", choices=["ce", "kl"], default="ce",
+                    help="ce: the cross-entropy hot path; kl: the soft-target KL between a "
+                         "student and a teacher softmax")
+    ap.add_argument("--kl-workload", default="soft_kl_24k_248k", choices=sorted(syn.KL_WORKLOADS))
     ap.add_argument("--kahan", action="store_true",
                     help="accumulate dE across steps with the Kahan-compensated bf16 path")
     ap.add_argument("--no-e2e", action="store_true")
@@ -203,6 +207,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.loss == "kl":
+        return kl_main(a, world, rank, local)
     wl = syn.WORKLOADS[a.workload]
     filt, sort = MODES[wl.name]
     if a.filter != "default":
@@ -404,6 +410,175 @@ def main():
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+KL_METRIC = "soft-target KL fwd+bwd positions/s (and % of B200 bf16 tensor peak)"
+
+
+def kl_oracle_sample(wl, Hs, Ht, E, seconds: float, eps: float):
+    """Time the fp64 oracle's KL forward + backward on a row sample."""
+    import oracle
+    E64 = oracle.widen_bf16(E)
+    dl = np.full(wl.N, 1.0 / wl.N)
+
+    def run(rows):
+        t = time.perf_counter()
+        oracle.kl_forward(Hs[rows], E64, Ht[rows], E64)
+        oracle.kl_backward(Hs[rows], E64, Ht[rows], E64, dl[rows], filter_eps=eps)
+        return time.perf_counter() - t
+
+    r0 = np.arange(4)
+    t0 = run(r0)
+    R = int(min(1024, wl.N, max(4, seconds / max(t0, 1e-6) * 4)))
+    rows = np.linspace(0, wl.N - 1, R).astype(np.int64)
+    t = run(rows)
+    desc = (f"fp64 numpy oracle, KL forward+backward over {R} rows of {wl.name} "
+            f"(N={wl.N}, D={wl.D}, V={wl.V}); full vocabulary and full dE per slice")
+    return R / t, R, t, desc
+
+
+def kl_main(a, world, rank, local):
+    """The soft-target KL path: cce_kl_fwd + cce_kl_bwd per step."""
+    wl = syn.KL_WORKLOADS[a.kl_workload]
+    eps = 0.0 if a.filter == "off" else EPS_BF16
+    Hs, Ht, E = syn.make_kl_inputs(wl, seed=rank)
+    if a.impl == "reference":
+        if rank != 0:
+            return
+        times, R = [], 0
+        for i in range(a.warmup + a.steps):
+            rps, R, t, desc = kl_oracle_sample(wl, Hs, Ht, E, max(2.0, 120.0 / (a.steps + a.warmup)), eps)
+            if i >= a.warmup:
+                times.append(t)
+        ms = 1e3 * float(np.mean(times))
+        v = R / (ms / 1e3)
+        print(json.dumps({"impl": "reference", "metric": KL_METRIC, "value": round(v, 3),
+                          "unit": "positions/s", "n_gpus": world, "steps": a.steps,
+                          "warmup": a.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": {"workload": wl.name, "rows_per_step": R},
+                          "cpu_baseline": {"value": round(v, 3), "unit": "positions/s",
+                                           "cores": host_cores(), "kind": "oracle", "sample": desc},
+                          "e2e": {"value": round(v, 3), "unit": "positions/s",
+                                  "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    from linear_cross_entropy_cce_b200 import cce
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    N, D, V = wl.N, wl.D, wl.V
+    Hs_d, Ht_d, E_d = (cce.bf16_from_bits(t, dev) for t in (Hs, Ht, E))
+    dl = torch.full((N,), 1.0 / N, dtype=torch.float32, device=dev)
+    ws_f = torch.empty(cce.lib().cce_kl_fwd_workspace_size(N, D, V), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(cce.lib().cce_kl_bwd_workspace_size(N, D, V, 0), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(hs=Hs_d, ht=Ht_d, e=E_d):
+        kl, ls, lt = cce.kl_fwd(hs, e, ht, e, workspace=ws_f, status=status)
+        cce.kl_bwd(hs, e, ht, e, ls, lt, dl, filter_eps=eps, workspace=ws_b, status=status)
+        return kl
+
+    def timed(fn, k):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        s = torch.cuda.current_stream(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(k):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        return max_over_ranks(e0.elapsed_time(e1) / k, world, dev)
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise SystemExit(f"device status {int(status.item())} during warm-up")
+    uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", ""))
+    uuid = uuid if uuid.startswith("GPU-") or not uuid else "GPU-" + uuid
+    l0 = cce.launch_count()
+    with ClockSampler(uuid) as clk:
+        ms_step = timed(step, a.steps)
+    launches = cce.launch_count() - l0
+    ms_fwd = timed(lambda: cce.kl_fwd(Hs_d, E_d, Ht_d, E_d, workspace=ws_f, status=status), a.steps)
+    cce.timing_enable(0b111111)
+    timed(step, a.steps)
+    per_class = cce.timing_read()
+    cce.timing_enable(0)
+
+    P = peaks()
+    ndv = float(N) * D * V
+    class_flops = {"fwd_tile_stream": 4 * ndv, "bwd_g_producer": 4 * ndv,
+                   "bwd_dE_contraction": 2 * ndv, "bwd_dH_contraction": 2 * ndv}
+    dom = max(class_flops, key=lambda k: per_class[k][0])
+    dom_ms, dom_n = per_class[dom]
+    achieved = class_flops[dom] * a.steps / (dom_ms / 1e3) / 1e12 if dom_ms > 0 else None
+    peak_sus = P.get("bf16_tflops_sustained", 1400.0)
+    step_tflops = 12 * ndv / (ms_step / 1e3) / 1e12
+
+    e2e = None
+    if not a.no_e2e:
+        hHs = torch.from_numpy(Hs.view(np.int16)).pin_memory()
+        hHt = torch.from_numpy(Ht.view(np.int16)).pin_memory()
+        hE = torch.from_numpy(E.view(np.int16)).pin_memory()
+        hkl = torch.empty(N, dtype=torch.float32).pin_memory()
+        bs, bt, be = torch.empty_like(Hs_d), torch.empty_like(Ht_d), torch.empty_like(E_d)
+
+        def e2e_step():
+            bs.view(torch.int16).copy_(hHs, non_blocking=True)
+            bt.view(torch.int16).copy_(hHt, non_blocking=True)
+            be.view(torch.int16).copy_(hE, non_blocking=True)
+            hkl.copy_(step(bs, bt, be), non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        ms_e2e = timed(e2e_step, a.steps)
+        e2e = {"value": round(tokens_per_s(N, world, ms_e2e), 1), "unit": "positions/s",
+               "h2d_bytes_per_step": int((Hs.size + Ht.size + E.size) * 2),
+               "d2h_bytes_per_step": int(N * 4), "ms_per_step": round(ms_e2e, 3)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        rps, R, t, desc = kl_oracle_sample(wl, Hs, Ht, E, a.cpu_seconds, eps)
+        cpu = {"value": round(rps, 3), "unit": "positions/s", "cores": host_cores(),
+               "kind": "oracle", "sample": desc, "seconds": round(t, 2)}
+    out = {
+        "metric": KL_METRIC, "value": round(tokens_per_s(N, world, ms_step), 1),
+        "unit": "positions/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded student and teacher rows, one shared head)",
+        "config": {"workload": wl.name, "N": N, "D": D, "V": V, "logit_std": wl.logit_std,
+                   "filter_eps": eps, "parallelism": f"dp{world} (independent batches)",
+                   "l2": f"inputs larger than L2 (E = {E.size * 2 / 2**20:.0f} MiB > 126 MiB)"},
+        "tensor_peak_frac": {"of_measured_burst": round(step_tflops / P.get("bf16_tflops", 1590.0), 4),
+                             "of_measured_sustained": round(step_tflops / peak_sus, 4),
+                             "tflops_unfiltered_12NDV": round(step_tflops, 1)},
+        "fwd_ms": round(ms_fwd, 3), "fwd_bwd_ms": round(ms_step, 3),
+        "roofline": {"bound": "tensor", "kernel": dom,
+                     "achieved": round(achieved, 1) if achieved else None,
+                     "peak": peak_sus, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_sus, 4) if achieved else None,
+                     "traffic": None,
+                     "peak_kind": "sustained bf16 (measured, cuBLAS)",
+                     "launches_per_step": dom_n // max(1, a.steps)},
+        "per_kernel_ms_per_step": {k: round(v[0] / a.steps, 3) for k, v in per_class.items()},
+        "gpu_launches": int(launches), "gpu_launches_per_step": int(launches // max(1, a.steps)),
+        "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
     }
     if rank == 0:
         print(json.dumps(out), flush=True)

@@ -180,3 +180,32 @@ def make_inputs(wl: Workload, seed: int = 0, threads: Optional[int] = None) -> I
         y[sel] = b + local
     y[ignore] = IGNORE_INDEX
     return Inputs(wl, H, segs, y.astype(np.int32))
+
+
+# ---- soft-target KL workload ------------------------------------------------
+# The page on chunking the loss after an OOM trains with a soft KL term
+# between a student and a teacher softmax at 24,576 positions over a 248,320
+# vocabulary.  Stand-in inputs of that shape: student and teacher rows
+# H ~ N(0, 1) drawn independently, one shared head E ~ N(0, logit_std/sqrt(D)).
+@dataclass(frozen=True)
+class KLWorkload:
+    name: str
+    N: int
+    D: int
+    V: int
+    logit_std: float
+
+
+KL_WORKLOADS = {
+    "soft_kl_24k_248k": KLWorkload("soft_kl_24k_248k", N=24576, D=2048, V=248320, logit_std=6.0),
+    "soft_kl_small": KLWorkload("soft_kl_small", N=512, D=256, V=8192, logit_std=6.0),
+}
+
+
+def make_kl_inputs(wl: KLWorkload, seed: int = 0, threads: Optional[int] = None):
+    """(Hs, Ht, E) as bf16 bit patterns for a soft-target KL workload."""
+    ss_s, ss_t, ss_e = np.random.SeedSequence(seed).spawn(3)
+    Hs = _normal_bf16(ss_s, (wl.N, wl.D), 1.0, threads)
+    Ht = _normal_bf16(ss_t, (wl.N, wl.D), 1.0, threads)
+    E = _normal_bf16(ss_e, (wl.V, wl.D), wl.logit_std / np.sqrt(wl.D), threads)
+    return Hs, Ht, E
