@@ -83,6 +83,33 @@ int device_sms() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// A second stream (per host thread and device) for the permuted-E gathers of
+// the backward, so the gather of chunk k+1 overlaps the tensor work of chunk
+// k; events order it against the caller's stream (fork at the start, join
+// before returning), which also keeps stream capture valid.  Created on first
+// use and kept; NULL when creation fails (the gathers then run in order on
+// the caller's stream).
+struct SideStream {
+  cudaStream_t ss;
+  cudaEvent_t fork, join, ready[2], freed[2];
+};
+
+SideStream* side_stream() {
+  constexpr int kMaxDev = 64;
+  thread_local SideStream per[kMaxDev];
+  thread_local int state[kMaxDev];  // 0 untried, 1 ready, -1 failed
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  if (state[dev] == 0) {
+    SideStream& x = per[dev];
+    bool ok = cudaStreamCreateWithFlags(&x.ss, cudaStreamNonBlocking) == cudaSuccess;
+    cudaEvent_t* evs[6] = {&x.fork, &x.join, &x.ready[0], &x.ready[1], &x.freed[0], &x.freed[1]};
+    for (cudaEvent_t* e : evs) ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+    state[dev] = ok ? 1 : -1;
+  }
+  return state[dev] == 1 ? &per[dev] : nullptr;
+}
+
 // ------------------------------------------------------------ segment table
 struct Segs {
   int n = 0;
@@ -227,7 +254,7 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = fals
   p.off_hc = o; o += align_up((size_t)p.Npad * D * 2);
   p.off_dh = o; o += align_up((size_t)p.Npad * D * 4);
   p.off_g = o; o += align_up((size_t)p.Npad * p.Vc * 2);
-  p.off_ec = o; o += align_up((size_t)p.Vc * D * 2);
+  p.off_ec = o; o += 2 * align_up((size_t)p.Vc * D * 2);  // two buffers: gather k+1 while k runs
   // CCE_FULL_DE: a second slab with the unfiltered G, read by dE only
   p.off_gfull = o; o += (flags & CCE_FULL_DE) ? align_up((size_t)p.Npad * p.Vc * 2) : 0;
   p.dh_words = (int)cdiv(p.Vc, 512);
@@ -676,7 +703,6 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   memset(&cmap, 0, sizeof(cmap));
   cmap.n_segs = sg.n;
   for (int s = 0; s < sg.n; ++s) cmap.live_off[s] = table.s[s].live_off;
-  int chunk = 0;  // global chunk index
 
   GParams gp;
   DEParams ep;
@@ -696,33 +722,72 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   if (!make_map_t(&hp.mapC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dH_acc, D, pl.Npad, D, 32, 32))
     return CCE_ELAUNCH;
 
+  // the chunk list: per segment, equal chunks (multiples of 256) so the last
+  // one is not a sliver
+  struct ChunkRef {
+    int s, c0, cv;
+  };
+  std::vector<ChunkRef> chunks;
   for (int s = 0; s < sg.n; ++s) {
+    const int ns = table.s[s].n;
+    const int nch = (int)cdiv(ns, Vc);
+    const int cw = (int)std::min<int64_t>(Vc, cdiv(cdiv(ns, nch), BN) * BN);
+    cmap.chunk_begin[s] = (int)chunks.size();
+    cmap.width[s] = cw;
+    for (int c0 = 0; c0 < ns; c0 += cw) chunks.push_back({s, c0, std::min(cw, ns - c0)});
+  }
+  const int n_chunks = (int)chunks.size();
+  __nv_bfloat16* Ecb[2] = {Ec, Ec + align_up((size_t)Vc * D * 2) / sizeof(__nv_bfloat16)};
+  // permuted walk: chunk k's E rows gathered into Ecb[k % 2] (on the side
+  // stream one chunk ahead when there is one)
+  SideStream* side = vocab_perm ? side_stream() : nullptr;
+  auto gather = [&](int k, cudaStream_t gs) -> int {
+    const ChunkRef& c = chunks[k];
+    {
+      TimedLaunch tl_(KC_AUX, gs);
+      gather_perm_rows_kernel<<<sms * 4, 256, 0, gs>>>(
+          static_cast<const __nv_bfloat16*>(sg.s[c.s].E), vocab_perm + table.s[c.s].live_off + c.c0,
+          c.cv, (int)D, Ecb[side ? (k & 1) : 0]);
+    }
+    return launched();
+  };
+  if (side) {
+    if (cudaEventRecord(side->fork, st) != cudaSuccess ||
+        cudaStreamWaitEvent(side->ss, side->fork, 0) != cudaSuccess)
+      return CCE_ELAUNCH;
+  }
+  auto do_chunk = [&](const int chunk) -> int {
+    const int s = chunks[chunk].s, c0 = chunks[chunk].c0, cv = chunks[chunk].cv;
     const int ns = table.s[s].n;
     const int* perm_seg = vocab_perm ? vocab_perm + table.s[s].live_off : nullptr;
     CUtensorMap segK, segMN;
-    if (!perm_seg) {
+    int row0 = c0;
+    if (perm_seg) {
+      if (side) {
+        if (chunk == 0) {
+          if (int rc = gather(0, side->ss)) return rc;
+          if (cudaEventRecord(side->ready[0], side->ss) != cudaSuccess) return CCE_ELAUNCH;
+        }
+        if (chunk + 1 < n_chunks) {
+          // buffer (chunk+1) % 2 was last read by the dH contraction of chunk - 1
+          if (chunk >= 1 && cudaStreamWaitEvent(side->ss, side->freed[(chunk + 1) & 1], 0) != cudaSuccess)
+            return CCE_ELAUNCH;
+          if (int rc = gather(chunk + 1, side->ss)) return rc;
+          if (cudaEventRecord(side->ready[(chunk + 1) & 1], side->ss) != cudaSuccess)
+            return CCE_ELAUNCH;
+        }
+        if (cudaStreamWaitEvent(st, side->ready[chunk & 1], 0) != cudaSuccess) return CCE_ELAUNCH;
+      } else if (int rc = gather(chunk, st)) {
+        return rc;
+      }
+      const __nv_bfloat16* Eb = Ecb[side ? (chunk & 1) : 0];
+      if (!make_map(&segK, Eb, D, cv, D, BK, BN)) return CCE_ELAUNCH;
+      if (!make_map(&segMN, Eb, D, cv, D, 64, 64)) return CCE_ELAUNCH;
+      row0 = 0;
+    } else {
       if (!make_map(&segK, sg.s[s].E, D, ns, D, BK, BN)) return CCE_ELAUNCH;
       if (!make_map(&segMN, sg.s[s].E, D, ns, D, 64, 64)) return CCE_ELAUNCH;
     }
-    // equal chunks (multiples of 256) so the last one is not a sliver
-    const int nch = (int)cdiv(ns, Vc);
-    const int cw = (int)std::min<int64_t>(Vc, cdiv(cdiv(ns, nch), BN) * BN);
-    cmap.chunk_begin[s] = chunk;
-    cmap.width[s] = cw;
-    for (int c0 = 0; c0 < ns; c0 += cw, ++chunk) {
-      const int cv = std::min(cw, ns - c0);
-      int row0 = c0;
-      if (perm_seg) {
-        {
-          TimedLaunch tl_(KC_AUX, st);
-          gather_perm_rows_kernel<<<sms * 4, 256, 0, st>>>(
-              static_cast<const __nv_bfloat16*>(sg.s[s].E), perm_seg + c0, cv, (int)D, Ec);
-        }
-        if (launched()) return CCE_ELAUNCH;
-        if (!make_map(&segK, Ec, D, cv, D, BK, BN)) return CCE_ELAUNCH;
-        if (!make_map(&segMN, Ec, D, cv, D, 64, 64)) return CCE_ELAUNCH;
-        row0 = 0;
-      }
       // step 1: G for this chunk, with its zero-slice masks
       uint32_t* dh_mask = masks + (size_t)(chunk & 1) * mask_stride;
       uint32_t* de_mask = dh_mask + (size_t)(pl.Npad / BM) * pl.dh_words;
@@ -810,8 +875,18 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       hp.status = status;
       if (int rc = launch_tc<DHPolicy>(hp, (int)std::min<int64_t>(sms, (int64_t)mbs * dt), st, KC_DH))
         return rc;
-    }
+      if (side && cudaEventRecord(side->freed[chunk & 1], st) != cudaSuccess) return CCE_ELAUNCH;
+      return CCE_OK;
+  };
+  int loop_rc = CCE_OK;
+  for (int k = 0; k < n_chunks && loop_rc == CCE_OK; ++k) loop_rc = do_chunk(k);
+  if (side) {  // join the side stream back into the caller's stream
+    const bool ok = cudaEventRecord(side->join, side->ss) == cudaSuccess &&
+                    cudaStreamWaitEvent(st, side->join, 0) == cudaSuccess;
+    if (loop_rc == CCE_OK && !ok) loop_rc = CCE_ELAUNCH;
   }
+  if (loop_rc != CCE_OK) return loop_rc;
+  const int chunk = n_chunks;
   // sparse chunks: lists -> CSR by column (dE) and by row (dH), then the gathers
   const int gthreads = gather_threads(D);
   const int gblocks = sms * std::max(1, 2048 / gthreads);
