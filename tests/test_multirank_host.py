@@ -34,7 +34,7 @@ def _worker(rank, world, port, out):
 
 def test_max_over_ranks_and_job_throughput_world2():
     world, port = 2, _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_worker, args=(world, port, out), nprocs=world, start_method="spawn")
         res = dict(out)
