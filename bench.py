@@ -367,9 +367,14 @@ def main():
                 "frac": round(achieved / peak_sus, 4) if achieved else None,
                 "peak_kind": "sustained bf16 (measured, cuBLAS) - kernel timed inside the step",
                 "traffic": recorded_traffic(dom) if wl.name == "gemma2_2b_head" else None,
-                "traffic_note": "DRAM bytes of one launch of this kernel from the committed ncu capture "
+                "traffic_note": "DRAM bytes of one working launch of this kernel (one vocabulary chunk "
+                                "for the G producer) from the committed ncu capture "
                                 "(profiles/roofline_traffic.json, cold cache); null if the sources changed",
+                "achieved_note": "algorithmic FLOPs of the class per step over the summed CUDA-event "
+                                 "durations of all its launches in the step",
                 "launches_per_step": dom_n // max(1, a.steps),
+                "launches_note": "the G producer launches twice per vocabulary chunk; the second "
+                                 "(repair) launch exits at once unless the chunk overflowed its sparse list",
                 "avg_launch_ms": round(dom_ms / max(1, dom_n), 4)}
     step_tflops = flops_step / (ms_step / 1e3) / 1e12
 

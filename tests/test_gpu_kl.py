@@ -98,3 +98,30 @@ def test_soft_target_kl_autograd():
     rH, rE = oracle.kl_backward(Hs, Es, Ht, Et, dl, mask)
     assert normwise(to_np(Hl.grad), rH) <= TOL_GRAD
     assert normwise(to_np(El.grad), rE) <= TOL_GRAD
+
+
+def test_kl_full_size_sampled_rows_and_pairing_identity():
+    """The 24,576 x 248,320 stand-in workload of bench.py --loss kl: KL, both
+    lse and dH on sampled rows (each an independent oracle row); dE through
+    sum_i <dH_i, H_s,i> = <dE, E_s> (both equal sum_ij G_ij z_s,ij)."""
+    from linear_cross_entropy_cce_b200 import cce
+    wl = syn.KL_WORKLOADS["soft_kl_24k_248k"]
+    Hs, Ht, E = syn.make_kl_inputs(wl, seed=0)
+    a, b, e = _up(Hs), _up(Ht), _up(E)
+    kl, ls, lt = cce.kl_fwd(a, e, b, e)
+    dl = np.full(wl.N, 1.0 / wl.N)
+    dH, dE = cce.kl_bwd(a, e, b, e, ls, lt, torch.from_numpy(dl).float().cuda(),
+                        filter_eps=EPS_BF16, fp32_grads=True)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.concatenate([[0, wl.N - 1], rng.choice(wl.N, 10, replace=False)]))
+    E64 = oracle.widen_bf16(E)
+    rk, rls, rlt = oracle.kl_forward(Hs[rows], E64, Ht[rows], E64)
+    assert np.max(np.abs(to_np(kl)[rows] - rk)) <= TOL_ROW
+    assert np.max(np.abs(to_np(ls)[rows] - rls)) <= TOL_ROW
+    assert np.max(np.abs(to_np(lt)[rows] - rlt)) <= TOL_ROW
+    rH, _ = oracle.kl_backward(Hs[rows], E64, Ht[rows], E64, dl[rows], filter_eps=EPS_BF16)
+    assert normwise(to_np(dH)[rows], rH) <= TOL_GRAD_FILTER
+    lhs = float(torch.sum(dH.double() * a.double()))
+    rhs = float(torch.sum(dE.double() * e.double()))
+    assert abs(lhs - rhs) <= 1e-3 * max(abs(lhs), abs(rhs), 1e-12)
