@@ -217,17 +217,26 @@ KLFwdPlan plan_kl_fwd(int64_t N, int64_t D, int64_t V) {
 
 // ----------------------------------------------------------- backward plan
 struct BwdPlan {
-  int64_t Npad, Vc;
+  int64_t Npad, Vc;  // Vc: chunk width of unfiltered / Kahan calls
+  int64_t Vc_f;      // chunk width of filtered calls (the sparse route is likely)
   size_t off_nvalid, off_idx, off_pos, off_lse2, off_dl, off_tseg, off_tpos, off_inv, off_hc,
       off_dh, off_g, off_ec, off_gfull, off_masks, total;
-  int dh_words, de_words;
-  size_t mask_bytes;
+  int de_words;
+  size_t mask_bytes;  // one mask buffer, sized for the wider chunk width
   // sparse backward (filtered gradients)
-  int64_t nch_max, cap;
+  int64_t nch_max;
   size_t off_nzcnt, off_lists, off_colc, off_csorted, off_rowc, off_rsorted, off_scan, scan_bytes;
   size_t off_tcmax, off_blkmin;  // tile-skip bounds
   size_t off_htc, off_lt2;       // soft-target KL: teacher rows and lse
 };
+
+// Zero-slice mask words for chunk width vc: dH masks (per 128-row block, one
+// bit per 16 columns) and dE masks (per 128-column block, one bit per 16 rows).
+size_t mask_bytes_for(int64_t Npad, int64_t vc) {
+  return sizeof(uint32_t) * ((size_t)(Npad / BM) * cdiv(vc, 512) + (size_t)(vc / BM) * cdiv(Npad, 512));
+}
+// Sparse-list capacity of one chunk of width vc: density 1/2048.
+int64_t list_cap(int64_t Npad, int64_t vc) { return std::max<int64_t>(4096, Npad * vc / 2048); }
 
 BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = false) {
   BwdPlan p;
@@ -241,6 +250,13 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = fals
   vc = std::min<int64_t>(vc, (int64_t)(kGCapBytes / (2 * (size_t)p.Npad)));
   vc = std::min<int64_t>(16384, vc) / BN * BN;
   p.Vc = std::max<int64_t>(BN, std::min<int64_t>(vc, cdiv(V, BN) * BN));
+  // Filtered calls: twice as wide (fewer launches per step and a smaller
+  // last-wave tail per launch; their chunks mostly take the sparse route and
+  // write no slab), within the slab cap.
+  int64_t vf = std::min<int64_t>(2 * p.Vc, (int64_t)(kGCapBytes / (2 * (size_t)p.Npad)));
+  vf = std::min<int64_t>(16384, vf) / BN * BN;
+  p.Vc_f = std::max<int64_t>(p.Vc, std::min<int64_t>(vf, cdiv(V, BN) * BN));
+  const int64_t Vw = p.Vc_f;  // buffers scaled by the chunk width are sized for the wider one
   const size_t n4 = sizeof(int) * (size_t)std::max<int64_t>(N, 1);
   size_t o = 0;
   p.off_nvalid = o; o += align_up(16);
@@ -253,24 +269,25 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = fals
   p.off_inv = o; o += align_up(sizeof(int) * (size_t)V);
   p.off_hc = o; o += align_up((size_t)p.Npad * D * 2);
   p.off_dh = o; o += align_up((size_t)p.Npad * D * 4);
-  p.off_g = o; o += align_up((size_t)p.Npad * p.Vc * 2);
-  p.off_ec = o; o += 2 * align_up((size_t)p.Vc * D * 2);  // two buffers: gather k+1 while k runs
+  p.off_g = o; o += align_up((size_t)p.Npad * Vw * 2);
+  p.off_ec = o; o += 2 * align_up((size_t)Vw * D * 2);  // two buffers: gather k+1 while k runs
   // CCE_FULL_DE: a second slab with the unfiltered G, read by dE only
-  p.off_gfull = o; o += (flags & CCE_FULL_DE) ? align_up((size_t)p.Npad * p.Vc * 2) : 0;
-  p.dh_words = (int)cdiv(p.Vc, 512);
+  p.off_gfull = o; o += (flags & CCE_FULL_DE) ? align_up((size_t)p.Npad * Vw * 2) : 0;
   p.de_words = (int)cdiv(p.Npad, 512);
-  p.mask_bytes = sizeof(uint32_t) * ((size_t)(p.Npad / BM) * p.dh_words + (size_t)(p.Vc / BM) * p.de_words);
+  p.mask_bytes = mask_bytes_for(p.Npad, Vw);
   // two mask buffers: chunk c uses buffer c % 2 and its G launch clears the other
   p.off_masks = o; o += 2 * align_up(p.mask_bytes);
-  // sparse path: per chunk a list of up to `cap` non-zeros (density 1/2048)
+  // sparse path: per chunk a list of up to cap(Vc) non-zeros (density 1/2048);
+  // chunk count from the narrower width, list slots for whichever needs more
   p.nch_max = cdiv(V, p.Vc) + CCE_MAX_SEGMENTS;
-  p.cap = std::max<int64_t>(4096, p.Npad * p.Vc / 2048);
+  const int64_t slots = std::max(p.nch_max * list_cap(p.Npad, p.Vc),
+                                 (cdiv(V, p.Vc_f) + CCE_MAX_SEGMENTS) * list_cap(p.Npad, p.Vc_f));
   p.off_nzcnt = o; o += align_up(sizeof(int) * 2 * (size_t)p.nch_max);  // counts + slab flags
-  p.off_lists = o; o += align_up(sizeof(NzEntry) * (size_t)p.nch_max * p.cap);
+  p.off_lists = o; o += align_up(sizeof(NzEntry) * (size_t)slots);
   p.off_colc = o; o += align_up(sizeof(int) * 2 * (size_t)(V + 1));  // counts, offsets
-  p.off_csorted = o; o += align_up(sizeof(int2) * (size_t)p.nch_max * p.cap);
+  p.off_csorted = o; o += align_up(sizeof(int2) * (size_t)slots);
   p.off_rowc = o; o += align_up(sizeof(int) * 2 * (size_t)(p.Npad + 1));
-  p.off_rsorted = o; o += align_up(sizeof(int2) * (size_t)p.nch_max * p.cap);
+  p.off_rsorted = o; o += align_up(sizeof(int2) * (size_t)slots);
   // generous bound on cub's single-pass scan scratch (checked again at run time)
   p.scan_bytes = align_up(sizeof(int) * (size_t)(std::max<int64_t>(V, p.Npad) + 1) / 8 + (1u << 20));
   p.off_scan = o; o += p.scan_bytes;
@@ -642,7 +659,10 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   const size_t mask_stride = align_up(pl.mask_bytes) / sizeof(uint32_t);
   if (cudaMemsetAsync(masks, 0, 2 * align_up(pl.mask_bytes), st) != cudaSuccess) return CCE_ELAUNCH;
   __nv_bfloat16* Ec = at<__nv_bfloat16>(workspace, pl.off_ec);
-  const int Vc = (int)pl.Vc;
+  // chunk width of this call: wider when filtering can take the sparse route
+  const bool wide = filter_eps > 0.f && !kahan;
+  const int Vc = (int)(wide ? pl.Vc_f : pl.Vc);
+  const int dh_words = (int)cdiv(Vc, 512);
   const int dt = (int)cdiv(D, BN);
   const int nkbD = (int)cdiv(D, BK);
   const int mbs = (int)(pl.Npad / BM);
@@ -686,7 +706,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   bool sparse = filter_eps > 0.f && !kahan;
   for (int s = 0; s < sg.n; ++s) sparse = sparse && table.s[s].n < (1 << 29);
   const bool sparse_de = sparse && !full_de;
-  const int cap = (int)pl.cap;
+  const int cap = (int)list_cap(pl.Npad, Vc);
   int* nz_cnt = at<int>(workspace, pl.off_nzcnt);
   NzEntry* lists = at<NzEntry>(workspace, pl.off_lists);
   const int64_t v_live = sg.live;
@@ -790,11 +810,11 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
     }
       // step 1: G for this chunk, with its zero-slice masks
       uint32_t* dh_mask = masks + (size_t)(chunk & 1) * mask_stride;
-      uint32_t* de_mask = dh_mask + (size_t)(pl.Npad / BM) * pl.dh_words;
+      uint32_t* de_mask = dh_mask + (size_t)(pl.Npad / BM) * dh_words;
       gp.mask_clear = masks + (size_t)((chunk + 1) & 1) * mask_stride;
-      gp.mask_clear_words = (int)(pl.mask_bytes / sizeof(uint32_t));
+      gp.mask_clear_words = (int)(mask_bytes_for(pl.Npad, Vc) / sizeof(uint32_t));
       gp.dh_mask = dh_mask;
-      gp.dh_words = pl.dh_words;
+      gp.dh_words = dh_words;
       gp.de_mask = de_mask;
       gp.de_words = pl.de_words;
       gp.mapB = segK;
@@ -870,7 +890,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       hp.nz_cnt = sparse ? nz_cnt + chunk : nullptr;
       hp.nz_cap = cap;
       hp.mask = dh_mask;
-      hp.mwords = pl.dh_words;
+      hp.mwords = dh_words;
       hp.n_valid = cp.n_valid;
       hp.status = status;
       if (int rc = launch_tc<DHPolicy>(hp, (int)std::min<int64_t>(sms, (int64_t)mbs * dt), st, KC_DH))
