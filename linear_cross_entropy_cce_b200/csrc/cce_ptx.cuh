@@ -222,10 +222,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // Order-preserving map of fp32 onto int32 (for integer max reductions).
 __device__ __forceinline__ int f32_to_ordered(float f) {
   int i = __float_as_int(f);
