@@ -168,7 +168,11 @@ size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs,
  *            0..n_s-1, off_s = sum of the sizes of earlier segments).  The
  *            backward walks the vocabulary in that order so that surviving
  *            blocks cluster; results do not depend on it beyond rounding.
- *            NULL = identity.
+ *            NULL = identity.  With a permutation the E rows of each
+ *            vocabulary chunk are gathered on an internal stream (one per
+ *            host thread and device, created on first use), one chunk ahead,
+ *            ordered against `stream` by events; all of the call's work is
+ *            still complete when work enqueued after it on `stream` runs.
  *   colmax   optional [V_live] fp32, the colmax output of cce_fwd on the
  *            same H, E, y and segments (a bound on every logit of each
  *            vocabulary row).  With filtering on (and without
@@ -311,7 +315,8 @@ int cce_fwd_noalloc(const void* H, const void* E, const int32_t* y,
  * launched on.  Classes: bit 0 forward tile stream, bit 1 backward G
  * producer, bit 2 backward dE contraction, bit 3 backward dH contraction,
  * bit 4 row compaction, gathers and finalize passes, bit 5 the sparse
- * gradient kernels (list sorts, gathers, dH finalize).  cce_timing_read
+ * gradient kernels (list counting, scans and scatter, the CSR gathers of dE
+ * and dH, the dH fill).  cce_timing_read
  * synchronises on the recorded events, writes per class the summed
  * milliseconds and the number of timed launches (arrays of n_classes <= 6
  * entries, host memory), and clears the record.  Not thread-safe.  Returns
