@@ -199,6 +199,8 @@ class KLWorkload:
 KL_WORKLOADS = {
     "soft_kl_24k_248k": KLWorkload("soft_kl_24k_248k", N=24576, D=2048, V=248320, logit_std=6.0),
     "soft_kl_small": KLWorkload("soft_kl_small", N=512, D=256, V=8192, logit_std=6.0),
+    # kernel captures: E (268 MB) larger than L2, about 1 GB on the device
+    "soft_kl_8k_64k": KLWorkload("soft_kl_8k_64k", N=8192, D=2048, V=65536, logit_std=6.0),
 }
 
 
