@@ -240,3 +240,32 @@ def test_all_rows_ignored():
     torch.cuda.synchronize()
     assert (loss == 0).all() and (lse == 0).all()
     assert (dH.float() == 0).all() and (dE.float() == 0).all()
+
+
+@pytest.mark.parametrize("eps", [0.0, EPS_BF16])
+def test_segmented_head_equals_compact_head(data, eps):
+    """A head with a dead gap equals the compact head [E_A; E_B] with the
+    targets past the gap moved down by the gap width: the same logits, the
+    gap contributing nothing (GPU against GPU, no oracle)."""
+    from linear_cross_entropy_cce_b200 import cce
+    x = data["composite_small"]
+    H, segs, y = upload(x)
+    (a0, a1, EA), (b0, b1, EB) = segs
+    gap = b0 - a1
+    E_c = torch.cat([EA, EB]).contiguous()
+    y_c = torch.where(y >= b0, y - gap, y)
+    loss_s, lse_s = run_fwd(x, H, segs, y)
+    loss_c, lse_c = cce.fwd(H, E_c, y_c, x.ignore_index)
+    dl = torch.from_numpy(x.dloss_mean()).cuda()
+    dH_s, dE_s, _ = run_bwd(x, H, segs, y, lse_s, dl, filter_eps=eps, fp32_grads=True)
+    dH_c, dE_c, _ = cce.bwd(H, E_c, y_c, lse_c, dl, x.ignore_index, filter_eps=eps,
+                            fp32_grads=True)
+    torch.cuda.synchronize()
+    assert torch.max(torch.abs(lse_s - lse_c)).item() <= 1e-5
+    assert torch.max(torch.abs(loss_s - loss_c)).item() <= 1e-5
+    # filtered: the two layouts may route a chunk differently (bf16 slab on
+    # the dense route, fp32 lists on the sparse one), so bf16-level agreement
+    tol = 5e-3 if eps > 0 else 1e-5
+    assert normwise(to_np(dH_s), to_np(dH_c)) <= tol
+    assert normwise(to_np(dE_s[0]), to_np(dE_c[:a1 - a0])) <= tol
+    assert normwise(to_np(dE_s[1]), to_np(dE_c[a1 - a0:])) <= tol
