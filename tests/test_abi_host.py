@@ -112,3 +112,37 @@ def test_bwd_rejects_bad_flags_and_missing_kahan_buffer():
     assert call(flags=cce.KAHAN_DE) == cce.CCE_EINVAL           # no compensation buffer
     assert call(flags=cce.KAHAN_DE | cce.FP32_GRADS, comp=16) == cce.CCE_EINVAL
     assert call(dE=None) == cce.CCE_EINVAL
+
+
+def test_kl_and_shard_entry_points_reject_bad_arguments_on_host():
+    L = cce.lib()
+    EINVAL = cce.CCE_EINVAL
+    # cce_kl_fwd(Hs, Es, Ht, Et, row_mask, N, D, V, kl, lse_s, lse_t, ws, wsb, status, stream)
+    ok = dict(Hs=16, Es=16, Ht=16, Et=16, N=4, D=8, V=10)
+
+    def kl_fwd(**kw):
+        a = dict(ok, **kw)
+        return L.cce_kl_fwd(a["Hs"], a["Es"], a["Ht"], a["Et"], None, a["N"], a["D"], a["V"],
+                            16, 16, 16, 16, 1 << 30, 16, None)
+    assert kl_fwd(Hs=None) == EINVAL
+    assert kl_fwd(Et=None) == EINVAL
+    assert kl_fwd(Ht=24) == EINVAL          # not 16-byte aligned
+    assert kl_fwd(D=12) == EINVAL           # D % 8 != 0
+    assert kl_fwd(N=0) == cce.CCE_OK        # nothing to do
+
+    # cce_kl_bwd(Hs, Es, Ht, Et, mask, lse_s, lse_t, dloss, N, D, V, eps, flags, dH, dE, dE_comp,
+    #            ws, wsb, status, stream)
+    def kl_bwd(flags=0, Ht=16):
+        return L.cce_kl_bwd(16, 16, Ht, 16, None, 16, 16, 16, 4, 8, 10, 0.0, flags, 16, 16, None,
+                            16, 1 << 30, 16, None)
+    assert kl_bwd(flags=cce.FULL_DE) == EINVAL
+    assert kl_bwd(flags=cce.VOCAB_SHARD) == EINVAL
+    assert kl_bwd(Ht=None) == EINVAL
+    assert L.cce_kl_bwd_workspace_size(256, 256, 4096, 0) > L.cce_bwd_workspace_size(256, 256, 4096, 0, 0)
+    assert L.cce_kl_fwd_workspace_size(256, 250, 4096) == 0
+
+    # cce_fwd_shard: the cce_fwd argument checks
+    assert L.cce_fwd_shard(None, 16, 16, 4, 8, 10, -100, None, 0, 16, 16, None, 16, 1 << 30, 16,
+                           None) == EINVAL
+    assert L.cce_fwd_shard(16, 16, 16, 4, 8, 10, -100, None, 0, None, 16, None, 16, 1 << 30, 16,
+                           None) == EINVAL
