@@ -28,7 +28,7 @@ A composite head is a list of segments on the logical vocabulary; ids that no
 segment covers form the dead gap whose logits are -inf ([LM] §What transfers
 to us, third bullet).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   * no bias, temperature or soft-capping on the logits;
   * ignored rows (y == ignore_index) have loss = lse = 0 and zero gradient;
   * a target outside [0, V) or inside the gap yields NaN loss/lse for its row;
@@ -248,7 +248,7 @@ def kahan_reference(parts: Sequence[np.ndarray]) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # Soft-target KL ([DE] §The OOM: the KL divergence between the student and the
 # teacher softmax over the whole vocabulary, computed in position chunks).
-# Readings where the page is silent (each also listed in the design doc):
+# Readings where the page is silent:
 #   * direction KL(p_t || p_s): the teacher distribution is the target;
 #   * temperature 1, no bias; p_s = softmax(H_s E_s^T), p_t = softmax(H_t E_t^T)
 #     (E_s and E_t may be the same head);
