@@ -100,14 +100,30 @@ def exchange_backward(dH_part: torch.Tensor, group=None) -> torch.Tensor:
     return dH_part
 
 
+def shard_forward_parts(H: torch.Tensor, y: torch.Tensor, local: Sequence[SegSpec], V: int,
+                        ignore_index: int = -100, want_colmax: bool = False):
+    """This rank's (lse part, correct-token logit part, ownership[, colmax]).
+    A rank whose range holds no ids (more ranks than 256-aligned ranges)
+    contributes -inf to the log-add-exp and nothing else, without a launch."""
+    if not local:
+        n = H.shape[0]
+        lse_p = torch.full((n,), float("-inf"), dtype=torch.float32, device=H.device)
+        zero = torch.zeros(n, dtype=torch.float32, device=H.device)
+        parts = (lse_p, zero, zero.clone())
+        return parts + (torch.empty(0, dtype=torch.float32, device=H.device),) if want_colmax else parts
+    out = cce.fwd(H, None, y, ignore_index, segments=list(local), V=V, shard=True,
+                  want_colmax=want_colmax)
+    parts = (out[1], out[0], owned(y, local))
+    return parts + (out[2],) if want_colmax else parts
+
+
 def vp_forward(H: torch.Tensor, y: torch.Tensor, local: Sequence[SegSpec], V: int,
                ignore_index: int = -100, group=None, want_colmax: bool = False):
     """Forward over this rank's shard plus the exchange; returns (loss, lse)
     for every row (identical on all ranks), and the shard's colmax if asked."""
-    out = cce.fwd(H, None, y, ignore_index, segments=list(local), V=V, shard=True,
-                  want_colmax=want_colmax)
-    loss, lse = exchange_forward(out[1], out[0], owned(y, local), y, ignore_index, group)
-    return (loss, lse, out[2]) if want_colmax else (loss, lse)
+    parts = shard_forward_parts(H, y, local, V, ignore_index, want_colmax)
+    loss, lse = exchange_forward(parts[0], parts[1], parts[2], y, ignore_index, group)
+    return (loss, lse, parts[3]) if want_colmax else (loss, lse)
 
 
 def vp_backward(H: torch.Tensor, y: torch.Tensor, lse: torch.Tensor, dloss: torch.Tensor,
@@ -117,6 +133,11 @@ def vp_backward(H: torch.Tensor, y: torch.Tensor, lse: torch.Tensor, dloss: torc
     """Backward over this rank's shard with the full lse; returns (dH summed
     over ranks, this shard's dE per local segment), bf16."""
     bad = torch.isnan(lse) & (y != ignore_index)
+    if not local:  # a rank without ids: a zero share of dH, no dE
+        dH = torch.zeros(H.shape, dtype=torch.float32, device=H.device)
+        exchange_backward(dH, group)
+        dH[bad] = float("nan")
+        return dH.to(torch.bfloat16), []
     lse_b = torch.where(bad, torch.zeros_like(lse), lse)
     dl = torch.where(bad, torch.zeros_like(dloss), dloss).to(torch.float32).contiguous()
     dH, dEs, _ = cce.bwd(H, None, y, lse_b, dl, ignore_index, segments=list(local), V=V,

@@ -132,3 +132,20 @@ def test_exchanges_world2_gloo():
         assert np.allclose(loss[~bad], rl[~bad], atol=1e-9, rtol=0)
         assert np.allclose(lse[~bad], rlse[~bad], atol=1e-9, rtol=0)
         assert np.allclose(dH[~bad], rH[~bad], atol=1e-10, rtol=1e-8)
+
+
+def test_rank_without_ids_contributes_nothing():
+    """More ranks than 256-aligned ranges leave some ranks an empty shard:
+    their parts are -inf / 0 / 0 (no launch), and the combine is unchanged."""
+    ranges = vp.shard_ranges(600, 4)
+    assert ranges[-1] == (600, 600)
+    H = torch.zeros((6, 8))
+    y = torch.tensor([0, 5, -100, 599, 300, 1], dtype=torch.int32)
+    lse_p, zy_p, own = vp.shard_forward_parts(H, y, [], 600)
+    assert torch.all(torch.isinf(lse_p) & (lse_p < 0)) and torch.all(zy_p == 0) and torch.all(own == 0)
+    full = torch.tensor([[1.0, 2.0, 0.0, 3.0, 0.5, 1.5], [0.2, 0.1, 0.0, 0.3, 0.4, 0.2],
+                         [1.0, 1.0, 0.0, 1.0, 1.0, 1.0]])
+    parts = torch.stack([full, torch.stack([lse_p, zy_p, own])])
+    loss, lse = vp.combine_shards(parts, y)
+    ref_loss, ref_lse = vp.combine_shards(full[None], y)
+    assert torch.equal(loss, ref_loss) and torch.equal(lse, ref_lse)
