@@ -146,3 +146,22 @@ def test_kl_and_shard_entry_points_reject_bad_arguments_on_host():
                            None) == EINVAL
     assert L.cce_fwd_shard(16, 16, 16, 4, 8, 10, -100, None, 0, None, 16, None, 16, 1 << 30, 16,
                            None) == EINVAL
+
+
+def test_plain_c_consumer(tmp_path):
+    """tests/c_abi_check.c: a C99 program that includes only include/cce.h and
+    links libcce.so checks the host-side contract."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    cce.lib()  # built
+    libdir = os.path.join(ROOT, "linear_cross_entropy_cce_b200")
+    exe = str(tmp_path / "c_abi_check")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-D_DEFAULT_SOURCE",
+                    "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_abi_check.c"),
+                    "-L", libdir, "-lcce", "-Wl,-rpath," + libdir, "-o", exe], check=True)
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert "c abi ok" in out.stdout
