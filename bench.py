@@ -228,7 +228,9 @@ def main():
     dev = torch.device("cuda", local)
     if world > 1:
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        # the bound on ranks waiting for one another; generous because every
+        # rank first draws its inputs on the shared host cores
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
 
     x = syn.make_inputs(wl, seed=rank)
     H = cce.bf16_from_bits(x.H, dev)
@@ -480,7 +482,7 @@ def kl_main(a, world, rank, local):
     dev = torch.device("cuda", local)
     if world > 1:
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
     N, D, V = wl.N, wl.D, wl.V
     Hs_d, Ht_d, E_d = (cce.bf16_from_bits(t, dev) for t in (Hs, Ht, E))
     dl = torch.full((N,), 1.0 / N, dtype=torch.float32, device=dev)
