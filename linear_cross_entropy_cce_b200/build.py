@@ -4,6 +4,7 @@
 """
 from __future__ import annotations
 
+import glob
 import os
 import subprocess
 import sys
@@ -13,12 +14,14 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libcce.so")
 SOURCES = ["cce_api.cu", "cce_noalloc.cu"]
-HEADERS = ["cce_ptx.cuh", "cce_engine.cuh", "cce_kernels.cuh", "cce_sparse.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 
 def _inputs():
-    return [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(ROOT, "include", "cce.h")]
+    """Every file the library is built from: all CUDA sources and headers
+    under csrc/ (so an edit to any kernel header triggers a rebuild) and the
+    public header."""
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu*"))) + [os.path.join(ROOT, "include", "cce.h")]
 
 
 def needs_build() -> bool:
