@@ -1,14 +1,20 @@
 #!/usr/bin/env python
 """Fused classifier matmul + cross-entropy, forward+backward, on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--parallel dp|vocab] [--impl ours|reference]
 
 One step = the whole hot path on one batch of synthetic input, inputs already
 resident in HBM: cce_fwd (loss, lse, and the colmax statistic when the
 vocabulary sort is on) -> cce_vocab_sort (when on) -> cce_bwd (dH, dE).
-Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one process per GPU)
-every rank runs its own batch (weak scaling, no collective on the data path);
-the time is the max over ranks.
+Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one process per GPU):
+  --parallel dp     every rank runs its own batch (weak scaling, no collective
+                    on the data path);
+  --parallel vocab  the classifier is split by vocabulary over the ranks and
+                    all ranks run the same batch (strong scaling): shard
+                    forward, an all-gather of the [2, N] per-row parts and the
+                    combine kernel, shard backward, an all-reduce of dH.
+The time is the max over ranks.
 
 `--impl reference` times the fp64 CPU oracle on a bounded row sample of the
 same workload on the host cores (the only other place this file runs the
@@ -45,12 +51,39 @@ MODES = {
 L2_BYTES = 126 * 2 ** 20
 
 
+# The peaks measured on this machine's B200s by the benchmark driver (cuBLAS bf16
+# 8192^3 burst and 4 s sustained under the power cap; STREAM-style copy),
+# used when the driver's MEASURED_PEAKS.json is not in the tree.
+RECORDED_PEAKS = {"bf16_tflops": 1665.4, "bf16_tflops_sustained": 1339.0, "hbm_gbs": 6547.0}
+
+
 def peaks():
+    """(peaks, source): MEASURED_PEAKS.json when present, else the recorded
+    measurement of this machine."""
     try:
-        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "MEASURED_PEAKS.json"
     except Exception:
-        return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0,
-                "fallback": True}
+        return dict(RECORDED_PEAKS), "recorded measurement of this pool (MEASURED_PEAKS.json absent)"
+
+
+def tensor_roofline(kernel: str, flops_per_step: float, steps: int, ms_total: float, n_launches: int,
+                    P: dict, src: str) -> dict:
+    """Roofline entry of a tensor-core kernel class: achieved = its
+    algorithmic FLOPs over the summed CUDA-event durations of its launches;
+    frac against the measured burst bf16 peak (the kernels are timed as
+    millisecond launches), the sustained figure beside it."""
+    achieved = flops_per_step * steps / (ms_total / 1e3) / 1e12 if ms_total > 0 else None
+    burst = float(P["bf16_tflops"])
+    sus = float(P.get("bf16_tflops_sustained", burst))
+    return {"bound": "tensor", "kernel": kernel,
+            "achieved": round(achieved, 1) if achieved else None, "peak": burst,
+            "unit": "TFLOP/s", "frac": round(achieved / burst, 4) if achieved else None,
+            "peak_kind": "burst bf16 (measured, cuBLAS), of measured",
+            "peak_source": src,
+            "frac_of_sustained": round(achieved / sus, 4) if achieved else None,
+            "sustained_peak": sus,
+            "launches_per_step": n_launches // max(1, steps),
+            "avg_launch_ms": round(ms_total / max(1, n_launches), 4)}
 
 
 def src_hash16():
@@ -181,6 +214,16 @@ def tokens_per_s(tokens_per_rank: int, world: int, ms: float) -> float:
     return tokens_per_rank * world / (ms / 1e3)
 
 
+def vocab_shard_plan(segments, V: int, world: int, rank: int):
+    """This rank's part of the head for --parallel vocab: the segments
+    [(begin, end, E_rows)] of the head cut to the rank's 256-aligned vocabulary
+    range (rows sliced, no copy; empty for a rank whose range holds no ids)."""
+    from linear_cross_entropy_cce_b200 import vocab_parallel as vp
+    v0, v1 = vp.shard_ranges(V, world)[rank]
+    return [(lo, hi, E[lo - b:hi - b]) for b, e, E in segments
+            for lo, hi in [(max(b, v0), min(e, v1))] if lo < hi]
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -189,6 +232,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="gemma2_2b_head", choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--parallel", default="dp", choices=["dp", "vocab"],
+                    help="dp: one batch per rank; vocab: the classifier split by vocabulary "
+                         "over the ranks, one shared batch")
     ap.add_argument("--filter", choices=["on", "off", "default"], default="default")
     ap.add_argument("--sort", choices=["on", "off", "default"], default="default")
     ap.add_argument("--loss", choices=["ce", "kl"], default="ce",
@@ -223,6 +269,7 @@ def main():
     import torch
     import torch.distributed as dist
     from linear_cross_entropy_cce_b200 import cce
+    from linear_cross_entropy_cce_b200 import vocab_parallel as vp
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -232,15 +279,25 @@ def main():
         # rank first draws its inputs on the shared host cores
         dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
 
-    x = syn.make_inputs(wl, seed=rank)
+    vocab = a.parallel == "vocab"
+    # vocabulary parallel: one batch shared by all ranks, each holding the E
+    # rows of its vocabulary range; data parallel: one batch per rank
+    x = syn.make_inputs(wl, seed=0 if vocab else rank)
+    N, D, V = wl.N, wl.D, wl.V
+    n_valid = x.n_valid
+    if vocab:
+        host_segs = vocab_shard_plan(x.segments, V, world, rank)
+    else:
+        host_segs = list(x.segments)
+    head_ranges = list(wl.segs())
     H = cce.bf16_from_bits(x.H, dev)
-    segs = [(b, e, cce.bf16_from_bits(E, dev)) for b, e, E in x.segments]
-    single = len(segs) == 1 and segs[0][0] == 0 and segs[0][1] == wl.V
+    segs = [(b, e, cce.bf16_from_bits(E, dev)) for b, e, E in host_segs]
+    single = (not vocab) and len(segs) == 1 and segs[0][0] == 0 and segs[0][1] == V
     y = torch.from_numpy(x.y).to(dev)
     dloss = torch.from_numpy(x.dloss_mean()).to(dev)
-    N, D, V = wl.N, wl.D, wl.V
-    nseg = 0 if single else len(segs)
-    n_valid, v_live = x.n_valid, wl.v_live
+    nseg = 0 if single else max(1, len(segs))
+    v_live_rank = sum(e - b for b, e, _ in segs)
+    v_live = wl.v_live
     ws_f = torch.empty(cce.fwd_workspace_size(N, D, V, nseg), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(cce.bwd_workspace_size(N, D, V, nseg), dtype=torch.uint8, device=dev)
     ws_s = torch.empty(cce.vocab_sort_workspace_size(N, V, nseg), dtype=torch.uint8, device=dev)
@@ -248,11 +305,13 @@ def main():
     input_bytes = H.numel() * 2 + sum(s[2].numel() * 2 for s in segs) + y.numel() * 4
     kahan_kw = {}
     if a.kahan:  # running bf16 sum and compensation, kept across steps
+        if vocab:
+            ap.error("--kahan runs with --parallel dp")
         S = [torch.zeros_like(t) for _, _, t in segs]
         C = [torch.zeros_like(t) for _, _, t in segs]
         kahan_kw = dict(kahan=True, dE_out=S[0] if single else S, dE_comp=C[0] if single else C)
 
-    def step(Hd=H, segd=segs, yd=y):
+    def dp_step(Hd=H, segd=segs, yd=y):
         kw = dict(workspace=ws_f, status=status)
         if single:
             out = cce.fwd(Hd, segd[0][2], yd, x.ignore_index, want_colmax=sort, **kw)
@@ -271,7 +330,23 @@ def main():
             dH, dE, _ = cce.bwd(Hd, None, yd, lse, dloss, x.ignore_index, segments=segd, V=V, **kw)
         return loss, dH, dE
 
+    def vocab_step(Hd=H, segd=segs, yd=y):
+        # shard forward + all-gather + combine kernel; shard backward + all-reduce
+        out = vp.vp_forward(Hd, yd, segd, V, x.ignore_index, want_colmax=sort,
+                            head_ranges=head_ranges)
+        loss, lse = out[0], out[1]
+        perm = None
+        if sort and segd:
+            perm = cce.vocab_sort(out[2], yd, V, x.ignore_index, segments=segd, workspace=ws_s)
+        dH, dE = vp.vp_backward(Hd, yd, lse, dloss, segd, V, x.ignore_index, filter_eps=eps,
+                                vocab_perm=perm, colmax=out[2] if (sort and segd) else None)
+        return loss, dH, dE
+
+    step = vocab_step if vocab else dp_step
+
     def fwd_only():
+        if vocab:
+            return vp.vp_forward(H, y, segs, V, x.ignore_index, head_ranges=head_ranges)
         if single:
             return cce.fwd(H, segs[0][2], y, x.ignore_index, workspace=ws_f, status=status)
         return cce.fwd(H, None, y, x.ignore_index, segments=segs, V=V, workspace=ws_f,
@@ -330,7 +405,7 @@ def main():
     e2e = None
     if not a.no_e2e:
         hH = torch.from_numpy(x.H.view(np.int16)).pin_memory()
-        hE = [torch.from_numpy(E.view(np.int16)).pin_memory() for _, _, E in x.segments]
+        hE = [torch.from_numpy(E.view(np.int16)).pin_memory() for _, _, E in host_segs]
         hy = torch.from_numpy(x.y).pin_memory()
         hloss = torch.empty(N, dtype=torch.float32).pin_memory()
         dH_ = torch.empty_like(H)
@@ -350,35 +425,32 @@ def main():
             e2e_step()
         ms_e2e = timed(e2e_step, a.steps)
         h2d = hH.numel() * 2 + sum(h.numel() * 2 for h in hE) + hy.numel() * 4
-        e2e = {"value": round(tokens_per_s(N, world, ms_e2e), 1), "unit": UNIT,
+        tok_e2e = N / (ms_e2e / 1e3) if vocab else tokens_per_s(N, world, ms_e2e)
+        e2e = {"value": round(tok_e2e, 1), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(N * 4),
                "ms_per_step": round(ms_e2e, 3)}
 
-    P = peaks()
-    flops_fwd = 2.0 * n_valid * D * v_live
-    flops_step = 8.0 * n_valid * D * v_live
+    P, psrc = peaks()
+    flops_fwd = 2.0 * n_valid * D * v_live_rank  # per rank (its vocabulary shard in vocab mode)
+    flops_step_job = 8.0 * n_valid * D * v_live * (1 if vocab else world)
     class_flops = {"fwd_tile_stream": flops_fwd, "bwd_g_producer": flops_fwd,
                    "bwd_dE_contraction": flops_fwd, "bwd_dH_contraction": flops_fwd}
     dom = max(class_flops, key=lambda k: per_class[k][0])
     dom_ms, dom_n = per_class[dom]
-    achieved = class_flops[dom] * a.steps / (dom_ms / 1e3) / 1e12 if dom_ms > 0 else None
-    peak_sus = float(P.get("bf16_tflops_sustained", P.get("bf16_tflops")))
-    peak_burst = float(P["bf16_tflops"])
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1) if achieved else None,
-                "peak": peak_sus, "unit": "TFLOP/s",
-                "frac": round(achieved / peak_sus, 4) if achieved else None,
-                "peak_kind": "sustained bf16 (measured, cuBLAS) - kernel timed inside the step",
-                "traffic": recorded_traffic(dom) if wl.name == "gemma2_2b_head" else None,
-                "traffic_note": "DRAM bytes of one working launch of this kernel (one vocabulary chunk "
-                                "for the G producer) from the committed ncu capture "
-                                "(profiles/roofline_traffic.json, cold cache); null if the sources changed",
-                "achieved_note": "algorithmic FLOPs of the class per step over the summed CUDA-event "
-                                 "durations of all its launches in the step",
-                "launches_per_step": dom_n // max(1, a.steps),
-                "launches_note": "the G producer launches twice per vocabulary chunk; the second "
-                                 "(repair) launch exits at once unless the chunk overflowed its sparse list",
-                "avg_launch_ms": round(dom_ms / max(1, dom_n), 4)}
-    step_tflops = flops_step / (ms_step / 1e3) / 1e12
+    roofline = tensor_roofline(dom, class_flops[dom], a.steps, dom_ms, dom_n, P, psrc)
+    roofline.update({
+        "traffic": recorded_traffic(dom) if (wl.name == "gemma2_2b_head" and not vocab) else None,
+        "traffic_note": "DRAM bytes of one working launch of this kernel (one vocabulary chunk "
+                        "for the G producer) from the committed ncu capture "
+                        "(profiles/roofline_traffic.json, cold cache); null if the sources changed",
+        "achieved_note": "algorithmic FLOPs of the class per step (2 N_v D V_live of this rank) "
+                         "over the summed CUDA-event durations of all its launches in the step",
+        "launches_note": "the G producer launches twice per vocabulary chunk when filtering; the "
+                         "second (repair) launch exits at once unless the chunk overflowed its "
+                         "sparse list"})
+    step_tflops = flops_step_job / (ms_step / 1e3) / 1e12
+    burst = float(P["bf16_tflops"])
+    sustained = float(P.get("bf16_tflops_sustained", burst))
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -386,22 +458,28 @@ def main():
         cpu = {"value": round(rps, 3), "unit": UNIT, "cores": host_cores(), "kind": "oracle",
                "sample": desc, "seconds": round(t, 2)}
 
+    value = N / (ms_step / 1e3) if vocab else tokens_per_s(N, world, ms_step)
+    parallelism = (f"vocab{world} (E split by vocabulary, one shared batch)" if vocab
+                   else f"dp{world} (independent batches)")
     out = {
-        "metric": METRIC, "value": round(tokens_per_s(N, world, ms_step), 1), "unit": UNIT,
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT,
         "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_step, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if vocab else "weak", "vs_baseline": None,
+        "dtype": "bf16",
         "data": "synthetic (seeded; shapes and value recipe of the workload; no dataset or trained weights)",
         "config": {"workload": wl.name, "N": N, "N_valid": n_valid, "D": D, "V": V,
-                   "V_live": v_live, "segments": [list(s) for s in wl.segs()],
+                   "V_live": v_live, "V_live_per_rank": v_live_rank,
+                   "segments": [list(s) for s in wl.segs()],
                    "logit_std": wl.logit_std, "filter_eps": eps, "vocab_sort": sort,
                    "kahan_dE": bool(a.kahan),
-                   "global_batch_tokens": N * world, "parallelism": f"dp{world} (independent batches)",
-                   "l2": f"inputs larger than L2 (E = {sum(s[2].numel() for s in segs) * 2 / 2**20:.0f} MiB > 126 MiB)",
-                   "tokens_per_s_valid_rows": round(n_valid * world / (ms_step / 1e3), 1)},
-        "tensor_peak_frac": {"of_measured_burst": round(step_tflops / peak_burst, 4),
-                             "of_measured_sustained": round(step_tflops / peak_sus, 4),
+                   "global_batch_tokens": N if vocab else N * world, "parallelism": parallelism,
+                   "l2": f"inputs larger than L2 (E = {sum(s[2].numel() for s in segs) * 2 / 2**20:.0f} MiB per rank > 126 MiB)",
+                   "tokens_per_s_valid_rows": round(value * n_valid / N, 1)},
+        "tensor_peak_frac": {"of_measured_burst": round(step_tflops / burst, 4),
+                             "of_measured_sustained": round(step_tflops / sustained, 4),
                              "of_spec_2250": round(step_tflops / 2250.0, 4),
-                             "tflops_unfiltered_8NDV": round(step_tflops, 1)},
+                             "tflops_unfiltered_8NDV": round(step_tflops, 1),
+                             "peak_source": psrc},
         "fwd_ms": round(ms_fwd, 3), "fwd_bwd_ms": round(ms_step, 3),
         "peak_mb": round((peak_extra + ws_bytes) / 2 ** 20, 1),
         "peak_mb_detail": {"workspaces_mb": round(ws_bytes / 2 ** 20, 1),
@@ -527,14 +605,15 @@ def kl_main(a, world, rank, local):
     per_class = cce.timing_read()
     cce.timing_enable(0)
 
-    P = peaks()
+    P, psrc = peaks()
     ndv = float(N) * D * V
     class_flops = {"fwd_tile_stream": 4 * ndv, "bwd_g_producer": 4 * ndv,
                    "bwd_dE_contraction": 2 * ndv, "bwd_dH_contraction": 2 * ndv}
     dom = max(class_flops, key=lambda k: per_class[k][0])
     dom_ms, dom_n = per_class[dom]
-    achieved = class_flops[dom] * a.steps / (dom_ms / 1e3) / 1e12 if dom_ms > 0 else None
-    peak_sus = P.get("bf16_tflops_sustained", 1400.0)
+    roofline = tensor_roofline(dom, class_flops[dom], a.steps, dom_ms, dom_n, P, psrc)
+    roofline["traffic"] = None
+    peak_sus = float(P.get("bf16_tflops_sustained", P["bf16_tflops"]))
     step_tflops = 12 * ndv / (ms_step / 1e3) / 1e12
 
     e2e = None
@@ -572,17 +651,11 @@ def kl_main(a, world, rank, local):
         "config": {"workload": wl.name, "N": N, "D": D, "V": V, "logit_std": wl.logit_std,
                    "filter_eps": eps, "parallelism": f"dp{world} (independent batches)",
                    "l2": f"inputs larger than L2 (E = {E.size * 2 / 2**20:.0f} MiB > 126 MiB)"},
-        "tensor_peak_frac": {"of_measured_burst": round(step_tflops / P.get("bf16_tflops", 1590.0), 4),
+        "tensor_peak_frac": {"of_measured_burst": round(step_tflops / float(P["bf16_tflops"]), 4),
                              "of_measured_sustained": round(step_tflops / peak_sus, 4),
                              "tflops_unfiltered_12NDV": round(step_tflops, 1)},
         "fwd_ms": round(ms_fwd, 3), "fwd_bwd_ms": round(ms_step, 3),
-        "roofline": {"bound": "tensor", "kernel": dom,
-                     "achieved": round(achieved, 1) if achieved else None,
-                     "peak": peak_sus, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak_sus, 4) if achieved else None,
-                     "traffic": None,
-                     "peak_kind": "sustained bf16 (measured, cuBLAS)",
-                     "launches_per_step": dom_n // max(1, a.steps)},
+        "roofline": roofline,
         "per_kernel_ms_per_step": {k: round(v[0] / a.steps, 3) for k, v in per_class.items()},
         "gpu_launches": int(launches), "gpu_launches_per_step": int(launches // max(1, a.steps)),
         "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,

@@ -61,6 +61,7 @@ extern "C" {
 #define CCE_FP32_GRADS 2u /* dH and dE are written as fp32 instead of bf16     */
 #define CCE_FULL_DE 4u    /* filter only dH; the classifier gradient dE is full */
 #define CCE_VOCAB_SHARD 8u /* E is one rank's vocabulary shard (see cce_fwd_shard) */
+#define CCE_FP32_DH 16u   /* dH alone is written as fp32 (dE keeps its type)    */
 
 #define CCE_MAX_SEGMENTS 8
 
@@ -148,6 +149,29 @@ int cce_fwd_shard(const void* H, const void* E, const int32_t* y,
                   void* workspace, size_t workspace_bytes,
                   int32_t* status, void* stream);
 
+/*
+ * Combine step of the vocabulary-parallel forward, run by every rank after
+ * the all-gather of the shards' per-row parts.
+ *   parts    [R, 2, N] fp32 device: for each of the R shards (ranks), the
+ *            lse_part and zy_part rows of cce_fwd_shard.  A shard without
+ *            vocabulary ids passes -inf and 0.
+ *   y        [N] int32 targets.
+ *   V, segs, n_segs  the whole head's logical vocabulary and live ranges
+ *            (as for cce_fwd; only vocab_begin / vocab_end are read, E may
+ *            be NULL); NULL / 0 = one range [0, V).
+ *   loss,lse [N] fp32 outputs: lse = log-add-exp of lse_part over shards,
+ *            loss = lse - sum of zy_part ("Cut Your Losses in Large-Vocabulary
+ *            Language Models", research-map entry §Limitations: log-add-exp
+ *            of partial results; first page §What transfers to us: the lse
+ *            of a composite head composes over its parts, a dead gap adding
+ *            -inf).  Ignored rows give 0; a target outside the live ranges
+ *            (no shard holds it) gives NaN, as a bad target does in cce_fwd.
+ * Returns CCE_EINVAL for R outside [1, 4096], bad ranges or a NULL pointer.
+ */
+int cce_vocab_combine(const float* parts, int32_t R, const int32_t* y, int64_t N, int64_t V,
+                      int32_t ignore_index, const cce_segment* segs, int32_t n_segs,
+                      float* loss, float* lse, void* stream);
+
 /* Workspace bytes cce_bwd needs (0 on invalid sizes). */
 size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs,
                               uint32_t flags);
@@ -184,9 +208,12 @@ size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs,
  *            and of the research-map entry's §Approach, taken exactly.  The
  *            skip never changes which entries are kept.  A colmax that is not such a bound
  *            drops gradient entries.  NULL = no tile skip.
- *   flags    CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE | CCE_VOCAB_SHARD
- *            (the backward of cce_fwd_shard: lse is the combined one, dH this
- *            shard's share).  CCE_FULL_DE keeps
+ *   flags    CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE | CCE_VOCAB_SHARD |
+ *            CCE_FP32_DH
+ *            (CCE_VOCAB_SHARD: the backward of cce_fwd_shard: lse is the
+ *            combined one, dH this shard's share; CCE_FP32_DH writes dH in
+ *            fp32 while dE stays bf16 (or Kahan), for dH shares that are
+ *            summed over ranks before rounding).  CCE_FULL_DE keeps
  *            the classifier gradient dE unfiltered while dH uses the filtered
  *            softmax (the "FullC" variant of "Cut Your Losses in
  *            Large-Vocabulary Language Models", research-map entry, §Key
@@ -303,6 +330,19 @@ int cce_fwd_noalloc(const void* H, const void* E, const int32_t* y,
                     const cce_segment* segs, int32_t n_segs,
                     float* loss, float* lse, float* colmax,
                     int32_t* status, void* stream);
+
+/*
+ * Diagnostic of the bounded waits (not needed for computing anything).
+ * Launches one CTA of the tensor-core tile engine whose producer never fills
+ * a stage: the MMA issuer's wait runs out after wait_ns nanoseconds of wall
+ * clock, the CTA aborts, drains, frees its tensor memory and returns, and
+ * CCE_STATUS_TIMEOUT is OR-ed into *status.  Every other kernel of the
+ * library handles a wait that cannot complete this way (with a 2 s limit),
+ * so the stream and the context stay usable.  No copy or MMA is issued.
+ *   wait_ns  1 .. 1e9 (else CCE_EINVAL).
+ *   status   device int32.
+ */
+int cce_debug_stall(uint64_t wait_ns, int32_t* status, void* stream);
 
 /*
  * Diagnostics (not needed for computing anything).

@@ -21,44 +21,54 @@ from . import cce
 
 class _LinearCrossEntropy(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, H, E, y, ignore_index, filter_eps, full_de, vocab_sort, segments_meta, *seg_E):
+    def forward(ctx, H, E, y, ignore_index, filter_eps, full_de, vocab_sort, check, segments_meta,
+                *seg_E):
         segments = [(b, e, t) for (b, e), t in zip(segments_meta, seg_E)] if segments_meta else None
         V = segments_meta[-1][1] if segments_meta else None
+        st = torch.zeros(1, dtype=torch.int32, device=H.device) if check else None
         if vocab_sort:
             loss, lse, colmax = cce.fwd(H, E, y, ignore_index, segments=segments, V=V,
-                                        want_colmax=True)
+                                        want_colmax=True, status=st)
             perm = cce.vocab_sort(colmax, y, V if segments else E.shape[0], ignore_index,
                                   segments=segments)
         else:
-            loss, lse = cce.fwd(H, E, y, ignore_index, segments=segments, V=V)
+            loss, lse = cce.fwd(H, E, y, ignore_index, segments=segments, V=V, status=st)
             perm = colmax = None
+        if check:
+            cce.check_status(st, "cce_fwd")
         ctx.save_for_backward(H, E if E is not None else torch.empty(0), y, lse,
                               perm if perm is not None else torch.empty(0),
                               colmax if colmax is not None else torch.empty(0), *seg_E)
-        ctx.meta = (ignore_index, filter_eps, full_de, segments_meta, E is not None, perm is not None)
+        ctx.meta = (ignore_index, filter_eps, full_de, check, segments_meta, E is not None,
+                    perm is not None)
         return loss
 
     @staticmethod
     def backward(ctx, grad_loss):
         H, E, y, lse, perm, colmax, *seg_E = ctx.saved_tensors
-        ignore_index, filter_eps, full_de, segments_meta, has_E, has_perm = ctx.meta
+        ignore_index, filter_eps, full_de, check, segments_meta, has_E, has_perm = ctx.meta
         segments = [(b, e, t) for (b, e), t in zip(segments_meta, seg_E)] if segments_meta else None
         V = segments_meta[-1][1] if segments_meta else None
         dloss = grad_loss.contiguous().to(torch.float32)
+        st = torch.zeros(1, dtype=torch.int32, device=H.device) if check else None
         dH, dE, _ = cce.bwd(H, E if has_E else None, y, lse, dloss, ignore_index, segments=segments,
                             V=V, filter_eps=filter_eps, vocab_perm=perm if has_perm else None,
-                            colmax=colmax if has_perm else None, full_de=full_de)
+                            colmax=colmax if has_perm else None, full_de=full_de, status=st)
+        if check:
+            cce.check_status(st, "cce_bwd")
         dH = dH.to(H.dtype)
         if segments:
-            return (dH, None, None, None, None, None, None, None, *[g.to(t.dtype) for g, t in zip(dE, seg_E)])
-        return (dH, dE.to(E.dtype), None, None, None, None, None, None)
+            return (dH, None, None, None, None, None, None, None, None,
+                    *[g.to(t.dtype) for g, t in zip(dE, seg_E)])
+        return (dH, dE.to(E.dtype), None, None, None, None, None, None, None)
 
 
 def linear_cross_entropy(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor,
                          ignore_index: int = -100, reduction: str = "mean",
                          filter_eps: float = 2.0 ** -12, full_de: bool = False,
                          vocab_sort: bool = False,
-                         segments: Optional[Sequence] = None) -> torch.Tensor:
+                         segments: Optional[Sequence] = None,
+                         check_status: bool = False) -> torch.Tensor:
     """Cross-entropy of the logits H @ E^T (never materialised) against y.
 
     H [N, D] bf16, E [V, D] bf16 (or `segments` = [(begin, end, E_s), ...] for
@@ -69,13 +79,16 @@ def linear_cross_entropy(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Te
     vocab_sort walks the vocabulary in descending max-logit order in the
     backward and, with the filter on, skips the tiles whose every softmax
     entry the forward's column maxima bound below filter_eps.
+    check_status: after each library call, synchronise and raise CCEError if
+    a kernel reported a bad target (NaN rows) or a wait that ran out
+    (incomplete outputs); off by default because it costs a host sync.
     """
     if y.dtype != torch.int32:
         y = y.to(torch.int32)
     meta = tuple((int(b), int(e)) for b, e, _ in segments) if segments else ()
     seg_E = tuple(t for _, _, t in segments) if segments else ()
     per_row = _LinearCrossEntropy.apply(H, E, y, ignore_index, float(filter_eps), bool(full_de),
-                                        bool(vocab_sort), meta, *seg_E)
+                                        bool(vocab_sort), bool(check_status), meta, *seg_E)
     if reduction == "none":
         return per_row
     if reduction == "sum":

@@ -18,13 +18,14 @@ LIB_PATH = os.path.join(_PKG, "libcce.so")
 
 CCE_OK, CCE_EINVAL, CCE_EWORKSPACE, CCE_ELAUNCH, CCE_EDEVICE = 0, 1, 2, 3, 4
 STATUS_BADTARGET, STATUS_TIMEOUT = 1, 2
-KAHAN_DE, FP32_GRADS, FULL_DE, VOCAB_SHARD = 1, 2, 4, 8
+KAHAN_DE, FP32_GRADS, FULL_DE, VOCAB_SHARD, FP32_DH = 1, 2, 4, 8, 16
 MAX_SEGMENTS = 8
 
 EXPORTS = ("cce_version", "cce_strerror", "cce_fwd_workspace_size", "cce_fwd", "cce_fwd_shard",
            "cce_bwd_workspace_size", "cce_bwd", "cce_vocab_sort_workspace_size",
            "cce_vocab_sort", "cce_launch_count", "cce_timing_enable", "cce_timing_read",
-           "cce_kl_fwd_workspace_size", "cce_kl_fwd", "cce_kl_bwd_workspace_size", "cce_kl_bwd")
+           "cce_kl_fwd_workspace_size", "cce_kl_fwd", "cce_kl_bwd_workspace_size", "cce_kl_bwd",
+           "cce_vocab_combine", "cce_fwd_noalloc", "cce_debug_stall")
 # kernel classes for cce_timing_enable / cce_timing_read
 KC_FWD, KC_G, KC_DE, KC_DH, KC_AUX, KC_SPARSE = 0, 1, 2, 3, 4, 5
 KC_NAMES = ("fwd_tile_stream", "bwd_g_producer", "bwd_dE_contraction", "bwd_dH_contraction", "aux",
@@ -82,6 +83,11 @@ def lib() -> ctypes.CDLL:
     L.cce_vocab_sort_workspace_size.argtypes = [i64, i64, i32]
     L.cce_vocab_sort.restype = ctypes.c_int
     L.cce_vocab_sort.argtypes = [vp, vp, i64, i64, i32, ctypes.POINTER(Segment), i32, vp, vp, sz, vp]
+    L.cce_vocab_combine.restype = ctypes.c_int
+    L.cce_vocab_combine.argtypes = [vp, i32, vp, i64, i64, i32, ctypes.POINTER(Segment), i32,
+                                    vp, vp, vp]
+    L.cce_debug_stall.restype = ctypes.c_int
+    L.cce_debug_stall.argtypes = [ctypes.c_uint64, vp, vp]
     L.cce_launch_count.restype = ctypes.c_uint64
     L.cce_timing_enable.restype = ctypes.c_int
     L.cce_timing_enable.argtypes = [u32]
@@ -183,7 +189,8 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
         dloss: torch.Tensor, ignore_index: int = -100,
         segments: Optional[Sequence[SegSpec]] = None, V: Optional[int] = None,
         filter_eps: float = 0.0, vocab_perm: Optional[torch.Tensor] = None,
-        colmax: Optional[torch.Tensor] = None, kahan: bool = False, shard: bool = False, fp32_grads: bool = False, full_de: bool = False,
+        colmax: Optional[torch.Tensor] = None, kahan: bool = False, shard: bool = False,
+        fp32_grads: bool = False, full_de: bool = False, fp32_dh: bool = False,
         dE_out=None, dE_comp=None, debug_rows: int = 0,
         workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
     """Gradients (dH, dE) of sum_i dloss_i loss_i.  See cce_bwd.
@@ -191,7 +198,8 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
     dE is one tensor for a single head, a list (one per segment) otherwise.
     With kahan=True, dE_out and dE_comp (bf16, same shape(s)) are required
     and updated in place.  colmax (the forward's, same inputs) enables the
-    exact tile skip when filtering.  Returns (dH, dE, debug_keep or None).
+    exact tile skip when filtering.  fp32_dh=True returns dH in fp32 with dE
+    in bf16.  Returns (dH, dE, debug_keep or None).
     """
     N, D = H.shape
     dev = H.device
@@ -212,9 +220,10 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
     comps = None
     if kahan:
         comps = list(dE_comp) if isinstance(dE_comp, (list, tuple)) else [dE_comp]
-    dH = torch.empty((N, D), dtype=gdt, device=dev)
+    dH = torch.empty((N, D), dtype=torch.float32 if fp32_dh else gdt, device=dev)
     flags = ((KAHAN_DE if kahan else 0) | (FP32_GRADS if fp32_grads else 0) |
-             (FULL_DE if full_de else 0) | (VOCAB_SHARD if shard else 0))
+             (FULL_DE if full_de else 0) | (VOCAB_SHARD if shard else 0) |
+             (FP32_DH if fp32_dh else 0))
     words = (V + 31) // 32
     dbg = torch.empty((debug_rows, words), dtype=torch.int32, device=dev) if debug_rows > 0 else None
     segarr, nseg = _seg_array(segments, dEs if segments else None, comps if segments else None)
@@ -242,6 +251,48 @@ def vocab_sort(colmax: Optional[torch.Tensor], y: torch.Tensor, V: int, ignore_i
                               _ptr(perm), _ptr(ws), ws.numel(), _stream_ptr(dev))
     _check(rc, "cce_vocab_sort")
     return perm
+
+
+def vocab_combine(parts: torch.Tensor, y: torch.Tensor, V: int, ignore_index: int = -100,
+                  ranges: Optional[Sequence[Tuple[int, int]]] = None):
+    """(loss, lse) [N] from the gathered shard parts [R, 2, N] (lse part,
+    correct-token logit part); `ranges` are the whole head's live
+    [begin, end) ranges (None: [0, V)).  See cce_vocab_combine."""
+    _require_cuda(parts, y)
+    R, two, N = parts.shape
+    if two != 2 or parts.dtype != torch.float32 or y.dtype != torch.int32 or y.numel() != N:
+        raise CCEError("parts must be [R, 2, N] float32 and y [N] int32")
+    arr, n = None, 0
+    if ranges:
+        arr = (Segment * len(ranges))()
+        for k, (b, e) in enumerate(ranges):
+            arr[k].vocab_begin, arr[k].vocab_end = int(b), int(e)
+        n = len(ranges)
+    loss = torch.empty(N, dtype=torch.float32, device=parts.device)
+    lse = torch.empty(N, dtype=torch.float32, device=parts.device)
+    rc = lib().cce_vocab_combine(_ptr(parts), R, _ptr(y), N, V, ignore_index, arr, n, _ptr(loss),
+                                 _ptr(lse), _stream_ptr(parts.device))
+    _check(rc, "cce_vocab_combine")
+    return loss, lse
+
+
+def check_status(status: torch.Tensor, what: str = "libcce"):
+    """Synchronise on the status word's stream and raise CCEError if a kernel
+    reported a bad target or a wait that ran out (the outputs of that call are
+    then incomplete).  Costs one device-to-host read."""
+    v = int(status.item())
+    if v & STATUS_TIMEOUT:
+        raise CCEError(f"{what}: a kernel wait ran out (CCE_STATUS_TIMEOUT); outputs are incomplete")
+    if v & STATUS_BADTARGET:
+        raise CCEError(f"{what}: a target outside the vocabulary or in a gap (CCE_STATUS_BADTARGET)")
+    return v
+
+
+def debug_stall(wait_ns: int, status: torch.Tensor):
+    """Run the bounded-wait diagnostic (see cce_debug_stall)."""
+    _require_cuda(status)
+    _check(lib().cce_debug_stall(int(wait_ns), _ptr(status), _stream_ptr(status.device)),
+           "cce_debug_stall")
 
 
 def launch_count() -> int:

@@ -566,11 +566,13 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
             void* dE, void* dE_comp, uint32_t* debug_keep, int64_t debug_rows, void* workspace,
             size_t workspace_bytes, int32_t* status, void* stream, const KLArgs* kl) {
   if (!sizes_ok(N, D, V)) return CCE_EINVAL;
-  if (flags & ~(CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE | CCE_VOCAB_SHARD)) return CCE_EINVAL;
+  if (flags & ~(CCE_KAHAN_DE | CCE_FP32_GRADS | CCE_FULL_DE | CCE_VOCAB_SHARD | CCE_FP32_DH))
+    return CCE_EINVAL;
   if (kl && (flags & (CCE_FULL_DE | CCE_VOCAB_SHARD))) return CCE_EINVAL;
   const bool full_de = flags & CCE_FULL_DE;
   const bool kahan = flags & CCE_KAHAN_DE;
-  const bool fp32 = flags & CCE_FP32_GRADS;
+  const bool fp32 = flags & CCE_FP32_GRADS;        // dE (and dH) in fp32
+  const bool fp32_dh = fp32 || (flags & CCE_FP32_DH);  // dH in fp32
   if (kahan && fp32) return CCE_EINVAL;
   Segs sg;
   if (int rc = build_segs(E, V, segs, n_segs, sg)) return rc;
@@ -987,7 +989,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   hr.D = (int)D;
   hr.range = gather_range(pl.Npad, gblocks);
   hr.dH = dH;
-  hr.fp32_out = fp32 ? 1 : 0;
+  hr.fp32_out = fp32_dh ? 1 : 0;
   for (int s = 0; s < sg.n; ++s) {
     hr.E[s] = table.s[s].E;
     hr.live_off[s] = table.s[s].live_off;
@@ -1002,7 +1004,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   {
     TimedLaunch tl_(KC_SPARSE, st);
     dh_fill_kernel<<<(int)std::min<int64_t>(cdiv(N * (D / 8), 256), sms * 8), 256, 0, st>>>(
-        cp.pos_of_row, N, (int)D, dH, fp32 ? 1 : 0);
+        cp.pos_of_row, N, (int)D, dH, fp32_dh ? 1 : 0);
   }
   return launched();
 }
@@ -1178,6 +1180,48 @@ int cce_vocab_sort(const float* colmax, const int32_t* y, int64_t N, int64_t V, 
     if (launched()) return CCE_ELAUNCH;  // counted as one (a short sequence of cub kernels)
   }
   return CCE_OK;
+}
+
+int cce_vocab_combine(const float* parts, int32_t R, const int32_t* y, int64_t N, int64_t V,
+                      int32_t ignore_index, const cce_segment* segs, int32_t n_segs, float* loss,
+                      float* lse, void* stream) {
+  if (N < 0 || N > (int64_t)INT32_MAX || R < 1 || R > 4096 || V <= 0) return CCE_EINVAL;
+  // only the head's logical ranges matter here: validate them with a stand-in
+  // classifier pointer
+  Segs sg;
+  if (segs == nullptr || n_segs == 0) {
+    sg.n = 1;
+    sg.s[0] = cce_segment{0, V, parts, nullptr, nullptr};
+  } else {
+    if (n_segs < 0 || n_segs > CCE_MAX_SEGMENTS) return CCE_EINVAL;
+    cce_segment tmp[CCE_MAX_SEGMENTS];
+    for (int i = 0; i < n_segs; ++i) {
+      tmp[i] = segs[i];
+      tmp[i].E = parts;
+    }
+    if (build_segs(nullptr, V, tmp, n_segs, sg) != CCE_OK) return CCE_EINVAL;
+  }
+  if (N == 0) return CCE_OK;
+  if (!parts || !y || !loss || !lse) return CCE_EINVAL;
+  const int sms = device_sms();
+  if (sms <= 0) return CCE_EDEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const SegTable table = dev_table(sg, nullptr);
+  {
+    TimedLaunch tl_(KC_AUX, st);
+    vocab_combine_kernel<<<(int)std::min<int64_t>(cdiv(N, 256), sms * 8), 256, 0, st>>>(
+        parts, R, y, (int)N, ignore_index, table, V, loss, lse);
+  }
+  return launched();
+}
+
+int cce_debug_stall(uint64_t wait_ns, int32_t* status, void* stream) {
+  if (!status || wait_ns == 0 || wait_ns > 1000000000ull) return CCE_EINVAL;
+  if (device_sms() <= 0) return CCE_EDEVICE;
+  StallParams sp;
+  sp.status = status;
+  sp.wait_ns = wait_ns;
+  return launch_tc<StallPolicy>(sp, 1, static_cast<cudaStream_t>(stream), KC_AUX);
 }
 
 uint64_t cce_launch_count(void) { return g_launches.load(); }

@@ -16,6 +16,9 @@
 // swizzling, which the UMMA descriptors describe.
 #pragma once
 
+#include <type_traits>
+#include <utility>
+
 #include "cce_ptx.cuh"
 
 namespace cce {
@@ -93,6 +96,49 @@ struct MaskCursor {
   }
 };
 
+// ---------------------------------------------------------------------------
+// Order of (row block, inner index) work items that keeps the row operand
+// resident in L2.  Every item re-reads its 128-row block of H (the A operand,
+// K = D) from L2 once per vocabulary tile; if all row blocks were live at once
+// (inner-major order), their blocks together (N x D x 2 bytes, 134 MB at
+// N = 16384, D = 4096) would exceed L2 and every re-read would go to DRAM.
+// Instead the row blocks are taken in groups whose bytes stay below
+// kRowGroupBytes; within a group the inner index (vocabulary split or tile)
+// is the major one, so the CTAs running at the same time share each vocabulary
+// tile and keep re-reading the same group of row blocks.  E is then read from
+// DRAM once per group.
+#ifndef CCE_ROW_GROUP_MB
+#define CCE_ROW_GROUP_MB 40
+#endif
+constexpr long long kRowGroupBytes = (long long)CCE_ROW_GROUP_MB << 20;
+
+// Row blocks per group for num_mb blocks of blk_bytes each: as few groups as
+// the budget allows, of near-equal size.
+__device__ __forceinline__ int row_group_blocks(int num_mb, long long blk_bytes) {
+  const long long total = (long long)num_mb * blk_bytes;
+  const int ngroups = (int)max(1ll, (total + kRowGroupBytes - 1) / kRowGroupBytes);
+  return max(1, (num_mb + ngroups - 1) / ngroups);
+}
+
+// Item -> (row block, inner index) for items 0 .. num_mb * n_inner - 1, in
+// groups of gm row blocks (the last group may be smaller).
+__device__ __forceinline__ void grouped_item(int item, int num_mb, int n_inner, int gm, int& mb,
+                                             int& inner) {
+  const int full = num_mb / gm;  // complete groups
+  const int per = gm * n_inner;  // items per complete group
+  const int g = item / per;
+  if (g < full) {
+    const int r = item - g * per;
+    inner = r / gm;
+    mb = g * gm + (r - inner * gm);
+  } else {
+    const int rem = num_mb - full * gm;  // > 0 here
+    const int r = item - full * per;
+    inner = r / rem;
+    mb = full * gm + (r - inner * rem);
+  }
+}
+
 // Per-role state handed to policies.
 struct Engine {
   Ctl* ctl;
@@ -103,8 +149,13 @@ struct Engine {
   Pipe pipe;
   int tcount = 0;  // accumulator tiles handled by this role
   int fills = 0;   // stage fills issued (producer) / consumed (MMA)
+  uint64_t wait_ns = kWaitLimitNs;  // limit of every wait of this launch
 
   __device__ __forceinline__ volatile int* abort_flag() { return &ctl->abort; }
+  // Bounded wait on a barrier phase (see wait_parity).
+  __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) {
+    return wait_parity(bar, parity, abort_flag(), status, wait_ns);
+  }
 
   // ---- producer: load nkb stages of one tile.  (ax, ay) / (bx, by) are the
   // tensor-map coordinates of the tile origin; K advances along x for a
@@ -118,7 +169,7 @@ struct Engine {
     mc.init(kmask, nkb);
     for (int kb = 0; kb < nkb; ++kb) {
       if (!mc.bits(kb)) continue;
-      if (!wait_parity(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u, abort_flag(), status))
+      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u))
         return false;
       const uint32_t fb = smem_u32(&ctl->full[pipe.stage]);
       mbar_arrive_expect_tx(fb, STAGE_BYTES);
@@ -151,8 +202,7 @@ struct Engine {
   template <bool A_MN, bool B_MN>
   __device__ __forceinline__ bool mma(int nkb, const uint32_t* kmask = nullptr) {
     const int acc = tcount & 1;
-    if (!wait_parity(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u,
-                     abort_flag(), status))
+    if (!wait(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u))
       return false;
     tc_fence_after();
     const uint32_t d = tmem + acc * BN;
@@ -163,7 +213,7 @@ struct Engine {
     for (int kb = 0; kb < nkb; ++kb) {
       const uint32_t bits = mc.bits(kb);
       if (!bits) continue;  // the producer skipped this stage too
-      if (!wait_parity(smem_u32(&ctl->full[pipe.stage]), pipe.phase, abort_flag(), status))
+      if (!wait(smem_u32(&ctl->full[pipe.stage]), pipe.phase))
         return false;
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + pipe.stage * STAGE_BYTES);
@@ -204,7 +254,7 @@ struct Engine {
     for (int kb = 0; kb < nkb; ++kb) {
       const uint32_t bits = mc.bits(kb);
       if (!bits) continue;
-      if (!wait_parity(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u, abort_flag(), status))
+      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u))
         return false;
       const uint32_t fb = smem_u32(&ctl->full[pipe.stage]);
       mbar_expect_tx(fb, STAGE_BYTES);
@@ -232,7 +282,7 @@ struct Engine {
       ++fills;
     }
     if (pend < 0) {  // nothing to load: one empty stage ends the tile
-      if (!wait_parity(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u, abort_flag(), status))
+      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u))
         return false;
       pend = pipe.stage;
       pend_bits = 0;
@@ -248,8 +298,7 @@ struct Engine {
   template <bool A_MN, bool B_MN>
   __device__ __forceinline__ bool mma_rec() {
     const int acc = tcount & 1;
-    if (!wait_parity(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u,
-                     abort_flag(), status))
+    if (!wait(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u))
       return false;
     tc_fence_after();
     const uint32_t d = tmem + acc * BN;
@@ -262,7 +311,7 @@ struct Engine {
                               : smem_desc_sw128(smem_u32(smem) + A_BYTES, 16, 1024);
     uint32_t issued = 0;
     for (;;) {
-      if (!wait_parity(smem_u32(&ctl->full[pipe.stage]), pipe.phase, abort_flag(), status))
+      if (!wait(smem_u32(&ctl->full[pipe.stage]), pipe.phase))
         return false;
       const uint32_t rec = *reinterpret_cast<volatile uint32_t*>(&ctl->rec[pipe.stage]);
       const uint64_t so = (uint64_t)((pipe.stage * STAGE_BYTES) >> 4);
@@ -286,8 +335,7 @@ struct Engine {
   // for this thread's lane quarter (column 0).
   __device__ __forceinline__ bool epi_acquire(int quarter, uint32_t& taddr) {
     const int acc = tcount & 1;
-    if (!wait_parity(smem_u32(&ctl->tfull[acc]), ((uint32_t)tcount >> 1) & 1u, abort_flag(),
-                     status))
+    if (!wait(smem_u32(&ctl->tfull[acc]), ((uint32_t)tcount >> 1) & 1u))
       return false;
     tc_fence_after();
     taddr = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
@@ -308,7 +356,7 @@ struct Engine {
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int t = tcount + k;
-      if (!wait_parity(smem_u32(&ctl->tfull[t & 1]), ((uint32_t)t >> 1) & 1u, abort_flag(), status))
+      if (!wait(smem_u32(&ctl->tfull[t & 1]), ((uint32_t)t >> 1) & 1u))
         return false;
     }
     tc_fence_after();
@@ -331,6 +379,21 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return;
     if ((it & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) return;
   }
+}
+
+// Wait limit of a policy's launch: Policy::wait_limit(p) when the policy
+// defines it, else kWaitLimitNs.
+template <class P, class = void>
+struct HasWaitLimit : std::false_type {};
+template <class P>
+struct HasWaitLimit<P, std::void_t<decltype(P::wait_limit(std::declval<const typename P::Params&>()))>>
+    : std::true_type {};
+template <class Policy>
+__device__ __forceinline__ uint64_t policy_wait_limit(const typename Policy::Params& p) {
+  if constexpr (HasWaitLimit<Policy>::value)
+    return Policy::wait_limit(p);
+  else
+    return kWaitLimitNs;
 }
 
 // The kernel body: set-up, role dispatch, drain, TMEM release.
@@ -374,6 +437,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
   eng.extra = extra;
   eng.tmem = ctl->tmem_base;
   eng.status = p.status;
+  eng.wait_ns = policy_wait_limit<Policy>(p);
 
   if (warp == 0) {
     if (lane == 0) Policy::producer(p, eng);

@@ -205,9 +205,11 @@ __global__ void gather_perm_rows_kernel(const __nv_bfloat16* __restrict__ src,
 // =====================================================================
 // Forward tile stream ([LM] §Contribution; [MAP] §Approach).
 // Work item = (row block mb, vocabulary split): tpi consecutive 256-wide
-// vocabulary tiles (tiles never straddle segments).  Items are ordered
-// split-major so the CTAs running at the same time share E tiles through
-// L2.  Each epilogue thread keeps (m, s) of its row in base-2 units:
+// vocabulary tiles (tiles never straddle segments).  Items follow the grouped
+// order of grouped_item(): split-major within an L2-sized group of row
+// blocks, so the CTAs running at the same time share E tiles through L2 and
+// re-read row blocks that stay in L2.  Each epilogue thread keeps (m, s) of
+// its row in base-2 units:
 //   m = max_j z_j log2 e,  s = sum_j 2^(z_j log2 e - m).
 // =====================================================================
 struct FwdParams {
@@ -235,9 +237,10 @@ struct FwdPolicy {
     const int nv = *p.n_valid;
     const int num_mb = (nv + BM - 1) / BM;
     const int num_items = num_mb * p.S;
+    const int gm = row_group_blocks(num_mb, (long long)BM * BK * 2 * p.nkb);
     for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
-      const int split = item / num_mb;
-      const int mb = item - split * num_mb;
+      int mb, split;
+      grouped_item(item, num_mb, p.S, gm, mb, split);
       const int t0 = split * p.tpi;
       const int t1 = min(p.T_v, t0 + p.tpi);
       int s = 0;
@@ -376,6 +379,42 @@ __global__ void fwd_finalize_kernel(const FinParams p) {
   }
 }
 
+// Combine of the vocabulary-parallel forward: per row, the parts of R
+// vocabulary shards [R][2][N] (log-sum-exp over the shard, correct-token
+// logit or 0) -> lse = log-add-exp over shards ([MAP] §Limitations:
+// log-add-exp of partial results; a shard with no ids contributes -inf),
+// loss = lse - sum of the logit parts (only the owning shard's is non-zero).
+// Ignored rows give 0; a target outside the head's live ranges (outside
+// [0, V) or in a dead gap: no shard holds it) gives NaN, as on one GPU.
+__global__ void vocab_combine_kernel(const float* __restrict__ parts, int R, const int* __restrict__ y,
+                                     int N, int ignore_index, const SegTable t, long long V,
+                                     float* __restrict__ loss, float* __restrict__ lse) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < N; i += gridDim.x * blockDim.x) {
+    const int yi = y[i];
+    if (yi == ignore_index) {
+      loss[i] = 0.f;
+      lse[i] = 0.f;
+      continue;
+    }
+    if (yi < 0 || (long long)yi >= V || segment_of(t, (long long)yi) < 0) {
+      loss[i] = __int_as_float(0x7fc00000);
+      lse[i] = __int_as_float(0x7fc00000);
+      continue;
+    }
+    float m = -INFINITY, zy = 0.f;
+    for (int r = 0; r < R; ++r) {
+      const float* pr = parts + (size_t)r * 2 * N;
+      m = fmaxf(m, pr[i]);
+      zy += pr[(size_t)N + i];
+    }
+    float sum = 0.f;
+    for (int r = 0; r < R; ++r) sum += expf(parts[(size_t)r * 2 * N + i] - m);
+    const float l = m + logf(sum);  // m is finite: the shard holding y_i has ids
+    lse[i] = l;
+    loss[i] = l - zy;
+  }
+}
+
 __global__ void colmax_init_kernel(int* colmax, int n) {
   const int neg = f32_to_ordered(-INFINITY);
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
@@ -488,9 +527,13 @@ struct GPolicyT {
     const int nv = *p.n_valid;
     const int num_mb = (nv + BM - 1) / BM;
     const int tiles = active(p) ? num_mb * p.ct : 0;
+    // grouped order (vocabulary-tile-major within L2-sized row groups); the
+    // KL producer's A operand is two row blocks (teacher and student)
+    const int gm = row_group_blocks(num_mb, (long long)BM * BK * 2 * p.nkb * (KL ? 2 : 1));
     for (int i = blockIdx.x; i < tiles; i += gridDim.x) {
-      const int vt = i / num_mb;
-      if (!f(i - vt * num_mb, vt, nv)) return;
+      int mb, vt;
+      grouped_item(i, num_mb, p.ct, gm, mb, vt);
+      if (!f(mb, vt, nv)) return;
     }
   }
   static __device__ void prefetch(const Params& p) {
@@ -976,6 +1019,34 @@ __global__ void skip_bounds_kernel(const SkipBoundParams p) {
     }
   }
 }
+
+// =====================================================================
+// Diagnostic: the tile engine with a stage that never fills.  The producer
+// loads nothing, so the MMA issuer's wait for its first stage runs out after
+// wait_ns, sets the CTA's abort flag and CCE_STATUS_TIMEOUT; the epilogue,
+// waiting for an accumulator, sees the abort and returns; the kernel then
+// takes its normal drain and TMEM release path.  No copy or MMA is ever in
+// flight.  This is how a wait that cannot complete (a lost copy, a peer that
+// never arrives) surfaces: a status bit and a returning launch.
+// =====================================================================
+struct StallParams {
+  int* status;
+  unsigned long long wait_ns;
+};
+
+struct StallPolicy {
+  using Params = StallParams;
+  static constexpr int EXTRA_SMEM = 0;
+  static __device__ __forceinline__ bool active(const Params&) { return true; }
+  static __device__ __forceinline__ uint64_t wait_limit(const Params& p) { return p.wait_ns; }
+  static __device__ void prefetch(const Params&) {}
+  static __device__ void producer(const Params&, Engine&) {}  // never fills a stage
+  static __device__ void mma(const Params&, Engine& eng) { eng.mma<false, false>(1); }
+  static __device__ void epilogue(const Params&, Engine& eng, int q, int) {
+    uint32_t taddr;
+    eng.epi_acquire(q, taddr);
+  }
+};
 
 // inv[perm[k]] = k for one segment (perm and inv point at the segment's
 // slice of the concatenated live vocabulary; entries are segment-local).

@@ -46,9 +46,11 @@ struct KLFwdPolicy {
     const int nv = *p.n_valid;
     const int num_mb = (nv + BM - 1) / BM;
     const int num_items = num_mb * p.S;
+    // grouped order (see grouped_item); each item re-reads two row blocks
+    const int gm = row_group_blocks(num_mb, (long long)BM * BK * 2 * p.nkb * 2);
     for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
-      const int split = item / num_mb;
-      const int mb = item - split * num_mb;
+      int mb, split;
+      grouped_item(item, num_mb, p.S, gm, mb, split);
       const int t0 = split * p.tpi;
       const int t1 = min(p.T_v, t0 + p.tpi);
       for (int t = t0; t < t1; ++t)

@@ -59,17 +59,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with the given parity to complete.  Returns
-// false (and sets *abort, ORs the timeout bit into *status) when the limit is
-// reached, or when another role of the CTA has already aborted.
+// false (and sets *abort, ORs the timeout bit into *status) when limit_ns of
+// wall-clock time pass, or when another role of the CTA has already aborted.
 __device__ __forceinline__ bool wait_parity(uint32_t bar, uint32_t parity, volatile int* abort,
-                                            int* status) {
+                                            int* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0u) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort = 1;
         if (status) atomicOr(status, kStatusTimeout);
         return false;

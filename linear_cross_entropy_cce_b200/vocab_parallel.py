@@ -10,15 +10,16 @@ entry §Limitations: log-add-exp of partial results).  So:
 
   forward   cce_fwd_shard on the local shard gives per row the shard's
             log-sum-exp and, where the shard holds the target, the correct
-            token logit; one all-gather of these [3, N] values (with an
-            ownership count) and a local log-add-exp give every rank the full
-            lse and loss.
+            token logit; one all-gather of these [2, N] values and
+            cce_vocab_combine (log-add-exp over shards) give every rank the
+            full lse and loss.
   backward  cce_bwd with CCE_VOCAB_SHARD and the full lse gives the shard's
-            dE rows (complete: they depend only on local columns) and its
-            share of dH, which an all-reduce sums over ranks.
+            dE rows (bf16, complete: they depend only on local columns) and
+            its share of dH in fp32 (CCE_FP32_DH), which one all-reduce sums
+            over ranks before the cast to bf16.
 
-The kernels are those of the single-GPU path; torch.distributed carries the
-two exchanges.
+The kernels are those of the single-GPU path plus the combine kernel;
+torch.distributed carries the two exchanges.
 """
 from typing import List, Optional, Sequence, Tuple
 
@@ -50,47 +51,26 @@ def shard_segments(segments: Sequence[SegSpec], v0: int, v1: int) -> List[SegSpe
     return out
 
 
-def combine_shards(parts: torch.Tensor, y: torch.Tensor, ignore_index: int = -100):
-    """Per-rank parts [R, 3, N] (lse over the shard, correct-token logit or 0,
-    1 where the shard holds the target) -> (loss, lse) [N].
-
-    lse = log-add-exp over ranks; loss = lse - the owner's logit.  Ignored
-    rows give 0; a target that no shard holds (outside [0, V) or in a dead
-    gap of the head) gives NaN, as on one GPU."""
-    lse_p, zy_p, own = parts[:, 0], parts[:, 1], parts[:, 2]
-    lse = torch.logsumexp(lse_p, dim=0)
-    zy = zy_p.sum(dim=0)
-    ignored = y == ignore_index
-    bad = (~ignored) & (own.sum(dim=0) == 0)
-    zero = torch.zeros_like(lse)
-    nan = torch.full_like(lse, float("nan"))
-    lse = torch.where(ignored, zero, torch.where(bad, nan, lse))
-    loss = torch.where(ignored, zero, torch.where(bad, nan, lse - zy))
-    return loss, lse
-
-
-def owned(y: torch.Tensor, local: Sequence[SegSpec]) -> torch.Tensor:
-    """1.0 where this shard's segments hold the target, else 0.0."""
-    o = torch.zeros(y.shape, dtype=torch.float32, device=y.device)
-    for b, e, _ in local:
-        o += ((y >= int(b)) & (y < int(e))).to(torch.float32)
-    return o
-
-
 def _all_gather(x: torch.Tensor, group) -> torch.Tensor:
+    """[R, *x.shape]: every rank's x, gathered into one buffer."""
     import torch.distributed as dist
     world = dist.get_world_size(group)
-    bufs = [torch.empty_like(x) for _ in range(world)]
-    dist.all_gather(bufs, x.contiguous(), group=group)
-    return torch.stack(bufs)
+    out = torch.empty((world * x.shape[0],) + tuple(x.shape[1:]), dtype=x.dtype, device=x.device)
+    dist.all_gather_into_tensor(out, x.contiguous(), group=group)  # ranks along dim 0
+    return out.view((world,) + tuple(x.shape))
 
 
-def exchange_forward(lse_part: torch.Tensor, zy_part: torch.Tensor, own: torch.Tensor,
-                     y: torch.Tensor, ignore_index: int = -100, group=None):
-    """The forward's one exchange: all-gather every rank's [3, N] parts, then
-    combine_shards locally.  Returns (loss, lse), the same on every rank."""
-    return combine_shards(_all_gather(torch.stack([lse_part, zy_part, own]), group), y,
-                          ignore_index)
+def exchange_forward(lse_part: torch.Tensor, zy_part: torch.Tensor, y: torch.Tensor, V: int,
+                     head_ranges: Optional[Sequence[Tuple[int, int]]] = None,
+                     ignore_index: int = -100, group=None, combine=None):
+    """The forward's one exchange: all-gather every rank's [2, N] parts, then
+    combine them (cce.vocab_combine; `combine` substitutes another function
+    of the same signature, e.g. a host one for CPU process groups).
+    head_ranges: the whole head's live [begin, end) ranges (None: [0, V)).
+    Returns (loss, lse), the same on every rank."""
+    parts = _all_gather(torch.stack([lse_part, zy_part]), group)
+    fn = combine if combine is not None else cce.vocab_combine
+    return fn(parts, y, V, ignore_index, head_ranges)
 
 
 def exchange_backward(dH_part: torch.Tensor, group=None) -> torch.Tensor:
@@ -102,28 +82,28 @@ def exchange_backward(dH_part: torch.Tensor, group=None) -> torch.Tensor:
 
 def shard_forward_parts(H: torch.Tensor, y: torch.Tensor, local: Sequence[SegSpec], V: int,
                         ignore_index: int = -100, want_colmax: bool = False):
-    """This rank's (lse part, correct-token logit part, ownership[, colmax]).
-    A rank whose range holds no ids (more ranks than 256-aligned ranges)
-    contributes -inf to the log-add-exp and nothing else, without a launch."""
+    """This rank's (lse part, correct-token logit part[, colmax]).  A rank
+    whose range holds no ids (more ranks than 256-aligned ranges) contributes
+    -inf to the log-add-exp and a zero logit part, without a launch."""
     if not local:
         n = H.shape[0]
         lse_p = torch.full((n,), float("-inf"), dtype=torch.float32, device=H.device)
-        zero = torch.zeros(n, dtype=torch.float32, device=H.device)
-        parts = (lse_p, zero, zero.clone())
+        parts = (lse_p, torch.zeros(n, dtype=torch.float32, device=H.device))
         return parts + (torch.empty(0, dtype=torch.float32, device=H.device),) if want_colmax else parts
     out = cce.fwd(H, None, y, ignore_index, segments=list(local), V=V, shard=True,
                   want_colmax=want_colmax)
-    parts = (out[1], out[0], owned(y, local))
+    parts = (out[1], out[0])
     return parts + (out[2],) if want_colmax else parts
 
 
 def vp_forward(H: torch.Tensor, y: torch.Tensor, local: Sequence[SegSpec], V: int,
-               ignore_index: int = -100, group=None, want_colmax: bool = False):
+               ignore_index: int = -100, group=None, want_colmax: bool = False,
+               head_ranges: Optional[Sequence[Tuple[int, int]]] = None):
     """Forward over this rank's shard plus the exchange; returns (loss, lse)
     for every row (identical on all ranks), and the shard's colmax if asked."""
     parts = shard_forward_parts(H, y, local, V, ignore_index, want_colmax)
-    loss, lse = exchange_forward(parts[0], parts[1], parts[2], y, ignore_index, group)
-    return (loss, lse, parts[3]) if want_colmax else (loss, lse)
+    loss, lse = exchange_forward(parts[0], parts[1], y, V, head_ranges, ignore_index, group)
+    return (loss, lse, parts[2]) if want_colmax else (loss, lse)
 
 
 def vp_backward(H: torch.Tensor, y: torch.Tensor, lse: torch.Tensor, dloss: torch.Tensor,
@@ -131,7 +111,8 @@ def vp_backward(H: torch.Tensor, y: torch.Tensor, lse: torch.Tensor, dloss: torc
                 filter_eps: float = 0.0, vocab_perm: Optional[torch.Tensor] = None,
                 colmax: Optional[torch.Tensor] = None, group=None):
     """Backward over this rank's shard with the full lse; returns (dH summed
-    over ranks, this shard's dE per local segment), bf16."""
+    over ranks, bf16; this shard's dE per local segment, bf16).  A row with a
+    NaN lse (a target no shard holds) gets a NaN dH row and no gradient."""
     bad = torch.isnan(lse) & (y != ignore_index)
     if not local:  # a rank without ids: a zero share of dH, no dE
         dH = torch.zeros(H.shape, dtype=torch.float32, device=H.device)
@@ -142,17 +123,17 @@ def vp_backward(H: torch.Tensor, y: torch.Tensor, lse: torch.Tensor, dloss: torc
     dl = torch.where(bad, torch.zeros_like(dloss), dloss).to(torch.float32).contiguous()
     dH, dEs, _ = cce.bwd(H, None, y, lse_b, dl, ignore_index, segments=list(local), V=V,
                          filter_eps=filter_eps, vocab_perm=vocab_perm, colmax=colmax,
-                         fp32_grads=True, shard=True)
+                         fp32_dh=True, shard=True)
     exchange_backward(dH, group)
     dH[bad] = float("nan")
-    return dH.to(torch.bfloat16), [d.to(torch.bfloat16) for d in dEs]
+    return dH.to(torch.bfloat16), dEs
 
 
 class _VocabParallelCE(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, H, y, V, ignore_index, filter_eps, group, bounds, *E_local):
+    def forward(ctx, H, y, V, ignore_index, filter_eps, group, bounds, head_ranges, *E_local):
         local = [(b, e, t) for (b, e), t in zip(bounds, E_local)]
-        loss, lse = vp_forward(H, y, local, V, ignore_index, group)
+        loss, lse = vp_forward(H, y, local, V, ignore_index, group, head_ranges=head_ranges)
         ctx.save_for_backward(H, y, lse, *E_local)
         ctx.meta = (V, ignore_index, filter_eps, group, bounds)
         return loss
@@ -163,21 +144,25 @@ class _VocabParallelCE(torch.autograd.Function):
         V, ignore_index, filter_eps, group, bounds = ctx.meta
         local = [(b, e, t) for (b, e), t in zip(bounds, E_local)]
         dH, dEs = vp_backward(H, y, lse, grad_loss, local, V, ignore_index, filter_eps, group=group)
-        return (dH.to(H.dtype), None, None, None, None, None, None,
+        return (dH.to(H.dtype), None, None, None, None, None, None, None,
                 *[g.to(t.dtype) for g, t in zip(dEs, E_local)])
 
 
 def vocab_parallel_cross_entropy(H: torch.Tensor, y: torch.Tensor, local: Sequence[SegSpec],
                                  V: int, ignore_index: int = -100, reduction: str = "mean",
-                                 filter_eps: float = 2.0 ** -12, group=None) -> torch.Tensor:
+                                 filter_eps: float = 2.0 ** -12, group=None,
+                                 head_ranges: Optional[Sequence[Tuple[int, int]]] = None
+                                 ) -> torch.Tensor:
     """Cross-entropy of H @ E^T against y with E split by vocabulary over the
     ranks of `group`: `local` is this rank's [(begin, end, E_rows)] (see
-    shard_segments).  Every rank passes the same H and y and gets the same
-    loss; dE flows to its own rows only."""
+    shard_segments), `head_ranges` the whole head's live [begin, end) ranges
+    (None: one range [0, V)).  Every rank passes the same H and y and gets
+    the same loss; dE flows to its own rows only."""
     if y.dtype != torch.int32:
         y = y.to(torch.int32)
     bounds = tuple((int(b), int(e)) for b, e, _ in local)
-    per_row = _VocabParallelCE.apply(H, y, V, ignore_index, float(filter_eps), group, bounds,
+    head = tuple((int(b), int(e)) for b, e in head_ranges) if head_ranges else None
+    per_row = _VocabParallelCE.apply(H, y, V, ignore_index, float(filter_eps), group, bounds, head,
                                      *[t for _, _, t in local])
     if reduction == "none":
         return per_row

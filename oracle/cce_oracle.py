@@ -228,6 +228,48 @@ def dE_columns(H, segments, y, V: int, dloss, cols: Sequence[int],
     return out
 
 
+def full_pass(H, segments, y, V: int, dloss, cols: Sequence[int], ignore_index: int = -100,
+              filter_eps: Sequence[float] = (0.0,), slice_rows: int = SLICE_ROWS):
+    """One pass over every row for the checks at full size: the per-row loss
+    and lse of forward() and, for each threshold in ``filter_eps``, the dE
+    rows of dE_columns() for the logical ids ``cols``.
+
+    The same slice arithmetic as those two functions (logits, textbook
+    log-sum-exp, loss = lse - z_y; G = dloss (p keep - onehot) on the sampled
+    columns, dE_j = sum_i G_ij h_i), done once per slice instead of once per
+    function, because at full size each pass is the whole N x V x D product.
+    Returns (loss[N], lse[N], {eps: dE_cols[len(cols), D]}).
+    """
+    segs64 = _segments_f64(segments)
+    y = np.asarray(y, dtype=np.int64)
+    N, D = H.shape
+    cols = np.asarray(cols, dtype=np.int64)
+    dloss = np.asarray(dloss, dtype=np.float64)
+    ignored, good, bad = _valid_targets(y, V, ignore_index, segs64)
+    loss = np.zeros(N)
+    lse_all = np.zeros(N)
+    out = {float(e): np.zeros((cols.shape[0], D)) for e in filter_eps}
+    for s in range(0, N, slice_rows):
+        r = np.arange(s, min(N, s + slice_rows))
+        r = r[good[r]]
+        if r.shape[0] == 0:
+            continue
+        H64 = as_f64(H[r])
+        Z = logits_rows(H64, segs64, V)
+        lse = logsumexp_rows(Z)
+        loss[r] = lse - Z[np.arange(r.shape[0]), y[r]]
+        lse_all[r] = lse
+        Pc = np.exp(Z[:, cols] - lse[:, None])
+        onehot = y[r][:, None] == cols[None, :]
+        for e, acc in out.items():
+            P = np.where(Pc >= e, Pc, 0.0) if e > 0.0 else Pc.copy()
+            P -= onehot
+            acc += (dloss[r][:, None] * P).T @ H64
+    loss[bad] = np.nan
+    lse_all[bad] = np.nan
+    return loss, lse_all, out
+
+
 def mean_loss(loss: np.ndarray, valid: np.ndarray) -> float:
     """Mean over valid rows, exactly rounded (math.fsum); N_v = 0 gives NaN."""
     n_v = int(np.count_nonzero(valid))
@@ -237,12 +279,19 @@ def mean_loss(loss: np.ndarray, valid: np.ndarray) -> float:
 
 
 def kahan_reference(parts: Sequence[np.ndarray]) -> np.ndarray:
-    """Exact (fp64) sum of several gradient contributions, the target that a
-    compensated accumulation approaches ([MAP] §Limitations, Kahan variants)."""
-    acc = np.zeros_like(parts[0], dtype=np.float64)
-    for p in parts:
-        acc += p
-    return acc
+    """The exactly rounded element-wise sum of several gradient contributions:
+    the value a compensated (Kahan) accumulation of the classifier gradient
+    over micro-batches approaches ([MAP] §Limitations, Kahan variants).
+
+    Each element is summed with math.fsum (Shewchuk's exact partials), so the
+    result does not depend on the order of the parts and is the fp64 number
+    nearest to the true sum, even when the parts cancel.
+    """
+    stack = np.stack([np.asarray(p, dtype=np.float64) for p in parts])
+    flat = stack.reshape(stack.shape[0], -1)
+    out = np.fromiter((math.fsum(flat[:, k]) for k in range(flat.shape[1])), dtype=np.float64,
+                      count=flat.shape[1])
+    return out.reshape(stack.shape[1:])
 
 
 # ---------------------------------------------------------------------------

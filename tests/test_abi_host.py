@@ -108,10 +108,30 @@ def test_bwd_rejects_bad_flags_and_missing_kahan_buffer():
     def call(flags=0, dE=16, comp=None):
         return L.cce_bwd(16, 16, 16, 16, 16, 4, 8, 10, -100, None, 0, 0.0, None, None, flags,
                          16, dE, comp, None, 0, 16, 1 << 30, 16, None)
-    assert call(flags=16) == cce.CCE_EINVAL                      # unknown flag bit
+    assert call(flags=32) == cce.CCE_EINVAL                      # unknown flag bit
     assert call(flags=cce.KAHAN_DE) == cce.CCE_EINVAL           # no compensation buffer
     assert call(flags=cce.KAHAN_DE | cce.FP32_GRADS, comp=16) == cce.CCE_EINVAL
     assert call(dE=None) == cce.CCE_EINVAL
+
+
+def test_vocab_combine_rejects_bad_arguments_on_host():
+    L = cce.lib()
+    EINVAL = cce.CCE_EINVAL
+
+    def comb(parts=16, R=2, y=16, N=4, V=10, segs=None, nseg=0, loss=16, lse=16):
+        return L.cce_vocab_combine(parts, R, y, N, V, -100, segs, nseg, loss, lse, None)
+    assert comb(R=0) == EINVAL and comb(R=5000) == EINVAL
+    assert comb(N=-1) == EINVAL and comb(V=0) == EINVAL
+    assert comb(parts=None) == EINVAL and comb(y=None) == EINVAL
+    assert comb(loss=None) == EINVAL and comb(lse=None) == EINVAL
+    assert comb(N=0, parts=None) == cce.CCE_OK  # nothing to do: no launch
+    seg = (cce.Segment * 2)()
+    seg[0].vocab_begin, seg[0].vocab_end = 0, 6
+    seg[1].vocab_begin, seg[1].vocab_end = 5, 10  # overlapping ranges
+    assert comb(segs=seg, nseg=2) == EINVAL
+    seg[1].vocab_begin, seg[1].vocab_end = 7, 11  # beyond V
+    assert comb(segs=seg, nseg=2) == EINVAL
+    assert comb(segs=seg, nseg=9) == EINVAL
 
 
 def test_kl_and_shard_entry_points_reject_bad_arguments_on_host():

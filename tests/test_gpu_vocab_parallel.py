@@ -39,8 +39,8 @@ def test_vocab_parallel_matches_oracle(head, R, eps):
     parts = []
     for local in shards:
         zy_p, lse_p = cce.fwd(H, None, y, x.ignore_index, segments=local, V=wl.V, shard=True)
-        parts.append(torch.stack([lse_p, zy_p, vp.owned(y, local)]))
-    loss, lse = vp.combine_shards(torch.stack(parts), y, x.ignore_index)
+        parts.append(torch.stack([lse_p, zy_p]))
+    loss, lse = cce.vocab_combine(torch.stack(parts), y, wl.V, x.ignore_index, list(wl.segs()))
     torch.cuda.synchronize()
     rl, rlse = oracle.forward(x.H, x.segments, x.y, wl.V, x.ignore_index)
     bad = np.isnan(rl)
@@ -57,7 +57,8 @@ def test_vocab_parallel_matches_oracle(head, R, eps):
     dE = {}
     for local in shards:
         dH_p, dEs, _ = cce.bwd(H, None, y, lse_b, dlt, x.ignore_index, segments=local, V=wl.V,
-                               filter_eps=eps, fp32_grads=True, shard=True)
+                               filter_eps=eps, fp32_dh=True, shard=True)
+        assert dH_p.dtype == torch.float32 and all(g.dtype == torch.bfloat16 for g in dEs)
         dH += torch.nan_to_num(dH_p, nan=0.0)
         for (b, e, _), g in zip(local, dEs):
             dE[(b, e)] = g
@@ -67,7 +68,7 @@ def test_vocab_parallel_matches_oracle(head, R, eps):
     tol = TOL_GRAD_FILTER if eps > 0 else TOL_GRAD
     assert normwise(to_np(dH)[~bad], rH[~bad]) <= tol
     for (b, e, _), r in zip(x.segments, rE):
-        got = torch.cat([dE[k] for k in sorted(dE) if b <= k[0] < e]).cpu().numpy()
+        got = torch.cat([dE[k] for k in sorted(dE) if b <= k[0] < e]).float().cpu().numpy()
         assert got.shape == r.shape
         assert normwise(got, r) <= tol
 
@@ -80,11 +81,51 @@ def test_one_shard_is_the_single_call():
     H, segs, y = upload(x)
     loss0, lse0 = cce.fwd(H, segs[0][2], y, x.ignore_index)
     zy_p, lse_p = cce.fwd(H, segs[0][2], y, x.ignore_index, shard=True)
-    loss1, lse1 = vp.combine_shards(torch.stack([lse_p, zy_p, vp.owned(y, segs)])[None], y,
-                                    x.ignore_index)
+    loss1, lse1 = cce.vocab_combine(torch.stack([lse_p, zy_p])[None], y, wl.V, x.ignore_index)
     torch.cuda.synchronize()
     assert torch.equal(lse0, lse1)
     assert torch.allclose(loss0, loss1, atol=1e-5, rtol=0)
+
+
+@pytest.mark.parametrize("R", [1, 2, 5])
+def test_combine_kernel_matches_oracle_with_empty_shards(R):
+    """cce_vocab_combine on shard parts computed by the oracle, with two
+    extra ranks that hold no ids (-inf, 0): per-row loss and lse equal the
+    oracle's full-vocabulary forward; ignored rows 0; targets in the dead gap
+    or outside the vocabulary NaN."""
+    from linear_cross_entropy_cce_b200 import cce
+    wl = HEADS["composite"]
+    x = syn.make_inputs(wl, seed=24)
+    x.y[3] = 4600        # dead gap
+    x.y[5] = wl.V + 11   # outside the vocabulary
+    x.y[6] = -7          # negative, not the ignore index
+    segs64 = [(b, e, oracle.widen_bf16(E)) for b, e, E in x.segments]
+    Z = oracle.logits_rows(oracle.widen_bf16(x.H), segs64, wl.V)
+    parts = []
+    for v0, v1 in vp.shard_ranges(wl.V, R) + [(wl.V, wl.V)] * 2:
+        cols = np.zeros(wl.V, bool)
+        cols[v0:v1] = True
+        Zs = np.where(cols[None, :], Z, -np.inf)
+        m = Zs.max(axis=1)
+        with np.errstate(invalid="ignore", divide="ignore"):
+            lse = np.where(np.isfinite(m), m + np.log(np.exp(Zs - np.where(np.isfinite(m), m, 0)[:, None]).sum(1)), -np.inf)
+        yc = np.clip(x.y, 0, wl.V - 1)
+        held = (x.y >= v0) & (x.y < v1) & np.isfinite(Z[np.arange(wl.N), yc])
+        zy = np.where(held, Z[np.arange(wl.N), yc], 0.0)
+        parts.append(np.stack([lse, zy]))
+    P = torch.from_numpy(np.stack(parts).astype(np.float32)).cuda()
+    y = torch.from_numpy(x.y).cuda()
+    loss, lse = cce.vocab_combine(P, y, wl.V, x.ignore_index, list(wl.segs()))
+    torch.cuda.synchronize()
+    rl, rs = oracle.forward(x.H, x.segments, x.y, wl.V, x.ignore_index)
+    bad = np.isnan(rl)
+    assert bad[3] and bad[5] and bad[6]
+    assert np.array_equal(np.isnan(to_np(loss)), bad) and np.array_equal(np.isnan(to_np(lse)), bad)
+    ign = x.y == x.ignore_index
+    assert np.all(to_np(loss)[ign] == 0) and np.all(to_np(lse)[ign] == 0)
+    ok = ~bad & ~ign
+    assert np.max(np.abs(to_np(loss)[ok] - rl[ok])) <= TOL_ROW
+    assert np.max(np.abs(to_np(lse)[ok] - rs[ok])) <= TOL_ROW
 
 
 def test_autograd_over_a_one_rank_nccl_group():
@@ -105,7 +146,8 @@ def test_autograd_over_a_one_rank_nccl_group():
         H, segs, y = upload(x)
         Hl = H.detach().clone().requires_grad_(True)
         local = [(b, e, t.detach().clone().requires_grad_(True)) for b, e, t in segs]
-        loss = vp.vocab_parallel_cross_entropy(Hl, y, local, wl.V, x.ignore_index)
+        loss = vp.vocab_parallel_cross_entropy(Hl, y, local, wl.V, x.ignore_index,
+                                               head_ranges=list(wl.segs()))
         loss.backward()
         torch.cuda.synchronize()
         rl, _ = oracle.forward(x.H, x.segments, x.y, wl.V, x.ignore_index)

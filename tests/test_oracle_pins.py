@@ -305,6 +305,22 @@ def test_dE_columns_match_backward():
     assert np.allclose(got, ref, rtol=1e-12, atol=1e-16)
 
 
+def test_full_pass_equals_forward_and_dE_columns():
+    """The one-pass helper of the full-size checks reproduces forward() (bit
+    for bit: same slice arithmetic) and dE_columns() for each threshold."""
+    x = _small(N=70, D=8, V=50, std=6.0, segments=[(0, 20), (26, 50)])
+    dl = x.dloss_mean()
+    cols = [0, 7, 19, 26, 31, 49]
+    loss, lse, dEc = oracle.full_pass(x.H, x.segments, x.y, 50, dl, cols, IGN,
+                                      filter_eps=(0.0, 1e-3), slice_rows=16)
+    rl, rs = oracle.forward(x.H, x.segments, x.y, 50, IGN, slice_rows=16)
+    assert np.array_equal(loss, rl, equal_nan=True) and np.array_equal(lse, rs, equal_nan=True)
+    for e in (0.0, 1e-3):
+        ref = oracle.dE_columns(x.H, x.segments, x.y, 50, dl, cols, IGN, filter_eps=e, slice_rows=16)
+        assert np.allclose(dEc[e], ref, rtol=1e-12, atol=1e-16)
+    assert not np.allclose(dEc[0.0], dEc[1e-3], rtol=1e-6, atol=0)
+
+
 def test_full_classifier_gradient_variant():
     """filter_dE=False ("FullC"): dE equals the unfiltered dE, dH the filtered
     dH; and the filter does change both on this peaky case (so the variant is
@@ -317,6 +333,41 @@ def test_full_classifier_gradient_variant():
     cH, cE = oracle.backward(x.H, x.segments, x.y, 200, dl, IGN, filter_eps=eps, filter_dE=False)
     assert np.array_equal(cH, fH) and np.array_equal(cE[0], uE[0])
     assert not np.allclose(fE[0], uE[0], rtol=1e-9, atol=0) and not np.allclose(fH, uH, rtol=1e-9, atol=0)
+
+
+# --------------------------------------------------- exact sum of gradient parts
+def test_kahan_reference_survives_cancellation():
+    """Parts built to cancel: 1e16 + 1 - 1e16 is exactly 1 (a running fp64 sum
+    gives 0 or 2); the order of the parts does not matter.
+    Catches: a plain left-to-right fp64 accumulation."""
+    a = np.array([1e16, 1.0, 3.0, -2.5])
+    parts = [a, np.array([1.0, 1e-30, -1e20, 2.5]), np.array([-1e16, -1.0, 1e20, 0.0])]
+    want = np.array([1.0, 1e-30, 3.0, 0.0])
+    assert np.array_equal(oracle.kahan_reference(parts), want)
+    assert np.array_equal(oracle.kahan_reference(parts[::-1]), want)
+
+
+def test_kahan_reference_is_the_exactly_rounded_rational_sum():
+    """Against exact rational arithmetic (fractions.Fraction): the result is
+    the fp64 number nearest to the true sum, bit for bit, on parts spanning 60
+    binary orders of magnitude with mixed signs.
+    Catches: any order-dependent or compensated-but-inexact summation."""
+    from fractions import Fraction
+    rng = np.random.default_rng(7)
+    K, M = 23, 41
+    parts = [rng.standard_normal(M) * np.exp2(rng.integers(-30, 30, M)) for _ in range(K)]
+    got = oracle.kahan_reference([p.reshape(1, M) for p in parts]).reshape(M)
+    for k in range(M):
+        exact = sum((Fraction(float(p[k])) for p in parts), Fraction(0))
+        assert got[k] == float(exact)  # Fraction -> float rounds to nearest
+
+
+def test_kahan_reference_keeps_shape_and_closed_form():
+    """n copies of 0.1 sum to the double nearest n/10, and shapes survive."""
+    parts = [np.full((3, 4), 0.1) for _ in range(10)]
+    got = oracle.kahan_reference(parts)
+    assert got.shape == (3, 4) and np.all(got == 1.0)  # fsum: 10 x 0.1 == 1.0 exactly rounded
+    assert np.all(oracle.kahan_reference([np.full(5, 0.1)] * 3) == 0.30000000000000004)
 
 
 # ------------------------------------------------------------- soft-target KL

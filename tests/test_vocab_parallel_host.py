@@ -26,6 +26,31 @@ def _inputs(seed=0):
     return x, y
 
 
+def _combine_ref(parts, y, V, ignore_index, head_ranges):
+    """Host restatement of the combine (the library's is a CUDA kernel, which
+    a CPU process group cannot run): lse = log-add-exp of the shards' lse
+    parts, loss = lse - sum of their logit parts; ignored rows 0; a target
+    outside the head's live ranges NaN."""
+    ranges = head_ranges or [(0, V)]
+    lse_p, zy_p = parts[:, 0].double(), parts[:, 1].double()
+    lse = torch.logsumexp(lse_p, dim=0)
+    zy = zy_p.sum(dim=0)
+    yl = y.long()
+    held = torch.zeros_like(yl, dtype=torch.bool)
+    for b, e in ranges:
+        held |= (yl >= b) & (yl < e)
+    ign = yl == ignore_index
+    bad = ~ign & ~held
+    nan = torch.full_like(lse, float("nan"))
+    zero = torch.zeros_like(lse)
+    lse = torch.where(ign, zero, torch.where(bad, nan, lse))
+    loss = torch.where(ign, zero, torch.where(bad, nan, lse - zy))
+    return loss, lse
+
+
+HEAD = [(b, e) for b, e in WL.segments]
+
+
 def _oracle_parts(x, y, v0, v1):
     """Shard [v0, v1): (lse over its live ids, correct-token logit if held,
     1 if held) per row, from the oracle's logits."""
@@ -68,8 +93,8 @@ def test_shard_segments_cut_the_head():
 @pytest.mark.parametrize("R", [2, 3])
 def test_combine_matches_full_oracle(R):
     x, y = _inputs()
-    parts = np.stack([_oracle_parts(x, y, v0, v1)[0] for v0, v1 in vp.shard_ranges(WL.V, R)])
-    loss, lse = vp.combine_shards(torch.from_numpy(parts), torch.from_numpy(y), x.ignore_index)
+    parts = np.stack([_oracle_parts(x, y, v0, v1)[0][:2] for v0, v1 in vp.shard_ranges(WL.V, R)])
+    loss, lse = _combine_ref(torch.from_numpy(parts), torch.from_numpy(y), WL.V, x.ignore_index, HEAD)
     rl, rlse = _expected(x, y)
     bad = np.isnan(rl)
     assert bad[3] and bad[5] and np.array_equal(np.isnan(loss.numpy()), bad)
@@ -96,7 +121,8 @@ def _worker(rank, world, port, out):
     v0, v1 = vp.shard_ranges(WL.V, world)[rank]
     parts, Z = _oracle_parts(x, y, v0, v1)
     t = [torch.from_numpy(p.copy()) for p in parts]
-    loss, lse = vp.exchange_forward(t[0], t[1], t[2], torch.from_numpy(y), x.ignore_index)
+    loss, lse = vp.exchange_forward(t[0], t[1], torch.from_numpy(y), WL.V, HEAD, x.ignore_index,
+                                    combine=_combine_ref)
     # this shard's share of dH with the full lse: dloss * (softmax - onehot) over its ids
     lse_full = lse.numpy()
     dl = x.dloss_mean()
@@ -141,11 +167,10 @@ def test_rank_without_ids_contributes_nothing():
     assert ranges[-1] == (600, 600)
     H = torch.zeros((6, 8))
     y = torch.tensor([0, 5, -100, 599, 300, 1], dtype=torch.int32)
-    lse_p, zy_p, own = vp.shard_forward_parts(H, y, [], 600)
-    assert torch.all(torch.isinf(lse_p) & (lse_p < 0)) and torch.all(zy_p == 0) and torch.all(own == 0)
-    full = torch.tensor([[1.0, 2.0, 0.0, 3.0, 0.5, 1.5], [0.2, 0.1, 0.0, 0.3, 0.4, 0.2],
-                         [1.0, 1.0, 0.0, 1.0, 1.0, 1.0]])
-    parts = torch.stack([full, torch.stack([lse_p, zy_p, own])])
-    loss, lse = vp.combine_shards(parts, y)
-    ref_loss, ref_lse = vp.combine_shards(full[None], y)
+    lse_p, zy_p = vp.shard_forward_parts(H, y, [], 600)
+    assert torch.all(torch.isinf(lse_p) & (lse_p < 0)) and torch.all(zy_p == 0)
+    full = torch.tensor([[1.0, 2.0, 0.0, 3.0, 0.5, 1.5], [0.2, 0.1, 0.0, 0.3, 0.4, 0.2]])
+    parts = torch.stack([full, torch.stack([lse_p, zy_p])])
+    loss, lse = _combine_ref(parts, y, 600, -100, None)
+    ref_loss, ref_lse = _combine_ref(full[None], y, 600, -100, None)
     assert torch.equal(loss, ref_loss) and torch.equal(lse, ref_lse)
