@@ -298,9 +298,13 @@ def main():
     nseg = 0 if single else max(1, len(segs))
     v_live_rank = sum(e - b for b, e, _ in segs)
     v_live = wl.v_live
-    ws_f = torch.empty(cce.fwd_workspace_size(N, D, V, nseg), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(cce.bwd_workspace_size(N, D, V, nseg), dtype=torch.uint8, device=dev)
-    ws_s = torch.empty(cce.vocab_sort_workspace_size(N, V, nseg), dtype=torch.uint8, device=dev)
+    # one caller-owned workspace serves the three calls of a step in turn (no
+    # call's scratch outlives it: loss, lse, colmax and the permutation are
+    # separate outputs)
+    ws_all = torch.empty(max(cce.fwd_workspace_size(N, D, V, nseg),
+                             cce.bwd_workspace_size(N, D, V, nseg),
+                             cce.vocab_sort_workspace_size(N, V, nseg)), dtype=torch.uint8, device=dev)
+    ws_f = ws_b = ws_s = ws_all
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     input_bytes = H.numel() * 2 + sum(s[2].numel() * 2 for s in segs) + y.numel() * 4
     kahan_kw = {}
@@ -399,7 +403,7 @@ def main():
     step()
     torch.cuda.synchronize(dev)
     peak_extra = torch.cuda.max_memory_allocated(dev) - base
-    ws_bytes = ws_f.numel() + ws_b.numel() + ws_s.numel()
+    ws_bytes = ws_all.numel()
 
     # end to end through the public API from pinned host buffers
     e2e = None

@@ -277,6 +277,9 @@ int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
  *            (its gradient is then smaller than filter_eps); <= 0 = off.
  *   flags    CCE_FP32_GRADS and/or CCE_KAHAN_DE (with dE_comp) as for
  *            cce_bwd; CCE_FULL_DE and CCE_VOCAB_SHARD are rejected.
+ *   debug_keep, debug_rows  optional per-element keep bits as for cce_bwd
+ *            (set where the entry kept a non-zero gradient, i.e. where
+ *            p_s or p_t reached filter_eps); NULL / 0 to skip.
  * Workspace: cce_kl_bwd_workspace_size(); errors as for cce_bwd.
  */
 size_t cce_kl_bwd_workspace_size(int64_t N, int64_t D, int64_t V, uint32_t flags);
@@ -284,6 +287,7 @@ int cce_kl_bwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
                const int32_t* row_mask, const float* lse_s, const float* lse_t,
                const float* dloss, int64_t N, int64_t D, int64_t V,
                float filter_eps, uint32_t flags, void* dH, void* dE, void* dE_comp,
+               uint32_t* debug_keep, int64_t debug_rows,
                void* workspace, size_t workspace_bytes,
                int32_t* status, void* stream);
 

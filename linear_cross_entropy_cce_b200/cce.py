@@ -73,7 +73,7 @@ def lib() -> ctypes.CDLL:
     L.cce_kl_bwd_workspace_size.argtypes = [i64, i64, i64, u32]
     L.cce_kl_bwd.restype = ctypes.c_int
     L.cce_kl_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, fp, u32, vp, vp, vp,
-                             vp, sz, vp, vp]
+                             vp, i64, vp, sz, vp, vp]
     L.cce_bwd_workspace_size.restype = sz
     L.cce_bwd_workspace_size.argtypes = [i64, i64, i64, i32, u32]
     L.cce_bwd.restype = ctypes.c_int
@@ -343,8 +343,10 @@ def kl_bwd(Hs: torch.Tensor, Es: torch.Tensor, Ht: torch.Tensor, Et: torch.Tenso
            lse_s: torch.Tensor, lse_t: torch.Tensor, dloss: torch.Tensor,
            row_mask: Optional[torch.Tensor] = None, filter_eps: float = 0.0,
            fp32_grads: bool = False, kahan: bool = False, dE_out=None, dE_comp=None,
-           workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
-    """Student gradients (dH, dE) of sum_i dloss_i KL_i.  See cce_kl_bwd."""
+           debug_rows: int = 0, workspace: Optional[torch.Tensor] = None,
+           status: Optional[torch.Tensor] = None):
+    """Student gradients (dH, dE) of sum_i dloss_i KL_i.  See cce_kl_bwd.
+    With debug_rows > 0 returns (dH, dE, keep bits [debug_rows, ceil(V/32)])."""
     N, D = Hs.shape
     V = int(Es.shape[0])
     _require_cuda(Hs, Es, Ht, Et, lse_s, lse_t, dloss, row_mask)
@@ -357,9 +359,13 @@ def kl_bwd(Hs: torch.Tensor, Es: torch.Tensor, Ht: torch.Tensor, Et: torch.Tenso
     flags = (KAHAN_DE if kahan else 0) | (FP32_GRADS if fp32_grads else 0)
     ws = _workspace(int(lib().cce_kl_bwd_workspace_size(N, D, V, flags)), dev, workspace)
     st = status if status is not None else torch.zeros(1, dtype=torch.int32, device=dev)
+    dbg = (torch.empty((debug_rows, (V + 31) // 32), dtype=torch.int32, device=dev)
+           if debug_rows > 0 else None)
     rc = lib().cce_kl_bwd(_ptr(Hs), _ptr(Es), _ptr(Ht), _ptr(Et), _ptr(row_mask), _ptr(lse_s),
                           _ptr(lse_t), _ptr(dloss), N, D, V, float(filter_eps), flags, _ptr(dH),
-                          _ptr(dE), _ptr(dE_comp) if kahan else None, _ptr(ws), ws.numel(),
-                          _ptr(st), _stream_ptr(dev))
+                          _ptr(dE), _ptr(dE_comp) if kahan else None, _ptr(dbg), debug_rows,
+                          _ptr(ws), ws.numel(), _ptr(st), _stream_ptr(dev))
     _check(rc, "cce_kl_bwd")
+    if debug_rows > 0:
+        return dH, dE, dbg
     return dH, dE

@@ -348,6 +348,41 @@ int launch_tc(const typename Policy::Params& prm, int grid, cudaStream_t st, int
   return cudaGetLastError() == cudaSuccess ? CCE_OK : CCE_ELAUNCH;
 }
 
+// Launch of a CTA-pair kernel: clusters of two CTAs along x; `pairs` pairs.
+template <class Policy>
+int launch_tc_pair(const typename Policy::Params& prm, int pairs, cudaStream_t st, int cls) {
+  auto k = tc_pair_kernel<Policy>;
+  constexpr int smem = pair_smem_bytes<Policy>();
+  static_assert(smem <= 232448, "shared memory per CTA exceeds 227 KB");
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return CCE_ELAUNCH;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const long slot = timing_begin(cls, st);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, prm);
+  timing_end(slot, st);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? CCE_OK : CCE_ELAUNCH;
+}
+
+// The dE / dH contractions of dense chunks run on CTA pairs (256 x 256 tiles,
+// tcgen05 cta_group::2) unless built with CCE_PAIR_DEDH=0.
+#ifndef CCE_PAIR_DEDH
+#define CCE_PAIR_DEDH 1
+#endif
+constexpr bool kPairDEDH = CCE_PAIR_DEDH != 0;
+
 // Brackets a plain kernel launch of class `cls` with timing events (when
 // that class is being timed); use as  { TimedLaunch t(cls, st); k<<<..>>>(); }
 struct TimedLaunch {
@@ -868,7 +903,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       ep.nz_cnt = sparse_de ? nz_cnt + chunk : nullptr;
       ep.nz_cap = cap;
       ep.chunk_valid = cv;
-      ep.mt = (int)cdiv(cv, BM);
+      ep.mt = (int)cdiv(cv, kPairDEDH ? 2 * BM : BM);
       ep.dt = dt;
       ep.D = (int)D;
       ep.c0 = c0;
@@ -880,7 +915,11 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       ep.mwords = pl.de_words;
       ep.n_valid = cp.n_valid;
       ep.status = status;
-      if (int rc = launch_tc<DEPolicy>(ep, (int)std::min<int64_t>(sms, (int64_t)ep.mt * dt), st, KC_DE))
+      if (int rc = kPairDEDH
+                       ? launch_tc_pair<DEPairPolicy>(
+                             ep, (int)std::min<int64_t>(sms / 2, (int64_t)ep.mt * dt), st, KC_DE)
+                       : launch_tc<DEPolicy>(ep, (int)std::min<int64_t>(sms, (int64_t)ep.mt * dt),
+                                             st, KC_DE))
         return rc;
       // step 3: dH += G E_chunk
       hp.mapB = segMN;
@@ -893,9 +932,14 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       hp.nz_cap = cap;
       hp.mask = dh_mask;
       hp.mwords = dh_words;
+      hp.mblocks = mbs;
       hp.n_valid = cp.n_valid;
       hp.status = status;
-      if (int rc = launch_tc<DHPolicy>(hp, (int)std::min<int64_t>(sms, (int64_t)mbs * dt), st, KC_DH))
+      if (int rc = kPairDEDH
+                       ? launch_tc_pair<DHPairPolicy>(
+                             hp, (int)std::min<int64_t>(sms / 2, cdiv(mbs, 2) * dt), st, KC_DH)
+                       : launch_tc<DHPolicy>(hp, (int)std::min<int64_t>(sms, (int64_t)mbs * dt), st,
+                                             KC_DH))
         return rc;
       if (side && cudaEventRecord(side->freed[chunk & 1], st) != cudaSuccess) return CCE_ELAUNCH;
       return CCE_OK;
@@ -1107,12 +1151,13 @@ size_t cce_kl_bwd_workspace_size(int64_t N, int64_t D, int64_t V, uint32_t flags
 int cce_kl_bwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
                const int32_t* row_mask, const float* lse_s, const float* lse_t,
                const float* dloss, int64_t N, int64_t D, int64_t V, float filter_eps,
-               uint32_t flags, void* dH, void* dE, void* dE_comp, void* workspace,
-               size_t workspace_bytes, int32_t* status, void* stream) {
+               uint32_t flags, void* dH, void* dE, void* dE_comp, uint32_t* debug_keep,
+               int64_t debug_rows, void* workspace, size_t workspace_bytes, int32_t* status,
+               void* stream) {
   const KLArgs a{Ht, Et, lse_t};
   return bwd_impl(Hs, Es, row_mask, lse_s, dloss, N, D, V, 0, nullptr, 0, filter_eps, nullptr,
-                  nullptr, flags, dH, dE, dE_comp, nullptr, 0, workspace, workspace_bytes, status,
-                  stream, &a);
+                  nullptr, flags, dH, dE, dE_comp, debug_keep, debug_rows, workspace,
+                  workspace_bytes, status, stream, &a);
 }
 
 

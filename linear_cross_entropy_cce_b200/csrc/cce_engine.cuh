@@ -371,6 +371,210 @@ struct Engine {
   }
 };
 
+// ===========================================================================
+// CTA-pair engine (tcgen05 cta_group::2).  A cluster of two CTAs computes one
+// 256 x 256 accumulator tile: each CTA stages its own 128 rows of A and 128 of
+// B's 256 columns per K step (32 KiB stages, PAIR_STAGES deep), the rank-0
+// CTA's single MMA thread issues M = 256 MMAs that read both CTAs' shared
+// memory, and each CTA's tensor memory holds its own 128 accumulator rows
+// (two 256-column accumulators, so the epilogue of a tile overlaps the MMAs of
+// the next).  Compared with one CTA per 128 x 256 tile, every CTA moves a
+// third fewer operand bytes per FLOP from L2 and keeps 1.5x more bytes in
+// flight.
+//   Barriers: full[s] lives in the rank-0 CTA (one arrival, by its producer,
+//   with the bytes of both CTAs' copies, which complete on it); empty[s] and
+//   tfull[a] live in both CTAs and are signalled by the MMA thread's commits
+//   (one commit arrives on the same barrier in both CTAs);
+//   tempty[a] lives in the rank-0 CTA and receives the arrivals of both CTAs'
+//   epilogue warps.  Every wait is bounded (wait_parity).
+// ===========================================================================
+constexpr int PAIR_STAGES = 6;
+constexpr int PA_BYTES = 128 * BK * 2;  // this CTA's A rows of one stage
+constexpr int PB_BYTES = 128 * BK * 2;  // this CTA's half of B's columns
+constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
+
+struct PairCtl {
+  uint64_t full[PAIR_STAGES];
+  uint64_t empty[PAIR_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int consumed;
+  int pad;
+  uint32_t rec[PAIR_STAGES];
+};
+
+template <class Policy>
+constexpr int pair_smem_bytes() {
+  return PAIR_STAGES * PSTAGE_BYTES + Policy::EXTRA_SMEM + static_cast<int>(sizeof(PairCtl)) +
+         1024 + 64;
+}
+
+struct PairPipe {
+  int stage = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void advance() {
+    if (++stage == PAIR_STAGES) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+// K-step bits of stage kb in the union of two masks (see MaskCursor); a null
+// mask issues every step.
+struct MaskPair {
+  MaskCursor a, b;
+  bool any_null;
+  __device__ __forceinline__ void init(const uint32_t* m0, const uint32_t* m1, int nkb) {
+    any_null = (m0 == nullptr) || (m1 == nullptr);
+    a.init(m0, nkb);
+    b.init(m1, nkb);
+  }
+  __device__ __forceinline__ uint32_t bits(int kb) {
+    const uint32_t x = a.bits(kb), y = b.bits(kb);
+    return any_null ? 0xFu : (x | y);
+  }
+};
+
+struct PairEngine {
+  PairCtl* ctl;
+  uint8_t* smem;
+  uint8_t* extra;
+  uint32_t tmem;
+  int* status;
+  uint32_t rank;  // 0: issues the MMAs; 1: its peer
+  PairPipe pipe;
+  int tcount = 0;
+  int fills = 0;
+  uint64_t wait_ns = kWaitLimitNs;
+
+  __device__ __forceinline__ volatile int* abort_flag() { return &ctl->abort; }
+  __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) {
+    return wait_parity(bar, parity, abort_flag(), status, wait_ns);
+  }
+  // shared::cluster address of a barrier of this CTA's layout in CTA `r`
+  __device__ __forceinline__ uint32_t in_cta(const uint64_t* bar, uint32_t r) const {
+    return mapa_shared(smem_u32(bar), r);
+  }
+
+  // ---- producer (each CTA, lane 0 of warp 0): this CTA's halves of one
+  // tile's stages.  (ax, ay) / (bx, by) are the tensor-map coordinates of this
+  // CTA's A rows and B columns; K advances along x for a K-major operand, y
+  // for an MN-major one.  Stages whose K steps are zero in both CTAs' masks
+  // are skipped by both; each loaded stage carries a record for the MMA
+  // thread (its K steps, REC_LAST on the tile's last stage), written and
+  // announced by the rank-0 producer once the next loaded stage is known.
+  template <bool A_MN, bool B_MN>
+  __device__ __forceinline__ bool produce_rec(const CUtensorMap* mA, const CUtensorMap* mB, int ax,
+                                              int ay, int bx, int by, int nkb, const uint32_t* m0,
+                                              const uint32_t* m1) {
+    MaskPair mc;
+    mc.init(m0, m1, nkb);
+    int pend = -1;
+    uint32_t pend_bits = 0;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const uint32_t bits = mc.bits(kb);
+      if (!bits) continue;
+      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
+      const uint32_t fb_local = smem_u32(&ctl->full[pipe.stage]);
+      if (rank == 0) mbar_expect_tx(fb_local, 2 * PSTAGE_BYTES);
+      const uint32_t fb = in_cta(&ctl->full[pipe.stage], 0);
+      const uint32_t sa = smem_u32(smem + pipe.stage * PSTAGE_BYTES);
+      const uint32_t sb = sa + PA_BYTES;
+      if (!A_MN) {
+        tma_load_2d_pair(sa, mA, fb, ax + kb * BK, ay);
+      } else {
+        tma_load_2d_pair(sa, mA, fb, ax, ay + kb * BK);
+        tma_load_2d_pair(sa + 8192, mA, fb, ax + 64, ay + kb * BK);
+      }
+      if (!B_MN) {
+        tma_load_2d_pair(sb, mB, fb, bx + kb * BK, by);
+      } else {
+        tma_load_2d_pair(sb, mB, fb, bx, by + kb * BK);
+        tma_load_2d_pair(sb + 8192, mB, fb, bx + 64, by + kb * BK);
+      }
+      if (rank == 0 && pend >= 0) {
+        ctl->rec[pend] = pend_bits;
+        mbar_arrive(smem_u32(&ctl->full[pend]));
+      }
+      pend = pipe.stage;
+      pend_bits = bits;
+      pipe.advance();
+      ++fills;
+    }
+    if (pend < 0) {  // nothing to load: one empty stage ends the tile (both CTAs keep step)
+      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
+      pend = pipe.stage;
+      pend_bits = 0;
+      pipe.advance();
+      ++fills;
+    }
+    if (rank == 0) {
+      ctl->rec[pend] = pend_bits | REC_LAST;
+      mbar_arrive(smem_u32(&ctl->full[pend]));
+    }
+    return true;
+  }
+
+  // ---- MMA issuer (rank 0 only, one thread): consumes the records until
+  // REC_LAST; each stage is released to both CTAs' producers by a commit to
+  // each CTA's empty barrier, the tile's accumulator to both epilogues.
+  template <bool A_MN, bool B_MN>
+  __device__ __forceinline__ bool mma_rec() {
+    const int acc = tcount & 1;
+    if (!wait(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u)) return false;
+    tc_fence_after();
+    const uint32_t d = tmem + acc * BN;
+    constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
+    constexpr uint32_t a_step = A_MN ? 2048 : 32;  // bytes per K=16 step
+    constexpr uint32_t b_step = B_MN ? 2048 : 32;
+    const uint64_t ad0 = A_MN ? smem_desc_sw128(smem_u32(smem), 8192, 1024)
+                              : smem_desc_sw128(smem_u32(smem), 16, 1024);
+    const uint64_t bd0 = B_MN ? smem_desc_sw128(smem_u32(smem) + PA_BYTES, 8192, 1024)
+                              : smem_desc_sw128(smem_u32(smem) + PA_BYTES, 16, 1024);
+    uint32_t issued = 0;
+    for (;;) {
+      if (!wait(smem_u32(&ctl->full[pipe.stage]), pipe.phase)) return false;
+      tc_fence_after();
+      const uint32_t rec = *reinterpret_cast<volatile uint32_t*>(&ctl->rec[pipe.stage]);
+      const uint64_t so = (uint64_t)((pipe.stage * PSTAGE_BYTES) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        if (!(rec & (1u << kk))) continue;
+        umma_bf16_pair(d, ad0 + so + kk * (a_step >> 4), bd0 + so + kk * (b_step >> 4), idesc,
+                       issued);
+        issued = 1;
+      }
+      umma_commit_pair_both(smem_u32(&ctl->empty[pipe.stage]));
+      pipe.advance();
+      ++fills;
+      if (rec & REC_LAST) break;
+    }
+    umma_commit_pair_both(smem_u32(&ctl->tfull[acc]));
+    ++tcount;
+    return true;
+  }
+
+  // ---- epilogue (both CTAs): this CTA's 128 accumulator rows.
+  __device__ __forceinline__ bool epi_acquire(int quarter, uint32_t& taddr) {
+    const int acc = tcount & 1;
+    if (!wait(smem_u32(&ctl->tfull[acc]), ((uint32_t)tcount >> 1) & 1u)) return false;
+    tc_fence_after();
+    taddr = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
+    return true;
+  }
+  __device__ __forceinline__ void epi_release(int lane) {
+    const int acc = tcount & 1;
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(in_cta(&ctl->tempty[acc], 0));
+    ++tcount;
+  }
+};
+
 // Bounded wait that ignores the abort flag (used only while draining).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return;
@@ -464,6 +668,90 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(ctl->tmem_base, TMEM_COLS);
+  }
+}
+
+// The CTA-pair kernel body: launched with clusters of two CTAs along x.
+template <class Policy>
+__global__ void __launch_bounds__(THREADS, 1)
+    tc_pair_kernel(const __grid_constant__ typename Policy::Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (base & 1023u)) & 1023u);
+  uint8_t* extra = smem + PAIR_STAGES * PSTAGE_BYTES;
+  PairCtl* ctl = reinterpret_cast<PairCtl*>(extra + Policy::EXTRA_SMEM);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // active() depends only on the parameters and on device values every CTA
+  // reads alike, so both CTAs of a pair leave here together or not at all
+  if (!Policy::active(p)) return;
+  const uint32_t rank = cluster_ctarank();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PAIR_STAGES; ++s) {
+      mbar_init(smem_u32(&ctl->full[s]), 1);
+      mbar_init(smem_u32(&ctl->empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&ctl->tfull[a]), 1);
+      mbar_init(smem_u32(&ctl->tempty[a]), 2 * EPI_THREADS / 32);
+    }
+    mbar_init(smem_u32(&ctl->drain), 1);
+    ctl->abort = 0;
+    ctl->consumed = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) Policy::prefetch(p);
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(&ctl->tmem_base), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote arrive
+  tc_fence_after();
+
+  PairEngine eng;
+  eng.ctl = ctl;
+  eng.smem = smem;
+  eng.extra = extra;
+  eng.tmem = ctl->tmem_base;
+  eng.status = p.status;
+  eng.rank = rank;
+  eng.wait_ns = policy_wait_limit<Policy>(p);
+
+  if (warp == 0) {
+    if (lane == 0) Policy::producer(p, eng);
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      Policy::mma(p, eng);
+      ctl->consumed = eng.fills;
+      // every pair MMA this thread issued has completed (they read both
+      // CTAs' shared memory, so neither CTA may leave before this)
+      umma_commit_pair_own(smem_u32(&ctl->drain));
+      drain_wait(smem_u32(&ctl->drain), 0);
+    }
+  } else {
+    Policy::epilogue(p, eng, warp & 3, lane);
+  }
+  __syncthreads();
+  tc_fence_before();
+  cluster_sync_all();
+  // After an abort, copies issued by either CTA may still be landing (their
+  // bytes count on the rank-0 CTA's barriers, which a phase that will never
+  // complete cannot report): both CTAs give them a fixed grace period before
+  // leaving.  Never taken on the normal path, where every issued stage was
+  // consumed by an MMA that waited for all of its bytes.
+  const int any_abort =
+      ctl->abort | (int)ld_shared_cluster_u32(mapa_shared(smem_u32(&ctl->abort), rank ^ 1u));
+  if (any_abort) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 2000000ull) {
+    }
+  }
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(ctl->tmem_base, TMEM_COLS);
   }
 }
 

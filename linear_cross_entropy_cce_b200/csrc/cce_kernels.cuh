@@ -775,19 +775,33 @@ __device__ __forceinline__ bool mask_empty(const uint32_t* m, int nkb, int lane)
   return __all_sync(0xffffffffu, any == 0u);
 }
 
-struct DEPolicy {
+// One CTA per 128 x 256 tile of dE (PAIR = false) or one CTA pair per
+// 256 x 256 tile (PAIR = true, tcgen05 cta_group::2; the host sets mt to the
+// number of 128- or 256-row vocabulary tiles accordingly).
+template <bool PAIR>
+struct DEPolicyT {
   using Params = DEParams;
   static constexpr int EXTRA_SMEM = 0;
+  static constexpr int ROWS = PAIR ? 2 * BM : BM;  // vocabulary rows per tile
   // a chunk taken by the sparse route has no dense work
   static __device__ __forceinline__ bool active(const Params& p) {
     return !(p.nz_cnt && *p.nz_cnt <= p.nz_cap);
+  }
+  // K-step masks of the (one or two) 128-row vocabulary blocks of tile vt
+  static __device__ __forceinline__ const uint32_t* mask_lo(const Params& p, int vt) {
+    return p.mask + (size_t)(PAIR ? 2 * vt : vt) * p.mwords;
+  }
+  static __device__ __forceinline__ const uint32_t* mask_hi(const Params& p, int vt) {
+    return PAIR ? p.mask + (size_t)(2 * vt + 1) * p.mwords : mask_lo(p, vt);
   }
 
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
     const int nkb = (*p.n_valid + BK - 1) / BK;
     const int tiles = (p.nz_cnt && *p.nz_cnt <= p.nz_cap) ? 0 : p.mt * p.dt;
-    for (int i = blockIdx.x; i < tiles; i += gridDim.x) {
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    for (int i = unit; i < tiles; i += units) {
       const int vt = i / p.dt;
       if (!f(vt, i - vt * p.dt, nkb)) return;
     }
@@ -796,24 +810,35 @@ struct DEPolicy {
     tma_prefetch_map(&p.mapA);
     tma_prefetch_map(&p.mapB);
   }
-  static __device__ void producer(const Params& p, Engine& eng) {
+  template <class Eng>
+  static __device__ void producer(const Params& p, Eng& eng) {
     schedule(p, [&](int vt, int dtile, int nkb) {
-      return eng.produce_rec<true, true>(&p.mapA, &p.mapB, vt * BM, 0, dtile * BN, 0, nkb,
-                                         p.mask + vt * p.mwords);
+      if constexpr (PAIR) {
+        const int r = (int)eng.rank * BM;
+        return eng.template produce_rec<true, true>(&p.mapA, &p.mapB, vt * ROWS + r, 0,
+                                                    dtile * BN + r, 0, nkb, mask_lo(p, vt),
+                                                    mask_hi(p, vt));
+      } else {
+        return eng.template produce_rec<true, true>(&p.mapA, &p.mapB, vt * BM, 0, dtile * BN, 0,
+                                                    nkb, mask_lo(p, vt));
+      }
     });
   }
-  static __device__ void mma(const Params& p, Engine& eng) {
-    schedule(p, [&](int vt, int, int nkb) {
-      return nkb == 0 || eng.mma_rec<true, true>();
-    });
+  template <class Eng>
+  static __device__ void mma(const Params& p, Eng& eng) {
+    schedule(p, [&](int, int, int nkb) { return nkb == 0 || eng.template mma_rec<true, true>(); });
   }
-  static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
+  template <class Eng>
+  static __device__ void epilogue(const Params& p, Eng& eng, int q, int lane) {
     const int row = q * 32 + lane;
+    uint32_t rank = 0;
+    if constexpr (PAIR) rank = eng.rank;
     schedule(p, [&](int vt, int dtile, int nkb) {
-      const bool zero = nkb == 0 || mask_empty(p.mask + vt * p.mwords, nkb, lane);
+      const bool zero = nkb == 0 || (mask_empty(mask_lo(p, vt), nkb, lane) &&
+                                     (!PAIR || mask_empty(mask_hi(p, vt), nkb, lane)));
       uint32_t taddr = 0;
       if (nkb > 0 && !eng.epi_acquire(q, taddr)) return false;
-      const int r = vt * BM + row;
+      const int r = vt * ROWS + (int)rank * BM + row;
       const bool ok = r < p.chunk_valid;
       const int w = p.c0 + r;
       const size_t local = ok ? (size_t)(p.perm_seg ? p.perm_seg[w] : w) : 0;
@@ -873,6 +898,8 @@ struct DEPolicy {
     });
   }
 };
+using DEPolicy = DEPolicyT<false>;
+using DEPairPolicy = DEPolicyT<true>;
 
 // =====================================================================
 // Backward, step 3: dH_acc[j, :] += G[j, chunk] E_chunk, K = chunk.
@@ -890,24 +917,42 @@ struct DHParams {
   int nz_cap;
   const uint32_t* mask;  // dh_mask of the G producer (K-step mask per row block)
   int mwords;
+  int mblocks;  // 128-row blocks the mask buffer holds (Npad / 128)
   const int* n_valid;
   int* status;
 };
 
-struct DHPolicy {
+// One CTA per 128 x 256 tile of dH (PAIR = false) or one CTA pair per
+// 256 x 256 tile (PAIR = true).  In a pair tile whose second 128-row block
+// lies beyond the valid rows, that block's rows (zero or stale G rows) are
+// computed and reduced into dH_acc rows that nothing reads (rows >= Npad are
+// clipped by the tensor map).
+template <bool PAIR>
+struct DHPolicyT {
   using Params = DHParams;
+  static constexpr int ROWS = PAIR ? 2 * BM : BM;
   static __device__ __forceinline__ bool active(const Params& p) {
     return !(p.nz_cnt && *p.nz_cnt <= p.nz_cap);
   }
   // per epilogue warp: two 32 x 32 fp32 staging tiles for the TMA reduce-add
   static constexpr int EXTRA_SMEM = 4 * 2 * 4096;
+  static __device__ __forceinline__ const uint32_t* mask_lo(const Params& p, int mb) {
+    return p.mask + (size_t)(PAIR ? 2 * mb : mb) * p.mwords;
+  }
+  static __device__ __forceinline__ const uint32_t* mask_hi(const Params& p, int mb) {
+    // the mask buffer has one entry per 128-row block of Npad
+    return (PAIR && 2 * mb + 1 < p.mblocks) ? p.mask + (size_t)(2 * mb + 1) * p.mwords
+                                            : mask_lo(p, mb);
+  }
 
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
     const int nv = *p.n_valid;
-    const int num_mb = (nv + BM - 1) / BM;
+    const int num_mb = (nv + ROWS - 1) / ROWS;
     const int tiles = (p.nz_cnt && *p.nz_cnt <= p.nz_cap) ? 0 : num_mb * p.dt;
-    for (int i = blockIdx.x; i < tiles; i += gridDim.x) {
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    for (int i = unit; i < tiles; i += units) {
       const int mb = i / p.dt;
       if (!f(mb, i - mb * p.dt, nv)) return;
     }
@@ -917,29 +962,47 @@ struct DHPolicy {
     tma_prefetch_map(&p.mapB);
     tma_prefetch_map(&p.mapC);
   }
-  static __device__ void producer(const Params& p, Engine& eng) {
+  template <class Eng>
+  static __device__ void producer(const Params& p, Eng& eng) {
     schedule(p, [&](int mb, int dtile, int) {
-      return eng.produce_rec<false, true>(&p.mapA, &p.mapB, 0, mb * BM, dtile * BN, p.b_row0,
-                                          p.nkb, p.mask + mb * p.mwords);
+      if constexpr (PAIR) {
+        const int r = (int)eng.rank * BM;
+        return eng.template produce_rec<false, true>(&p.mapA, &p.mapB, 0, mb * ROWS + r,
+                                                     dtile * BN + r, p.b_row0, p.nkb,
+                                                     mask_lo(p, mb), mask_hi(p, mb));
+      } else {
+        return eng.template produce_rec<false, true>(&p.mapA, &p.mapB, 0, mb * BM, dtile * BN,
+                                                     p.b_row0, p.nkb, mask_lo(p, mb));
+      }
     });
   }
-  static __device__ void mma(const Params& p, Engine& eng) {
-    schedule(p, [&](int, int, int) { return eng.mma_rec<false, true>(); });
+  template <class Eng>
+  static __device__ void mma(const Params& p, Eng& eng) {
+    schedule(p, [&](int, int, int) { return eng.template mma_rec<false, true>(); });
   }
   // Each warp adds its 32 accumulator rows into dH_acc 32 columns at a time:
   // tcgen05.ld -> swizzled staging tile in shared memory -> TMA reduce-add
   // (performed in L2), double-buffered so the next chunk is staged while the
   // previous reduction still reads shared memory.  Rows past n_valid hold
   // zeros (their G rows are zero), columns past D are clipped by the map.
-  static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
+  template <class Eng>
+  static __device__ void epilogue(const Params& p, Eng& eng, int q, int lane) {
     uint8_t* stage = eng.extra + q * 2 * 4096;
     const uint32_t st0 = smem_u32(stage);
     int nbuf = 0;
+    uint32_t rank = 0;
+    if constexpr (PAIR) rank = eng.rank;
     schedule(p, [&](int mb, int dtile, int) {
-      const bool zero = mask_empty(p.mask + mb * p.mwords, p.nkb, lane);  // nothing to add
+      // nothing to add when no K step of the tile was issued
+      const bool zero = mask_empty(mask_lo(p, mb), p.nkb, lane) &&
+                        (!PAIR || mask_empty(mask_hi(p, mb), p.nkb, lane));
       uint32_t taddr;
       if (!eng.epi_acquire(q, taddr)) return false;
-      for (int c = 0; c < BN / 32 && !zero; ++c) {
+      const int row0 = mb * ROWS + (int)rank * BM + q * 32;
+      // rows at or beyond Npad (the upper half of a pair tile past the end)
+      // have no dH_acc rows: nothing to add
+      const bool skip = zero || row0 >= p.mblocks * BM;
+      for (int c = 0; c < BN / 32 && !skip; ++c) {
         const int col0 = dtile * BN + c * 32;
         if (col0 >= p.D) break;
         uint32_t v[32];
@@ -957,7 +1020,7 @@ struct DHPolicy {
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_reduce_add_2d(&p.mapC, st0 + b * 4096, col0, mb * BM + q * 32);
+          tma_reduce_add_2d(&p.mapC, st0 + b * 4096, col0, row0);
           bulk_commit();
         }
         ++nbuf;
@@ -969,6 +1032,8 @@ struct DHPolicy {
     __syncwarp();
   }
 };
+using DHPolicy = DHPolicyT<false>;
+using DHPairPolicy = DHPolicyT<true>;
 
 // Bounds for the exact tile skip of the G producer.  One warp per output:
 //   tile_cmax2[tile_off[s] + t] = log2 e * max colmax over walk positions

@@ -40,8 +40,12 @@ int main(void) {
         CCE_EINVAL);
   CHECK(cce_bwd(p, p, y, f, f, 4, 8, 10, -100, NULL, 0, 0.f, NULL, NULL, 64u, p, p, NULL, NULL, 0,
                 p, 1u << 30, st, NULL) == CCE_EINVAL); /* unknown flag */
-  CHECK(cce_kl_bwd(p, p, p, p, NULL, f, f, f, 4, 8, 10, 0.f, CCE_FULL_DE, p, p, NULL, p, 1u << 30,
-                   st, NULL) == CCE_EINVAL);
+  CHECK(cce_kl_bwd(p, p, p, p, NULL, f, f, f, 4, 8, 10, 0.f, CCE_FULL_DE, p, p, NULL, NULL, 0, p,
+                   1u << 30, st, NULL) == CCE_EINVAL);
+  /* the vocabulary-parallel combine and the wait diagnostic check their arguments */
+  CHECK(cce_vocab_combine(f, 0, y, 4, 10, -100, NULL, 0, f, f, NULL) == CCE_EINVAL);
+  CHECK(cce_vocab_combine(NULL, 0, y, 0, 10, -100, NULL, 0, f, f, NULL) == CCE_EINVAL);
+  CHECK(cce_debug_stall(0, st, NULL) == CCE_EINVAL);
   /* an empty batch is a no-op */
   CHECK(cce_fwd(p, p, y, 0, 8, 10, -100, NULL, 0, f, f, NULL, p, 1u << 30, st, NULL) == CCE_OK);
 

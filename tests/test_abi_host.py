@@ -151,13 +151,14 @@ def test_kl_and_shard_entry_points_reject_bad_arguments_on_host():
     assert kl_fwd(N=0) == cce.CCE_OK        # nothing to do
 
     # cce_kl_bwd(Hs, Es, Ht, Et, mask, lse_s, lse_t, dloss, N, D, V, eps, flags, dH, dE, dE_comp,
-    #            ws, wsb, status, stream)
-    def kl_bwd(flags=0, Ht=16):
+    #            debug_keep, debug_rows, ws, wsb, status, stream)
+    def kl_bwd(flags=0, Ht=16, dbg_rows=0):
         return L.cce_kl_bwd(16, 16, Ht, 16, None, 16, 16, 16, 4, 8, 10, 0.0, flags, 16, 16, None,
-                            16, 1 << 30, 16, None)
+                            16 if dbg_rows else None, dbg_rows, 16, 1 << 30, 16, None)
     assert kl_bwd(flags=cce.FULL_DE) == EINVAL
     assert kl_bwd(flags=cce.VOCAB_SHARD) == EINVAL
     assert kl_bwd(Ht=None) == EINVAL
+    assert kl_bwd(dbg_rows=5) == EINVAL  # more debug rows than rows
     assert L.cce_kl_bwd_workspace_size(256, 256, 4096, 0) > L.cce_bwd_workspace_size(256, 256, 4096, 0, 0)
     assert L.cce_kl_fwd_workspace_size(256, 250, 4096) == 0
 

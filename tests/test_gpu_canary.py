@@ -175,8 +175,10 @@ def test_soft_target_kl_writes_only_its_buffers(eps):
     dH = g.alloc((N, D), torch.bfloat16)
     dE = g.alloc((V, D), torch.bfloat16)
     ws_b = g.alloc((L.cce_kl_bwd_workspace_size(N, D, V, 0),), torch.uint8)
+    keep = g.alloc((N, (V + 31) // 32), torch.int32) if eps > 0 else None
     rc = L.cce_kl_bwd(_p(Hs), _p(E), _p(Ht), _p(E), _p(mask), _p(ls), _p(lt), _p(dl), N, D, V,
-                      float(eps), 0, _p(dH), _p(dE), None, _p(ws_b), ws_b.numel(), _p(st), _stream())
+                      float(eps), 0, _p(dH), _p(dE), None, _p(keep), N if keep is not None else 0,
+                      _p(ws_b), ws_b.numel(), _p(st), _stream())
     assert rc == 0
     g.check()
     assert int(st.item()) == 0

@@ -125,3 +125,37 @@ def test_kl_full_size_sampled_rows_and_pairing_identity():
     lhs = float(torch.sum(dH.double() * a.double()))
     rhs = float(torch.sum(dE.double() * e.double()))
     assert abs(lhs - rhs) <= 1e-3 * max(abs(lhs), abs(rhs), 1e-12)
+
+
+@pytest.mark.parametrize("case", ["separate_heads", "sparse"])
+def test_kl_filter_criterion_per_element(case):
+    """Every entry the KL backward drops has both oracle probabilities below
+    eps (its gradient dloss (p_s - p_t) is then below eps in magnitude); every
+    entry where either reaches eps (with a margin for fp32 rounding) is kept."""
+    from linear_cross_entropy_cce_b200 import cce
+    Hs, Es, Ht, Et, mask = _kl_case(**CASES[case])
+    tm = torch.from_numpy(mask).cuda() if mask is not None else None
+    Hs_d, Es_d, Ht_d = _up(Hs), _up(Es), _up(Ht)
+    Et_d = Es_d if CASES[case]["shared"] else _up(Et)
+    kl, ls, lt = cce.kl_fwd(Hs_d, Es_d, Ht_d, Et_d, tm)
+    N, V = Hs.shape[0], Es.shape[0]
+    dl = torch.full((N,), 1.0 / N, dtype=torch.float32, device="cuda")
+    _, _, keep = cce.kl_bwd(Hs_d, Es_d, Ht_d, Et_d, ls, lt, dl, tm, filter_eps=EPS_BF16,
+                            debug_rows=N)
+    torch.cuda.synchronize()
+    bits = keep.cpu().numpy().view(np.uint32)
+    kept = np.unpackbits(bits.view(np.uint8), bitorder="little").reshape(N, -1)[:, :V].astype(bool)
+    rows = np.arange(N) if mask is None else np.nonzero(mask)[0]
+    Es64, Et64 = oracle.widen_bf16(Es), oracle.widen_bf16(Et)
+    Zs = oracle.widen_bf16(Hs[rows]) @ Es64.T
+    Zt = oracle.widen_bf16(Ht[rows]) @ Et64.T
+    Ps = np.exp(Zs - oracle.logsumexp_rows(Zs)[:, None])
+    Pt = np.exp(Zt - oracle.logsumexp_rows(Zt)[:, None])
+    k = kept[rows]
+    dropped = ~k
+    assert np.all((Ps[dropped] < EPS_BF16) & (Pt[dropped] < EPS_BF16))
+    must_keep = (Ps >= EPS_BF16 * 1.001) | (Pt >= EPS_BF16 * 1.001)
+    assert np.all(k[must_keep])
+    if mask is not None:  # masked rows keep nothing
+        assert not kept[mask == 0].any()
+    assert dropped.any() and k.any()  # the criterion is exercised both ways
