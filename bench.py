@@ -45,6 +45,7 @@ MODES = {
     "tiny": (False, False),
     "gemma2_2b_head": (True, True),
     "llama3_8b_head": (False, False),
+    "llama3_8b_head_8k": (False, False),
     "phi35_mini_head": (True, False),
     "composite_two_segment": (True, False),
 }

@@ -197,10 +197,11 @@ struct KLFwdPlan {
   size_t off_nvalid, off_idx, off_pos, off_hs, off_ht, off_part, total;
 };
 
-KLFwdPlan plan_kl_fwd(int64_t N, int64_t D, int64_t V) {
+// tile: vocabulary ids per tile (256, or 128 for a shared head's dual tiles)
+KLFwdPlan plan_kl_fwd(int64_t N, int64_t D, int64_t V, int tile = BN) {
   KLFwdPlan p;
   p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
-  p.T_v = (int)cdiv(V, BN);
+  p.T_v = (int)cdiv(V, tile);
   const int64_t num_mb = p.Npad / BM;
   p.tpi = (int)std::min<int64_t>(16, std::max<int64_t>(2, num_mb * p.T_v / (kPlanSMs * 24)));
   p.S = (int)cdiv(p.T_v, p.tpi);
@@ -1071,7 +1072,8 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
 // ------------------------------------------------------------ soft-target KL
 size_t cce_kl_fwd_workspace_size(int64_t N, int64_t D, int64_t V) {
   if (!sizes_ok(N, D, V)) return 0;
-  return plan_kl_fwd(N, D, V).total;
+  // enough for either tile width
+  return std::max(plan_kl_fwd(N, D, V, BN).total, plan_kl_fwd(N, D, V, BN / 2).total);
 }
 
 int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
@@ -1083,7 +1085,9 @@ int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
   if (!Hs || !Es || !Ht || !Et || !kl || !lse_s || !lse_t || !status || !aligned16(Hs) ||
       !aligned16(Es) || !aligned16(Ht) || !aligned16(Et))
     return CCE_EINVAL;
-  const KLFwdPlan pl = plan_kl_fwd(N, D, V);
+  // one head for teacher and student: dual 128-id tiles (see KLFwdPolicyT)
+  const bool dual = Es == Et;
+  const KLFwdPlan pl = plan_kl_fwd(N, D, V, dual ? BN / 2 : BN);
   if (!workspace || workspace_bytes < pl.total) return CCE_EWORKSPACE;
   const int sms = device_sms();
   if (sms <= 0 || !encode_fn()) return CCE_EDEVICE;
@@ -1113,7 +1117,8 @@ int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
   memset(&kp, 0, sizeof(kp));
   if (!make_map(&kp.mapAs, Hs_c, D, pl.Npad, D, BK, BM) ||
       !make_map(&kp.mapAt, Ht_c, D, pl.Npad, D, BK, BM) ||
-      !make_map(&kp.mapBs, Es, D, V, D, BK, BN) || !make_map(&kp.mapBt, Et, D, V, D, BK, BN))
+      !make_map(&kp.mapBs, Es, D, V, D, BK, BN) || !make_map(&kp.mapBt, Et, D, V, D, BK, BN) ||
+      !make_map(&kp.mapB128, Es, D, V, D, BK, BN / 2))
     return CCE_ELAUNCH;
   kp.V = (int)V;
   kp.T_v = pl.T_v;
@@ -1125,7 +1130,9 @@ int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
   kp.part = at<float>(workspace, pl.off_part);
   kp.status = status;
   const int64_t items = (pl.Npad / BM) * pl.S;
-  if (int rc = launch_tc<KLFwdPolicy>(kp, (int)std::min<int64_t>(sms, items), st, KC_FWD))
+  const int grid = (int)std::min<int64_t>(sms, items);
+  if (int rc = dual ? launch_tc<KLFwdDualPolicy>(kp, grid, st, KC_FWD)
+                    : launch_tc<KLFwdPolicy>(kp, grid, st, KC_FWD))
     return rc;
   KLFinParams fin;
   fin.pos_of_row = cp.pos_of_row;

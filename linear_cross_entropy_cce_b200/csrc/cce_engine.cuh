@@ -331,7 +331,57 @@ struct Engine {
     return true;
   }
 
-  // ---- epilogue: wait for the next accumulator; returns its TMEM address
+  // ---- two products over one staged head tile (one 48 KiB stage: rows of
+  // two row operands, 128 x 64 each, and 128 rows of the shared B operand):
+  // the MMA thread issues both N = 128 products from it, into columns
+  // [0, 128) and [128, 256) of one accumulator, so a tile pair takes 256
+  // TMEM columns and the two accumulators still alternate (the epilogue of a
+  // pair overlaps the MMAs of the next).  Per FLOP this moves as many operand
+  // bytes as a single N = 256 product.
+  __device__ __forceinline__ bool produce_dual(const CUtensorMap* mA0, const CUtensorMap* mA1,
+                                               const CUtensorMap* mB, int ay, int by, int nkb) {
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
+      const uint32_t fb = smem_u32(&ctl->full[pipe.stage]);
+      mbar_arrive_expect_tx(fb, STAGE_BYTES);
+      const uint32_t sa = smem_u32(smem + pipe.stage * STAGE_BYTES);
+      tma_load_2d(sa, mA0, fb, kb * BK, ay);
+      tma_load_2d(sa + A_BYTES, mA1, fb, kb * BK, ay);
+      tma_load_2d(sa + 2 * A_BYTES, mB, fb, kb * BK, by);
+      pipe.advance();
+      ++fills;
+    }
+    return true;
+  }
+  __device__ __forceinline__ bool mma_dual(int nkb) {
+    const int acc = tcount & 1;
+    if (!wait(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u)) return false;
+    tc_fence_after();
+    const uint32_t d0 = tmem + acc * BN;
+    const uint32_t d1 = d0 + BN / 2;
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN / 2, false, false);
+    uint32_t issued = 0;
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!wait(smem_u32(&ctl->full[pipe.stage]), pipe.phase)) return false;
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + pipe.stage * STAGE_BYTES);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t bd = smem_desc_sw128(sa + 2 * A_BYTES + kk * 32, 16, 1024);
+        umma_bf16(d0, smem_desc_sw128(sa + kk * 32, 16, 1024), bd, idesc, issued);
+        umma_bf16(d1, smem_desc_sw128(sa + A_BYTES + kk * 32, 16, 1024), bd, idesc, issued);
+        issued = 1;
+      }
+      umma_commit(smem_u32(&ctl->empty[pipe.stage]));
+      pipe.advance();
+      ++fills;
+    }
+    umma_commit(smem_u32(&ctl->tfull[acc]));
+    ++tcount;
+    return true;
+  }
+
+  // ---- epilogue: wait for the next accumulator; returns its TMEM address  // ---- epilogue: wait for the next accumulator; returns its TMEM address
   // for this thread's lane quarter (column 0).
   __device__ __forceinline__ bool epi_acquire(int quarter, uint32_t& taddr) {
     const int acc = tcount & 1;

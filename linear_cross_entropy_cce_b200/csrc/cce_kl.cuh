@@ -25,8 +25,9 @@ namespace cce {
 struct KLFwdParams {
   CUtensorMap mapAs, mapAt;  // H_s,c / H_t,c [Npad, D], box {64, 128}
   CUtensorMap mapBs, mapBt;  // E_s / E_t [V, D], box {64, 256}
+  CUtensorMap mapB128;       // the shared head E [V, D], box {64, 128} (dual tiles)
   int V;
-  int T_v;   // vocabulary tiles
+  int T_v;   // vocabulary tiles (of the policy's width)
   int tpi;   // tiles per work item
   int S;     // splits
   int Npad;  // partial row stride
@@ -36,9 +37,17 @@ struct KLFwdParams {
   int* status;
 };
 
-struct KLFwdPolicy {
+// DUAL = false: separate heads; each 256-id tile is a pair of N = 256
+// products (teacher, then student), one per accumulator, so the pair's
+// epilogue waits for both and does not overlap the next pair's MMAs.
+// DUAL = true: one head shared by teacher and student; each 128-id tile is
+// two N = 128 products from one staged head tile (Engine::produce_dual /
+// mma_dual) in one accumulator, and the two accumulators alternate.
+template <bool DUAL>
+struct KLFwdPolicyT {
   using Params = KLFwdParams;
   static constexpr int EXTRA_SMEM = 0;
+  static constexpr int TN = DUAL ? BN / 2 : BN;  // vocabulary ids per tile
   static __device__ __forceinline__ bool active(const Params&) { return true; }
 
   template <class F>
@@ -61,20 +70,30 @@ struct KLFwdPolicy {
   static __device__ void prefetch(const Params& p) {
     tma_prefetch_map(&p.mapAs);
     tma_prefetch_map(&p.mapAt);
-    tma_prefetch_map(&p.mapBs);
-    tma_prefetch_map(&p.mapBt);
+    if constexpr (DUAL) {
+      tma_prefetch_map(&p.mapB128);
+    } else {
+      tma_prefetch_map(&p.mapBs);
+      tma_prefetch_map(&p.mapBt);
+    }
   }
 
   static __device__ void producer(const Params& p, Engine& eng) {
     schedule(p, [&](int mb, int, int t, bool, int) {
-      return eng.produce<false, false>(&p.mapAt, &p.mapBt, 0, mb * BM, 0, t * BN, p.nkb) &&
-             eng.produce<false, false>(&p.mapAs, &p.mapBs, 0, mb * BM, 0, t * BN, p.nkb);
+      if constexpr (DUAL)
+        return eng.produce_dual(&p.mapAt, &p.mapAs, &p.mapB128, mb * BM, t * TN, p.nkb);
+      else
+        return eng.produce<false, false>(&p.mapAt, &p.mapBt, 0, mb * BM, 0, t * BN, p.nkb) &&
+               eng.produce<false, false>(&p.mapAs, &p.mapBs, 0, mb * BM, 0, t * BN, p.nkb);
     });
   }
 
   static __device__ void mma(const Params& p, Engine& eng) {
     schedule(p, [&](int, int, int, bool, int) {
-      return eng.mma<false, false>(p.nkb) && eng.mma<false, false>(p.nkb);
+      if constexpr (DUAL)
+        return eng.mma_dual(p.nkb);
+      else
+        return eng.mma<false, false>(p.nkb) && eng.mma<false, false>(p.nkb);
     });
   }
 
@@ -84,10 +103,15 @@ struct KLFwdPolicy {
     float ms = -INFINITY, ss = 0.f;           // student
     schedule(p, [&](int mb, int split, int t, bool last, int nv) {
       uint32_t ta, tb;
-      if (!eng.epi_acquire2(q, ta, tb)) return false;
-      const int valid = min(BN, p.V - t * BN);
+      if constexpr (DUAL) {
+        if (!eng.epi_acquire(q, ta)) return false;
+        tb = ta + TN;  // student columns follow the teacher's in the same accumulator
+      } else {
+        if (!eng.epi_acquire2(q, ta, tb)) return false;
+      }
+      const int valid = min(TN, p.V - t * TN);
       const bool row_ok = mb * BM + row < nv;
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < TN / 32; ++c) {
         if (c * 32 >= valid) break;  // uniform over the CTA
         const int nvc = min(32, valid - c * 32);
         uint32_t rt[32], rs[32];
@@ -122,7 +146,10 @@ struct KLFwdPolicy {
         ms = ns;
         ss = as;
       }
-      eng.epi_release2(lane);
+      if constexpr (DUAL)
+        eng.epi_release(lane);
+      else
+        eng.epi_release2(lane);
       if (last) {
         if (row_ok) {
           float* o = p.part + (size_t)split * 5 * p.Npad + mb * BM + row;
@@ -142,6 +169,8 @@ struct KLFwdPolicy {
     });
   }
 };
+using KLFwdPolicy = KLFwdPolicyT<false>;
+using KLFwdDualPolicy = KLFwdPolicyT<true>;
 
 // Splits combined per row (one warp per original row): KL = A - lse_t +
 // lse_s with A = w / s_t after both are rescaled to the teacher's overall

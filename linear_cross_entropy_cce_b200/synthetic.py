@@ -74,6 +74,10 @@ WORKLOADS = {
         "composite_two_segment", N=24576, D=2048, V=248320, logit_std=6.0,
         ignore_frac=0.50, segments=((0, 151936), (153090, 248320)),
         segment_mix=(0.7, 0.3)),
+    # the Llama-3-8B-shaped head at half the rows: sized for kernel captures
+    # (a few GB on the device; H_c still larger than L2)
+    "llama3_8b_head_8k": Workload("llama3_8b_head_8k", N=8192, D=4096, V=128256,
+                                  logit_std=1.0, ignore_frac=0.0),
 }
 
 

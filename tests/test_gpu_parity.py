@@ -325,3 +325,50 @@ def test_degenerate_shapes(N, D, V, eps):
         tol = TOL_GRAD_FILTER if eps > 0 else TOL_GRAD
         assert normwise(to_np(dH), rH) <= tol
         assert normwise(to_np(dEs[0]), rE[0]) <= tol
+
+
+def test_mispredicted_chunks_and_mixed_routes():
+    """A filtered call whose vocabulary chunks alternate sparse / dense: with
+    N = 512 (list capacity 4096 entries per 16384-id chunk), chunks 1 and 3
+    hold 256 "hot" ids per row (every row's logit there is about 8 while the
+    other ~65k logits are ~N(0, 1), so each hot entry keeps p ~ 3e-3 and the
+    chunk holds 131k kept entries), chunks 0 and 2 keep almost nothing but the
+    targets.  The backward predicts chunk 1 sparse from chunk 0 and must repair
+    it with a second, dense launch; it predicts chunk 2 dense from chunk 1 (the
+    slab is written) but takes the sparse route there; chunk 3 is mispredicted
+    again.  dH then sums the dense chunks' accumulator with the sparse
+    chunks' gathers.  Parity with the oracle, and every hot entry kept."""
+    from linear_cross_entropy_cce_b200 import cce
+    N, D, V = 512, 64, 4 * 16384
+    rng = np.random.default_rng(11)
+    H = rng.standard_normal((N, D)).astype(np.float32)
+    H[:, 0] = 4.0
+    E = (rng.standard_normal((V, D)) / np.sqrt(D)).astype(np.float32)
+    E[:, 0] = 0.0
+    hot = np.concatenate([np.arange(16384 + 1000, 16384 + 1256), np.arange(3 * 16384 + 77, 3 * 16384 + 333)])
+    E[hot] = 0.01 * E[hot]
+    E[hot, 0] = 2.0  # logit 8 for every row
+    y = rng.integers(0, V, N).astype(np.int32)
+    y[::9] = -100
+    Hb, Eb = syn.fp32_to_bf16_bits(H), syn.fp32_to_bf16_bits(E)
+    Hd, Ed = cce.bf16_from_bits(Hb, "cuda"), cce.bf16_from_bits(Eb, "cuda")
+    yd = torch.from_numpy(y).cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    loss, lse = cce.fwd(Hd, Ed, yd, status=st)
+    valid = y != -100
+    dl = np.where(valid, 1.0 / valid.sum(), 0.0)
+    dH, dE, keep = cce.bwd(Hd, Ed, yd, lse, torch.from_numpy(dl).float().cuda(),
+                           filter_eps=EPS_BF16, debug_rows=N, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rH, rE = oracle.backward(Hb, [(0, V, Eb)], y, V, dl, -100, filter_eps=EPS_BF16)
+    assert normwise(to_np(dH), rH) <= TOL_GRAD_FILTER
+    assert normwise(to_np(dE), rE[0]) <= TOL_GRAD_FILTER
+    bits = keep.cpu().numpy().view(np.uint32)
+    kept = np.unpackbits(bits.view(np.uint8), bitorder="little").reshape(N, -1)[:, :V].astype(bool)
+    assert kept[np.ix_(valid, hot)].all()
+    per_chunk = kept[valid].reshape(-1, 4, 16384).sum(axis=(0, 2))
+    assert per_chunk[1] > 4096 and per_chunk[3] > 4096  # dense: beyond the list capacity
+    assert per_chunk[0] < 1024 and per_chunk[2] < 1024  # sparse
+    # the hot columns' dE rows are the large ones, and they are right
+    assert normwise(to_np(dE)[hot], rE[0][hot]) <= TOL_GRAD_FILTER
