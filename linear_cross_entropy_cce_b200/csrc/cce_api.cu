@@ -769,6 +769,8 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   memset(&ep, 0, sizeof(ep));
   memset(&hp, 0, sizeof(hp));
   if (!make_map(&gp.mapA, Hc, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
+  // soft-target KL with one head for student and teacher: dual 128-id tiles
+  const bool kl_dual = kl != nullptr && kl->Et == E;
   if (kl) {
     if (!make_map(&gp.mapA2, Ht_c, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
     if (!make_map(&gp.mapB2, kl->Et, D, V, D, BK, BN)) return CCE_ELAUNCH;
@@ -858,7 +860,8 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       gp.mapB = segK;
       gp.b_row0 = row0;
       gp.chunk_valid = cv;
-      gp.ct = (int)cdiv(cv, BN);
+      gp.ct = (int)cdiv(cv, kl_dual ? BN / 2 : BN);
+      if (kl_dual && !make_map(&gp.mapB128, sg.s[s].E, D, ns, D, BK, BN / 2)) return CCE_ELAUNCH;
       gp.seg = s;
       gp.c0 = c0;
       gp.Vc = Vc;
@@ -889,16 +892,16 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       gp.blk_lse2min = blk_lse2min;
       gp.skip_l2 = gp.l2eps - 1.0f / 16.0f;  // margin over fp32 differences of the two logits
       const int g_grid = (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct);
-      if (int rc = kl ? launch_tc<GPolicyKL>(gp, g_grid, st, KC_G)
-                      : full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
-                                : launch_tc<GPolicy>(gp, g_grid, st, KC_G))
-        return rc;
+      auto launch_g = [&]() {
+        return kl_dual ? launch_tc<GPolicyKLDual>(gp, g_grid, st, KC_G)
+               : kl    ? launch_tc<GPolicyKL>(gp, g_grid, st, KC_G)
+               : full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
+                         : launch_tc<GPolicy>(gp, g_grid, st, KC_G);
+      };
+      if (int rc = launch_g()) return rc;
       if (sparse) {  // recompute with the dense fallback if the chunk was mispredicted
         gp.repair = 1;
-        if (int rc = kl ? launch_tc<GPolicyKL>(gp, g_grid, st, KC_G)
-                        : full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
-                                  : launch_tc<GPolicy>(gp, g_grid, st, KC_G))
-          return rc;
+        if (int rc = launch_g()) return rc;
       }
       // step 2: dE rows of this chunk (chunks on the sparse route: after the loop)
       ep.nz_cnt = sparse_de ? nz_cnt + chunk : nullptr;

@@ -493,6 +493,7 @@ struct GParams {
   // an entry kept when either probability reaches the threshold.
   CUtensorMap mapA2;  // H_t,c [Npad, D], box {64, 128}
   CUtensorMap mapB2;  // E_t rows, K-major, box {64, 256}
+  CUtensorMap mapB128;  // shared head rows, K-major, box {64, 128} (dual tiles)
   const float* lt2_c;
   // optional per-element keep bits of original rows < debug_rows
   uint32_t* debug_keep;
@@ -504,10 +505,15 @@ struct GParams {
   int* status;
 };
 
-template <bool FULL, bool KL = false>
+// KL && DUAL: the student and teacher share one head; each 128-id tile is
+// two N = 128 products from one staged head tile (Engine::produce_dual), in
+// one accumulator (teacher columns 0..127, student 128..255), so the two
+// accumulators alternate and the epilogue overlaps the next tile's MMAs.
+template <bool FULL, bool KL = false, bool DUAL = false>
 struct GPolicyT {
   using Params = GParams;
   static constexpr int EXTRA_SMEM = 0;
+  static constexpr int TN = (KL && DUAL) ? BN / 2 : BN;  // vocabulary ids per tile
 
   // Whether this launch writes the dense fallback (slab + masks), and
   // whether it runs at all (a repair launch usually has nothing to do).
@@ -539,10 +545,16 @@ struct GPolicyT {
   static __device__ void prefetch(const Params& p) {
     tma_prefetch_map(&p.mapA);
     tma_prefetch_map(&p.mapB);
+    if constexpr (KL) {
+      tma_prefetch_map(&p.mapA2);
+      tma_prefetch_map(DUAL ? &p.mapB128 : &p.mapB2);
+    }
   }
   static __device__ void producer(const Params& p, Engine& eng) {
     schedule(p, [&](int mb, int vt, int) {
       if (skip(p, mb, vt)) return true;
+      if constexpr (KL && DUAL)  // teacher rows, student rows, one head tile
+        return eng.produce_dual(&p.mapA2, &p.mapA, &p.mapB128, mb * BM, p.b_row0 + vt * TN, p.nkb);
       if constexpr (KL) {  // teacher tile first: it lands in the even accumulator
         if (!eng.produce<false, false>(&p.mapA2, &p.mapB2, 0, mb * BM, 0, p.b_row0 + vt * BN,
                                        p.nkb))
@@ -554,6 +566,7 @@ struct GPolicyT {
   static __device__ void mma(const Params& p, Engine& eng) {
     schedule(p, [&](int mb, int vt, int) {
       if (skip(p, mb, vt)) return true;
+      if constexpr (KL && DUAL) return eng.mma_dual(p.nkb);
       if constexpr (KL) {
         if (!eng.mma<false, false>(p.nkb)) return false;
       }
@@ -577,7 +590,10 @@ struct GPolicyT {
       const bool sk = skip(p, mb, vt);
       uint32_t taddr = 0, tteach = 0;
       if (!sk) {
-        if constexpr (KL) {
+        if constexpr (KL && DUAL) {
+          if (!eng.epi_acquire(q, tteach)) return false;
+          taddr = tteach + TN;  // student columns after the teacher's
+        } else if constexpr (KL) {
           if (!eng.epi_acquire2(q, tteach, taddr)) return false;
         } else {
           if (!eng.epi_acquire(q, taddr)) return false;
@@ -588,13 +604,13 @@ struct GPolicyT {
       const float lse2 = ok ? p.lse2_c[jrow] : 0.f;
       const float lt2 = (KL && ok) ? p.lt2_c[jrow] : 0.f;
       const float dl = ok ? p.dloss_c[jrow] : 0.f;
-      const int tcol = (ok && p.tseg[jrow] == p.seg) ? p.tpos[jrow] - p.c0 - vt * BN : -1;
-      const int valid = p.chunk_valid - vt * BN;  // valid columns of this tile
-      __nv_bfloat16* grow = p.G + (size_t)jrow * p.Vc + vt * BN;
-      __nv_bfloat16* frow = FULL ? p.G_full + (size_t)jrow * p.Vc + vt * BN : nullptr;
+      const int tcol = (ok && p.tseg[jrow] == p.seg) ? p.tpos[jrow] - p.c0 - vt * TN : -1;
+      const int valid = p.chunk_valid - vt * TN;  // valid columns of this tile
+      __nv_bfloat16* grow = p.G + (size_t)jrow * p.Vc + vt * TN;
+      __nv_bfloat16* frow = FULL ? p.G_full + (size_t)jrow * p.Vc + vt * TN : nullptr;
       const bool dbg = p.debug_keep != nullptr && ok && p.idx[jrow] < p.debug_rows;
       uint32_t half_nz = 0;  // bit h: this row has a non-zero in tile columns 128h..128h+127
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < TN / 32; ++c) {
         uint32_t r[32];
         uint32_t rt[KL ? 32 : 1];  // teacher log2 softmax (KL)
         // keep bits: softmax part retained (p >= eps, decided in base-2 log
@@ -660,7 +676,7 @@ struct GPolicyT {
             const uint32_t b0 = __ballot_sync(0xffffffffu, (nzb & 0xFFFFu) != 0u);
             const uint32_t b1 = __ballot_sync(0xffffffffu, (nzb >> 16) != 0u);
             if (lane == 0 && (b0 | b1)) {
-              const int g = vt * (BN / 16) + c * 2;
+              const int g = vt * (TN / 16) + c * 2;
               atomicOr(&p.dh_mask[mb * p.dh_words + (g >> 5)],
                        ((b0 ? 1u : 0u) | (b1 ? 2u : 0u)) << (g & 31));
             }
@@ -698,7 +714,7 @@ struct GPolicyT {
                 if (!((nzb >> j) & 1u)) continue;
                 const float v = ((kb >> j) & 1u) ? pval(j) : 0.f;
                 const float g = dl * (v - (((tb >> j) & 1u) ? 1.f : 0.f));
-                if (pos < p.nz_cap) p.nz_list[pos] = NzEntry{jrow, vt * BN + c * 32 + j, g, 0};
+                if (pos < p.nz_cap) p.nz_list[pos] = NzEntry{jrow, vt * TN + c * 32 + j, g, 0};
                 ++pos;
               }
             }
@@ -708,7 +724,7 @@ struct GPolicyT {
           const int orig = p.idx[jrow];
           for (int j = 0; j < 32; ++j) {
             if (!((kb >> j) & 1u)) continue;
-            const int w = p.c0 + vt * BN + c * 32 + j;
+            const int w = p.c0 + vt * TN + c * 32 + j;
             const long long lid = p.seg_begin + (p.perm_seg ? p.perm_seg[w] : w);
             atomicOr(&p.debug_keep[(size_t)orig * p.words_per_row + (lid >> 5)], 1u << (lid & 31));
           }
@@ -717,17 +733,17 @@ struct GPolicyT {
       if (de_bits) {
         // warp vote per 16-row group for the dE contraction's K slices
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < TN / 128; ++h) {
           const uint32_t b = __ballot_sync(0xffffffffu, (half_nz >> h) & 1u);
           if (lane == 0 && b) {
             const int g = mb * (BM / 16) + q * 2;
-            atomicOr(&p.de_mask[(vt * 2 + h) * p.de_words + (g >> 5)],
+            atomicOr(&p.de_mask[(vt * (TN / 128) + h) * p.de_words + (g >> 5)],
                      (((b & 0xFFFFu) ? 1u : 0u) | ((b >> 16) ? 2u : 0u)) << (g & 31));
           }
         }
       }
       if (!sk) {
-        if constexpr (KL)
+        if constexpr (KL && !DUAL)
           eng.epi_release2(lane);
         else
           eng.epi_release(lane);
@@ -740,6 +756,7 @@ struct GPolicyT {
 using GPolicy = GPolicyT<false>;
 using GPolicyFull = GPolicyT<true>;
 using GPolicyKL = GPolicyT<false, true>;
+using GPolicyKLDual = GPolicyT<false, true, true>;
 
 // =====================================================================
 // Backward, step 2: dE_chunk = G^T H_c, K = compact rows, accumulated on
