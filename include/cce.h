@@ -177,6 +177,23 @@ size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs,
                               uint32_t flags);
 
 /*
+ * The same workspace split by what each of its buffers scales with (host
+ * pointers; the three add up to cce_bwd_workspace_size):
+ *   rows    per-row arrays and [N, D] buffers (the compact copy of H, the
+ *           fp32 dH accumulator),
+ *   vocab   per-id arrays and [chunk, D] buffers of E rows,
+ *   logits  buffers that hold parts of the [N, V] product: the bf16 G slab(s)
+ *           of one vocabulary chunk (N x chunk width, the width capped so a
+ *           slab stays below 512 MiB) and the sparse lists of kept entries.
+ * The point of the method ("Cut Your Losses in Large-Vocabulary Language
+ * Models", first page §Contribution: the logits are never written to global
+ * memory in full) is that `logits` stays a small fraction of N x V x 2
+ * bytes.  Returns CCE_OK or CCE_EINVAL.
+ */
+int cce_bwd_workspace_parts(int64_t N, int64_t D, int64_t V, int32_t n_segs, uint32_t flags,
+                            size_t* rows, size_t* vocab, size_t* logits);
+
+/*
  * Backward: gradients of sum_i dloss_i * loss_i.
  *   H, E, y, N, D, V, ignore_index, segs, n_segs  as for cce_fwd.
  *   lse      [N] fp32, the forward's lse output for the same inputs.

@@ -25,7 +25,8 @@ EXPORTS = ("cce_version", "cce_strerror", "cce_fwd_workspace_size", "cce_fwd", "
            "cce_bwd_workspace_size", "cce_bwd", "cce_vocab_sort_workspace_size",
            "cce_vocab_sort", "cce_launch_count", "cce_timing_enable", "cce_timing_read",
            "cce_kl_fwd_workspace_size", "cce_kl_fwd", "cce_kl_bwd_workspace_size", "cce_kl_bwd",
-           "cce_vocab_combine", "cce_fwd_noalloc", "cce_debug_stall")
+           "cce_vocab_combine", "cce_fwd_noalloc", "cce_debug_stall",
+           "cce_bwd_workspace_parts")
 # kernel classes for cce_timing_enable / cce_timing_read
 KC_FWD, KC_G, KC_DE, KC_DH, KC_AUX, KC_SPARSE = 0, 1, 2, 3, 4, 5
 KC_NAMES = ("fwd_tile_stream", "bwd_g_producer", "bwd_dE_contraction", "bwd_dH_contraction", "aux",
@@ -76,6 +77,9 @@ def lib() -> ctypes.CDLL:
                              vp, i64, vp, sz, vp, vp]
     L.cce_bwd_workspace_size.restype = sz
     L.cce_bwd_workspace_size.argtypes = [i64, i64, i64, i32, u32]
+    L.cce_bwd_workspace_parts.restype = ctypes.c_int
+    L.cce_bwd_workspace_parts.argtypes = [i64, i64, i64, i32, u32, ctypes.POINTER(sz),
+                                          ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.cce_bwd.restype = ctypes.c_int
     L.cce_bwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, ctypes.POINTER(Segment), i32,
                           fp, vp, vp, u32, vp, vp, vp, vp, i64, vp, sz, vp, vp]
@@ -137,6 +141,15 @@ def fwd_workspace_size(N: int, D: int, V: int, n_segs: int = 0) -> int:
 
 def bwd_workspace_size(N: int, D: int, V: int, n_segs: int = 0, flags: int = 0) -> int:
     return int(lib().cce_bwd_workspace_size(N, D, V, n_segs, flags))
+
+
+def bwd_workspace_parts(N: int, D: int, V: int, n_segs: int = 0, flags: int = 0):
+    """{"rows", "vocab", "logits"}: the backward workspace by size class
+    (see cce_bwd_workspace_parts)."""
+    r, v, l = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().cce_bwd_workspace_parts(N, D, V, n_segs, flags, ctypes.byref(r), ctypes.byref(v),
+                                         ctypes.byref(l)), "cce_bwd_workspace_parts")
+    return {"rows": r.value, "vocab": v.value, "logits": l.value}
 
 
 def vocab_sort_workspace_size(N: int, V: int, n_segs: int = 0) -> int:

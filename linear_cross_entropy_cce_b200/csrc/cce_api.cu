@@ -27,6 +27,16 @@ constexpr size_t kGBudgetBytes = 64ull << 20;   // preferred bf16 G slab (about 
 constexpr size_t kGCapBytes = 512ull << 20;     // never more than this for the slab
 constexpr int64_t kDeWaves = 4;                 // dE tiles per chunk >= this many waves
 constexpr size_t kAlign = 256;
+// Filtered calls use vocabulary chunks this many times as wide as unfiltered
+// ones (their chunks mostly take the sparse route, which writes no slab).
+#ifndef CCE_FILTERED_WIDTH_MULT
+#define CCE_FILTERED_WIDTH_MULT 2
+#endif
+constexpr int64_t kFilteredWidthMult = CCE_FILTERED_WIDTH_MULT;
+#ifndef CCE_CAP_CHUNK_EIGHTH
+#define CCE_CAP_CHUNK_EIGHTH 0
+#endif
+constexpr bool kCapChunkToEighth = CCE_CAP_CHUNK_EIGHTH != 0;
 
 size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -229,6 +239,8 @@ struct BwdPlan {
   size_t off_nzcnt, off_lists, off_colc, off_csorted, off_rowc, off_rsorted, off_scan, scan_bytes;
   size_t off_tcmax, off_blkmin;  // tile-skip bounds
   size_t off_htc, off_lt2;       // soft-target KL: teacher rows and lse
+  // bytes by the size class of the buffers (see cce_bwd_workspace_parts)
+  size_t part_rows, part_vocab, part_logits;
 };
 
 // Zero-slice mask words for chunk width vc: dH masks (per 128-row block, one
@@ -250,52 +262,71 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = fals
   vc = std::max<int64_t>(vc, cdiv(kDeWaves * kPlanSMs * BM, dt));
   vc = std::min<int64_t>(vc, (int64_t)(kGCapBytes / (2 * (size_t)p.Npad)));
   vc = std::min<int64_t>(16384, vc) / BN * BN;
+  // no chunk's slab may hold a sizeable part of the logits: at most about an
+  // eighth of the vocabulary per chunk (binds only for heads with a small V)
+  const int64_t vc_nv = std::max<int64_t>(BN, (V * 9 / 80) / BN * BN);
+  if (kCapChunkToEighth) vc = std::min(vc, vc_nv);
   p.Vc = std::max<int64_t>(BN, std::min<int64_t>(vc, cdiv(V, BN) * BN));
   // Filtered calls: twice as wide (fewer launches per step and a smaller
   // last-wave tail per launch; their chunks mostly take the sparse route and
   // write no slab), within the slab cap.
-  int64_t vf = std::min<int64_t>(2 * p.Vc, (int64_t)(kGCapBytes / (2 * (size_t)p.Npad)));
+  int64_t vf = std::min<int64_t>(kFilteredWidthMult * p.Vc,
+                                 (int64_t)(kGCapBytes / (2 * (size_t)p.Npad)));
   vf = std::min<int64_t>(16384, vf) / BN * BN;
+  if (kCapChunkToEighth) vf = std::min(vf, vc_nv);
   p.Vc_f = std::max<int64_t>(p.Vc, std::min<int64_t>(vf, cdiv(V, BN) * BN));
   const int64_t Vw = p.Vc_f;  // buffers scaled by the chunk width are sized for the wider one
   const size_t n4 = sizeof(int) * (size_t)std::max<int64_t>(N, 1);
+  // Carve the workspace; every buffer is counted in the class its size
+  // scales with: rows (N, N x D), vocabulary (V, V x D) or the logits (N x V:
+  // the bf16 G slabs of one chunk and the sparse lists of all chunks).
   size_t o = 0;
-  p.off_nvalid = o; o += align_up(16);
-  p.off_idx = o; o += align_up(n4);
-  p.off_pos = o; o += align_up(n4);
-  p.off_lse2 = o; o += align_up(n4);
-  p.off_dl = o; o += align_up(n4);
-  p.off_tseg = o; o += align_up(n4);
-  p.off_tpos = o; o += align_up(n4);
-  p.off_inv = o; o += align_up(sizeof(int) * (size_t)V);
-  p.off_hc = o; o += align_up((size_t)p.Npad * D * 2);
-  p.off_dh = o; o += align_up((size_t)p.Npad * D * 4);
-  p.off_g = o; o += align_up((size_t)p.Npad * Vw * 2);
-  p.off_ec = o; o += 2 * align_up((size_t)Vw * D * 2);  // two buffers: gather k+1 while k runs
+  p.part_rows = p.part_vocab = p.part_logits = 0;
+  auto take = [&](size_t bytes, size_t& cls) {
+    const size_t at = o;
+    o += bytes;
+    cls += bytes;
+    return at;
+  };
+  size_t& R = p.part_rows;
+  size_t& Vb = p.part_vocab;
+  size_t& L = p.part_logits;
+  p.off_nvalid = take(align_up(16), R);
+  p.off_idx = take(align_up(n4), R);
+  p.off_pos = take(align_up(n4), R);
+  p.off_lse2 = take(align_up(n4), R);
+  p.off_dl = take(align_up(n4), R);
+  p.off_tseg = take(align_up(n4), R);
+  p.off_tpos = take(align_up(n4), R);
+  p.off_inv = take(align_up(sizeof(int) * (size_t)V), Vb);
+  p.off_hc = take(align_up((size_t)p.Npad * D * 2), R);
+  p.off_dh = take(align_up((size_t)p.Npad * D * 4), R);
+  p.off_g = take(align_up((size_t)p.Npad * Vw * 2), L);
+  p.off_ec = take(2 * align_up((size_t)Vw * D * 2), Vb);  // two buffers: gather k+1 while k runs
   // CCE_FULL_DE: a second slab with the unfiltered G, read by dE only
-  p.off_gfull = o; o += (flags & CCE_FULL_DE) ? align_up((size_t)p.Npad * Vw * 2) : 0;
+  p.off_gfull = take((flags & CCE_FULL_DE) ? align_up((size_t)p.Npad * Vw * 2) : 0, L);
   p.de_words = (int)cdiv(p.Npad, 512);
   p.mask_bytes = mask_bytes_for(p.Npad, Vw);
   // two mask buffers: chunk c uses buffer c % 2 and its G launch clears the other
-  p.off_masks = o; o += 2 * align_up(p.mask_bytes);
+  p.off_masks = take(2 * align_up(p.mask_bytes), L);
   // sparse path: per chunk a list of up to cap(Vc) non-zeros (density 1/2048);
   // chunk count from the narrower width, list slots for whichever needs more
   p.nch_max = cdiv(V, p.Vc) + CCE_MAX_SEGMENTS;
   const int64_t slots = std::max(p.nch_max * list_cap(p.Npad, p.Vc),
                                  (cdiv(V, p.Vc_f) + CCE_MAX_SEGMENTS) * list_cap(p.Npad, p.Vc_f));
-  p.off_nzcnt = o; o += align_up(sizeof(int) * 2 * (size_t)p.nch_max);  // counts + slab flags
-  p.off_lists = o; o += align_up(sizeof(NzEntry) * (size_t)slots);
-  p.off_colc = o; o += align_up(sizeof(int) * 2 * (size_t)(V + 1));  // counts, offsets
-  p.off_csorted = o; o += align_up(sizeof(int2) * (size_t)slots);
-  p.off_rowc = o; o += align_up(sizeof(int) * 2 * (size_t)(p.Npad + 1));
-  p.off_rsorted = o; o += align_up(sizeof(int2) * (size_t)slots);
+  p.off_nzcnt = take(align_up(sizeof(int) * 2 * (size_t)p.nch_max), Vb);  // counts + slab flags
+  p.off_lists = take(align_up(sizeof(NzEntry) * (size_t)slots), L);
+  p.off_colc = take(align_up(sizeof(int) * 2 * (size_t)(V + 1)), Vb);  // counts, offsets
+  p.off_csorted = take(align_up(sizeof(int2) * (size_t)slots), L);
+  p.off_rowc = take(align_up(sizeof(int) * 2 * (size_t)(p.Npad + 1)), R);
+  p.off_rsorted = take(align_up(sizeof(int2) * (size_t)slots), L);
   // generous bound on cub's single-pass scan scratch (checked again at run time)
   p.scan_bytes = align_up(sizeof(int) * (size_t)(std::max<int64_t>(V, p.Npad) + 1) / 8 + (1u << 20));
-  p.off_scan = o; o += p.scan_bytes;
-  p.off_tcmax = o; o += align_up(sizeof(float) * (size_t)(cdiv(V, BN) + CCE_MAX_SEGMENTS));
-  p.off_blkmin = o; o += align_up(sizeof(float) * (size_t)(p.Npad / BM));
-  p.off_htc = o; o += kl ? align_up((size_t)p.Npad * D * 2) : 0;
-  p.off_lt2 = o; o += kl ? align_up(sizeof(float) * (size_t)std::max<int64_t>(N, 1)) : 0;
+  p.off_scan = take(p.scan_bytes, Vb);
+  p.off_tcmax = take(align_up(sizeof(float) * (size_t)(cdiv(V, BN) + CCE_MAX_SEGMENTS)), Vb);
+  p.off_blkmin = take(align_up(sizeof(float) * (size_t)(p.Npad / BM)), R);
+  p.off_htc = take(kl ? align_up((size_t)p.Npad * D * 2) : 0, R);
+  p.off_lt2 = take(kl ? align_up(sizeof(float) * (size_t)std::max<int64_t>(N, 1)) : 0, R);
   p.total = o;
   return p;
 }
@@ -478,6 +509,17 @@ size_t cce_fwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs) {
 size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs, uint32_t flags) {
   if (!sizes_ok(N, D, V) || n_segs < 0 || n_segs > CCE_MAX_SEGMENTS) return 0;
   return plan_bwd(N, D, V, flags).total;
+}
+
+int cce_bwd_workspace_parts(int64_t N, int64_t D, int64_t V, int32_t n_segs, uint32_t flags,
+                            size_t* rows, size_t* vocab, size_t* logits) {
+  if (!sizes_ok(N, D, V) || n_segs < 0 || n_segs > CCE_MAX_SEGMENTS || !rows || !vocab || !logits)
+    return CCE_EINVAL;
+  const BwdPlan p = plan_bwd(N, D, V, flags);
+  *rows = p.part_rows;
+  *vocab = p.part_vocab;
+  *logits = p.part_logits;
+  return CCE_OK;
 }
 
 }  // extern "C"

@@ -156,13 +156,22 @@ def run(request):
 
 
 def test_no_logit_sized_buffer(run):
-    """Nothing of the size class of the [N, V] logits is allocated: each
-    workspace stays below N V 2 / 8 bytes (an eighth of bf16 logits), and the
-    step's peak allocation is its workspaces plus its outputs (so no hidden
-    allocation exists either)."""
+    """Nothing of the size class of the [N, V] logits is allocated: the
+    buffers of the backward's workspace that hold parts of the product (the
+    G slab of one vocabulary chunk and the sparse lists,
+    cce_bwd_workspace_parts "logits") stay below N V 2 / 8 bytes, an eighth
+    of the bf16 logits; the rest of the scratch scales with the inputs (N x D
+    rows, chunk x D rows of E), and the step's peak allocation is its
+    workspaces plus its outputs (so no hidden allocation exists either)."""
+    from linear_cross_entropy_cce_b200 import cce
     x = run["x"]
-    bound = x.wl.N * x.wl.V * 2 / 8
-    assert max(run["ws"]) < bound, (run["ws"], bound)
+    wl = x.wl
+    bound = wl.N * wl.V * 2 / 8
+    nseg = 0 if len(wl.segs()) == 1 else len(wl.segs())
+    parts = cce.bwd_workspace_parts(wl.N, wl.D, wl.V, nseg, 0)  # Kahan needs no more scratch
+    assert sum(parts.values()) == run["ws"][1]
+    assert parts["logits"] < bound, (parts, bound)
+    assert run["ws"][0] < bound and run["ws"][2] < bound  # forward and sort scratch
     slack = 8 << 20  # allocator rounding and a few small tensors (dloss, status)
     assert run["peak"] <= sum(run["ws"]) + run["outputs"] + slack, (run["peak"], run["ws"],
                                                                      run["outputs"])
