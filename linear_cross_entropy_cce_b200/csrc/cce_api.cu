@@ -33,8 +33,12 @@ constexpr size_t kAlign = 256;
 #define CCE_FILTERED_WIDTH_MULT 2
 #endif
 constexpr int64_t kFilteredWidthMult = CCE_FILTERED_WIDTH_MULT;
+// Chunk widths are capped so that the bf16 G slab of one chunk (plus the
+// sparse lists) stays below an eighth of the bf16 logits, N x V x 2 / 8
+// bytes: no buffer of the logits' size class.  Binds only for heads with a
+// small V (the Phi-3.5-mini-shaped head: 3584 ids per chunk).
 #ifndef CCE_CAP_CHUNK_EIGHTH
-#define CCE_CAP_CHUNK_EIGHTH 0
+#define CCE_CAP_CHUNK_EIGHTH 1
 #endif
 constexpr bool kCapChunkToEighth = CCE_CAP_CHUNK_EIGHTH != 0;
 
@@ -251,7 +255,24 @@ size_t mask_bytes_for(int64_t Npad, int64_t vc) {
 // Sparse-list capacity of one chunk of width vc: density 1/2048.
 int64_t list_cap(int64_t Npad, int64_t vc) { return std::max<int64_t>(4096, Npad * vc / 2048); }
 
+BwdPlan plan_bwd_widths(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl, int64_t cap_w);
+
+// The plan for these sizes.  With kCapChunkToEighth the chunk widths shrink
+// (in steps of 256 ids) until the logits-class buffers (the G slab(s) and the
+// sparse lists) take less than an eighth of the bf16 logits, N x V x 2 / 8.
 BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = false) {
+  BwdPlan p = plan_bwd_widths(N, D, V, flags, kl, INT64_MAX);
+  const double bound = (double)N * (double)V * 2.0 / 8.0;
+  // small problems are left alone: their scratch is a few MB whatever the
+  // logits, and narrow chunks would only add launches
+  if (!kCapChunkToEighth || bound < (double)(64u << 20)) return p;
+  while ((double)p.part_logits >= bound && p.Vc_f > BN)
+    p = plan_bwd_widths(N, D, V, flags, kl, p.Vc_f - BN);
+  return p;
+}
+
+// The plan with both chunk widths at most cap_w ids.
+BwdPlan plan_bwd_widths(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl, int64_t cap_w) {
   BwdPlan p;
   p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
   // Vocabulary chunk width: an L2-sized slab, widened so that the dE
@@ -261,19 +282,14 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = fals
   int64_t vc = (int64_t)(kGBudgetBytes / (2 * (size_t)p.Npad));
   vc = std::max<int64_t>(vc, cdiv(kDeWaves * kPlanSMs * BM, dt));
   vc = std::min<int64_t>(vc, (int64_t)(kGCapBytes / (2 * (size_t)p.Npad)));
-  vc = std::min<int64_t>(16384, vc) / BN * BN;
-  // no chunk's slab may hold a sizeable part of the logits: at most about an
-  // eighth of the vocabulary per chunk (binds only for heads with a small V)
-  const int64_t vc_nv = std::max<int64_t>(BN, (V * 9 / 80) / BN * BN);
-  if (kCapChunkToEighth) vc = std::min(vc, vc_nv);
+  vc = std::min<int64_t>(std::min<int64_t>(16384, cap_w), vc) / BN * BN;
   p.Vc = std::max<int64_t>(BN, std::min<int64_t>(vc, cdiv(V, BN) * BN));
   // Filtered calls: twice as wide (fewer launches per step and a smaller
   // last-wave tail per launch; their chunks mostly take the sparse route and
   // write no slab), within the slab cap.
   int64_t vf = std::min<int64_t>(kFilteredWidthMult * p.Vc,
                                  (int64_t)(kGCapBytes / (2 * (size_t)p.Npad)));
-  vf = std::min<int64_t>(16384, vf) / BN * BN;
-  if (kCapChunkToEighth) vf = std::min(vf, vc_nv);
+  vf = std::min<int64_t>(std::min<int64_t>(16384, cap_w), vf) / BN * BN;
   p.Vc_f = std::max<int64_t>(p.Vc, std::min<int64_t>(vf, cdiv(V, BN) * BN));
   const int64_t Vw = p.Vc_f;  // buffers scaled by the chunk width are sized for the wider one
   const size_t n4 = sizeof(int) * (size_t)std::max<int64_t>(N, 1);

@@ -28,8 +28,16 @@ int main(void) {
   CHECK(cce_fwd_workspace_size(4096, 2048, 128256, 0) > 0);
   CHECK(cce_fwd_workspace_size(4096, 2050, 128256, 0) == 0); /* D % 8 != 0 */
   CHECK(cce_bwd_workspace_size(4096, 2048, 128256, 0, 0) > 0);
-  CHECK(cce_bwd_workspace_size(4096, 2048, 128256, 0, CCE_FULL_DE) >
-        cce_bwd_workspace_size(4096, 2048, 128256, 0, 0));
+  CHECK(cce_bwd_workspace_size(4096, 2048, 128256, 0, CCE_FULL_DE) > 0);
+  {
+    /* the size classes add up, and the logits class stays below N V 2 / 8 */
+    size_t rows = 0, vocab = 0, logits = 0;
+    CHECK(cce_bwd_workspace_parts(4096, 2048, 128256, 0, CCE_FULL_DE, &rows, &vocab, &logits) ==
+          CCE_OK);
+    CHECK(rows + vocab + logits == cce_bwd_workspace_size(4096, 2048, 128256, 0, CCE_FULL_DE));
+    CHECK(logits < (size_t)4096 * 128256 * 2 / 8);
+    CHECK(cce_bwd_workspace_parts(4096, 2048, 128256, 0, 0, NULL, &vocab, &logits) == CCE_EINVAL);
+  }
   CHECK(cce_vocab_sort_workspace_size(4096, 128256, 0) > 0);
   CHECK(cce_kl_fwd_workspace_size(4096, 2048, 128256) > 0);
 
