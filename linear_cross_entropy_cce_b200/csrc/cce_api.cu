@@ -977,12 +977,24 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       ep.mwords = pl.de_words;
       ep.n_valid = cp.n_valid;
       ep.status = status;
-      if (int rc = kPairDEDH
-                       ? launch_tc_pair<DEPairPolicy>(
-                             ep, (int)std::min<int64_t>(sms / 2, (int64_t)ep.mt * dt), st, KC_DE)
-                       : launch_tc<DEPolicy>(ep, (int)std::min<int64_t>(sms, (int64_t)ep.mt * dt),
-                                             st, KC_DE))
-        return rc;
+      int de_rc;
+      if (kPairDEDH) {
+        // 256 x 128 pair tiles when they fill the SM pairs' waves better
+        // than 256 x 256 ones (narrow chunks, e.g. a small vocabulary)
+        const int pairs = sms / 2;
+        const int64_t t256 = (int64_t)ep.mt * dt, t128 = (int64_t)ep.mt * cdiv(D, BN / 2);
+        auto wave_eff = [&](int64_t t) { return (double)t / (double)(cdiv(t, pairs) * pairs); };
+        const bool narrow = wave_eff(t128) > wave_eff(t256) + 0.05;
+        ep.dt = narrow ? (int)cdiv(D, BN / 2) : dt;
+        const int64_t tiles = narrow ? t128 : t256;
+        de_rc = narrow ? launch_tc_pair<DEPairNarrowPolicy>(
+                             ep, (int)std::min<int64_t>(pairs, tiles), st, KC_DE)
+                       : launch_tc_pair<DEPairPolicy>(ep, (int)std::min<int64_t>(pairs, tiles), st,
+                                                      KC_DE);
+      } else {
+        de_rc = launch_tc<DEPolicy>(ep, (int)std::min<int64_t>(sms, (int64_t)ep.mt * dt), st, KC_DE);
+      }
+      if (de_rc) return de_rc;
       // step 3: dH += G E_chunk
       hp.mapB = segMN;
       hp.b_row0 = row0;

@@ -517,10 +517,14 @@ struct PairEngine {
   // are skipped by both; each loaded stage carries a record for the MMA
   // thread (its K steps, REC_LAST on the tile's last stage), written and
   // announced by the rank-0 producer once the next loaded stage is known.
-  template <bool A_MN, bool B_MN>
+  // NT: the pair tile's columns (256, or 128 for narrow problems): each CTA
+  // stages NT / 2 of them.
+  template <bool A_MN, bool B_MN, int NT = BN>
   __device__ __forceinline__ bool produce_rec(const CUtensorMap* mA, const CUtensorMap* mB, int ax,
                                               int ay, int bx, int by, int nkb, const uint32_t* m0,
                                               const uint32_t* m1) {
+    static_assert(NT == BN || (NT == BN / 2 && B_MN), "128-column pair tiles need an MN-major B");
+    constexpr uint32_t tx = 2u * (PA_BYTES + (NT / 2) * BK * 2);
     MaskPair mc;
     mc.init(m0, m1, nkb);
     int pend = -1;
@@ -530,7 +534,7 @@ struct PairEngine {
       if (!bits) continue;
       if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
       const uint32_t fb_local = smem_u32(&ctl->full[pipe.stage]);
-      if (rank == 0) mbar_expect_tx(fb_local, 2 * PSTAGE_BYTES);
+      if (rank == 0) mbar_expect_tx(fb_local, tx);
       const uint32_t fb = in_cta(&ctl->full[pipe.stage], 0);
       const uint32_t sa = smem_u32(smem + pipe.stage * PSTAGE_BYTES);
       const uint32_t sb = sa + PA_BYTES;
@@ -544,7 +548,7 @@ struct PairEngine {
         tma_load_2d_pair(sb, mB, fb, bx + kb * BK, by);
       } else {
         tma_load_2d_pair(sb, mB, fb, bx, by + kb * BK);
-        tma_load_2d_pair(sb + 8192, mB, fb, bx + 64, by + kb * BK);
+        if (NT == BN) tma_load_2d_pair(sb + 8192, mB, fb, bx + 64, by + kb * BK);
       }
       if (rank == 0 && pend >= 0) {
         ctl->rec[pend] = pend_bits;
@@ -572,13 +576,13 @@ struct PairEngine {
   // ---- MMA issuer (rank 0 only, one thread): consumes the records until
   // REC_LAST; each stage is released to both CTAs' producers by a commit to
   // each CTA's empty barrier, the tile's accumulator to both epilogues.
-  template <bool A_MN, bool B_MN>
+  template <bool A_MN, bool B_MN, int NT = BN>
   __device__ __forceinline__ bool mma_rec() {
     const int acc = tcount & 1;
     if (!wait(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u)) return false;
     tc_fence_after();
     const uint32_t d = tmem + acc * BN;
-    constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
+    constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, NT, A_MN, B_MN);
     constexpr uint32_t a_step = A_MN ? 2048 : 32;  // bytes per K=16 step
     constexpr uint32_t b_step = B_MN ? 2048 : 32;
     const uint64_t ad0 = A_MN ? smem_desc_sw128(smem_u32(smem), 8192, 1024)

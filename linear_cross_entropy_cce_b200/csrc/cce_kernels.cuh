@@ -793,9 +793,10 @@ __device__ __forceinline__ bool mask_empty(const uint32_t* m, int nkb, int lane)
 }
 
 // One CTA per 128 x 256 tile of dE (PAIR = false) or one CTA pair per
-// 256 x 256 tile (PAIR = true, tcgen05 cta_group::2; the host sets mt to the
-// number of 128- or 256-row vocabulary tiles accordingly).
-template <bool PAIR>
+// 256 x NT tile (PAIR = true, tcgen05 cta_group::2; NT = 256, or 128 when a
+// narrow chunk would leave the SMs few 256-column tiles; the host sets mt and
+// dt to the number of vocabulary and D tiles accordingly).
+template <bool PAIR, int NT = BN>
 struct DEPolicyT {
   using Params = DEParams;
   static constexpr int EXTRA_SMEM = 0;
@@ -831,10 +832,9 @@ struct DEPolicyT {
   static __device__ void producer(const Params& p, Eng& eng) {
     schedule(p, [&](int vt, int dtile, int nkb) {
       if constexpr (PAIR) {
-        const int r = (int)eng.rank * BM;
-        return eng.template produce_rec<true, true>(&p.mapA, &p.mapB, vt * ROWS + r, 0,
-                                                    dtile * BN + r, 0, nkb, mask_lo(p, vt),
-                                                    mask_hi(p, vt));
+        return eng.template produce_rec<true, true, NT>(
+            &p.mapA, &p.mapB, vt * ROWS + (int)eng.rank * BM, 0, dtile * NT + (int)eng.rank * (NT / 2),
+            0, nkb, mask_lo(p, vt), mask_hi(p, vt));
       } else {
         return eng.template produce_rec<true, true>(&p.mapA, &p.mapB, vt * BM, 0, dtile * BN, 0,
                                                     nkb, mask_lo(p, vt));
@@ -843,7 +843,12 @@ struct DEPolicyT {
   }
   template <class Eng>
   static __device__ void mma(const Params& p, Eng& eng) {
-    schedule(p, [&](int, int, int nkb) { return nkb == 0 || eng.template mma_rec<true, true>(); });
+    schedule(p, [&](int, int, int nkb) {
+      if constexpr (PAIR)
+        return nkb == 0 || eng.template mma_rec<true, true, NT>();
+      else
+        return nkb == 0 || eng.template mma_rec<true, true>();
+    });
   }
   template <class Eng>
   static __device__ void epilogue(const Params& p, Eng& eng, int q, int lane) {
@@ -859,8 +864,8 @@ struct DEPolicyT {
       const bool ok = r < p.chunk_valid;
       const int w = p.c0 + r;
       const size_t local = ok ? (size_t)(p.perm_seg ? p.perm_seg[w] : w) : 0;
-      for (int c = 0; c < BN / 32; ++c) {
-        const int col0 = dtile * BN + c * 32;
+      for (int c = 0; c < NT / 32; ++c) {
+        const int col0 = dtile * NT + c * 32;
         if (col0 >= p.D) break;
         uint32_t v[32];
         if (!zero) {
@@ -917,6 +922,7 @@ struct DEPolicyT {
 };
 using DEPolicy = DEPolicyT<false>;
 using DEPairPolicy = DEPolicyT<true>;
+using DEPairNarrowPolicy = DEPolicyT<true, BN / 2>;
 
 // =====================================================================
 // Backward, step 3: dH_acc[j, :] += G[j, chunk] E_chunk, K = chunk.
