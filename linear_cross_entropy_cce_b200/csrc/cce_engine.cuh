@@ -139,6 +139,20 @@ __device__ __forceinline__ void grouped_item(int item, int num_mb, int n_inner, 
   }
 }
 
+// Index of the last stage of a K-step mask (see MaskCursor) with any step to
+// issue, among stages 0 .. nkb-1; -1 if none; nkb - 1 for a null mask.
+__device__ __forceinline__ int mask_last_stage(const uint32_t* m, int nkb) {
+  if (!m) return nkb - 1;
+  const int nwords = (nkb + 7) >> 3;
+  for (int w = nwords - 1; w >= 0; --w) {
+    uint32_t v = __ldg(m + w);
+    const int stages = min(8, nkb - w * 8);
+    if (stages < 8) v &= (1u << (stages * 4)) - 1u;
+    if (v) return w * 8 + ((31 - __clz(v)) >> 2);
+  }
+  return -1;
+}
+
 // Per-role state handed to policies.
 struct Engine {
   Ctl* ctl;
@@ -239,25 +253,32 @@ struct Engine {
 
   // ---- masked producer (lane 0): like produce() with a K-step mask, but the
   // MMA issuer never reads the mask: each loaded stage carries a record (its
-  // non-zero K steps, and REC_LAST on the tile's last loaded stage).  A stage
-  // is announced (record + arrive) only once the next non-zero stage is found
-  // or the tile ends, so REC_LAST is known; a tile with no non-zero stage
-  // still sends one empty REC_LAST stage.
+  // non-zero K steps, and REC_LAST on the tile's last loaded stage, found by
+  // scanning the mask first), written before the stage is announced.  A tile
+  // with no non-zero stage still sends one empty REC_LAST stage.
   template <bool A_MN, bool B_MN>
   __device__ __forceinline__ bool produce_rec(const CUtensorMap* mA, const CUtensorMap* mB, int ax,
                                               int ay, int bx, int by, int nkb,
                                               const uint32_t* kmask) {
+    const int last = mask_last_stage(kmask, nkb);
+    if (last < 0) {  // nothing to load: one empty stage ends the tile
+      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
+      ctl->rec[pipe.stage] = REC_LAST;
+      mbar_arrive(smem_u32(&ctl->full[pipe.stage]));
+      pipe.advance();
+      ++fills;
+      return true;
+    }
     MaskCursor mc;
     mc.init(kmask, nkb);
-    int pend = -1;         // stage announced last (awaiting its record)
-    uint32_t pend_bits = 0;
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int kb = 0; kb <= last; ++kb) {
       const uint32_t bits = mc.bits(kb);
       if (!bits) continue;
       if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u))
         return false;
       const uint32_t fb = smem_u32(&ctl->full[pipe.stage]);
-      mbar_expect_tx(fb, STAGE_BYTES);
+      ctl->rec[pipe.stage] = bits | (kb == last ? REC_LAST : 0u);
+      mbar_arrive_expect_tx(fb, STAGE_BYTES);
       const uint32_t sa = smem_u32(smem + pipe.stage * STAGE_BYTES);
       const uint32_t sb = sa + A_BYTES;
       if (!A_MN) {
@@ -272,25 +293,9 @@ struct Engine {
 #pragma unroll
         for (int b = 0; b < 4; ++b) tma_load_2d(sb + b * 8192, mB, fb, bx + b * 64, by + kb * BK);
       }
-      if (pend >= 0) {  // the previous stage was not the last one
-        ctl->rec[pend] = pend_bits;
-        mbar_arrive(smem_u32(&ctl->full[pend]));
-      }
-      pend = pipe.stage;
-      pend_bits = bits;
       pipe.advance();
       ++fills;
     }
-    if (pend < 0) {  // nothing to load: one empty stage ends the tile
-      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u))
-        return false;
-      pend = pipe.stage;
-      pend_bits = 0;
-      pipe.advance();
-      ++fills;
-    }
-    ctl->rec[pend] = pend_bits | REC_LAST;
-    mbar_arrive(smem_u32(&ctl->full[pend]));
     return true;
   }
 
@@ -515,8 +520,9 @@ struct PairEngine {
   // CTA's A rows and B columns; K advances along x for a K-major operand, y
   // for an MN-major one.  Stages whose K steps are zero in both CTAs' masks
   // are skipped by both; each loaded stage carries a record for the MMA
-  // thread (its K steps, REC_LAST on the tile's last stage), written and
-  // announced by the rank-0 producer once the next loaded stage is known.
+  // thread (its K steps, REC_LAST on the tile's last stage, found by scanning
+  // both masks first), written by the rank-0 producer before it announces
+  // the stage with the bytes of both CTAs' copies.
   // NT: the pair tile's columns (256, or 128 for narrow problems): each CTA
   // stages NT / 2 of them.
   template <bool A_MN, bool B_MN, int NT = BN>
@@ -525,16 +531,29 @@ struct PairEngine {
                                               const uint32_t* m1) {
     static_assert(NT == BN || (NT == BN / 2 && B_MN), "128-column pair tiles need an MN-major B");
     constexpr uint32_t tx = 2u * (PA_BYTES + (NT / 2) * BK * 2);
+    const int last = (m0 == nullptr || m1 == nullptr)
+                         ? nkb - 1
+                         : max(mask_last_stage(m0, nkb), mask_last_stage(m1, nkb));
+    if (last < 0) {  // nothing to load: one empty stage ends the tile (both CTAs keep step)
+      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
+      if (rank == 0) {
+        ctl->rec[pipe.stage] = REC_LAST;
+        mbar_arrive(smem_u32(&ctl->full[pipe.stage]));
+      }
+      pipe.advance();
+      ++fills;
+      return true;
+    }
     MaskPair mc;
     mc.init(m0, m1, nkb);
-    int pend = -1;
-    uint32_t pend_bits = 0;
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int kb = 0; kb <= last; ++kb) {
       const uint32_t bits = mc.bits(kb);
       if (!bits) continue;
       if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
-      const uint32_t fb_local = smem_u32(&ctl->full[pipe.stage]);
-      if (rank == 0) mbar_expect_tx(fb_local, tx);
+      if (rank == 0) {
+        ctl->rec[pipe.stage] = bits | (kb == last ? REC_LAST : 0u);
+        mbar_arrive_expect_tx(smem_u32(&ctl->full[pipe.stage]), tx);
+      }
       const uint32_t fb = in_cta(&ctl->full[pipe.stage], 0);
       const uint32_t sa = smem_u32(smem + pipe.stage * PSTAGE_BYTES);
       const uint32_t sb = sa + PA_BYTES;
@@ -550,25 +569,8 @@ struct PairEngine {
         tma_load_2d_pair(sb, mB, fb, bx, by + kb * BK);
         if (NT == BN) tma_load_2d_pair(sb + 8192, mB, fb, bx + 64, by + kb * BK);
       }
-      if (rank == 0 && pend >= 0) {
-        ctl->rec[pend] = pend_bits;
-        mbar_arrive(smem_u32(&ctl->full[pend]));
-      }
-      pend = pipe.stage;
-      pend_bits = bits;
       pipe.advance();
       ++fills;
-    }
-    if (pend < 0) {  // nothing to load: one empty stage ends the tile (both CTAs keep step)
-      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
-      pend = pipe.stage;
-      pend_bits = 0;
-      pipe.advance();
-      ++fills;
-    }
-    if (rank == 0) {
-      ctl->rec[pend] = pend_bits | REC_LAST;
-      mbar_arrive(smem_u32(&ctl->full[pend]));
     }
     return true;
   }
