@@ -274,13 +274,23 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    vocab = a.parallel == "vocab"
     if world > 1:
         from datetime import timedelta
         # the bound on ranks waiting for one another; generous because every
         # rank first draws its inputs on the shared host cores
         dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
-
-    vocab = a.parallel == "vocab"
+    elif vocab:
+        # the vocabulary-parallel step runs its exchanges over a process
+        # group; a single GPU gets a group of one
+        import socket
+        from datetime import timedelta
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+        sk.close()
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, timeout=timedelta(seconds=120), device_id=dev)
     # vocabulary parallel: one batch shared by all ranks, each holding the E
     # rows of its vocabulary range; data parallel: one batch per rank
     x = syn.make_inputs(wl, seed=0 if vocab else rank)
@@ -505,6 +515,7 @@ def main():
         print(json.dumps(out), flush=True)
     if world > 1:
         dist.barrier()
+    if dist.is_initialized():
         dist.destroy_process_group()
 
 

@@ -255,24 +255,51 @@ size_t mask_bytes_for(int64_t Npad, int64_t vc) {
 // Sparse-list capacity of one chunk of width vc: density 1/2048.
 int64_t list_cap(int64_t Npad, int64_t vc) { return std::max<int64_t>(4096, Npad * vc / 2048); }
 
-BwdPlan plan_bwd_widths(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl, int64_t cap_w);
+BwdPlan plan_bwd_widths(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl, int64_t cap_u,
+                        int64_t cap_f);
+
+// Among chunk widths w in [lo, hi] (multiples of 256), the one that needs the
+// fewest rounds of dE tiles over the whole vocabulary: chunks(w) x waves of
+// one chunk's tiles (`rows` vocabulary rows per tile, `slots` tiles at once);
+// the widest on ties.  Narrowing a chunk below the cap can save a nearly
+// empty last wave in every chunk.
+int64_t best_dE_width(int64_t V, int64_t D, int64_t lo, int64_t hi, int rows, int slots) {
+  int64_t best = hi, best_cost = INT64_MAX;
+  for (int64_t w = hi; w >= std::max<int64_t>(BN, lo); w -= BN) {
+    const int64_t tiles = cdiv(w, rows) * cdiv(D, BN);
+    const int64_t cost = cdiv(V, w) * cdiv(tiles, slots);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = w;
+    }
+  }
+  return best;
+}
 
 // The plan for these sizes.  With kCapChunkToEighth the chunk widths shrink
 // (in steps of 256 ids) until the logits-class buffers (the G slab(s) and the
-// sparse lists) take less than an eighth of the bf16 logits, N x V x 2 / 8.
+// sparse lists) take less than an eighth of the bf16 logits, N x V x 2 / 8,
+// and are then trimmed to the width below that cap whose dE contraction
+// wastes the least of its last waves.
 BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = false) {
-  BwdPlan p = plan_bwd_widths(N, D, V, flags, kl, INT64_MAX);
+  BwdPlan p = plan_bwd_widths(N, D, V, flags, kl, INT64_MAX, INT64_MAX);
   const double bound = (double)N * (double)V * 2.0 / 8.0;
   // small problems are left alone: their scratch is a few MB whatever the
   // logits, and narrow chunks would only add launches
   if (!kCapChunkToEighth || bound < (double)(64u << 20)) return p;
+  if ((double)p.part_logits < bound) return p;
   while ((double)p.part_logits >= bound && p.Vc_f > BN)
-    p = plan_bwd_widths(N, D, V, flags, kl, p.Vc_f - BN);
-  return p;
+    p = plan_bwd_widths(N, D, V, flags, kl, p.Vc_f - BN, p.Vc_f - BN);
+  // unfiltered calls run the dE contraction on CTA pairs (256-row tiles,
+  // kPlanSMs / 2 at once), filtered ones on single CTAs (128-row tiles)
+  const int64_t wu = best_dE_width(V, D, p.Vc / 2, p.Vc, 2 * BM, kPlanSMs / 2);
+  const int64_t wf = best_dE_width(V, D, p.Vc_f / 2, p.Vc_f, BM, kPlanSMs);
+  return plan_bwd_widths(N, D, V, flags, kl, wu, wf);
 }
 
-// The plan with both chunk widths at most cap_w ids.
-BwdPlan plan_bwd_widths(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl, int64_t cap_w) {
+// The plan with the unfiltered / filtered chunk widths at most cap_u / cap_f.
+BwdPlan plan_bwd_widths(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl, int64_t cap_u,
+                        int64_t cap_f) {
   BwdPlan p;
   p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
   // Vocabulary chunk width: an L2-sized slab, widened so that the dE
@@ -282,14 +309,14 @@ BwdPlan plan_bwd_widths(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl
   int64_t vc = (int64_t)(kGBudgetBytes / (2 * (size_t)p.Npad));
   vc = std::max<int64_t>(vc, cdiv(kDeWaves * kPlanSMs * BM, dt));
   vc = std::min<int64_t>(vc, (int64_t)(kGCapBytes / (2 * (size_t)p.Npad)));
-  vc = std::min<int64_t>(std::min<int64_t>(16384, cap_w), vc) / BN * BN;
+  vc = std::min<int64_t>(std::min<int64_t>(16384, cap_u), vc) / BN * BN;
   p.Vc = std::max<int64_t>(BN, std::min<int64_t>(vc, cdiv(V, BN) * BN));
   // Filtered calls: twice as wide (fewer launches per step and a smaller
   // last-wave tail per launch; their chunks mostly take the sparse route and
   // write no slab), within the slab cap.
   int64_t vf = std::min<int64_t>(kFilteredWidthMult * p.Vc,
                                  (int64_t)(kGCapBytes / (2 * (size_t)p.Npad)));
-  vf = std::min<int64_t>(std::min<int64_t>(16384, cap_w), vf) / BN * BN;
+  vf = std::min<int64_t>(std::min<int64_t>(16384, cap_f), vf) / BN * BN;
   p.Vc_f = std::max<int64_t>(p.Vc, std::min<int64_t>(vf, cdiv(V, BN) * BN));
   const int64_t Vw = p.Vc_f;  // buffers scaled by the chunk width are sized for the wider one
   const size_t n4 = sizeof(int) * (size_t)std::max<int64_t>(N, 1);
@@ -424,8 +451,11 @@ int launch_tc_pair(const typename Policy::Params& prm, int pairs, cudaStream_t s
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? CCE_OK : CCE_ELAUNCH;
 }
 
-// The dE / dH contractions of dense chunks run on CTA pairs (256 x 256 tiles,
-// tcgen05 cta_group::2) unless built with CCE_PAIR_DEDH=0.
+// The dE / dH contractions of unfiltered calls run on CTA pairs (256 x 256
+// tiles, tcgen05 cta_group::2) unless built with CCE_PAIR_DEDH=0.  Filtered
+// calls keep single-CTA tiles: their K steps are skipped when a 16-wide slice
+// of G is zero across the tile's rows (or columns), which happens less often
+// over 256 of them than over 128.
 #ifndef CCE_PAIR_DEDH
 #define CCE_PAIR_DEDH 1
 #endif
@@ -757,6 +787,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   __nv_bfloat16* Ec = at<__nv_bfloat16>(workspace, pl.off_ec);
   // chunk width of this call: wider when filtering can take the sparse route
   const bool wide = filter_eps > 0.f && !kahan;
+  const bool pair_dedh = kPairDEDH && filter_eps <= 0.f;
   const int Vc = (int)(wide ? pl.Vc_f : pl.Vc);
   const int dh_words = (int)cdiv(Vc, 512);
   const int dt = (int)cdiv(D, BN);
@@ -965,7 +996,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       ep.nz_cnt = sparse_de ? nz_cnt + chunk : nullptr;
       ep.nz_cap = cap;
       ep.chunk_valid = cv;
-      ep.mt = (int)cdiv(cv, kPairDEDH ? 2 * BM : BM);
+      ep.mt = (int)cdiv(cv, pair_dedh ? 2 * BM : BM);
       ep.dt = dt;
       ep.D = (int)D;
       ep.c0 = c0;
@@ -978,19 +1009,9 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       ep.n_valid = cp.n_valid;
       ep.status = status;
       int de_rc;
-      if (kPairDEDH) {
-        // 256 x 128 pair tiles when they fill the SM pairs' waves better
-        // than 256 x 256 ones (narrow chunks, e.g. a small vocabulary)
-        const int pairs = sms / 2;
-        const int64_t t256 = (int64_t)ep.mt * dt, t128 = (int64_t)ep.mt * cdiv(D, BN / 2);
-        auto wave_eff = [&](int64_t t) { return (double)t / (double)(cdiv(t, pairs) * pairs); };
-        const bool narrow = wave_eff(t128) > wave_eff(t256) + 0.05;
-        ep.dt = narrow ? (int)cdiv(D, BN / 2) : dt;
-        const int64_t tiles = narrow ? t128 : t256;
-        de_rc = narrow ? launch_tc_pair<DEPairNarrowPolicy>(
-                             ep, (int)std::min<int64_t>(pairs, tiles), st, KC_DE)
-                       : launch_tc_pair<DEPairPolicy>(ep, (int)std::min<int64_t>(pairs, tiles), st,
-                                                      KC_DE);
+      if (pair_dedh) {
+        de_rc = launch_tc_pair<DEPairPolicy>(
+            ep, (int)std::min<int64_t>(sms / 2, (int64_t)ep.mt * dt), st, KC_DE);
       } else {
         de_rc = launch_tc<DEPolicy>(ep, (int)std::min<int64_t>(sms, (int64_t)ep.mt * dt), st, KC_DE);
       }
@@ -1009,7 +1030,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       hp.mblocks = mbs;
       hp.n_valid = cp.n_valid;
       hp.status = status;
-      if (int rc = kPairDEDH
+      if (int rc = pair_dedh
                        ? launch_tc_pair<DHPairPolicy>(
                              hp, (int)std::min<int64_t>(sms / 2, cdiv(mbs, 2) * dt), st, KC_DH)
                        : launch_tc<DHPolicy>(hp, (int)std::min<int64_t>(sms, (int64_t)mbs * dt), st,

@@ -922,7 +922,6 @@ struct DEPolicyT {
 };
 using DEPolicy = DEPolicyT<false>;
 using DEPairPolicy = DEPolicyT<true>;
-using DEPairNarrowPolicy = DEPolicyT<true, BN / 2>;
 
 // =====================================================================
 // Backward, step 3: dH_acc[j, :] += G[j, chunk] E_chunk, K = chunk.
