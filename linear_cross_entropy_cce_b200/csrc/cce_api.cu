@@ -41,6 +41,12 @@ constexpr int64_t kFilteredWidthMult = CCE_FILTERED_WIDTH_MULT;
 #define CCE_CAP_CHUNK_EIGHTH 1
 #endif
 constexpr bool kCapChunkToEighth = CCE_CAP_CHUNK_EIGHTH != 0;
+// Soft-target KL with one head: dual 128-id tiles (see KLFwdPolicyT) unless
+// built with CCE_KL_DUAL=0.
+#ifndef CCE_KL_DUAL
+#define CCE_KL_DUAL 1
+#endif
+constexpr bool kKLDual = CCE_KL_DUAL != 0;
 
 size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -788,6 +794,8 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   // chunk width of this call: wider when filtering can take the sparse route
   const bool wide = filter_eps > 0.f && !kahan;
   const bool pair_dedh = kPairDEDH && filter_eps <= 0.f;
+  // zero-slice masks only pay where G has zeros: filtered calls
+  const bool use_masks = filter_eps > 0.f;
   const int Vc = (int)(wide ? pl.Vc_f : pl.Vc);
   const int dh_words = (int)cdiv(Vc, 512);
   const int dt = (int)cdiv(D, BN);
@@ -859,7 +867,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   memset(&hp, 0, sizeof(hp));
   if (!make_map(&gp.mapA, Hc, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
   // soft-target KL with one head for student and teacher: dual 128-id tiles
-  const bool kl_dual = kl != nullptr && kl->Et == E;
+  const bool kl_dual = kKLDual && kl != nullptr && kl->Et == E;
   if (kl) {
     if (!make_map(&gp.mapA2, Ht_c, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
     if (!make_map(&gp.mapB2, kl->Et, D, V, D, BK, BN)) return CCE_ELAUNCH;
@@ -940,11 +948,12 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       // step 1: G for this chunk, with its zero-slice masks
       uint32_t* dh_mask = masks + (size_t)(chunk & 1) * mask_stride;
       uint32_t* de_mask = dh_mask + (size_t)(pl.Npad / BM) * dh_words;
-      gp.mask_clear = masks + (size_t)((chunk + 1) & 1) * mask_stride;
+      // unfiltered calls keep no zero-slice masks (every K step is issued)
+      gp.mask_clear = use_masks ? masks + (size_t)((chunk + 1) & 1) * mask_stride : nullptr;
       gp.mask_clear_words = (int)(mask_bytes_for(pl.Npad, Vc) / sizeof(uint32_t));
-      gp.dh_mask = dh_mask;
+      gp.dh_mask = use_masks ? dh_mask : nullptr;
       gp.dh_words = dh_words;
-      gp.de_mask = de_mask;
+      gp.de_mask = use_masks ? de_mask : nullptr;
       gp.de_words = pl.de_words;
       gp.mapB = segK;
       gp.b_row0 = row0;
@@ -1004,7 +1013,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       ep.dE = sg.s[s].dE;
       ep.dE_comp = static_cast<__nv_bfloat16*>(sg.s[s].dE_comp);
       ep.mode = kahan ? 2 : (fp32 ? 1 : 0);
-      ep.mask = de_mask;
+      ep.mask = use_masks ? de_mask : nullptr;
       ep.mwords = pl.de_words;
       ep.n_valid = cp.n_valid;
       ep.status = status;
@@ -1025,7 +1034,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       hp.dH_acc = dH_acc;
       hp.nz_cnt = sparse ? nz_cnt + chunk : nullptr;
       hp.nz_cap = cap;
-      hp.mask = dh_mask;
+      hp.mask = use_masks ? dh_mask : nullptr;
       hp.mwords = dh_words;
       hp.mblocks = mbs;
       hp.n_valid = cp.n_valid;
@@ -1180,7 +1189,7 @@ int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
       !aligned16(Es) || !aligned16(Ht) || !aligned16(Et))
     return CCE_EINVAL;
   // one head for teacher and student: dual 128-id tiles (see KLFwdPolicyT)
-  const bool dual = Es == Et;
+  const bool dual = kKLDual && Es == Et;
   const KLFwdPlan pl = plan_kl_fwd(N, D, V, dual ? BN / 2 : BN);
   if (!workspace || workspace_bytes < pl.total) return CCE_EWORKSPACE;
   const int sms = device_sms();

@@ -575,6 +575,66 @@ struct PairEngine {
     return true;
   }
 
+  // ---- unmasked producer (each CTA): all nkb stages of this CTA's halves,
+  // each announced by the rank-0 producer as soon as it is issued.
+  template <bool A_MN, bool B_MN>
+  __device__ __forceinline__ bool produce(const CUtensorMap* mA, const CUtensorMap* mB, int ax,
+                                          int ay, int bx, int by, int nkb) {
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
+      if (rank == 0) mbar_arrive_expect_tx(smem_u32(&ctl->full[pipe.stage]), 2 * PSTAGE_BYTES);
+      const uint32_t fb = in_cta(&ctl->full[pipe.stage], 0);
+      const uint32_t sa = smem_u32(smem + pipe.stage * PSTAGE_BYTES);
+      const uint32_t sb = sa + PA_BYTES;
+      if (!A_MN) {
+        tma_load_2d_pair(sa, mA, fb, ax + kb * BK, ay);
+      } else {
+        tma_load_2d_pair(sa, mA, fb, ax, ay + kb * BK);
+        tma_load_2d_pair(sa + 8192, mA, fb, ax + 64, ay + kb * BK);
+      }
+      if (!B_MN) {
+        tma_load_2d_pair(sb, mB, fb, bx + kb * BK, by);
+      } else {
+        tma_load_2d_pair(sb, mB, fb, bx, by + kb * BK);
+        tma_load_2d_pair(sb + 8192, mB, fb, bx + 64, by + kb * BK);
+      }
+      pipe.advance();
+      ++fills;
+    }
+    return true;
+  }
+
+  // ---- unmasked MMA issuer (rank 0): every K step of nkb stages.
+  template <bool A_MN, bool B_MN>
+  __device__ __forceinline__ bool mma(int nkb) {
+    const int acc = tcount & 1;
+    if (!wait(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u)) return false;
+    tc_fence_after();
+    const uint32_t d = tmem + acc * BN;
+    constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
+    constexpr uint32_t a_step = A_MN ? 2048 : 32;
+    constexpr uint32_t b_step = B_MN ? 2048 : 32;
+    const uint64_t ad0 = A_MN ? smem_desc_sw128(smem_u32(smem), 8192, 1024)
+                              : smem_desc_sw128(smem_u32(smem), 16, 1024);
+    const uint64_t bd0 = B_MN ? smem_desc_sw128(smem_u32(smem) + PA_BYTES, 8192, 1024)
+                              : smem_desc_sw128(smem_u32(smem) + PA_BYTES, 16, 1024);
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!wait(smem_u32(&ctl->full[pipe.stage]), pipe.phase)) return false;
+      tc_fence_after();
+      const uint64_t so = (uint64_t)((pipe.stage * PSTAGE_BYTES) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        umma_bf16_pair(d, ad0 + so + kk * (a_step >> 4), bd0 + so + kk * (b_step >> 4), idesc,
+                       (kb | kk) != 0);
+      umma_commit_pair_both(smem_u32(&ctl->empty[pipe.stage]));
+      pipe.advance();
+      ++fills;
+    }
+    umma_commit_pair_both(smem_u32(&ctl->tfull[acc]));
+    ++tcount;
+    return true;
+  }
+
   // ---- MMA issuer (rank 0 only, one thread): consumes the records until
   // REC_LAST; each stage is released to both CTAs' producers by a commit to
   // each CTA's empty barrier, the tile's accumulator to both epilogues.

@@ -577,7 +577,8 @@ struct GPolicyT {
     const int row = q * 32 + lane;
     const bool slab = writes_slab(p);
     const bool full = FULL && !p.repair;        // this launch writes G_full
-    const bool de_bits = FULL ? full : slab;    // ... and the dE contraction's masks
+    // ... and the dE contraction's masks (none for unfiltered calls)
+    const bool de_bits = (FULL ? full : slab) && p.de_mask != nullptr;
     bool emit = p.nz_list != nullptr && !p.repair;  // this warp still lists non-zeros
     if (slab && p.slab_flag && !p.repair && blockIdx.x == 0 && threadIdx.x == 64)
       *p.slab_flag = 1;
@@ -673,12 +674,15 @@ struct GPolicyT {
             dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
             dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
             // warp vote: which 16-column slices of this chunk hold any non-zero
-            const uint32_t b0 = __ballot_sync(0xffffffffu, (nzb & 0xFFFFu) != 0u);
-            const uint32_t b1 = __ballot_sync(0xffffffffu, (nzb >> 16) != 0u);
-            if (lane == 0 && (b0 | b1)) {
-              const int g = vt * (TN / 16) + c * 2;
-              atomicOr(&p.dh_mask[mb * p.dh_words + (g >> 5)],
-                       ((b0 ? 1u : 0u) | (b1 ? 2u : 0u)) << (g & 31));
+            // (unfiltered calls keep no masks: every slice is issued)
+            if (p.dh_mask != nullptr) {
+              const uint32_t b0 = __ballot_sync(0xffffffffu, (nzb & 0xFFFFu) != 0u);
+              const uint32_t b1 = __ballot_sync(0xffffffffu, (nzb >> 16) != 0u);
+              if (lane == 0 && (b0 | b1)) {
+                const int g = vt * (TN / 16) + c * 2;
+                atomicOr(&p.dh_mask[mb * p.dh_words + (g >> 5)],
+                         ((b0 ? 1u : 0u) | (b1 ? 2u : 0u)) << (g & 31));
+              }
             }
           }
           if constexpr (FULL) {
@@ -806,11 +810,12 @@ struct DEPolicyT {
     return !(p.nz_cnt && *p.nz_cnt <= p.nz_cap);
   }
   // K-step masks of the (one or two) 128-row vocabulary blocks of tile vt
+  // (null without masks: an unfiltered call issues every K step)
   static __device__ __forceinline__ const uint32_t* mask_lo(const Params& p, int vt) {
-    return p.mask + (size_t)(PAIR ? 2 * vt : vt) * p.mwords;
+    return p.mask ? p.mask + (size_t)(PAIR ? 2 * vt : vt) * p.mwords : nullptr;
   }
   static __device__ __forceinline__ const uint32_t* mask_hi(const Params& p, int vt) {
-    return PAIR ? p.mask + (size_t)(2 * vt + 1) * p.mwords : mask_lo(p, vt);
+    return (PAIR && p.mask) ? p.mask + (size_t)(2 * vt + 1) * p.mwords : mask_lo(p, vt);
   }
 
   template <class F>
@@ -831,6 +836,13 @@ struct DEPolicyT {
   template <class Eng>
   static __device__ void producer(const Params& p, Eng& eng) {
     schedule(p, [&](int vt, int dtile, int nkb) {
+      if (p.mask == nullptr) {  // unfiltered: every K step, no records
+        if constexpr (PAIR)
+          return eng.template produce<true, true>(&p.mapA, &p.mapB, vt * ROWS + (int)eng.rank * BM,
+                                                  0, dtile * NT + (int)eng.rank * (NT / 2), 0, nkb);
+        else
+          return eng.template produce<true, true>(&p.mapA, &p.mapB, vt * BM, 0, dtile * BN, 0, nkb);
+      }
       if constexpr (PAIR) {
         return eng.template produce_rec<true, true, NT>(
             &p.mapA, &p.mapB, vt * ROWS + (int)eng.rank * BM, 0, dtile * NT + (int)eng.rank * (NT / 2),
@@ -844,10 +856,12 @@ struct DEPolicyT {
   template <class Eng>
   static __device__ void mma(const Params& p, Eng& eng) {
     schedule(p, [&](int, int, int nkb) {
+      if (nkb == 0) return true;
+      if (p.mask == nullptr) return eng.template mma<true, true>(nkb);
       if constexpr (PAIR)
-        return nkb == 0 || eng.template mma_rec<true, true, NT>();
+        return eng.template mma_rec<true, true, NT>();
       else
-        return nkb == 0 || eng.template mma_rec<true, true>();
+        return eng.template mma_rec<true, true>();
     });
   }
   template <class Eng>
@@ -958,13 +972,14 @@ struct DHPolicyT {
   }
   // per epilogue warp: two 32 x 32 fp32 staging tiles for the TMA reduce-add
   static constexpr int EXTRA_SMEM = 4 * 2 * 4096;
+  // (null without masks: an unfiltered call issues every K step)
   static __device__ __forceinline__ const uint32_t* mask_lo(const Params& p, int mb) {
-    return p.mask + (size_t)(PAIR ? 2 * mb : mb) * p.mwords;
+    return p.mask ? p.mask + (size_t)(PAIR ? 2 * mb : mb) * p.mwords : nullptr;
   }
   static __device__ __forceinline__ const uint32_t* mask_hi(const Params& p, int mb) {
     // the mask buffer has one entry per 128-row block of Npad
-    return (PAIR && 2 * mb + 1 < p.mblocks) ? p.mask + (size_t)(2 * mb + 1) * p.mwords
-                                            : mask_lo(p, mb);
+    return (PAIR && p.mask && 2 * mb + 1 < p.mblocks) ? p.mask + (size_t)(2 * mb + 1) * p.mwords
+                                                      : mask_lo(p, mb);
   }
 
   template <class F>
@@ -987,6 +1002,15 @@ struct DHPolicyT {
   template <class Eng>
   static __device__ void producer(const Params& p, Eng& eng) {
     schedule(p, [&](int mb, int dtile, int) {
+      if (p.mask == nullptr) {  // unfiltered: every K step, no records
+        if constexpr (PAIR)
+          return eng.template produce<false, true>(&p.mapA, &p.mapB, 0,
+                                                   mb * ROWS + (int)eng.rank * BM,
+                                                   dtile * BN + (int)eng.rank * BM, p.b_row0, p.nkb);
+        else
+          return eng.template produce<false, true>(&p.mapA, &p.mapB, 0, mb * BM, dtile * BN,
+                                                   p.b_row0, p.nkb);
+      }
       if constexpr (PAIR) {
         const int r = (int)eng.rank * BM;
         return eng.template produce_rec<false, true>(&p.mapA, &p.mapB, 0, mb * ROWS + r,
@@ -1000,7 +1024,10 @@ struct DHPolicyT {
   }
   template <class Eng>
   static __device__ void mma(const Params& p, Eng& eng) {
-    schedule(p, [&](int, int, int) { return eng.template mma_rec<false, true>(); });
+    schedule(p, [&](int, int, int) {
+      if (p.mask == nullptr) return eng.template mma<false, true>(p.nkb);
+      return eng.template mma_rec<false, true>();
+    });
   }
   // Each warp adds its 32 accumulator rows into dH_acc 32 columns at a time:
   // tcgen05.ld -> swizzled staging tile in shared memory -> TMA reduce-add
