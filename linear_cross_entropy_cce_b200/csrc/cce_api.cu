@@ -41,12 +41,6 @@ constexpr int64_t kFilteredWidthMult = CCE_FILTERED_WIDTH_MULT;
 #define CCE_CAP_CHUNK_EIGHTH 1
 #endif
 constexpr bool kCapChunkToEighth = CCE_CAP_CHUNK_EIGHTH != 0;
-// Soft-target KL with one head: dual 128-id tiles (see KLFwdPolicyT) unless
-// built with CCE_KL_DUAL=0.
-#ifndef CCE_KL_DUAL
-#define CCE_KL_DUAL 1
-#endif
-constexpr bool kKLDual = CCE_KL_DUAL != 0;
 
 size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -217,11 +211,10 @@ struct KLFwdPlan {
   size_t off_nvalid, off_idx, off_pos, off_hs, off_ht, off_part, total;
 };
 
-// tile: vocabulary ids per tile (256, or 128 for a shared head's dual tiles)
-KLFwdPlan plan_kl_fwd(int64_t N, int64_t D, int64_t V, int tile = BN) {
+KLFwdPlan plan_kl_fwd(int64_t N, int64_t D, int64_t V) {
   KLFwdPlan p;
   p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
-  p.T_v = (int)cdiv(V, tile);
+  p.T_v = (int)cdiv(V, BN);
   const int64_t num_mb = p.Npad / BM;
   p.tpi = (int)std::min<int64_t>(16, std::max<int64_t>(2, num_mb * p.T_v / (kPlanSMs * 24)));
   p.S = (int)cdiv(p.T_v, p.tpi);
@@ -866,8 +859,9 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   memset(&ep, 0, sizeof(ep));
   memset(&hp, 0, sizeof(hp));
   if (!make_map(&gp.mapA, Hc, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
-  // soft-target KL with one head for student and teacher: dual 128-id tiles
-  const bool kl_dual = kKLDual && kl != nullptr && kl->Et == E;
+  // soft-target KL with one head for student and teacher: dual 128-id
+  // tiles on CTA pairs (GPolicyKLPair)
+  const bool kl_pair = kl != nullptr && kl->Et == E;
   if (kl) {
     if (!make_map(&gp.mapA2, Ht_c, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
     if (!make_map(&gp.mapB2, kl->Et, D, V, D, BK, BN)) return CCE_ELAUNCH;
@@ -958,8 +952,9 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       gp.mapB = segK;
       gp.b_row0 = row0;
       gp.chunk_valid = cv;
-      gp.ct = (int)cdiv(cv, kl_dual ? BN / 2 : BN);
-      if (kl_dual && !make_map(&gp.mapB128, sg.s[s].E, D, ns, D, BK, BN / 2)) return CCE_ELAUNCH;
+      gp.ct = (int)cdiv(cv, kl_pair ? BN / 2 : BN);
+      // this CTA's 64 of a dual tile's 128 head rows
+      if (kl_pair && !make_map(&gp.mapBdual, sg.s[s].E, D, ns, D, BK, BN / 4)) return CCE_ELAUNCH;
       gp.seg = s;
       gp.c0 = c0;
       gp.Vc = Vc;
@@ -990,8 +985,9 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       gp.blk_lse2min = blk_lse2min;
       gp.skip_l2 = gp.l2eps - 1.0f / 16.0f;  // margin over fp32 differences of the two logits
       const int g_grid = (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct);
+      const int g_pairs = (int)std::min<int64_t>(sms / 2, cdiv(mbs, 2) * gp.ct);
       auto launch_g = [&]() {
-        return kl_dual ? launch_tc<GPolicyKLDual>(gp, g_grid, st, KC_G)
+        return kl_pair ? launch_tc_pair<GPolicyKLPair>(gp, g_pairs, st, KC_G)
                : kl    ? launch_tc<GPolicyKL>(gp, g_grid, st, KC_G)
                : full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
                          : launch_tc<GPolicy>(gp, g_grid, st, KC_G);
@@ -1175,8 +1171,7 @@ int cce_bwd(const void* H, const void* E, const int32_t* y, const float* lse, co
 // ------------------------------------------------------------ soft-target KL
 size_t cce_kl_fwd_workspace_size(int64_t N, int64_t D, int64_t V) {
   if (!sizes_ok(N, D, V)) return 0;
-  // enough for either tile width
-  return std::max(plan_kl_fwd(N, D, V, BN).total, plan_kl_fwd(N, D, V, BN / 2).total);
+  return plan_kl_fwd(N, D, V).total;
 }
 
 int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
@@ -1188,9 +1183,7 @@ int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
   if (!Hs || !Es || !Ht || !Et || !kl || !lse_s || !lse_t || !status || !aligned16(Hs) ||
       !aligned16(Es) || !aligned16(Ht) || !aligned16(Et))
     return CCE_EINVAL;
-  // one head for teacher and student: dual 128-id tiles (see KLFwdPolicyT)
-  const bool dual = kKLDual && Es == Et;
-  const KLFwdPlan pl = plan_kl_fwd(N, D, V, dual ? BN / 2 : BN);
+  const KLFwdPlan pl = plan_kl_fwd(N, D, V);
   if (!workspace || workspace_bytes < pl.total) return CCE_EWORKSPACE;
   const int sms = device_sms();
   if (sms <= 0 || !encode_fn()) return CCE_EDEVICE;
@@ -1220,8 +1213,7 @@ int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
   memset(&kp, 0, sizeof(kp));
   if (!make_map(&kp.mapAs, Hs_c, D, pl.Npad, D, BK, BM) ||
       !make_map(&kp.mapAt, Ht_c, D, pl.Npad, D, BK, BM) ||
-      !make_map(&kp.mapBs, Es, D, V, D, BK, BN) || !make_map(&kp.mapBt, Et, D, V, D, BK, BN) ||
-      !make_map(&kp.mapB128, Es, D, V, D, BK, BN / 2))
+      !make_map(&kp.mapBs, Es, D, V, D, BK, BN) || !make_map(&kp.mapBt, Et, D, V, D, BK, BN))
     return CCE_ELAUNCH;
   kp.V = (int)V;
   kp.T_v = pl.T_v;
@@ -1233,10 +1225,7 @@ int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
   kp.part = at<float>(workspace, pl.off_part);
   kp.status = status;
   const int64_t items = (pl.Npad / BM) * pl.S;
-  const int grid = (int)std::min<int64_t>(sms, items);
-  if (int rc = dual ? launch_tc<KLFwdDualPolicy>(kp, grid, st, KC_FWD)
-                    : launch_tc<KLFwdPolicy>(kp, grid, st, KC_FWD))
-    return rc;
+  if (int rc = launch_tc<KLFwdPolicy>(kp, (int)std::min<int64_t>(sms, items), st, KC_FWD)) return rc;
   KLFinParams fin;
   fin.pos_of_row = cp.pos_of_row;
   fin.part = kp.part;

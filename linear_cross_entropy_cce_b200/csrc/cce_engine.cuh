@@ -336,57 +336,7 @@ struct Engine {
     return true;
   }
 
-  // ---- two products over one staged head tile (one 48 KiB stage: rows of
-  // two row operands, 128 x 64 each, and 128 rows of the shared B operand):
-  // the MMA thread issues both N = 128 products from it, into columns
-  // [0, 128) and [128, 256) of one accumulator, so a tile pair takes 256
-  // TMEM columns and the two accumulators still alternate (the epilogue of a
-  // pair overlaps the MMAs of the next).  Per FLOP this moves as many operand
-  // bytes as a single N = 256 product.
-  __device__ __forceinline__ bool produce_dual(const CUtensorMap* mA0, const CUtensorMap* mA1,
-                                               const CUtensorMap* mB, int ay, int by, int nkb) {
-    for (int kb = 0; kb < nkb; ++kb) {
-      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
-      const uint32_t fb = smem_u32(&ctl->full[pipe.stage]);
-      mbar_arrive_expect_tx(fb, STAGE_BYTES);
-      const uint32_t sa = smem_u32(smem + pipe.stage * STAGE_BYTES);
-      tma_load_2d(sa, mA0, fb, kb * BK, ay);
-      tma_load_2d(sa + A_BYTES, mA1, fb, kb * BK, ay);
-      tma_load_2d(sa + 2 * A_BYTES, mB, fb, kb * BK, by);
-      pipe.advance();
-      ++fills;
-    }
-    return true;
-  }
-  __device__ __forceinline__ bool mma_dual(int nkb) {
-    const int acc = tcount & 1;
-    if (!wait(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u)) return false;
-    tc_fence_after();
-    const uint32_t d0 = tmem + acc * BN;
-    const uint32_t d1 = d0 + BN / 2;
-    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN / 2, false, false);
-    uint32_t issued = 0;
-    for (int kb = 0; kb < nkb; ++kb) {
-      if (!wait(smem_u32(&ctl->full[pipe.stage]), pipe.phase)) return false;
-      tc_fence_after();
-      const uint32_t sa = smem_u32(smem + pipe.stage * STAGE_BYTES);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t bd = smem_desc_sw128(sa + 2 * A_BYTES + kk * 32, 16, 1024);
-        umma_bf16(d0, smem_desc_sw128(sa + kk * 32, 16, 1024), bd, idesc, issued);
-        umma_bf16(d1, smem_desc_sw128(sa + A_BYTES + kk * 32, 16, 1024), bd, idesc, issued);
-        issued = 1;
-      }
-      umma_commit(smem_u32(&ctl->empty[pipe.stage]));
-      pipe.advance();
-      ++fills;
-    }
-    umma_commit(smem_u32(&ctl->tfull[acc]));
-    ++tcount;
-    return true;
-  }
-
-  // ---- epilogue: wait for the next accumulator; returns its TMEM address  // ---- epilogue: wait for the next accumulator; returns its TMEM address
+  // ---- epilogue: wait for the next accumulator; returns its TMEM address
   // for this thread's lane quarter (column 0).
   __device__ __forceinline__ bool epi_acquire(int quarter, uint32_t& taddr) {
     const int acc = tcount & 1;
@@ -447,10 +397,15 @@ constexpr int PAIR_STAGES = 6;
 constexpr int PA_BYTES = 128 * BK * 2;  // this CTA's A rows of one stage
 constexpr int PB_BYTES = 128 * BK * 2;  // this CTA's half of B's columns
 constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
+// Dual-product stages (PairEngineT::produce_dual): two A operands of 128 rows
+// and this CTA's 64 rows of a 128-row B operand, 40 KiB, five deep.
+constexpr int PAIR_DUAL_STAGES = 5;
+constexpr int PDUAL_STAGE_BYTES = 2 * PA_BYTES + 64 * BK * 2;
 
-struct PairCtl {
-  uint64_t full[PAIR_STAGES];
-  uint64_t empty[PAIR_STAGES];
+template <int NST>
+struct PairCtlT {
+  uint64_t full[NST];
+  uint64_t empty[NST];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -458,20 +413,35 @@ struct PairCtl {
   int abort;
   int consumed;
   int pad;
-  uint32_t rec[PAIR_STAGES];
+  uint32_t rec[NST];
+};
+
+// Stage geometry of a pair policy: Policy::PAIR_NST stages of
+// Policy::PAIR_SB bytes when it declares them, else the 32 KiB default.
+template <class P, class = void>
+struct PairGeom {
+  static constexpr int NST = PAIR_STAGES;
+  static constexpr int SB = PSTAGE_BYTES;
+};
+template <class P>
+struct PairGeom<P, std::void_t<decltype(P::PAIR_NST), decltype(P::PAIR_SB)>> {
+  static constexpr int NST = P::PAIR_NST;
+  static constexpr int SB = P::PAIR_SB;
 };
 
 template <class Policy>
 constexpr int pair_smem_bytes() {
-  return PAIR_STAGES * PSTAGE_BYTES + Policy::EXTRA_SMEM + static_cast<int>(sizeof(PairCtl)) +
-         1024 + 64;
+  using G = PairGeom<Policy>;
+  return G::NST * G::SB + Policy::EXTRA_SMEM + static_cast<int>(sizeof(PairCtlT<G::NST>)) + 1024 +
+         64;
 }
 
+template <int NST>
 struct PairPipe {
   int stage = 0;
   uint32_t phase = 0;
   __device__ __forceinline__ void advance() {
-    if (++stage == PAIR_STAGES) {
+    if (++stage == NST) {
       stage = 0;
       phase ^= 1u;
     }
@@ -494,14 +464,15 @@ struct MaskPair {
   }
 };
 
-struct PairEngine {
-  PairCtl* ctl;
+template <int NST, int SB>
+struct PairEngineT {
+  PairCtlT<NST>* ctl;
   uint8_t* smem;
   uint8_t* extra;
   uint32_t tmem;
   int* status;
   uint32_t rank;  // 0: issues the MMAs; 1: its peer
-  PairPipe pipe;
+  PairPipe<NST> pipe;
   int tcount = 0;
   int fills = 0;
   uint64_t wait_ns = kWaitLimitNs;
@@ -523,14 +494,11 @@ struct PairEngine {
   // thread (its K steps, REC_LAST on the tile's last stage, found by scanning
   // both masks first), written by the rank-0 producer before it announces
   // the stage with the bytes of both CTAs' copies.
-  // NT: the pair tile's columns (256, or 128 for narrow problems): each CTA
-  // stages NT / 2 of them.
-  template <bool A_MN, bool B_MN, int NT = BN>
+  template <bool A_MN, bool B_MN>
   __device__ __forceinline__ bool produce_rec(const CUtensorMap* mA, const CUtensorMap* mB, int ax,
                                               int ay, int bx, int by, int nkb, const uint32_t* m0,
                                               const uint32_t* m1) {
-    static_assert(NT == BN || (NT == BN / 2 && B_MN), "128-column pair tiles need an MN-major B");
-    constexpr uint32_t tx = 2u * (PA_BYTES + (NT / 2) * BK * 2);
+    constexpr uint32_t tx = 2u * SB;
     const int last = (m0 == nullptr || m1 == nullptr)
                          ? nkb - 1
                          : max(mask_last_stage(m0, nkb), mask_last_stage(m1, nkb));
@@ -555,7 +523,7 @@ struct PairEngine {
         mbar_arrive_expect_tx(smem_u32(&ctl->full[pipe.stage]), tx);
       }
       const uint32_t fb = in_cta(&ctl->full[pipe.stage], 0);
-      const uint32_t sa = smem_u32(smem + pipe.stage * PSTAGE_BYTES);
+      const uint32_t sa = smem_u32(smem + pipe.stage * SB);
       const uint32_t sb = sa + PA_BYTES;
       if (!A_MN) {
         tma_load_2d_pair(sa, mA, fb, ax + kb * BK, ay);
@@ -567,7 +535,7 @@ struct PairEngine {
         tma_load_2d_pair(sb, mB, fb, bx + kb * BK, by);
       } else {
         tma_load_2d_pair(sb, mB, fb, bx, by + kb * BK);
-        if (NT == BN) tma_load_2d_pair(sb + 8192, mB, fb, bx + 64, by + kb * BK);
+        tma_load_2d_pair(sb + 8192, mB, fb, bx + 64, by + kb * BK);
       }
       pipe.advance();
       ++fills;
@@ -582,9 +550,9 @@ struct PairEngine {
                                           int ay, int bx, int by, int nkb) {
     for (int kb = 0; kb < nkb; ++kb) {
       if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
-      if (rank == 0) mbar_arrive_expect_tx(smem_u32(&ctl->full[pipe.stage]), 2 * PSTAGE_BYTES);
+      if (rank == 0) mbar_arrive_expect_tx(smem_u32(&ctl->full[pipe.stage]), 2 * SB);
       const uint32_t fb = in_cta(&ctl->full[pipe.stage], 0);
-      const uint32_t sa = smem_u32(smem + pipe.stage * PSTAGE_BYTES);
+      const uint32_t sa = smem_u32(smem + pipe.stage * SB);
       const uint32_t sb = sa + PA_BYTES;
       if (!A_MN) {
         tma_load_2d_pair(sa, mA, fb, ax + kb * BK, ay);
@@ -621,7 +589,7 @@ struct PairEngine {
     for (int kb = 0; kb < nkb; ++kb) {
       if (!wait(smem_u32(&ctl->full[pipe.stage]), pipe.phase)) return false;
       tc_fence_after();
-      const uint64_t so = (uint64_t)((pipe.stage * PSTAGE_BYTES) >> 4);
+      const uint64_t so = (uint64_t)((pipe.stage * SB) >> 4);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         umma_bf16_pair(d, ad0 + so + kk * (a_step >> 4), bd0 + so + kk * (b_step >> 4), idesc,
@@ -638,13 +606,13 @@ struct PairEngine {
   // ---- MMA issuer (rank 0 only, one thread): consumes the records until
   // REC_LAST; each stage is released to both CTAs' producers by a commit to
   // each CTA's empty barrier, the tile's accumulator to both epilogues.
-  template <bool A_MN, bool B_MN, int NT = BN>
+  template <bool A_MN, bool B_MN>
   __device__ __forceinline__ bool mma_rec() {
     const int acc = tcount & 1;
     if (!wait(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u)) return false;
     tc_fence_after();
     const uint32_t d = tmem + acc * BN;
-    constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, NT, A_MN, B_MN);
+    constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
     constexpr uint32_t a_step = A_MN ? 2048 : 32;  // bytes per K=16 step
     constexpr uint32_t b_step = B_MN ? 2048 : 32;
     const uint64_t ad0 = A_MN ? smem_desc_sw128(smem_u32(smem), 8192, 1024)
@@ -656,7 +624,7 @@ struct PairEngine {
       if (!wait(smem_u32(&ctl->full[pipe.stage]), pipe.phase)) return false;
       tc_fence_after();
       const uint32_t rec = *reinterpret_cast<volatile uint32_t*>(&ctl->rec[pipe.stage]);
-      const uint64_t so = (uint64_t)((pipe.stage * PSTAGE_BYTES) >> 4);
+      const uint64_t so = (uint64_t)((pipe.stage * SB) >> 4);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         if (!(rec & (1u << kk))) continue;
@@ -668,6 +636,62 @@ struct PairEngine {
       pipe.advance();
       ++fills;
       if (rec & REC_LAST) break;
+    }
+    umma_commit_pair_both(smem_u32(&ctl->tfull[acc]));
+    ++tcount;
+    return true;
+  }
+
+  // ---- two products over one staged 128-row B tile (each CTA, lane 0 of
+  // warp 0; needs the dual geometry PAIR_DUAL_STAGES x PDUAL_STAGE_BYTES):
+  // a stage holds this CTA's 128 rows of each of two A operands (rows ay ..
+  // ay+127 of mA0 and mA1) and its 64 of B's 128 rows (rows by .. by+63).
+  // The rank-0 MMA thread issues two M = 256, N = 128 products per K step
+  // into columns [0, 128) and [128, 256) of one accumulator, so a tile takes
+  // 256 TMEM columns and the two accumulators still alternate (the epilogue
+  // of a tile overlaps the MMAs of the next), at the shared-memory operand
+  // bytes per FLOP of a single-CTA N = 256 product.
+  __device__ __forceinline__ bool produce_dual(const CUtensorMap* mA0, const CUtensorMap* mA1,
+                                               const CUtensorMap* mB64, int ay, int by, int nkb) {
+    static_assert(SB == PDUAL_STAGE_BYTES, "dual products need the dual stage geometry");
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!wait(smem_u32(&ctl->empty[pipe.stage]), pipe.phase ^ 1u)) return false;
+      if (rank == 0) mbar_arrive_expect_tx(smem_u32(&ctl->full[pipe.stage]), 2 * SB);
+      const uint32_t fb = in_cta(&ctl->full[pipe.stage], 0);
+      const uint32_t sa = smem_u32(smem + pipe.stage * SB);
+      tma_load_2d_pair(sa, mA0, fb, kb * BK, ay);
+      tma_load_2d_pair(sa + PA_BYTES, mA1, fb, kb * BK, ay);
+      tma_load_2d_pair(sa + 2 * PA_BYTES, mB64, fb, kb * BK, by);
+      pipe.advance();
+      ++fills;
+    }
+    return true;
+  }
+  __device__ __forceinline__ bool mma_dual(int nkb) {
+    static_assert(SB == PDUAL_STAGE_BYTES, "dual products need the dual stage geometry");
+    const int acc = tcount & 1;
+    if (!wait(smem_u32(&ctl->tempty[acc]), (((uint32_t)tcount >> 1) & 1u) ^ 1u)) return false;
+    tc_fence_after();
+    const uint32_t d0 = tmem + acc * BN;
+    const uint32_t d1 = d0 + BN / 2;
+    constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN / 2, false, false);
+    const uint32_t s0 = smem_u32(smem);
+    const uint64_t a0 = smem_desc_sw128(s0, 16, 1024);
+    const uint64_t a1 = smem_desc_sw128(s0 + PA_BYTES, 16, 1024);
+    const uint64_t b0 = smem_desc_sw128(s0 + 2 * PA_BYTES, 16, 1024);
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!wait(smem_u32(&ctl->full[pipe.stage]), pipe.phase)) return false;
+      tc_fence_after();
+      const uint64_t so = (uint64_t)((pipe.stage * SB) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t k = so + kk * (32 >> 4);  // 32 bytes per K = 16 step
+        umma_bf16_pair(d0, a0 + k, b0 + k, idesc, (kb | kk) != 0);
+        umma_bf16_pair(d1, a1 + k, b0 + k, idesc, (kb | kk) != 0);
+      }
+      umma_commit_pair_both(smem_u32(&ctl->empty[pipe.stage]));
+      pipe.advance();
+      ++fills;
     }
     umma_commit_pair_both(smem_u32(&ctl->tfull[acc]));
     ++tcount;
@@ -690,6 +714,7 @@ struct PairEngine {
     ++tcount;
   }
 };
+using PairEngine = PairEngineT<PAIR_STAGES, PSTAGE_BYTES>;
 
 // Bounded wait that ignores the abort flag (used only while draining).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
@@ -791,11 +816,12 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
 template <class Policy>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_pair_kernel(const __grid_constant__ typename Policy::Params p) {
+  using G = PairGeom<Policy>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (base & 1023u)) & 1023u);
-  uint8_t* extra = smem + PAIR_STAGES * PSTAGE_BYTES;
-  PairCtl* ctl = reinterpret_cast<PairCtl*>(extra + Policy::EXTRA_SMEM);
+  uint8_t* extra = smem + G::NST * G::SB;
+  PairCtlT<G::NST>* ctl = reinterpret_cast<PairCtlT<G::NST>*>(extra + Policy::EXTRA_SMEM);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   // active() depends only on the parameters and on device values every CTA
@@ -804,7 +830,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t rank = cluster_ctarank();
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < PAIR_STAGES; ++s) {
+    for (int s = 0; s < G::NST; ++s) {
       mbar_init(smem_u32(&ctl->full[s]), 1);
       mbar_init(smem_u32(&ctl->empty[s]), 1);
     }
@@ -826,7 +852,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   cluster_sync_all();  // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
 
-  PairEngine eng;
+  PairEngineT<G::NST, G::SB> eng;
   eng.ctl = ctl;
   eng.smem = smem;
   eng.extra = extra;

@@ -29,6 +29,10 @@
 //           back to the original rows.
 #pragma once
 
+#ifndef CCE_DE_PAIR_STAGES
+#define CCE_DE_PAIR_STAGES 6
+#endif
+
 #include <cub/block/block_scan.cuh>
 
 #include "cce_engine.cuh"
@@ -493,7 +497,9 @@ struct GParams {
   // an entry kept when either probability reaches the threshold.
   CUtensorMap mapA2;  // H_t,c [Npad, D], box {64, 128}
   CUtensorMap mapB2;  // E_t rows, K-major, box {64, 256}
-  CUtensorMap mapB128;  // shared head rows, K-major, box {64, 128} (dual tiles)
+  // shared head rows, K-major, for dual tiles: box {64, 128} on one CTA,
+  // {64, 64} per CTA of a pair
+  CUtensorMap mapBdual;
   const float* lt2_c;
   // optional per-element keep bits of original rows < debug_rows
   uint32_t* debug_keep;
@@ -505,15 +511,23 @@ struct GParams {
   int* status;
 };
 
-// KL && DUAL: the student and teacher share one head; each 128-id tile is
-// two N = 128 products from one staged head tile (Engine::produce_dual), in
-// one accumulator (teacher columns 0..127, student 128..255), so the two
-// accumulators alternate and the epilogue overlaps the next tile's MMAs.
-template <bool FULL, bool KL = false, bool DUAL = false>
+// KL (separate heads): each 256-id tile is a teacher and a student N = 256
+// product, one per accumulator, so a tile's epilogue waits for both and does
+// not overlap the next tile's MMAs.
+// KL && PAIR (one head shared by student and teacher): on CTA pairs
+// (tc_pair_kernel), each 128-id tile is two M = 256, N = 128 products from
+// one staged head tile (PairEngineT::produce_dual) in one accumulator
+// (teacher columns 0..127, student 128..255), so the two accumulators
+// alternate and the epilogue overlaps the next tile's MMAs.  Work unit mbu is
+// then a pair of row blocks, 2 mbu (rank 0) and 2 mbu + 1 (rank 1).
+template <bool FULL, bool KL = false, bool PAIR = false>
 struct GPolicyT {
+  static_assert(!PAIR || (KL && !FULL), "CTA pairs serve the shared-head KL producer");
   using Params = GParams;
   static constexpr int EXTRA_SMEM = 0;
-  static constexpr int TN = (KL && DUAL) ? BN / 2 : BN;  // vocabulary ids per tile
+  static constexpr int TN = PAIR ? BN / 2 : BN;  // vocabulary ids per tile
+  static constexpr int PAIR_NST = PAIR_DUAL_STAGES;  // stage geometry on CTA pairs
+  static constexpr int PAIR_SB = PDUAL_STAGE_BYTES;
 
   // Whether this launch writes the dense fallback (slab + masks), and
   // whether it runs at all (a repair launch usually has nothing to do).
@@ -524,22 +538,29 @@ struct GPolicyT {
   static __device__ __forceinline__ bool active(const Params& p) {
     return !p.repair || (*p.nz_cnt > p.nz_cap && *p.slab_flag == 0);
   }
+  // (no tile skip on CTA pairs: the KL producer never skips)
   static __device__ __forceinline__ bool skip(const Params& p, int mb, int vt) {
+    if constexpr (PAIR) return false;
     return p.tile_cmax2 != nullptr && p.tile_cmax2[vt] - p.blk_lse2min[mb] < p.skip_l2;
   }
 
+  // f(mbu, vt, nv) for this CTA's (or CTA pair's) work units: mbu a row
+  // block, or a pair of row blocks on CTA pairs
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
     const int nv = *p.n_valid;
-    const int num_mb = (nv + BM - 1) / BM;
-    const int tiles = active(p) ? num_mb * p.ct : 0;
+    const int rows_u = PAIR ? 2 * BM : BM;  // rows per work unit
+    const int num_u = (nv + rows_u - 1) / rows_u;
+    const int tiles = active(p) ? num_u * p.ct : 0;
     // grouped order (vocabulary-tile-major within L2-sized row groups); the
     // KL producer's A operand is two row blocks (teacher and student)
-    const int gm = row_group_blocks(num_mb, (long long)BM * BK * 2 * p.nkb * (KL ? 2 : 1));
-    for (int i = blockIdx.x; i < tiles; i += gridDim.x) {
-      int mb, vt;
-      grouped_item(i, num_mb, p.ct, gm, mb, vt);
-      if (!f(mb, vt, nv)) return;
+    const int gm = row_group_blocks(num_u, (long long)rows_u * BK * 2 * p.nkb * (KL ? 2 : 1));
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    for (int i = unit; i < tiles; i += units) {
+      int mbu, vt;
+      grouped_item(i, num_u, p.ct, gm, mbu, vt);
+      if (!f(mbu, vt, nv)) return;
     }
   }
   static __device__ void prefetch(const Params& p) {
@@ -547,34 +568,46 @@ struct GPolicyT {
     tma_prefetch_map(&p.mapB);
     if constexpr (KL) {
       tma_prefetch_map(&p.mapA2);
-      tma_prefetch_map(DUAL ? &p.mapB128 : &p.mapB2);
+      tma_prefetch_map(PAIR ? &p.mapBdual : &p.mapB2);
     }
   }
-  static __device__ void producer(const Params& p, Engine& eng) {
+  template <class Eng>
+  static __device__ void producer(const Params& p, Eng& eng) {
     schedule(p, [&](int mb, int vt, int) {
       if (skip(p, mb, vt)) return true;
-      if constexpr (KL && DUAL)  // teacher rows, student rows, one head tile
-        return eng.produce_dual(&p.mapA2, &p.mapA, &p.mapB128, mb * BM, p.b_row0 + vt * TN, p.nkb);
-      if constexpr (KL) {  // teacher tile first: it lands in the even accumulator
-        if (!eng.produce<false, false>(&p.mapA2, &p.mapB2, 0, mb * BM, 0, p.b_row0 + vt * BN,
-                                       p.nkb))
-          return false;
+      if constexpr (PAIR) {  // this CTA's 128 rows of each, 64 of the tile's head rows
+        return eng.produce_dual(&p.mapA2, &p.mapA, &p.mapBdual, (2 * mb + (int)eng.rank) * BM,
+                                p.b_row0 + vt * TN + (int)eng.rank * (TN / 2), p.nkb);
+      } else {
+        if constexpr (KL) {  // teacher tile first: it lands in the even accumulator
+          if (!eng.template produce<false, false>(&p.mapA2, &p.mapB2, 0, mb * BM, 0,
+                                                  p.b_row0 + vt * BN, p.nkb))
+            return false;
+        }
+        return eng.template produce<false, false>(&p.mapA, &p.mapB, 0, mb * BM, 0,
+                                                  p.b_row0 + vt * BN, p.nkb);
       }
-      return eng.produce<false, false>(&p.mapA, &p.mapB, 0, mb * BM, 0, p.b_row0 + vt * BN, p.nkb);
     });
   }
-  static __device__ void mma(const Params& p, Engine& eng) {
+  template <class Eng>
+  static __device__ void mma(const Params& p, Eng& eng) {
     schedule(p, [&](int mb, int vt, int) {
       if (skip(p, mb, vt)) return true;
-      if constexpr (KL && DUAL) return eng.mma_dual(p.nkb);
-      if constexpr (KL) {
-        if (!eng.mma<false, false>(p.nkb)) return false;
+      if constexpr (PAIR) {
+        return eng.mma_dual(p.nkb);
+      } else {
+        if constexpr (KL) {
+          if (!eng.template mma<false, false>(p.nkb)) return false;
+        }
+        return eng.template mma<false, false>(p.nkb);
       }
-      return eng.mma<false, false>(p.nkb);
     });
   }
-  static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
+  template <class Eng>
+  static __device__ void epilogue(const Params& p, Eng& eng, int q, int lane) {
     const int row = q * 32 + lane;
+    uint32_t rank = 0;
+    if constexpr (PAIR) rank = eng.rank;
     const bool slab = writes_slab(p);
     const bool full = FULL && !p.repair;        // this launch writes G_full
     // ... and the dE contraction's masks (none for unfiltered calls)
@@ -586,12 +619,16 @@ struct GPolicyT {
       for (int i = blockIdx.x * EPI_THREADS + q * 32 + lane; i < p.mask_clear_words;
            i += gridDim.x * EPI_THREADS)
         p.mask_clear[i] = 0u;
-    schedule(p, [&](int mb, int vt, int nv) {
+    schedule(p, [&](int mbu, int vt, int nv) {
+      const int mb = PAIR ? 2 * mbu + (int)rank : mbu;  // this CTA's row block
+      // rank 1's block past the last one (an odd count on CTA pairs): its
+      // rows are outside the slab and carry no entries
+      const bool blk_live = !PAIR || mb * BM < nv;
       // a skipped tile has no accumulator: no softmax entry is kept in it
       const bool sk = skip(p, mb, vt);
       uint32_t taddr = 0, tteach = 0;
       if (!sk) {
-        if constexpr (KL && DUAL) {
+        if constexpr (PAIR) {
           if (!eng.epi_acquire(q, tteach)) return false;
           taddr = tteach + TN;  // student columns after the teacher's
         } else if constexpr (KL) {
@@ -650,7 +687,7 @@ struct GPolicyT {
         const int tj = tcol - c * 32;
         const uint32_t tb = (tj >= 0 && tj < 32) ? (cm & (1u << tj)) : 0u;
         const uint32_t nzb = kb | tb;  // entries of G that are non-zero
-        if (slab || full) {
+        if ((slab || full) && blk_live) {
           // softmax entries evaluated: the kept ones, or all valid ones for G_full
           const uint32_t ks = full ? cm : kb;
           uint32_t pk[16], pf[FULL ? 16 : 1];
@@ -747,7 +784,7 @@ struct GPolicyT {
         }
       }
       if (!sk) {
-        if constexpr (KL && !DUAL)
+        if constexpr (KL && !PAIR)
           eng.epi_release2(lane);
         else
           eng.epi_release(lane);
@@ -760,7 +797,7 @@ struct GPolicyT {
 using GPolicy = GPolicyT<false>;
 using GPolicyFull = GPolicyT<true>;
 using GPolicyKL = GPolicyT<false, true>;
-using GPolicyKLDual = GPolicyT<false, true, true>;
+using GPolicyKLPair = GPolicyT<false, true, true>;
 
 // =====================================================================
 // Backward, step 2: dE_chunk = G^T H_c, K = compact rows, accumulated on
@@ -797,14 +834,17 @@ __device__ __forceinline__ bool mask_empty(const uint32_t* m, int nkb, int lane)
 }
 
 // One CTA per 128 x 256 tile of dE (PAIR = false) or one CTA pair per
-// 256 x NT tile (PAIR = true, tcgen05 cta_group::2; NT = 256, or 128 when a
-// narrow chunk would leave the SMs few 256-column tiles; the host sets mt and
-// dt to the number of vocabulary and D tiles accordingly).
-template <bool PAIR, int NT = BN>
+// 256 x 256 tile (PAIR = true, tcgen05 cta_group::2; the host sets mt to the
+// number of vocabulary tiles accordingly).
+template <bool PAIR>
 struct DEPolicyT {
   using Params = DEParams;
   static constexpr int EXTRA_SMEM = 0;
   static constexpr int ROWS = PAIR ? 2 * BM : BM;  // vocabulary rows per tile
+  // on CTA pairs: the default 32 KiB stages, CCE_DE_PAIR_STAGES deep (this
+  // epilogue needs no shared memory, so a seventh stage fits)
+  static constexpr int PAIR_NST = CCE_DE_PAIR_STAGES;
+  static constexpr int PAIR_SB = PSTAGE_BYTES;
   // a chunk taken by the sparse route has no dense work
   static __device__ __forceinline__ bool active(const Params& p) {
     return !(p.nz_cnt && *p.nz_cnt <= p.nz_cap);
@@ -839,13 +879,13 @@ struct DEPolicyT {
       if (p.mask == nullptr) {  // unfiltered: every K step, no records
         if constexpr (PAIR)
           return eng.template produce<true, true>(&p.mapA, &p.mapB, vt * ROWS + (int)eng.rank * BM,
-                                                  0, dtile * NT + (int)eng.rank * (NT / 2), 0, nkb);
+                                                  0, dtile * BN + (int)eng.rank * (BN / 2), 0, nkb);
         else
           return eng.template produce<true, true>(&p.mapA, &p.mapB, vt * BM, 0, dtile * BN, 0, nkb);
       }
       if constexpr (PAIR) {
-        return eng.template produce_rec<true, true, NT>(
-            &p.mapA, &p.mapB, vt * ROWS + (int)eng.rank * BM, 0, dtile * NT + (int)eng.rank * (NT / 2),
+        return eng.template produce_rec<true, true>(
+            &p.mapA, &p.mapB, vt * ROWS + (int)eng.rank * BM, 0, dtile * BN + (int)eng.rank * (BN / 2),
             0, nkb, mask_lo(p, vt), mask_hi(p, vt));
       } else {
         return eng.template produce_rec<true, true>(&p.mapA, &p.mapB, vt * BM, 0, dtile * BN, 0,
@@ -859,7 +899,7 @@ struct DEPolicyT {
       if (nkb == 0) return true;
       if (p.mask == nullptr) return eng.template mma<true, true>(nkb);
       if constexpr (PAIR)
-        return eng.template mma_rec<true, true, NT>();
+        return eng.template mma_rec<true, true>();
       else
         return eng.template mma_rec<true, true>();
     });
@@ -878,8 +918,8 @@ struct DEPolicyT {
       const bool ok = r < p.chunk_valid;
       const int w = p.c0 + r;
       const size_t local = ok ? (size_t)(p.perm_seg ? p.perm_seg[w] : w) : 0;
-      for (int c = 0; c < NT / 32; ++c) {
-        const int col0 = dtile * NT + c * 32;
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = dtile * BN + c * 32;
         if (col0 >= p.D) break;
         uint32_t v[32];
         if (!zero) {

@@ -25,9 +25,8 @@ namespace cce {
 struct KLFwdParams {
   CUtensorMap mapAs, mapAt;  // H_s,c / H_t,c [Npad, D], box {64, 128}
   CUtensorMap mapBs, mapBt;  // E_s / E_t [V, D], box {64, 256}
-  CUtensorMap mapB128;       // the shared head E [V, D], box {64, 128} (dual tiles)
   int V;
-  int T_v;   // vocabulary tiles (of the policy's width)
+  int T_v;   // 256-id vocabulary tiles
   int tpi;   // tiles per work item
   int S;     // splits
   int Npad;  // partial row stride
@@ -37,17 +36,80 @@ struct KLFwdParams {
   int* status;
 };
 
-// DUAL = false: separate heads; each 256-id tile is a pair of N = 256
-// products (teacher, then student), one per accumulator, so the pair's
-// epilogue waits for both and does not overlap the next pair's MMAs.
-// DUAL = true: one head shared by teacher and student; each 128-id tile is
-// two N = 128 products from one staged head tile (Engine::produce_dual /
-// mma_dual) in one accumulator, and the two accumulators alternate.
-template <bool DUAL>
-struct KLFwdPolicyT {
+// Per-row running state of the KL forward over a split's tiles (base-2
+// units): teacher max, sum and teacher-weighted sum of z_t - z_s; student
+// max and sum.
+struct KLRowState {
+  float mt, st, w, ms, ss;
+  __device__ __forceinline__ void reset() {
+    mt = -INFINITY;
+    st = 0.f;
+    w = 0.f;
+    ms = -INFINITY;
+    ss = 0.f;
+  }
+  // the split's partials of compact row r
+  __device__ __forceinline__ void store(const KLFwdParams& p, int split, int r) const {
+    float* o = p.part + (size_t)split * 5 * p.Npad + r;
+    o[0] = mt;
+    o[(size_t)p.Npad] = st;
+    o[(size_t)2 * p.Npad] = w;
+    o[(size_t)3 * p.Npad] = ms;
+    o[(size_t)4 * p.Npad] = ss;
+  }
+};
+
+// Folds one tile of this thread's row into the running state: teacher logits
+// at TMEM address ta, student logits at tb, `valid` (> 0) of TN columns.
+template <int TN>
+__device__ __forceinline__ void kl_fwd_tile(uint32_t ta, uint32_t tb, int valid, KLRowState& s) {
+  for (int c = 0; c < TN / 32; ++c) {
+    if (c * 32 >= valid) break;  // uniform over the CTA
+    const int nvc = min(32, valid - c * 32);
+    uint32_t rt[32], rs[32];
+    tmem_ld32(ta + c * 32, rt);
+    tmem_ld32(tb + c * 32, rs);
+    float cmt = -INFINITY, cms = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (j < nvc) {
+        cmt = fmaxf(cmt, __uint_as_float(rt[j]));
+        cms = fmaxf(cms, __uint_as_float(rs[j]));
+      }
+    }
+    const float nt = fmaxf(s.mt, cmt * kLog2e);
+    const float sct = ex2_approx(s.mt - nt);
+    float at = s.st * sct, aw = s.w * sct;
+    const float ns = fmaxf(s.ms, cms * kLog2e);
+    float as = s.ss * ex2_approx(s.ms - ns);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (j < nvc) {
+        const float zt = __uint_as_float(rt[j]), zs = __uint_as_float(rs[j]);
+        const float e = ex2_approx(fmaf(zt, kLog2e, -nt));
+        at += e;
+        aw = fmaf(e, zt - zs, aw);
+        as += ex2_approx(fmaf(zs, kLog2e, -ns));
+      }
+    }
+    s.mt = nt;
+    s.st = at;
+    s.w = aw;
+    s.ms = ns;
+    s.ss = as;
+  }
+}
+
+// Each 256-id tile is a pair of N = 256 products (teacher, then student),
+// one per accumulator, so the pair's epilogue waits for both and does not
+// overlap the next pair's MMAs.  (Two N = 128 products per 128-id tile from
+// one staged head tile, which do overlap, measured slower here on one CTA
+// and on CTA pairs alike: this epilogue is light, and N = 128 MMAs do half
+// the work per instruction.)
+struct KLFwdPolicy {
   using Params = KLFwdParams;
   static constexpr int EXTRA_SMEM = 0;
-  static constexpr int TN = DUAL ? BN / 2 : BN;  // vocabulary ids per tile
+  static constexpr int TN = BN;  // vocabulary ids per tile
   static __device__ __forceinline__ bool active(const Params&) { return true; }
 
   template <class F>
@@ -70,107 +132,40 @@ struct KLFwdPolicyT {
   static __device__ void prefetch(const Params& p) {
     tma_prefetch_map(&p.mapAs);
     tma_prefetch_map(&p.mapAt);
-    if constexpr (DUAL) {
-      tma_prefetch_map(&p.mapB128);
-    } else {
-      tma_prefetch_map(&p.mapBs);
-      tma_prefetch_map(&p.mapBt);
-    }
+    tma_prefetch_map(&p.mapBs);
+    tma_prefetch_map(&p.mapBt);
   }
 
   static __device__ void producer(const Params& p, Engine& eng) {
     schedule(p, [&](int mb, int, int t, bool, int) {
-      if constexpr (DUAL)
-        return eng.produce_dual(&p.mapAt, &p.mapAs, &p.mapB128, mb * BM, t * TN, p.nkb);
-      else
-        return eng.produce<false, false>(&p.mapAt, &p.mapBt, 0, mb * BM, 0, t * BN, p.nkb) &&
-               eng.produce<false, false>(&p.mapAs, &p.mapBs, 0, mb * BM, 0, t * BN, p.nkb);
+      return eng.produce<false, false>(&p.mapAt, &p.mapBt, 0, mb * BM, 0, t * BN, p.nkb) &&
+             eng.produce<false, false>(&p.mapAs, &p.mapBs, 0, mb * BM, 0, t * BN, p.nkb);
     });
   }
 
   static __device__ void mma(const Params& p, Engine& eng) {
     schedule(p, [&](int, int, int, bool, int) {
-      if constexpr (DUAL)
-        return eng.mma_dual(p.nkb);
-      else
-        return eng.mma<false, false>(p.nkb) && eng.mma<false, false>(p.nkb);
+      return eng.mma<false, false>(p.nkb) && eng.mma<false, false>(p.nkb);
     });
   }
 
   static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
     const int row = q * 32 + lane;
-    float mt = -INFINITY, st = 0.f, w = 0.f;  // teacher (log2 max, sum, weighted z_t - z_s)
-    float ms = -INFINITY, ss = 0.f;           // student
+    KLRowState st;
+    st.reset();
     schedule(p, [&](int mb, int split, int t, bool last, int nv) {
       uint32_t ta, tb;
-      if constexpr (DUAL) {
-        if (!eng.epi_acquire(q, ta)) return false;
-        tb = ta + TN;  // student columns follow the teacher's in the same accumulator
-      } else {
-        if (!eng.epi_acquire2(q, ta, tb)) return false;
-      }
-      const int valid = min(TN, p.V - t * TN);
-      const bool row_ok = mb * BM + row < nv;
-      for (int c = 0; c < TN / 32; ++c) {
-        if (c * 32 >= valid) break;  // uniform over the CTA
-        const int nvc = min(32, valid - c * 32);
-        uint32_t rt[32], rs[32];
-        tmem_ld32(ta + c * 32, rt);
-        tmem_ld32(tb + c * 32, rs);
-        float cmt = -INFINITY, cms = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (j < nvc) {
-            cmt = fmaxf(cmt, __uint_as_float(rt[j]));
-            cms = fmaxf(cms, __uint_as_float(rs[j]));
-          }
-        }
-        const float nt = fmaxf(mt, cmt * kLog2e);
-        const float sct = ex2_approx(mt - nt);
-        float at = st * sct, aw = w * sct;
-        const float ns = fmaxf(ms, cms * kLog2e);
-        float as = ss * ex2_approx(ms - ns);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (j < nvc) {
-            const float zt = __uint_as_float(rt[j]), zs = __uint_as_float(rs[j]);
-            const float e = ex2_approx(fmaf(zt, kLog2e, -nt));
-            at += e;
-            aw = fmaf(e, zt - zs, aw);
-            as += ex2_approx(fmaf(zs, kLog2e, -ns));
-          }
-        }
-        mt = nt;
-        st = at;
-        w = aw;
-        ms = ns;
-        ss = as;
-      }
-      if constexpr (DUAL)
-        eng.epi_release(lane);
-      else
-        eng.epi_release2(lane);
+      if (!eng.epi_acquire2(q, ta, tb)) return false;
+      kl_fwd_tile<BN>(ta, tb, min(BN, p.V - t * BN), st);
+      eng.epi_release2(lane);
       if (last) {
-        if (row_ok) {
-          float* o = p.part + (size_t)split * 5 * p.Npad + mb * BM + row;
-          o[0] = mt;
-          o[(size_t)p.Npad] = st;
-          o[(size_t)2 * p.Npad] = w;
-          o[(size_t)3 * p.Npad] = ms;
-          o[(size_t)4 * p.Npad] = ss;
-        }
-        mt = -INFINITY;
-        st = 0.f;
-        w = 0.f;
-        ms = -INFINITY;
-        ss = 0.f;
+        if (mb * BM + row < nv) st.store(p, split, mb * BM + row);
+        st.reset();
       }
       return true;
     });
   }
 };
-using KLFwdPolicy = KLFwdPolicyT<false>;
-using KLFwdDualPolicy = KLFwdPolicyT<true>;
 
 // Splits combined per row (one warp per original row): KL = A - lse_t +
 // lse_s with A = w / s_t after both are rescaled to the teacher's overall
