@@ -29,10 +29,6 @@
 //           back to the original rows.
 #pragma once
 
-#ifndef CCE_DE_PAIR_STAGES
-#define CCE_DE_PAIR_STAGES 6
-#endif
-
 #include <cub/block/block_scan.cuh>
 
 #include "cce_engine.cuh"
@@ -841,10 +837,6 @@ struct DEPolicyT {
   using Params = DEParams;
   static constexpr int EXTRA_SMEM = 0;
   static constexpr int ROWS = PAIR ? 2 * BM : BM;  // vocabulary rows per tile
-  // on CTA pairs: the default 32 KiB stages, CCE_DE_PAIR_STAGES deep (this
-  // epilogue needs no shared memory, so a seventh stage fits)
-  static constexpr int PAIR_NST = CCE_DE_PAIR_STAGES;
-  static constexpr int PAIR_SB = PSTAGE_BYTES;
   // a chunk taken by the sparse route has no dense work
   static __device__ __forceinline__ bool active(const Params& p) {
     return !(p.nz_cnt && *p.nz_cnt <= p.nz_cap);
