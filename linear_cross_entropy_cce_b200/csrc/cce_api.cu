@@ -459,6 +459,12 @@ int launch_tc_pair(const typename Policy::Params& prm, int pairs, cudaStream_t s
 #define CCE_PAIR_DEDH 1
 #endif
 constexpr bool kPairDEDH = CCE_PAIR_DEDH != 0;
+// The cross-entropy G producer runs on CTA pairs (256 x 256 tiles) unless
+// built with CCE_PAIR_G=0.
+#ifndef CCE_PAIR_G
+#define CCE_PAIR_G 1
+#endif
+constexpr bool kPairG = CCE_PAIR_G != 0;
 
 // Brackets a plain kernel launch of class `cls` with timing events (when
 // that class is being timed); use as  { TimedLaunch t(cls, st); k<<<..>>>(); }
@@ -862,6 +868,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   // soft-target KL with one head for student and teacher: dual 128-id
   // tiles on CTA pairs (GPolicyKLPair)
   const bool kl_pair = kl != nullptr && kl->Et == E;
+  const bool pair_g = kPairG && kl == nullptr;  // cross-entropy G on CTA pairs
   if (kl) {
     if (!make_map(&gp.mapA2, Ht_c, D, pl.Npad, D, BK, BM)) return CCE_ELAUNCH;
     if (!make_map(&gp.mapB2, kl->Et, D, V, D, BK, BN)) return CCE_ELAUNCH;
@@ -911,7 +918,9 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
     const int s = chunks[chunk].s, c0 = chunks[chunk].c0, cv = chunks[chunk].cv;
     const int ns = table.s[s].n;
     const int* perm_seg = vocab_perm ? vocab_perm + table.s[s].live_off : nullptr;
-    CUtensorMap segK, segMN;
+    // segKhalf: the head rows one CTA of a pair stages, 128 of a cross-entropy
+    // tile's 256 or 64 of a KL dual tile's 128
+    CUtensorMap segK, segMN, segKhalf;
     int row0 = c0;
     if (perm_seg) {
       if (side) {
@@ -934,10 +943,16 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       const __nv_bfloat16* Eb = Ecb[side ? (chunk & 1) : 0];
       if (!make_map(&segK, Eb, D, cv, D, BK, BN)) return CCE_ELAUNCH;
       if (!make_map(&segMN, Eb, D, cv, D, 64, 64)) return CCE_ELAUNCH;
+      if ((pair_g || kl_pair) &&
+          !make_map(&segKhalf, Eb, D, cv, D, BK, kl_pair ? BN / 4 : BN / 2))
+        return CCE_ELAUNCH;
       row0 = 0;
     } else {
       if (!make_map(&segK, sg.s[s].E, D, ns, D, BK, BN)) return CCE_ELAUNCH;
       if (!make_map(&segMN, sg.s[s].E, D, ns, D, 64, 64)) return CCE_ELAUNCH;
+      if ((pair_g || kl_pair) &&
+          !make_map(&segKhalf, sg.s[s].E, D, ns, D, BK, kl_pair ? BN / 4 : BN / 2))
+        return CCE_ELAUNCH;
     }
       // step 1: G for this chunk, with its zero-slice masks
       uint32_t* dh_mask = masks + (size_t)(chunk & 1) * mask_stride;
@@ -953,8 +968,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       gp.b_row0 = row0;
       gp.chunk_valid = cv;
       gp.ct = (int)cdiv(cv, kl_pair ? BN / 2 : BN);
-      // this CTA's 64 of a dual tile's 128 head rows
-      if (kl_pair && !make_map(&gp.mapBdual, sg.s[s].E, D, ns, D, BK, BN / 4)) return CCE_ELAUNCH;
+      if (pair_g || kl_pair) gp.mapBdual = segKhalf;
       gp.seg = s;
       gp.c0 = c0;
       gp.Vc = Vc;
@@ -987,10 +1001,13 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       const int g_grid = (int)std::min<int64_t>(sms, (int64_t)mbs * gp.ct);
       const int g_pairs = (int)std::min<int64_t>(sms / 2, cdiv(mbs, 2) * gp.ct);
       auto launch_g = [&]() {
-        return kl_pair ? launch_tc_pair<GPolicyKLPair>(gp, g_pairs, st, KC_G)
-               : kl    ? launch_tc<GPolicyKL>(gp, g_grid, st, KC_G)
-               : full_de ? launch_tc<GPolicyFull>(gp, g_grid, st, KC_G)
-                         : launch_tc<GPolicy>(gp, g_grid, st, KC_G);
+        if (kl_pair) return launch_tc_pair<GPolicyKLPair>(gp, g_pairs, st, KC_G);
+        if (kl) return launch_tc<GPolicyKL>(gp, g_grid, st, KC_G);
+        if (full_de)
+          return pair_g ? launch_tc_pair<GPolicyFullPair>(gp, g_pairs, st, KC_G)
+                        : launch_tc<GPolicyFull>(gp, g_grid, st, KC_G);
+        return pair_g ? launch_tc_pair<GPolicyPair>(gp, g_pairs, st, KC_G)
+                      : launch_tc<GPolicy>(gp, g_grid, st, KC_G);
       };
       if (int rc = launch_g()) return rc;
       if (sparse) {  // recompute with the dense fallback if the chunk was mispredicted

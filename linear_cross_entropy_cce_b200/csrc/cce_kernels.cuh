@@ -493,8 +493,9 @@ struct GParams {
   // an entry kept when either probability reaches the threshold.
   CUtensorMap mapA2;  // H_t,c [Npad, D], box {64, 128}
   CUtensorMap mapB2;  // E_t rows, K-major, box {64, 256}
-  // shared head rows, K-major, for dual tiles: box {64, 128} on one CTA,
-  // {64, 64} per CTA of a pair
+  // head rows, K-major, as one CTA of a pair stages them: box {64, 128}
+  // (cross-entropy, half a 256-id tile) or {64, 64} (KL dual tiles, half a
+  // 128-id tile)
   CUtensorMap mapBdual;
   const float* lt2_c;
   // optional per-element keep bits of original rows < debug_rows
@@ -510,20 +511,24 @@ struct GParams {
 // KL (separate heads): each 256-id tile is a teacher and a student N = 256
 // product, one per accumulator, so a tile's epilogue waits for both and does
 // not overlap the next tile's MMAs.
-// KL && PAIR (one head shared by student and teacher): on CTA pairs
-// (tc_pair_kernel), each 128-id tile is two M = 256, N = 128 products from
-// one staged head tile (PairEngineT::produce_dual) in one accumulator
-// (teacher columns 0..127, student 128..255), so the two accumulators
-// alternate and the epilogue overlaps the next tile's MMAs.  Work unit mbu is
-// then a pair of row blocks, 2 mbu (rank 0) and 2 mbu + 1 (rank 1).
+// PAIR: on CTA pairs (tc_pair_kernel); work unit mbu is a pair of row
+// blocks, 2 mbu (rank 0) and 2 mbu + 1 (rank 1), and each CTA keeps its own
+// 128 accumulator rows.  Cross-entropy: 256 x 256 tiles, M = 256 products,
+// each CTA staging 128 of the tile's 256 head rows.  KL && PAIR (one head
+// shared by student and teacher): each 128-id tile is two M = 256, N = 128
+// products from one staged head tile (PairEngineT::produce_dual) in one
+// accumulator (teacher columns 0..127, student 128..255), so the two
+// accumulators alternate and the epilogue overlaps the next tile's MMAs.
 template <bool FULL, bool KL = false, bool PAIR = false>
 struct GPolicyT {
-  static_assert(!PAIR || (KL && !FULL), "CTA pairs serve the shared-head KL producer");
+  static_assert(!(KL && FULL), "the KL producer has no unfiltered classifier gradient");
   using Params = GParams;
+  static constexpr bool DUALT = PAIR && KL;  // dual 128-id tiles
   static constexpr int EXTRA_SMEM = 0;
-  static constexpr int TN = PAIR ? BN / 2 : BN;  // vocabulary ids per tile
-  static constexpr int PAIR_NST = PAIR_DUAL_STAGES;  // stage geometry on CTA pairs
-  static constexpr int PAIR_SB = PDUAL_STAGE_BYTES;
+  static constexpr int TN = DUALT ? BN / 2 : BN;  // vocabulary ids per tile
+  // stage geometry on CTA pairs
+  static constexpr int PAIR_NST = DUALT ? PAIR_DUAL_STAGES : PAIR_STAGES;
+  static constexpr int PAIR_SB = DUALT ? PDUAL_STAGE_BYTES : PSTAGE_BYTES;
 
   // Whether this launch writes the dense fallback (slab + masks), and
   // whether it runs at all (a repair launch usually has nothing to do).
@@ -534,10 +539,19 @@ struct GPolicyT {
   static __device__ __forceinline__ bool active(const Params& p) {
     return !p.repair || (*p.nz_cnt > p.nz_cap && *p.slab_flag == 0);
   }
-  // (no tile skip on CTA pairs: the KL producer never skips)
-  static __device__ __forceinline__ bool skip(const Params& p, int mb, int vt) {
-    if constexpr (PAIR) return false;
-    return p.tile_cmax2 != nullptr && p.tile_cmax2[vt] - p.blk_lse2min[mb] < p.skip_l2;
+  // Exact tile skip of work unit (mbu, vt): every row block of the unit is
+  // below the bound (on CTA pairs both blocks, or the one that exists).
+  // Producer, MMA issuer and epilogue (of both CTAs) decide alike.
+  static __device__ __forceinline__ bool skip(const Params& p, int mbu, int vt, int nv) {
+    if (p.tile_cmax2 == nullptr) return false;
+    float m;
+    if constexpr (PAIR) {
+      m = p.blk_lse2min[2 * mbu];
+      if (2 * mbu + 1 < (nv + BM - 1) / BM) m = fminf(m, p.blk_lse2min[2 * mbu + 1]);
+    } else {
+      m = p.blk_lse2min[mbu];
+    }
+    return p.tile_cmax2[vt] - m < p.skip_l2;
   }
 
   // f(mbu, vt, nv) for this CTA's (or CTA pair's) work units: mbu a row
@@ -561,19 +575,24 @@ struct GPolicyT {
   }
   static __device__ void prefetch(const Params& p) {
     tma_prefetch_map(&p.mapA);
-    tma_prefetch_map(&p.mapB);
+    tma_prefetch_map(PAIR ? &p.mapBdual : &p.mapB);
     if constexpr (KL) {
       tma_prefetch_map(&p.mapA2);
-      tma_prefetch_map(PAIR ? &p.mapBdual : &p.mapB2);
+      if constexpr (!PAIR) tma_prefetch_map(&p.mapB2);
     }
   }
   template <class Eng>
   static __device__ void producer(const Params& p, Eng& eng) {
-    schedule(p, [&](int mb, int vt, int) {
-      if (skip(p, mb, vt)) return true;
-      if constexpr (PAIR) {  // this CTA's 128 rows of each, 64 of the tile's head rows
+    schedule(p, [&](int mb, int vt, int nv) {
+      if (skip(p, mb, vt, nv)) return true;
+      if constexpr (DUALT) {  // this CTA's 128 rows of each, 64 of the tile's head rows
         return eng.produce_dual(&p.mapA2, &p.mapA, &p.mapBdual, (2 * mb + (int)eng.rank) * BM,
                                 p.b_row0 + vt * TN + (int)eng.rank * (TN / 2), p.nkb);
+      } else if constexpr (PAIR) {  // this CTA's 128 rows, 128 of the tile's head rows
+        return eng.template produce<false, false>(&p.mapA, &p.mapBdual, 0,
+                                                  (2 * mb + (int)eng.rank) * BM, 0,
+                                                  p.b_row0 + vt * BN + (int)eng.rank * (BN / 2),
+                                                  p.nkb);
       } else {
         if constexpr (KL) {  // teacher tile first: it lands in the even accumulator
           if (!eng.template produce<false, false>(&p.mapA2, &p.mapB2, 0, mb * BM, 0,
@@ -587,9 +606,9 @@ struct GPolicyT {
   }
   template <class Eng>
   static __device__ void mma(const Params& p, Eng& eng) {
-    schedule(p, [&](int mb, int vt, int) {
-      if (skip(p, mb, vt)) return true;
-      if constexpr (PAIR) {
+    schedule(p, [&](int mb, int vt, int nv) {
+      if (skip(p, mb, vt, nv)) return true;
+      if constexpr (DUALT) {
         return eng.mma_dual(p.nkb);
       } else {
         if constexpr (KL) {
@@ -621,10 +640,10 @@ struct GPolicyT {
       // rows are outside the slab and carry no entries
       const bool blk_live = !PAIR || mb * BM < nv;
       // a skipped tile has no accumulator: no softmax entry is kept in it
-      const bool sk = skip(p, mb, vt);
+      const bool sk = skip(p, mbu, vt, nv);
       uint32_t taddr = 0, tteach = 0;
       if (!sk) {
-        if constexpr (PAIR) {
+        if constexpr (DUALT) {
           if (!eng.epi_acquire(q, tteach)) return false;
           taddr = tteach + TN;  // student columns after the teacher's
         } else if constexpr (KL) {
@@ -793,6 +812,8 @@ struct GPolicyT {
 using GPolicy = GPolicyT<false>;
 using GPolicyFull = GPolicyT<true>;
 using GPolicyKL = GPolicyT<false, true>;
+using GPolicyPair = GPolicyT<false, false, true>;
+using GPolicyFullPair = GPolicyT<true, false, true>;
 using GPolicyKLPair = GPolicyT<false, true, true>;
 
 // =====================================================================
