@@ -214,7 +214,7 @@ __global__ void gather_perm_rows_kernel(const __nv_bfloat16* __restrict__ src,
 // =====================================================================
 struct FwdParams {
   CUtensorMap mapA;            // H_c [Npad, D] bf16, box {64, 128}
-  CUtensorMap mapB[MAX_SEGS];  // E_s [n_s, D] bf16, box {64, 256}
+  CUtensorMap mapB[MAX_SEGS];  // E_s [n_s, D] bf16, box {64, 256} ({64, 128} on CTA pairs)
   SegTable segs;
   int T_v;     // total vocabulary tiles
   int tpi;     // tiles per work item
@@ -227,7 +227,12 @@ struct FwdParams {
   int* status;
 };
 
-struct FwdPolicy {
+// PAIR: on CTA pairs (tc_pair_kernel), 256 x 256 tiles as M = 256 products;
+// work unit mbu is a pair of row blocks, 2 mbu (rank 0) and 2 mbu + 1
+// (rank 1), and each CTA stages its 128 rows and 128 of the tile's 256 head
+// rows and keeps its own 128 accumulator rows.
+template <bool PAIR>
+struct FwdPolicyT {
   using Params = FwdParams;
   static constexpr int EXTRA_SMEM = 0;
   static __device__ __forceinline__ bool active(const Params&) { return true; }
@@ -235,18 +240,21 @@ struct FwdPolicy {
   template <class F>
   static __device__ __forceinline__ void schedule(const Params& p, F&& f) {
     const int nv = *p.n_valid;
-    const int num_mb = (nv + BM - 1) / BM;
-    const int num_items = num_mb * p.S;
-    const int gm = row_group_blocks(num_mb, (long long)BM * BK * 2 * p.nkb);
-    for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
-      int mb, split;
-      grouped_item(item, num_mb, p.S, gm, mb, split);
+    const int rows_u = PAIR ? 2 * BM : BM;  // rows per work unit
+    const int num_u = (nv + rows_u - 1) / rows_u;
+    const int num_items = num_u * p.S;
+    const int gm = row_group_blocks(num_u, (long long)rows_u * BK * 2 * p.nkb);
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    for (int item = unit; item < num_items; item += units) {
+      int mbu, split;
+      grouped_item(item, num_u, p.S, gm, mbu, split);
       const int t0 = split * p.tpi;
       const int t1 = min(p.T_v, t0 + p.tpi);
       int s = 0;
       for (int t = t0; t < t1; ++t) {
         while (s + 1 < p.segs.n_segs && t >= p.segs.s[s + 1].tile_off) ++s;
-        if (!f(mb, split, t, s, t == t1 - 1, nv)) return;
+        if (!f(mbu, split, t, s, t == t1 - 1, nv)) return;
       }
     }
   }
@@ -256,21 +264,34 @@ struct FwdPolicy {
     for (int s = 0; s < p.segs.n_segs; ++s) tma_prefetch_map(&p.mapB[s]);
   }
 
-  static __device__ void producer(const Params& p, Engine& eng) {
+  template <class Eng>
+  static __device__ void producer(const Params& p, Eng& eng) {
     schedule(p, [&](int mb, int, int t, int s, bool, int) {
-      return eng.produce<false, false>(&p.mapA, &p.mapB[s], 0, mb * BM, 0,
-                                       (t - p.segs.s[s].tile_off) * BN, p.nkb);
+      if constexpr (PAIR)
+        return eng.template produce<false, false>(
+            &p.mapA, &p.mapB[s], 0, (2 * mb + (int)eng.rank) * BM, 0,
+            (t - p.segs.s[s].tile_off) * BN + (int)eng.rank * (BN / 2), p.nkb);
+      else
+        return eng.template produce<false, false>(&p.mapA, &p.mapB[s], 0, mb * BM, 0,
+                                                  (t - p.segs.s[s].tile_off) * BN, p.nkb);
     });
   }
 
-  static __device__ void mma(const Params& p, Engine& eng) {
-    schedule(p, [&](int, int, int, int, bool, int) { return eng.mma<false, false>(p.nkb); });
+  template <class Eng>
+  static __device__ void mma(const Params& p, Eng& eng) {
+    schedule(p, [&](int, int, int, int, bool, int) {
+      return eng.template mma<false, false>(p.nkb);
+    });
   }
 
-  static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
+  template <class Eng>
+  static __device__ void epilogue(const Params& p, Eng& eng, int q, int lane) {
     const int row = q * 32 + lane;
+    uint32_t rank = 0;
+    if constexpr (PAIR) rank = eng.rank;
     float m2 = -INFINITY, sum = 0.f;
-    schedule(p, [&](int mb, int split, int t, int s, bool last, int nv) {
+    schedule(p, [&](int mbu, int split, int t, int s, bool last, int nv) {
+      const int mb = PAIR ? 2 * mbu + (int)rank : mbu;  // this CTA's row block
       uint32_t taddr;
       if (!eng.epi_acquire(q, taddr)) return false;
       const SegDev& sg = p.segs.s[s];
@@ -316,6 +337,8 @@ struct FwdPolicy {
     });
   }
 };
+using FwdPolicy = FwdPolicyT<false>;
+using FwdPairPolicy = FwdPolicyT<true>;
 
 // log-add-exp of the split partials, the correct-token logit as an indexed
 // dot product in fp32, loss = lse - z_y.  One warp per original row.
