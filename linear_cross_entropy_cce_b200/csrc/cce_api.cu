@@ -42,6 +42,28 @@ constexpr int64_t kFilteredWidthMult = CCE_FILTERED_WIDTH_MULT;
 #endif
 constexpr bool kCapChunkToEighth = CCE_CAP_CHUNK_EIGHTH != 0;
 
+// The dE / dH contractions of unfiltered calls run on CTA pairs (256 x 256
+// tiles, tcgen05 cta_group::2) unless built with CCE_PAIR_DEDH=0.  Filtered
+// calls keep single-CTA tiles: their K steps are skipped when a 16-wide slice
+// of G is zero across the tile's rows (or columns), which happens less often
+// over 256 of them than over 128.
+#ifndef CCE_PAIR_DEDH
+#define CCE_PAIR_DEDH 1
+#endif
+constexpr bool kPairDEDH = CCE_PAIR_DEDH != 0;
+// The cross-entropy G producer runs on CTA pairs (256 x 256 tiles) unless
+// built with CCE_PAIR_G=0.
+#ifndef CCE_PAIR_G
+#define CCE_PAIR_G 1
+#endif
+constexpr bool kPairG = CCE_PAIR_G != 0;
+// The cross-entropy forward runs on CTA pairs (256 x 256 tiles) unless built
+// with CCE_PAIR_FWD=0.
+#ifndef CCE_PAIR_FWD
+#define CCE_PAIR_FWD 1
+#endif
+constexpr bool kPairFwd = CCE_PAIR_FWD != 0;
+
 size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -187,12 +209,33 @@ struct FwdPlan {
   size_t off_nvalid, off_idx, off_pos, off_hc, off_part, total;
 };
 
+// Vocabulary tiles per forward work item.  Enough items for load balance
+// (about 24 per SM), at most 16; and few enough that the E tiles the running
+// items stream stay within kFwdInflightBytes of L2: the CTAs (or CTA pairs)
+// running at once cover about slots / gm vocabulary splits (gm = work units
+// per row group, as the kernel's grouped order forms them), each streaming
+// its own tiles.  Longer items let the units that share a split drift
+// apart, and a tile the laggards need is then re-read from DRAM (on the
+// Llama-shaped head: 18.2 GB per forward at 16 tiles per item, 7.6 GB at 2).
+constexpr int64_t kFwdInflightBytes = 32ll << 20;
+int fwd_tiles_per_item(int64_t Npad, int64_t D, int64_t T_v, bool pair) {
+  const int64_t num_mb = Npad / BM;
+  const int64_t units = pair ? cdiv(num_mb, 2) : num_mb;
+  const int64_t slots = pair ? kPlanSMs / 2 : kPlanSMs;
+  const int64_t unit_bytes = (pair ? 2 * BM : BM) * cdiv(D, BK) * BK * 2;
+  const int64_t groups = std::max<int64_t>(1, cdiv(units * unit_bytes, (int64_t)kRowGroupBytes));
+  const int64_t gm = std::max<int64_t>(1, cdiv(units, groups));
+  const int64_t splits = std::max<int64_t>(1, cdiv(slots, gm));
+  const int64_t by_l2 = kFwdInflightBytes / (splits * (int64_t)BN * D * 2);
+  const int64_t by_balance = num_mb * T_v / (kPlanSMs * 24);
+  return (int)std::max<int64_t>(2, std::min<int64_t>({16, by_l2, by_balance}));
+}
+
 FwdPlan plan_fwd(int64_t N, int64_t D, int64_t V, int32_t n_segs) {
   FwdPlan p;
   p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
   p.T_v_max = (int)(cdiv(V, BN) + std::max(1, (int)n_segs));
-  const int64_t num_mb = p.Npad / BM;
-  p.tpi = (int)std::min<int64_t>(16, std::max<int64_t>(2, num_mb * p.T_v_max / (kPlanSMs * 24)));
+  p.tpi = fwd_tiles_per_item(p.Npad, D, p.T_v_max, kPairFwd);
   p.S_max = (int)cdiv(p.T_v_max, p.tpi);
   size_t o = 0;
   p.off_nvalid = o; o += align_up(16);
@@ -215,6 +258,9 @@ KLFwdPlan plan_kl_fwd(int64_t N, int64_t D, int64_t V) {
   KLFwdPlan p;
   p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
   p.T_v = (int)cdiv(V, BN);
+  // (the rule of fwd_tiles_per_item measured neutral here, at four times
+  // the partial buffer: 4 tiles per item instead of 16 on the 24,576 x
+  // 248,320 step)
   const int64_t num_mb = p.Npad / BM;
   p.tpi = (int)std::min<int64_t>(16, std::max<int64_t>(2, num_mb * p.T_v / (kPlanSMs * 24)));
   p.S = (int)cdiv(p.T_v, p.tpi);
@@ -450,27 +496,6 @@ int launch_tc_pair(const typename Policy::Params& prm, int pairs, cudaStream_t s
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? CCE_OK : CCE_ELAUNCH;
 }
 
-// The dE / dH contractions of unfiltered calls run on CTA pairs (256 x 256
-// tiles, tcgen05 cta_group::2) unless built with CCE_PAIR_DEDH=0.  Filtered
-// calls keep single-CTA tiles: their K steps are skipped when a 16-wide slice
-// of G is zero across the tile's rows (or columns), which happens less often
-// over 256 of them than over 128.
-#ifndef CCE_PAIR_DEDH
-#define CCE_PAIR_DEDH 1
-#endif
-constexpr bool kPairDEDH = CCE_PAIR_DEDH != 0;
-// The cross-entropy G producer runs on CTA pairs (256 x 256 tiles) unless
-// built with CCE_PAIR_G=0.
-#ifndef CCE_PAIR_G
-#define CCE_PAIR_G 1
-#endif
-constexpr bool kPairG = CCE_PAIR_G != 0;
-// The cross-entropy forward runs on CTA pairs (256 x 256 tiles) unless built
-// with CCE_PAIR_FWD=0.
-#ifndef CCE_PAIR_FWD
-#define CCE_PAIR_FWD 1
-#endif
-constexpr bool kPairFwd = CCE_PAIR_FWD != 0;
 
 // Brackets a plain kernel launch of class `cls` with timing events (when
 // that class is being timed); use as  { TimedLaunch t(cls, st); k<<<..>>>(); }
