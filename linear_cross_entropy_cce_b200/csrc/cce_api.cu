@@ -454,13 +454,30 @@ void timing_end(long slot, cudaStream_t st) {
   if (slot >= 0) cudaEventRecord(g_timing.pool[slot + 1], st);
 }
 
+// Raises a kernel's dynamic shared-memory limit once per device (the call
+// is not repeated per launch, so launches can be captured into CUDA graphs
+// without it).
+template <class Policy, bool PAIR, class K>
+bool smem_attribute_once(K k, int smem) {
+  constexpr int kMaxDev = 64;
+  // bit d: set on device d; one word per kernel (policy and launch shape)
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+  const uint64_t bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return false;
+  done.fetch_or(bit, std::memory_order_release);
+  return true;
+}
+
 template <class Policy>
 int launch_tc(const typename Policy::Params& prm, int grid, cudaStream_t st, int cls) {
   auto k = tc_kernel<Policy>;
   constexpr int smem = smem_bytes<Policy>();
   static_assert(smem <= 232448, "shared memory per CTA exceeds 227 KB");
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return CCE_ELAUNCH;
+  if (!smem_attribute_once<Policy, false>(k, smem)) return CCE_ELAUNCH;
   const long slot = timing_begin(cls, st);
   k<<<grid, THREADS, smem, st>>>(prm);
   timing_end(slot, st);
@@ -474,8 +491,7 @@ int launch_tc_pair(const typename Policy::Params& prm, int pairs, cudaStream_t s
   auto k = tc_pair_kernel<Policy>;
   constexpr int smem = pair_smem_bytes<Policy>();
   static_assert(smem <= 232448, "shared memory per CTA exceeds 227 KB");
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return CCE_ELAUNCH;
+  if (!smem_attribute_once<Policy, true>(k, smem)) return CCE_ELAUNCH;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(2 * pairs, 1, 1);
