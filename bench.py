@@ -306,6 +306,8 @@ def main():
     ap.add_argument("--kahan", action="store_true",
                     help="accumulate dE across steps with the Kahan-compensated bf16 path")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip the CUDA-graph replay timing of the step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     a = ap.parse_args()
@@ -459,6 +461,23 @@ def main():
     launches = cce.launch_count() - l0
     clocks = clk.summary()
 
+    # the same step captured once into a CUDA graph and replayed (no host
+    # launch work per step; supplementary to the eager value above)
+    graph = None
+    if not vocab and not a.no_graph:
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        for _ in range(3):
+            g.replay()
+        ms_graph = timed(g.replay, a.steps)
+        graph = {"ms_per_step": round(ms_graph, 3),
+                 "value": round(tokens_per_s(N, world, ms_graph), 1), "unit": UNIT,
+                 "note": "the same step captured once into a CUDA graph, replayed K times"}
+        del g
+        torch.cuda.synchronize(dev)
+
     # forward alone (context), then a per-kernel-class timing pass
     for _ in range(3):
         fwd_only()
@@ -571,6 +590,7 @@ def main():
         "gpu_launches_per_step": int(launches // max(1, a.steps)),
         "clocks": clocks,
         "e2e": e2e,
+        "graph": graph,
         "cpu_baseline": cpu,
     }
     if rank == 0:
