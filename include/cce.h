@@ -366,6 +366,16 @@ int cce_fwd_noalloc(const void* H, const void* E, const int32_t* y,
 int cce_debug_stall(uint64_t wait_ns, int32_t* status, void* stream);
 
 /*
+ * The same on one CTA pair of the cluster engine (tcgen05 cta_group::2):
+ * the pair's MMA issuer waits for a stage its producers never fill, both
+ * CTAs' epilogues wait for an accumulator that is never committed; each wait
+ * runs out after wait_ns, both CTAs abort, hold a fixed grace period, free
+ * the pair's tensor memory and return, and CCE_STATUS_TIMEOUT is OR-ed into
+ * *status.  Arguments and errors as for cce_debug_stall.
+ */
+int cce_debug_stall_pair(uint64_t wait_ns, int32_t* status, void* stream);
+
+/*
  * Diagnostics (not needed for computing anything).
  *
  * cce_launch_count: number of kernels libcce has enqueued in this process

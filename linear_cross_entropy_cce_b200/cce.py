@@ -26,7 +26,7 @@ EXPORTS = ("cce_version", "cce_strerror", "cce_fwd_workspace_size", "cce_fwd", "
            "cce_vocab_sort", "cce_launch_count", "cce_timing_enable", "cce_timing_read",
            "cce_kl_fwd_workspace_size", "cce_kl_fwd", "cce_kl_bwd_workspace_size", "cce_kl_bwd",
            "cce_vocab_combine", "cce_fwd_noalloc", "cce_debug_stall",
-           "cce_bwd_workspace_parts")
+           "cce_debug_stall_pair", "cce_bwd_workspace_parts")
 # kernel classes for cce_timing_enable / cce_timing_read
 KC_FWD, KC_G, KC_DE, KC_DH, KC_AUX, KC_SPARSE = 0, 1, 2, 3, 4, 5
 KC_NAMES = ("fwd_tile_stream", "bwd_g_producer", "bwd_dE_contraction", "bwd_dH_contraction", "aux",
@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
                                     vp, vp, vp]
     L.cce_debug_stall.restype = ctypes.c_int
     L.cce_debug_stall.argtypes = [ctypes.c_uint64, vp, vp]
+    L.cce_debug_stall_pair.restype = ctypes.c_int
+    L.cce_debug_stall_pair.argtypes = [ctypes.c_uint64, vp, vp]
     L.cce_launch_count.restype = ctypes.c_uint64
     L.cce_timing_enable.restype = ctypes.c_int
     L.cce_timing_enable.argtypes = [u32]
@@ -301,11 +303,13 @@ def check_status(status: torch.Tensor, what: str = "libcce"):
     return v
 
 
-def debug_stall(wait_ns: int, status: torch.Tensor):
-    """Run the bounded-wait diagnostic (see cce_debug_stall)."""
+def debug_stall(wait_ns: int, status: torch.Tensor, pair: bool = False):
+    """Run the bounded-wait diagnostic (see cce_debug_stall; pair=True:
+    cce_debug_stall_pair, on one CTA pair)."""
     _require_cuda(status)
-    _check(lib().cce_debug_stall(int(wait_ns), _ptr(status), _stream_ptr(status.device)),
-           "cce_debug_stall")
+    fn = lib().cce_debug_stall_pair if pair else lib().cce_debug_stall
+    _check(fn(int(wait_ns), _ptr(status), _stream_ptr(status.device)),
+           "cce_debug_stall_pair" if pair else "cce_debug_stall")
 
 
 def launch_count() -> int:

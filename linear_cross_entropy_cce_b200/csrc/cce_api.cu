@@ -1444,6 +1444,15 @@ int cce_debug_stall(uint64_t wait_ns, int32_t* status, void* stream) {
   return launch_tc<StallPolicy>(sp, 1, static_cast<cudaStream_t>(stream), KC_AUX);
 }
 
+int cce_debug_stall_pair(uint64_t wait_ns, int32_t* status, void* stream) {
+  if (!status || wait_ns == 0 || wait_ns > 1000000000ull) return CCE_EINVAL;
+  if (device_sms() <= 0) return CCE_EDEVICE;
+  StallParams sp;
+  sp.status = status;
+  sp.wait_ns = wait_ns;
+  return launch_tc_pair<StallPairPolicy>(sp, 1, static_cast<cudaStream_t>(stream), KC_AUX);
+}
+
 uint64_t cce_launch_count(void) { return g_launches.load(); }
 
 int cce_timing_enable(uint32_t class_mask) {

@@ -1238,6 +1238,30 @@ struct StallPolicy {
   }
 };
 
+// The same on a CTA pair (tc_pair_kernel): the rank-0 MMA issuer's wait for
+// a stage runs out, the epilogues of both CTAs wait for an accumulator that
+// is never committed until their own limits run out; both CTAs then take the
+// abort path of the pair kernel (grace period, cluster barriers, freeing the
+// pair's tensor memory).
+struct StallPairPolicy {
+  using Params = StallParams;
+  static constexpr int EXTRA_SMEM = 0;
+  static __device__ __forceinline__ bool active(const Params&) { return true; }
+  static __device__ __forceinline__ uint64_t wait_limit(const Params& p) { return p.wait_ns; }
+  static __device__ void prefetch(const Params&) {}
+  template <class Eng>
+  static __device__ void producer(const Params&, Eng&) {}  // never fills a stage
+  template <class Eng>
+  static __device__ void mma(const Params&, Eng& eng) {
+    eng.template mma<false, false>(1);
+  }
+  template <class Eng>
+  static __device__ void epilogue(const Params&, Eng& eng, int q, int) {
+    uint32_t taddr;
+    eng.epi_acquire(q, taddr);
+  }
+};
+
 // inv[perm[k]] = k for one segment (perm and inv point at the segment's
 // slice of the concatenated live vocabulary; entries are segment-local).
 __global__ void invert_perm_kernel(const int* __restrict__ perm, int n, int* __restrict__ inv) {

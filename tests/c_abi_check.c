@@ -54,6 +54,8 @@ int main(void) {
   CHECK(cce_vocab_combine(f, 0, y, 4, 10, -100, NULL, 0, f, f, NULL) == CCE_EINVAL);
   CHECK(cce_vocab_combine(NULL, 0, y, 0, 10, -100, NULL, 0, f, f, NULL) == CCE_EINVAL);
   CHECK(cce_debug_stall(0, st, NULL) == CCE_EINVAL);
+  CHECK(cce_debug_stall_pair(0, st, NULL) == CCE_EINVAL);
+  CHECK(cce_debug_stall_pair(1000, NULL, NULL) == CCE_EINVAL);
   /* an empty batch is a no-op */
   CHECK(cce_fwd(p, p, y, 0, 8, 10, -100, NULL, 0, f, f, NULL, p, 1u << 30, st, NULL) == CCE_OK);
 
