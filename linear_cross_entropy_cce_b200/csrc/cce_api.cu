@@ -42,11 +42,13 @@ constexpr int64_t kFilteredWidthMult = CCE_FILTERED_WIDTH_MULT;
 #endif
 constexpr bool kCapChunkToEighth = CCE_CAP_CHUNK_EIGHTH != 0;
 
-// The dE / dH contractions of unfiltered calls run on CTA pairs (256 x 256
+// The dE / dH contractions of cross-entropy calls run on CTA pairs (256 x 256
 // tiles, tcgen05 cta_group::2) unless built with CCE_PAIR_DEDH=0.  Filtered
-// calls keep single-CTA tiles: their K steps are skipped when a 16-wide slice
-// of G is zero across the tile's rows (or columns), which happens less often
-// over 256 of them than over 128.
+// soft-target KL calls keep single-CTA tiles: their K steps are skipped when
+// a 16-wide slice of G is zero across the tile's rows (or columns), which
+// happens less often over 256 of them than over 128 (the KL step's dE went
+// from 20 to 34 ms on pairs; the filtered Phi-shaped cross-entropy step, also
+// on the dense route, gained 2% on pairs).
 #ifndef CCE_PAIR_DEDH
 #define CCE_PAIR_DEDH 1
 #endif
@@ -849,7 +851,8 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   __nv_bfloat16* Ec = at<__nv_bfloat16>(workspace, pl.off_ec);
   // chunk width of this call: wider when filtering can take the sparse route
   const bool wide = filter_eps > 0.f && !kahan;
-  const bool pair_dedh = kPairDEDH && filter_eps <= 0.f;
+  // (the soft-target KL's filtered chunks keep single-CTA tiles: see kPairDEDH)
+  const bool pair_dedh = kPairDEDH && (filter_eps <= 0.f || kl == nullptr);
   // zero-slice masks only pay where G has zeros: filtered calls
   const bool use_masks = filter_eps > 0.f;
   const int Vc = (int)(wide ? pl.Vc_f : pl.Vc);
