@@ -272,7 +272,8 @@ KLFwdPlan plan_kl_fwd(int64_t N, int64_t D, int64_t V) {
   p.off_pos = o; o += align_up(sizeof(int) * (size_t)std::max<int64_t>(N, 1));
   p.off_hs = o; o += align_up((size_t)p.Npad * D * 2);
   p.off_ht = o; o += align_up((size_t)p.Npad * D * 2);
-  p.off_part = o; o += align_up((size_t)p.S * 5 * p.Npad * sizeof(float));
+  // partials per split (and per column half of the epilogue, see KLFwdPolicy)
+  p.off_part = o; o += align_up((size_t)p.S * kKLFwdHalves * 5 * p.Npad * sizeof(float));
   p.total = o;
   return p;
 }
@@ -481,7 +482,7 @@ int launch_tc(const typename Policy::Params& prm, int grid, cudaStream_t st, int
   static_assert(smem <= 232448, "shared memory per CTA exceeds 227 KB");
   if (!smem_attribute_once<Policy, false>(k, smem)) return CCE_ELAUNCH;
   const long slot = timing_begin(cls, st);
-  k<<<grid, THREADS, smem, st>>>(prm);
+  k<<<grid, tc_threads<Policy>(), smem, st>>>(prm);
   timing_end(slot, st);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? CCE_OK : CCE_ELAUNCH;
@@ -1309,7 +1310,7 @@ int cce_kl_fwd(const void* Hs, const void* Es, const void* Ht, const void* Et,
   fin.pos_of_row = cp.pos_of_row;
   fin.part = kp.part;
   fin.N = (int)N;
-  fin.S = pl.S;
+  fin.S = pl.S * kKLFwdHalves;
   fin.Npad = (int)pl.Npad;
   fin.kl = kl;
   fin.lse_s = lse_s;

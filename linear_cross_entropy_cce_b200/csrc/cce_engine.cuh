@@ -741,9 +741,25 @@ __device__ __forceinline__ uint64_t policy_wait_limit(const typename Policy::Par
     return kWaitLimitNs;
 }
 
+// Epilogue warps of a policy: Policy::EPI_WARPS (4 or 8) when it declares
+// it, else 4.  With 8, two warps share each TMEM lane quarter; the policy's
+// epilogue then takes a fifth argument, 0 or 1, saying which of them it is.
+template <class P, class = void>
+struct EpiWarps : std::integral_constant<int, 4> {};
+template <class P>
+struct EpiWarps<P, std::void_t<decltype(P::EPI_WARPS)>>
+    : std::integral_constant<int, P::EPI_WARPS> {};
+template <class Policy>
+constexpr int tc_threads() {
+  static_assert(EpiWarps<Policy>::value == 4 || EpiWarps<Policy>::value == 8,
+                "4 or 8 epilogue warps");
+  return 64 + 32 * EpiWarps<Policy>::value;
+}
+
 // The kernel body: set-up, role dispatch, drain, TMEM release.
 template <class Policy>
-__global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ typename Policy::Params p) {
+__global__ void __launch_bounds__(tc_threads<Policy>(), 1)
+    tc_kernel(const __grid_constant__ typename Policy::Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (base & 1023u)) & 1023u);
@@ -760,7 +776,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&ctl->tfull[a]), 1);
-      mbar_init(smem_u32(&ctl->tempty[a]), EPI_THREADS / 32);
+      mbar_init(smem_u32(&ctl->tempty[a]), EpiWarps<Policy>::value);
     }
     mbar_init(smem_u32(&ctl->drain), 1);
     ctl->abort = 0;
@@ -795,7 +811,10 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
       drain_wait(smem_u32(&ctl->drain), 0);
     }
   } else {
-    Policy::epilogue(p, eng, warp & 3, lane);
+    if constexpr (EpiWarps<Policy>::value == 8)
+      Policy::epilogue(p, eng, warp & 3, lane, (warp - 2) >> 2);
+    else
+      Policy::epilogue(p, eng, warp & 3, lane);
   }
   __syncthreads();
   if (warp == 0 && lane == 0 && ctl->abort) {

@@ -106,10 +106,21 @@ __device__ __forceinline__ void kl_fwd_tile(uint32_t ta, uint32_t tb, int valid,
 // one staged head tile, which do overlap, measured slower here on one CTA
 // and on CTA pairs alike: this epilogue is light, and N = 128 MMAs do half
 // the work per instruction.)
+// With CCE_KL_FWD_SPLIT_COLS (default 1) the epilogue has 8 warps, two per
+// TMEM lane quarter, each folding 128 of a tile's 256 columns: this epilogue
+// does not overlap the MMAs, so halving it shortens every tile.  The two
+// column halves keep separate partials (split index 2 s + half), which the
+// finalize combines like any other splits.
+#ifndef CCE_KL_FWD_SPLIT_COLS
+#define CCE_KL_FWD_SPLIT_COLS 1
+#endif
+constexpr int kKLFwdHalves = CCE_KL_FWD_SPLIT_COLS ? 2 : 1;
+
 struct KLFwdPolicy {
   using Params = KLFwdParams;
   static constexpr int EXTRA_SMEM = 0;
   static constexpr int TN = BN;  // vocabulary ids per tile
+  static constexpr int EPI_WARPS = 4 * kKLFwdHalves;
   static __device__ __forceinline__ bool active(const Params&) { return true; }
 
   template <class F>
@@ -149,17 +160,19 @@ struct KLFwdPolicy {
     });
   }
 
-  static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane) {
+  static __device__ void epilogue(const Params& p, Engine& eng, int q, int lane, int half = 0) {
+    constexpr int CW = BN / kKLFwdHalves;  // columns this warp folds
     const int row = q * 32 + lane;
     KLRowState st;
     st.reset();
     schedule(p, [&](int mb, int split, int t, bool last, int nv) {
       uint32_t ta, tb;
       if (!eng.epi_acquire2(q, ta, tb)) return false;
-      kl_fwd_tile<BN>(ta, tb, min(BN, p.V - t * BN), st);
+      // (nothing to fold when the tile's valid columns end before this half)
+      kl_fwd_tile<CW>(ta + half * CW, tb + half * CW, min(CW, p.V - t * BN - half * CW), st);
       eng.epi_release2(lane);
       if (last) {
-        if (mb * BM + row < nv) st.store(p, split, mb * BM + row);
+        if (mb * BM + row < nv) st.store(p, split * kKLFwdHalves + half, mb * BM + row);
         st.reset();
       }
       return true;
