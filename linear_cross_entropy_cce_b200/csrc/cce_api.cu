@@ -1192,8 +1192,11 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
       dr.fp32_out = fp32 ? 1 : 0;
       {
         TimedLaunch tl_(KC_SPARSE, st);
-        csr_rows_kernel<DERows><<<(int)std::min<int64_t>(cdiv(v_live, dr.range), gblocks), gthreads, 0,
-                                  st>>>(dr);
+        const int grid = (int)std::min<int64_t>(cdiv(v_live, dr.range), gblocks);
+        if (fp32)
+          csr_rows_kernel<DERows, true><<<grid, gthreads, 0, st>>>(dr);
+        else
+          csr_rows_kernel<DERows, false><<<grid, gthreads, 0, st>>>(dr);
       }
       if (launched()) return CCE_ELAUNCH;
     }
@@ -1219,8 +1222,11 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
   hr.vocab_perm = vocab_perm;
   {
     TimedLaunch tl_(KC_SPARSE, st);
-    csr_rows_kernel<DHRows><<<(int)std::min<int64_t>(cdiv(pl.Npad, hr.range), gblocks), gthreads, 0,
-                              st>>>(hr);
+    const int grid = (int)std::min<int64_t>(cdiv(pl.Npad, hr.range), gblocks);
+    if (fp32_dh)
+      csr_rows_kernel<DHRows, true><<<grid, gthreads, 0, st>>>(hr);
+    else
+      csr_rows_kernel<DHRows, false><<<grid, gthreads, 0, st>>>(hr);
   }
   if (launched()) return CCE_ELAUNCH;
   {

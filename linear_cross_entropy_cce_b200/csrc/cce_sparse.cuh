@@ -183,6 +183,7 @@ struct DERows {
                     : (void*)(static_cast<__nv_bfloat16*>(dE[s]) + row * D);
   }
   __device__ const float* addend(long long) const { return nullptr; }
+  static constexpr bool kAddend = false;  // rows start from zero
 };
 
 // dH rows of the valid (compact) rows j: dH_acc row j (when some chunk took
@@ -215,9 +216,11 @@ struct DHRows {
                     : (void*)(static_cast<__nv_bfloat16*>(dH) + i * D);
   }
   __device__ const float* addend(long long j) const { return dH_acc + (size_t)j * D; }
+  static constexpr bool kAddend = true;  // dH_acc, when some chunk was dense
 };
 
-template <class R>
+// FP32: the output rows are fp32 (else bf16), fixed per launch.
+template <class R, bool FP32>
 __global__ void __launch_bounds__(GATHER_MAX_THREADS, 1) csr_rows_kernel(const R p) {
   __shared__ int sp[GATHER_RANGE + 1];
   __shared__ void* dst[GATHER_RANGE];
@@ -254,9 +257,12 @@ __global__ void __launch_bounds__(GATHER_MAX_THREADS, 1) csr_rows_kernel(const R
       const bool act = d < p.D;
       int cur = 0;  // row being accumulated
       float a[8];
+      bool touched = false;  // the current row has an entry (or an addend)
       auto start = [&](int r) {
-        const float* ad = add[r];
+        touched = false;
+        const float* ad = R::kAddend ? add[r] : nullptr;
         if (ad && act) {
+          touched = true;
           const float4 u = *reinterpret_cast<const float4*>(ad + d);
           const float4 v = *reinterpret_cast<const float4*>(ad + d + 4);
           a[0] = u.x; a[1] = u.y; a[2] = u.z; a[3] = u.w;
@@ -267,7 +273,16 @@ __global__ void __launch_bounds__(GATHER_MAX_THREADS, 1) csr_rows_kernel(const R
         }
       };
       auto finish = [&](int r) {
-        if (act && dst[r]) store_row8(dst[r], d, a, p.fp32_out);
+        if (!act || !dst[r]) return;
+        if (touched) {
+          store_row8(dst[r], d, a, FP32);
+        } else if (FP32) {  // an empty row: zeros, nothing to convert
+          float4* o = reinterpret_cast<float4*>(static_cast<float*>(dst[r]) + d);
+          o[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+          o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst[r]) + d) = make_uint4(0u, 0u, 0u, 0u);
+        }
       };
       start(0);
       for (int wb = E0; wb < E1; wb += GATHER_STAGE) {
@@ -298,6 +313,7 @@ __global__ void __launch_bounds__(GATHER_MAX_THREADS, 1) csr_rows_kernel(const R
               start(++cur);
             }
             fma8(a, stage[k + u].g, h[u]);
+            touched = true;
           }
         }
         for (; k < n; ++k) {
@@ -307,6 +323,7 @@ __global__ void __launch_bounds__(GATHER_MAX_THREADS, 1) csr_rows_kernel(const R
             start(++cur);
           }
           fma8(a, stage[k].g, __ldg(reinterpret_cast<const uint4*>(stage[k].src + d)));
+          touched = true;
         }
       }
       // the rows after the last entry (all of them if the range has none)

@@ -37,6 +37,9 @@ CASES = {
     "shared_head": dict(N=300, D=256, V=7001, std_s=2.0, std_t=2.0, shared=True, seed=2, masked=False),
     # peaky distributions: after filtering the sparse (CUDA-core) route runs
     "sparse": dict(N=700, D=192, V=30000, std_s=14.0, std_t=14.0, shared=True, seed=3, masked=True),
+    # 11 vocabulary tiles in splits of 2: the last split is one tile with 100
+    # valid ids, so the forward's second column half has an empty partial
+    "half_tail": dict(N=300, D=256, V=2660, std_s=3.0, std_t=3.0, shared=True, seed=5, masked=True),
 }
 
 
