@@ -304,7 +304,7 @@ size_t mask_bytes_for(int64_t Npad, int64_t vc) {
 int64_t list_cap(int64_t Npad, int64_t vc) { return std::max<int64_t>(4096, Npad * vc / 2048); }
 
 BwdPlan plan_bwd_widths(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl, int64_t cap_u,
-                        int64_t cap_f);
+                        int64_t cap_f, int nseg);
 
 // Among chunk widths w in [lo, hi] (multiples of 256), the one that needs the
 // fewest rounds of dE tiles over the whole vocabulary: chunks(w) x waves of
@@ -329,25 +329,26 @@ int64_t best_dE_width(int64_t V, int64_t D, int64_t lo, int64_t hi, int rows, in
 // sparse lists) take less than an eighth of the bf16 logits, N x V x 2 / 8,
 // and are then trimmed to the width below that cap whose dE contraction
 // wastes the least of its last waves.
-BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = false) {
-  BwdPlan p = plan_bwd_widths(N, D, V, flags, kl, INT64_MAX, INT64_MAX);
+// nseg: the head's segments (0: one segment); each adds at most one chunk.
+BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = false, int nseg = 0) {
+  BwdPlan p = plan_bwd_widths(N, D, V, flags, kl, INT64_MAX, INT64_MAX, nseg);
   const double bound = (double)N * (double)V * 2.0 / 8.0;
   // small problems are left alone: their scratch is a few MB whatever the
   // logits, and narrow chunks would only add launches
   if (!kCapChunkToEighth || bound < (double)(64u << 20)) return p;
   if ((double)p.part_logits < bound) return p;
   while ((double)p.part_logits >= bound && p.Vc_f > BN)
-    p = plan_bwd_widths(N, D, V, flags, kl, p.Vc_f - BN, p.Vc_f - BN);
+    p = plan_bwd_widths(N, D, V, flags, kl, p.Vc_f - BN, p.Vc_f - BN, nseg);
   // unfiltered calls run the dE contraction on CTA pairs (256-row tiles,
   // kPlanSMs / 2 at once), filtered ones on single CTAs (128-row tiles)
   const int64_t wu = best_dE_width(V, D, p.Vc / 2, p.Vc, 2 * BM, kPlanSMs / 2);
   const int64_t wf = best_dE_width(V, D, p.Vc_f / 2, p.Vc_f, BM, kPlanSMs);
-  return plan_bwd_widths(N, D, V, flags, kl, wu, wf);
+  return plan_bwd_widths(N, D, V, flags, kl, wu, wf, nseg);
 }
 
 // The plan with the unfiltered / filtered chunk widths at most cap_u / cap_f.
 BwdPlan plan_bwd_widths(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl, int64_t cap_u,
-                        int64_t cap_f) {
+                        int64_t cap_f, int nseg) {
   BwdPlan p;
   p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
   // Vocabulary chunk width: an L2-sized slab, widened so that the dE
@@ -402,9 +403,12 @@ BwdPlan plan_bwd_widths(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl
   p.off_masks = take(2 * align_up(p.mask_bytes), L);
   // sparse path: per chunk a list of up to cap(Vc) non-zeros (density 1/2048);
   // chunk count from the narrower width, list slots for whichever needs more
-  p.nch_max = cdiv(V, p.Vc) + CCE_MAX_SEGMENTS;
+  // chunks of one call: per segment ceil(n_s / width), at most ceil(V / width)
+  // plus one per segment
+  const int64_t extra = std::max(1, nseg);
+  p.nch_max = cdiv(V, p.Vc) + extra;
   const int64_t slots = std::max(p.nch_max * list_cap(p.Npad, p.Vc),
-                                 (cdiv(V, p.Vc_f) + CCE_MAX_SEGMENTS) * list_cap(p.Npad, p.Vc_f));
+                                 (cdiv(V, p.Vc_f) + extra) * list_cap(p.Npad, p.Vc_f));
   p.off_nzcnt = take(align_up(sizeof(int) * 2 * (size_t)p.nch_max), Vb);  // counts + slab flags
   p.off_lists = take(align_up(sizeof(NzEntry) * (size_t)slots), L);
   p.off_colc = take(align_up(sizeof(int) * 2 * (size_t)(V + 1)), Vb);  // counts, offsets
@@ -609,14 +613,14 @@ size_t cce_fwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs) {
 
 size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs, uint32_t flags) {
   if (!sizes_ok(N, D, V) || n_segs < 0 || n_segs > CCE_MAX_SEGMENTS) return 0;
-  return plan_bwd(N, D, V, flags).total;
+  return plan_bwd(N, D, V, flags, false, n_segs).total;
 }
 
 int cce_bwd_workspace_parts(int64_t N, int64_t D, int64_t V, int32_t n_segs, uint32_t flags,
                             size_t* rows, size_t* vocab, size_t* logits) {
   if (!sizes_ok(N, D, V) || n_segs < 0 || n_segs > CCE_MAX_SEGMENTS || !rows || !vocab || !logits)
     return CCE_EINVAL;
-  const BwdPlan p = plan_bwd(N, D, V, flags);
+  const BwdPlan p = plan_bwd(N, D, V, flags, false, n_segs);
   *rows = p.part_rows;
   *vocab = p.part_vocab;
   *logits = p.part_logits;
@@ -781,7 +785,7 @@ int bwd_impl(const void* H, const void* E, const int32_t* y, const float* lse, c
     return CCE_EINVAL;
   if (kl && (!kl->Ht || !kl->Et || !kl->lse_t || !aligned16(kl->Ht) || !aligned16(kl->Et)))
     return CCE_EINVAL;
-  const BwdPlan pl = plan_bwd(N, D, V, flags, kl != nullptr);
+  const BwdPlan pl = plan_bwd(N, D, V, flags, kl != nullptr, segs ? n_segs : 0);
   if (!workspace || workspace_bytes < pl.total) return CCE_EWORKSPACE;
   const int sms = device_sms();
   if (sms <= 0 || !encode_fn()) return CCE_EDEVICE;

@@ -114,6 +114,21 @@ def test_bwd_rejects_bad_flags_and_missing_kahan_buffer():
     assert call(dE=None) == cce.CCE_EINVAL
 
 
+def test_bwd_workspace_follows_the_segment_count():
+    # each segment may add one partial vocabulary chunk to the sparse lists,
+    # so the size grows with n_segs, and a call with more segments than the
+    # workspace was sized for is refused before anything reaches the device
+    L = cce.lib()
+    sizes = [cce.bwd_workspace_size(4, 8, 10, n) for n in (0, 1, 2, 8)]
+    assert sizes[0] == sizes[1] < sizes[2] < sizes[3]
+    seg = (cce.Segment * 2)()
+    seg[0].vocab_begin, seg[0].vocab_end, seg[0].E, seg[0].dE = 0, 6, 16, 16
+    seg[1].vocab_begin, seg[1].vocab_end, seg[1].E, seg[1].dE = 6, 10, 32, 32
+    rc = L.cce_bwd(16, None, 16, 16, 16, 4, 8, 10, -100, seg, 2, 0.0, None, None, 0,
+                   16, None, None, None, 0, 16, sizes[1], 16, None)
+    assert rc == cce.CCE_EWORKSPACE
+
+
 def test_vocab_combine_rejects_bad_arguments_on_host():
     L = cce.lib()
     EINVAL = cce.CCE_EINVAL
