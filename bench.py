@@ -121,15 +121,34 @@ def host_cores():
 
 
 # ------------------------------------------------------------------ oracle
-def oracle_sample(x, seconds: float, max_rows: int = 2048):
-    """Time the fp64 oracle (forward + backward) on a row sample; returns
-    (rows/s, rows, seconds, description)."""
+def grow_sample(run, n_max: int, seconds: float, r0: int, quantum: int):
+    """Size a CPU sample: time run(R) on growing R until one run takes at
+    least half of `seconds` (or R reaches n_max).  The oracle's fixed costs
+    per call (allocating and touching its full-vocabulary buffers) would make
+    a single small calibration run overstate the time per row.  Returns the
+    (R, seconds) of the last run."""
+    n_max = max(1, n_max)
+    R = min(r0, n_max)
+    while True:
+        t = run(R)
+        if t >= 0.5 * seconds or R >= n_max:
+            return R, t
+        nxt = int(min(n_max, max(2 * R, 0.9 * seconds / max(t, 1e-6) * R)))
+        if nxt < n_max:  # a multiple of the quantum, and always larger
+            nxt = max(R + 1, (nxt // quantum) * quantum)
+        R = nxt
+
+
+def oracle_runner(x):
+    """run(R): seconds of the fp64 oracle's forward + backward over R valid
+    rows of x spread evenly over the batch."""
     import oracle
     segs64 = [(b, e, oracle.widen_bf16(E)) for b, e, E in x.segments]
     valid = np.nonzero(x.valid)[0]
     dl = x.dloss_mean()
 
-    def run(rows):
+    def run(R):
+        rows = valid[np.linspace(0, len(valid) - 1, R).astype(np.int64)]
         Hs, ys, ds = x.H[rows], x.y[rows], dl[rows]
         t = time.perf_counter()
         oracle.forward(Hs, segs64, ys, x.wl.V, x.ignore_index)
@@ -137,15 +156,20 @@ def oracle_sample(x, seconds: float, max_rows: int = 2048):
                         filter_eps=EPS_BF16 if MODES.get(x.wl.name, (False,))[0] else 0.0)
         return time.perf_counter() - t
 
-    r0 = valid[:8]
-    t0 = run(r0)
-    R = int(min(max_rows, len(valid), max(8, seconds / max(t0, 1e-6) * len(r0))))
-    R = max(8, (R // 8) * 8)
-    rows = valid[np.linspace(0, len(valid) - 1, R).astype(np.int64)]
-    t = run(rows)
-    desc = (f"fp64 numpy oracle, forward+backward over {R} valid rows of {x.wl.name} "
+    return run, len(valid)
+
+
+def oracle_desc(x, R):
+    return (f"fp64 numpy oracle, forward+backward over {R} valid rows of {x.wl.name} "
             f"(N={x.wl.N}, D={x.wl.D}, V={x.wl.V}); full vocabulary and full dE per slice")
-    return R / t, R, t, desc
+
+
+def oracle_sample(x, seconds: float, max_rows: int = 2048):
+    """Time the fp64 oracle (forward + backward) on a row sample of about
+    `seconds`; returns (rows/s, rows, seconds, description)."""
+    run, n_valid = oracle_runner(x)
+    R, t = grow_sample(run, min(max_rows, n_valid), seconds, 8, 8)
+    return R / t, R, t, oracle_desc(x, R)
 
 
 # ------------------------------------------------------------------ clocks
@@ -604,26 +628,34 @@ def main():
 KL_METRIC = "soft-target KL fwd+bwd positions/s (and % of B200 bf16 tensor peak)"
 
 
-def kl_oracle_sample(wl, Hs, Ht, E, seconds: float, eps: float):
-    """Time the fp64 oracle's KL forward + backward on a row sample."""
+def kl_oracle_runner(wl, Hs, Ht, E, eps: float):
+    """run(R): seconds of the fp64 oracle's KL forward + backward over R rows
+    spread evenly over the batch."""
     import oracle
     E64 = oracle.widen_bf16(E)
     dl = np.full(wl.N, 1.0 / wl.N)
 
-    def run(rows):
+    def run(R):
+        rows = np.linspace(0, wl.N - 1, R).astype(np.int64)
         t = time.perf_counter()
         oracle.kl_forward(Hs[rows], E64, Ht[rows], E64)
         oracle.kl_backward(Hs[rows], E64, Ht[rows], E64, dl[rows], filter_eps=eps)
         return time.perf_counter() - t
 
-    r0 = np.arange(4)
-    t0 = run(r0)
-    R = int(min(1024, wl.N, max(4, seconds / max(t0, 1e-6) * 4)))
-    rows = np.linspace(0, wl.N - 1, R).astype(np.int64)
-    t = run(rows)
-    desc = (f"fp64 numpy oracle, KL forward+backward over {R} rows of {wl.name} "
+    return run
+
+
+def kl_oracle_desc(wl, R):
+    return (f"fp64 numpy oracle, KL forward+backward over {R} rows of {wl.name} "
             f"(N={wl.N}, D={wl.D}, V={wl.V}); full vocabulary and full dE per slice")
-    return R / t, R, t, desc
+
+
+def kl_oracle_sample(wl, Hs, Ht, E, seconds: float, eps: float):
+    """Time the fp64 oracle's KL forward + backward on a row sample of about
+    `seconds`; returns (rows/s, rows, seconds, description)."""
+    run = kl_oracle_runner(wl, Hs, Ht, E, eps)
+    R, t = grow_sample(run, min(1024, wl.N), seconds, 4, 4)
+    return R / t, R, t, kl_oracle_desc(wl, R)
 
 
 def kl_main(a, world, rank, local):
@@ -634,9 +666,13 @@ def kl_main(a, world, rank, local):
     if a.impl == "reference":
         if rank != 0:
             return
-        times, R = [], 0
+        # one sizing pass, then every step runs the same R rows
+        run = kl_oracle_runner(wl, Hs, Ht, E, eps)
+        R, _ = grow_sample(run, min(1024, wl.N), max(2.0, 120.0 / (a.steps + a.warmup)), 4, 4)
+        desc = kl_oracle_desc(wl, R)
+        times = []
         for i in range(a.warmup + a.steps):
-            rps, R, t, desc = kl_oracle_sample(wl, Hs, Ht, E, max(2.0, 120.0 / (a.steps + a.warmup)), eps)
+            t = run(R)
             if i >= a.warmup:
                 times.append(t)
         ms = 1e3 * float(np.mean(times))
@@ -773,11 +809,15 @@ def reference_arm(a, wl, world, rank, filt):
         return
     x = syn.make_inputs(wl, seed=0)
     per_step = max(2.0, 120.0 / max(1, a.steps + a.warmup))
-    times, R = [], 0
+    # one sizing pass, then every step runs the same R rows
+    run, n_valid = oracle_runner(x)
+    R, _ = grow_sample(run, min(2048, n_valid), per_step, 8, 8)
+    desc = oracle_desc(x, R)
+    times = []
     for i in range(a.warmup + a.steps):
-        rps, R, t, desc = oracle_sample(x, per_step)
+        t = run(R)
         if i >= a.warmup:
-            times.append(R / rps)
+            times.append(t)
     ms = 1e3 * float(np.mean(times))
     v = R / (ms / 1e3)
     out = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": UNIT,

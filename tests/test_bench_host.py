@@ -38,3 +38,28 @@ def test_warmup_below_three_is_rejected():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "2"],
                          capture_output=True, text=True, timeout=120, cwd=ROOT)
     assert out.returncode != 0
+
+
+def _bench_module():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_cpu_sample_grows_past_fixed_costs_and_stops():
+    grow = _bench_module().grow_sample
+    calls = []
+
+    def fixed_plus_rows(R):  # 1.5 s per call plus 8 ms per row
+        calls.append(R)
+        return 1.5 + 0.008 * R
+    R, t = grow(fixed_plus_rows, 2048, 15.0, 8, 8)
+    # one calibration run would have taken 8 rows' 1.56 s as the per-row cost
+    assert 7.5 <= t <= 15.0 and R % 8 == 0 and calls[-1] == R and calls == sorted(calls)
+    # a batch smaller than the target ends at all of its rows, quantum or not
+    calls.clear()
+    assert grow(lambda R: calls.append(R) or 1e-3 * R, 230, 2.0, 8, 8)[0] == 230
+    assert len(calls) <= 3
+    assert grow(lambda R: 1e-3 * R, 5, 2.0, 8, 8)[0] == 5
