@@ -130,8 +130,10 @@ def _seg_array(segments: Optional[Sequence], dEs=None, comps=None):
         return None, 0
     arr = (Segment * len(segments))()
     for k, s in enumerate(segments):
-        b, e, E = s[0], s[1], s[2]
-        arr[k].vocab_begin, arr[k].vocab_end, arr[k].E = int(b), int(e), E.data_ptr()
+        # (begin, end) ranges suffice where no head rows are read (vocab_sort)
+        b, e, E = s[0], s[1], (s[2] if len(s) > 2 else None)
+        arr[k].vocab_begin, arr[k].vocab_end = int(b), int(e)
+        arr[k].E = E.data_ptr() if E is not None else None
         arr[k].dE = dEs[k].data_ptr() if dEs is not None else None
         arr[k].dE_comp = comps[k].data_ptr() if comps is not None else None
     return arr, len(segments)
@@ -254,9 +256,11 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
 
 
 def vocab_sort(colmax: Optional[torch.Tensor], y: torch.Tensor, V: int, ignore_index: int = -100,
-               segments: Optional[Sequence[SegSpec]] = None,
+               segments: Optional[Sequence] = None,
                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Per-segment permutation of live vocabulary rows by descending key."""
+    """Per-segment permutation of live vocabulary rows by descending key.
+    `segments` are (begin, end) ranges, or the (begin, end, E_s) triples of
+    fwd / bwd (the head rows themselves are not read)."""
     dev = y.device
     v_live = sum(int(e) - int(b) for b, e, *_ in segments) if segments else V
     perm = torch.empty(v_live, dtype=torch.int32, device=dev)

@@ -1,0 +1,86 @@
+"""Seeded random combinations of shape and mode against the oracle.
+
+The parity suite pins each mode on hand-picked shapes; here every case draws
+its own N, D, V, segment layout (gaps before, between and after segments),
+logit scale, ignored fraction and backward mode (filter, vocabulary sort with
+the tile skip, FullC, fp32 gradients), so that modes meet shapes no
+hand-picked case combines.  Same acceptance tolerances as the parity suite.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_cross_entropy_cce_b200 import cce, synthetic as syn
+from _helpers import (EPS_BF16, TOL_GRAD, TOL_GRAD_FILTER, TOL_ROW, normwise, run_bwd, run_fwd,
+                      to_np, upload)
+
+pytestmark = pytest.mark.gpu
+
+N_CASES = 20
+
+
+def _draw(k):
+    rng = np.random.default_rng(5000 + k)
+    N = int(rng.integers(1, 641))
+    D = 8 * int(rng.integers(1, 65))
+    V = int(rng.integers(1, 12001))
+    nseg = int(rng.choice([1, 1, 2, 3])) if V >= 8 else 1
+    segments = ()
+    if nseg > 1 or rng.random() < 0.3:
+        # 2 nseg distinct cut points: segment s is [c[2s], c[2s+1]), so gaps
+        # fall before, between and after the segments
+        cuts = np.sort(rng.choice(np.arange(V + 1), size=2 * nseg, replace=False))
+        segments = tuple((int(cuts[2 * s]), int(cuts[2 * s + 1])) for s in range(nseg))
+    filt = bool(rng.random() < 0.6)
+    mode = {
+        "filter": filt,
+        "sort": filt and bool(rng.random() < 0.5),
+        "full_de": filt and bool(rng.random() < 0.3),
+        "fp32": bool(rng.random() < 0.25),
+    }
+    wl = syn.Workload(f"fuzz{k}", N=N, D=D, V=V,
+                      logit_std=float(rng.choice([0.5, 2.0, 6.0, 16.0])),
+                      ignore_frac=float(rng.choice([0.0, 0.1, 0.5, 1.0])),
+                      segments=segments,
+                      segment_mix=tuple(float(e - b) for b, e in segments) if segments else ())
+    return wl, mode
+
+
+def _close(got, ref, tol):
+    if not np.any(ref):
+        return np.max(np.abs(got), initial=0.0) <= 1e-6
+    return normwise(got, ref) <= tol
+
+
+@pytest.mark.parametrize("k", range(N_CASES))
+def test_random_case_matches_oracle(k):
+    wl, mode = _draw(k)
+    x = syn.make_inputs(wl, seed=k)
+    H, segs, y = upload(x)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run_fwd(x, H, segs, y, want_colmax=mode["sort"], status=st)
+    loss, lse = out[0], out[1]
+    kw = {}
+    if mode["sort"]:
+        colmax = out[2]
+        seg_arg = None if len(segs) == 1 and segs[0][:2] == (0, wl.V) else [s[:2] for s in segs]
+        kw["vocab_perm"] = cce.vocab_sort(colmax, y, wl.V, x.ignore_index, segments=seg_arg)
+        kw["colmax"] = colmax
+    eps = EPS_BF16 if mode["filter"] else 0.0
+    dl = x.dloss_mean()
+    dH, dEs, _ = run_bwd(x, H, segs, y, lse, torch.from_numpy(dl).cuda(), filter_eps=eps,
+                         full_de=mode["full_de"], fp32_grads=mode["fp32"], status=st, **kw)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, (wl, mode)
+
+    rl, rs = oracle.forward(x.H, x.segments, x.y, wl.V, x.ignore_index)
+    assert np.max(np.abs(to_np(loss) - rl), initial=0.0) <= TOL_ROW, (wl, mode)
+    assert np.max(np.abs(to_np(lse) - rs), initial=0.0) <= TOL_ROW, (wl, mode)
+    rH, rE = oracle.backward(x.H, x.segments, x.y, wl.V, dl, x.ignore_index, filter_eps=eps,
+                             filter_dE=not mode["full_de"])
+    tol = TOL_GRAD_FILTER if mode["filter"] else TOL_GRAD
+    assert _close(to_np(dH), rH, tol), (wl, mode, normwise(to_np(dH), rH))
+    for g, r in zip(dEs, rE):
+        assert _close(to_np(g), r, tol), (wl, mode, normwise(to_np(g), r))
+    assert np.all(to_np(dH)[~x.valid] == 0)
