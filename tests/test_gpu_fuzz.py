@@ -4,7 +4,9 @@ The parity suite pins each mode on hand-picked shapes; here every case draws
 its own N, D, V, segment layout (gaps before, between and after segments),
 logit scale, ignored fraction and backward mode (filter, vocabulary sort with
 the tile skip, FullC, fp32 gradients), so that modes meet shapes no
-hand-picked case combines.  Same acceptance tolerances as the parity suite.
+hand-picked case combines.  The soft-target KL cases draw shapes, the two
+logit scales, one or two heads, a row mask, the filter and fp32 gradients
+the same way.  Same acceptance tolerances as the parity suite.
 """
 import numpy as np
 import pytest
@@ -84,3 +86,54 @@ def test_random_case_matches_oracle(k):
     for g, r in zip(dEs, rE):
         assert _close(to_np(g), r, tol), (wl, mode, normwise(to_np(g), r))
     assert np.all(to_np(dH)[~x.valid] == 0)
+
+
+# ---- soft-target KL --------------------------------------------------------
+N_KL_CASES = 10
+
+
+def _draw_kl(k):
+    rng = np.random.default_rng(7000 + k)
+    N = int(rng.integers(1, 513))
+    D = 8 * int(rng.integers(1, 49))
+    V = int(rng.integers(2, 9001))
+    std_s, std_t = (float(v) for v in rng.choice([0.5, 2.0, 6.0, 14.0], size=2))
+    shared = bool(rng.random() < 0.5)
+    masked = bool(rng.random() < 0.5)
+    eps = EPS_BF16 if rng.random() < 0.6 else 0.0
+    fp32 = bool(rng.random() < 0.25)
+    return N, D, V, std_s, std_t, shared, masked, eps, fp32
+
+
+@pytest.mark.parametrize("k", range(N_KL_CASES))
+def test_random_kl_case_matches_oracle(k):
+    N, D, V, std_s, std_t, shared, masked, eps, fp32 = _draw_kl(k)
+    xs = syn.make_inputs(syn.Workload("kls", N=N, D=D, V=V, logit_std=std_s, ignore_frac=0.0),
+                         seed=k)
+    xt = syn.make_inputs(syn.Workload("klt", N=N, D=D, V=V, logit_std=std_t, ignore_frac=0.0),
+                         seed=k + 100)
+    Hs, Es, Ht = xs.H, xs.segments[0][2], xt.H
+    Et = Es if shared else xt.segments[0][2]
+    mask = (np.random.default_rng(k).random(N) > 0.3).astype(np.int32) if masked else None
+    up = lambda a: cce.bf16_from_bits(a, "cuda")
+    Hs_d, Es_d, Ht_d = up(Hs), up(Es), up(Ht)
+    Et_d = Es_d if shared else up(Et)
+    tm = torch.from_numpy(mask).cuda() if mask is not None else None
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kl, ls, lt = cce.kl_fwd(Hs_d, Es_d, Ht_d, Et_d, tm, status=st)
+    dl = np.linspace(0.2, 1.0, N) / N
+    dH, dE = cce.kl_bwd(Hs_d, Es_d, Ht_d, Et_d, ls, lt, torch.from_numpy(dl).float().cuda(), tm,
+                        filter_eps=eps, fp32_grads=fp32, status=st)
+    torch.cuda.synchronize()
+    case = (N, D, V, std_s, std_t, shared, masked, eps, fp32)
+    assert int(st.item()) == 0, case
+    rk, rls, rlt = oracle.kl_forward(Hs, Es, Ht, Et, mask)
+    assert np.max(np.abs(to_np(kl) - rk)) <= TOL_ROW, case
+    assert np.max(np.abs(to_np(ls) - rls)) <= TOL_ROW, case
+    assert np.max(np.abs(to_np(lt) - rlt)) <= TOL_ROW, case
+    rH, rE = oracle.kl_backward(Hs, Es, Ht, Et, dl, mask, filter_eps=eps)
+    tol = TOL_GRAD_FILTER if eps > 0 else TOL_GRAD
+    assert _close(to_np(dH), rH, tol), (case, normwise(to_np(dH), rH))
+    assert _close(to_np(dE), rE, tol), (case, normwise(to_np(dE), rE))
+    if mask is not None:
+        assert np.all(to_np(kl)[mask == 0] == 0) and np.all(to_np(dH)[mask == 0] == 0)
