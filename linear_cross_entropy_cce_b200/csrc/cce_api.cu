@@ -339,10 +339,12 @@ BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = fals
   if ((double)p.part_logits < bound) return p;
   while ((double)p.part_logits >= bound && p.Vc_f > BN)
     p = plan_bwd_widths(N, D, V, flags, kl, p.Vc_f - BN, p.Vc_f - BN, nseg);
-  // unfiltered calls run the dE contraction on CTA pairs (256-row tiles,
-  // kPlanSMs / 2 at once), filtered ones on single CTAs (128-row tiles)
+  // the dE contraction runs on CTA pairs (256-row tiles, kPlanSMs / 2 at
+  // once), except the soft-target KL's filtered chunks (single CTAs, 128-row
+  // tiles)
   const int64_t wu = best_dE_width(V, D, p.Vc / 2, p.Vc, 2 * BM, kPlanSMs / 2);
-  const int64_t wf = best_dE_width(V, D, p.Vc_f / 2, p.Vc_f, BM, kPlanSMs);
+  const int64_t wf = kl ? best_dE_width(V, D, p.Vc_f / 2, p.Vc_f, BM, kPlanSMs)
+                        : best_dE_width(V, D, p.Vc_f / 2, p.Vc_f, 2 * BM, kPlanSMs / 2);
   return plan_bwd_widths(N, D, V, flags, kl, wu, wf, nseg);
 }
 
