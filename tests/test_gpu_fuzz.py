@@ -137,3 +137,53 @@ def test_random_kl_case_matches_oracle(k):
     assert _close(to_np(dE), rE, tol), (case, normwise(to_np(dE), rE))
     if mask is not None:
         assert np.all(to_np(kl)[mask == 0] == 0) and np.all(to_np(dH)[mask == 0] == 0)
+
+
+# ---- vocabulary parallel (shards run one after another on one GPU) ---------
+N_VP_CASES = 8
+
+
+@pytest.mark.parametrize("k", range(N_VP_CASES))
+def test_random_vocab_parallel_case_matches_oracle(k):
+    from linear_cross_entropy_cce_b200 import vocab_parallel as vp
+    wl, _ = _draw(100 + k)
+    rng = np.random.default_rng(9000 + k)
+    R = int(rng.integers(2, 6))
+    eps = EPS_BF16 if rng.random() < 0.5 else 0.0
+    x = syn.make_inputs(wl, seed=100 + k)
+    H, segs, y = upload(x)
+    parts = []
+    shards = [vp.shard_segments(segs, v0, v1) for v0, v1 in vp.shard_ranges(wl.V, R)]
+    for local in shards:
+        if not local:  # a rank whose range holds no live ids
+            parts.append(torch.stack([torch.full((wl.N,), -float("inf"), device="cuda"),
+                                      torch.zeros(wl.N, device="cuda")]))
+            continue
+        zy_p, lse_p = cce.fwd(H, None, y, x.ignore_index, segments=local, V=wl.V, shard=True)
+        parts.append(torch.stack([lse_p, zy_p]))
+    loss, lse = cce.vocab_combine(torch.stack(parts), y, wl.V, x.ignore_index, list(wl.segs()))
+    rl, rlse = oracle.forward(x.H, x.segments, x.y, wl.V, x.ignore_index)
+    case = (wl, R, eps)
+    assert np.max(np.abs(to_np(loss) - rl), initial=0.0) <= TOL_ROW, case
+    assert np.max(np.abs(to_np(lse) - rlse), initial=0.0) <= TOL_ROW, case
+
+    dl = x.dloss_mean()
+    dlt = torch.from_numpy(dl).cuda()
+    dH = torch.zeros((wl.N, wl.D), dtype=torch.float32, device="cuda")
+    dE = {}
+    for local in shards:
+        if not local:
+            continue
+        dH_p, dEs, _ = cce.bwd(H, None, y, lse, dlt, x.ignore_index, segments=local, V=wl.V,
+                               filter_eps=eps, fp32_dh=True, shard=True)
+        dH += dH_p
+        for (b, e, _), g in zip(local, dEs):
+            dE[(b, e)] = g
+    torch.cuda.synchronize()
+    rH, rE = oracle.backward(x.H, x.segments, x.y, wl.V, dl, x.ignore_index, filter_eps=eps)
+    tol = TOL_GRAD_FILTER if eps > 0 else TOL_GRAD
+    assert _close(to_np(dH), rH, tol), (case, normwise(to_np(dH), rH))
+    for (b, e, _), r in zip(x.segments, rE):
+        got = torch.cat([dE[kk] for kk in sorted(dE) if b <= kk[0] < e]).float().cpu().numpy()
+        assert got.shape == r.shape, case
+        assert _close(got, r, tol), (case, normwise(got, r))
