@@ -20,7 +20,10 @@
  * Conventions shared by every entry point
  *   - Layouts are row-major and dense: H [N, D] bf16, E [V_s, D] bf16 per
  *     segment, y [N] int32.  D must be a positive multiple of 8 (16-byte rows,
- *     a TMA requirement); every device pointer must be 16-byte aligned.
+ *     a TMA requirement) and at most 65536; every device pointer must be
+ *     16-byte aligned.  0 <= N and 0 < V, both at most 2^31 - 257 (ids and
+ *     row indices are int32 on the device).  Sizes outside these ranges give
+ *     CCE_EINVAL, and a workspace size of 0.
  *   - All pointers except the ones marked "host" are device pointers.  The
  *     caller owns every buffer, including the workspace; the library never
  *     allocates device memory and never synchronises the stream.

@@ -50,6 +50,21 @@ def test_workspace_sizes_and_invalid_sizes():
     assert L.cce_vocab_sort_workspace_size(256, 4096, 0) > 0
 
 
+def test_size_limits_are_enforced():
+    L = cce.lib()
+    top = 2 ** 31 - 257
+    assert L.cce_fwd_workspace_size(1, 8, top, 0) > 0
+    assert L.cce_fwd_workspace_size(1, 8, top + 1, 0) == 0
+    assert L.cce_fwd_workspace_size(top + 1, 8, 16, 0) == 0
+    assert L.cce_fwd_workspace_size(1, 65536, 16, 0) > 0
+    assert L.cce_fwd_workspace_size(1, 65544, 16, 0) == 0
+    assert L.cce_bwd_workspace_size(1, 8, top + 1, 0, 0) == 0
+    assert L.cce_bwd_workspace_size(1, 65544, 16, 0, 0) == 0
+    assert _null_fwd(V=top + 1) == cce.CCE_EINVAL
+    assert _null_fwd(N=top + 1) == cce.CCE_EINVAL
+    assert _null_fwd(D=65544) == cce.CCE_EINVAL
+
+
 def test_workspace_is_far_below_materialised_logits():
     """The page on chunking CE after an OOM prints 12.2 GB for one bf16
     softmax over 24,576 positions x 248,320 vocabulary; the research-map
