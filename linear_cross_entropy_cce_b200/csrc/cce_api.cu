@@ -58,6 +58,16 @@ constexpr bool kPairDEDH = CCE_PAIR_DEDH != 0;
 #ifndef CCE_PAIR_G
 #define CCE_PAIR_G 1
 #endif
+// Tensor-core kernels are launched with programmatic stream serialization
+// (unless built with CCE_PDL=0): a launch may be scheduled while the
+// previous kernel in the stream drains, and its CTAs wait in-kernel
+// (griddepcontrol.wait) for that kernel to complete before touching global
+// memory, so the gap between dependent launches shrinks; most of the
+// backward's launches per chunk exit at once on chunks of the other route.
+#ifndef CCE_PDL
+#define CCE_PDL 1
+#endif
+constexpr bool kPDL = CCE_PDL != 0;
 constexpr bool kPairG = CCE_PAIR_G != 0;
 // The cross-entropy forward runs on CTA pairs (256 x 256 tiles) unless built
 // with CCE_PAIR_FWD=0.
@@ -487,11 +497,22 @@ int launch_tc(const typename Policy::Params& prm, int grid, cudaStream_t st, int
   constexpr int smem = smem_bytes<Policy>();
   static_assert(smem <= 232448, "shared memory per CTA exceeds 227 KB");
   if (!smem_attribute_once<Policy, false>(k, smem)) return CCE_ELAUNCH;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(tc_threads<Policy>(), 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = kPDL ? 1 : 0;
   const long slot = timing_begin(cls, st);
-  k<<<grid, tc_threads<Policy>(), smem, st>>>(prm);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, prm);
   timing_end(slot, st);
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  return cudaGetLastError() == cudaSuccess ? CCE_OK : CCE_ELAUNCH;
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? CCE_OK : CCE_ELAUNCH;
 }
 
 // Launch of a CTA-pair kernel: clusters of two CTAs along x; `pairs` pairs.
@@ -507,13 +528,15 @@ int launch_tc_pair(const typename Policy::Params& prm, int pairs, cudaStream_t s
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = kPDL ? 2 : 1;
   const long slot = timing_begin(cls, st);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, k, prm);
   timing_end(slot, st);

@@ -767,6 +767,10 @@ __global__ void __launch_bounds__(tc_threads<Policy>(), 1)
   Ctl* ctl = reinterpret_cast<Ctl*>(extra + Policy::EXTRA_SMEM);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // launched with programmatic serialization: nothing of global memory is
+  // touched before the previous grid in the stream has completed
+  grid_dep_launch();
+  grid_dep_wait();
   if (!Policy::active(p)) return;  // nothing to do in this launch: skip all set-up
 
   if (threadIdx.x == 0) {
@@ -843,6 +847,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   PairCtlT<G::NST>* ctl = reinterpret_cast<PairCtlT<G::NST>*>(extra + Policy::EXTRA_SMEM);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  grid_dep_launch();  // as in tc_kernel
+  grid_dep_wait();
   // active() depends only on the parameters and on device values every CTA
   // reads alike, so both CTAs of a pair leave here together or not at all
   if (!Policy::active(p)) return;

@@ -116,6 +116,16 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
+// Programmatic dependent launch.  grid_dep_wait: block until the grids this
+// launch depends on in its stream have completed and their memory operations
+// are visible (returns at once for a launch without the programmatic
+// attribute).  grid_dep_launch: allow the next launch in the stream, if it
+// carries the attribute, to be scheduled before this grid completes (its
+// CTAs then take SMs as this grid's CTAs leave, and wait in grid_dep_wait).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
