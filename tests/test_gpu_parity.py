@@ -372,3 +372,42 @@ def test_mispredicted_chunks_and_mixed_routes():
     assert per_chunk[0] < 1024 and per_chunk[2] < 1024  # sparse
     # the hot columns' dE rows are the large ones, and they are right
     assert normwise(to_np(dE)[hot], rE[0][hot]) <= TOL_GRAD_FILTER
+
+
+@pytest.mark.parametrize("eps", [0.0, EPS_BF16])
+def test_maximum_segment_count(eps):
+    """CCE_MAX_SEGMENTS (8) segments: single-id segments, gaps of one id and
+    of thousands, a segment ending at V; peaky logits so that filtered chunks
+    take the sparse route, with the vocabulary sort and the tile skip.  The
+    backward's workspace is sized for exactly 8 segments (each can add one
+    partial chunk to the sparse lists)."""
+    from linear_cross_entropy_cce_b200 import cce
+    segs = ((0, 1), (5, 6), (100, 3000), (3001, 3002), (4000, 9000), (9100, 9101),
+            (12000, 19000), (19999, 20000))
+    wl = syn.Workload("max_segs", N=500, D=64, V=20000, logit_std=16.0, ignore_frac=0.1,
+                      segments=segs, segment_mix=tuple(float(e - b) for b, e in segs))
+    x = syn.make_inputs(wl, seed=41)
+    H, dsegs, y = upload(x)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    loss, lse, colmax = run_fwd(x, H, dsegs, y, want_colmax=True, status=st)
+    perm = cce.vocab_sort(colmax, y, wl.V, x.ignore_index, segments=list(segs))
+    dl = x.dloss_mean()
+    assert cce.bwd_workspace_size(wl.N, wl.D, wl.V, 8) > cce.bwd_workspace_size(wl.N, wl.D, wl.V, 1)
+    dH, dEs, _ = run_bwd(x, H, dsegs, y, lse, torch.from_numpy(dl).cuda(), filter_eps=eps,
+                         vocab_perm=perm if eps > 0 else None, colmax=colmax if eps > 0 else None,
+                         status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rl, rs = oracle.forward(x.H, x.segments, x.y, wl.V, x.ignore_index)
+    assert np.max(np.abs(to_np(loss) - rl)) <= TOL_ROW
+    assert np.max(np.abs(to_np(lse) - rs)) <= TOL_ROW
+    rH, rE = oracle.backward(x.H, x.segments, x.y, wl.V, dl, x.ignore_index, filter_eps=eps)
+    tol = TOL_GRAD_FILTER if eps > 0 else TOL_GRAD
+    assert normwise(to_np(dH), rH) <= tol
+    for g, r in zip(dEs, rE):
+        got = to_np(g)
+        assert got.shape == r.shape
+        if np.any(r):
+            assert normwise(got, r) <= tol
+        else:
+            assert np.max(np.abs(got)) <= 1e-6
