@@ -125,6 +125,44 @@ def _require_cuda(*ts: torch.Tensor):
 SegSpec = Tuple[int, int, torch.Tensor]  # (vocab_begin, vocab_end, E_s)
 
 
+def _expect(t: Optional[torch.Tensor], name: str, dtype, shape):
+    """The C ABI takes bare pointers and trusts the sizes it is given, so a
+    tensor of the wrong type or shape would be read or written out of
+    bounds: refuse it here."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise CCEError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise CCEError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _expect_status(st: Optional[torch.Tensor]):
+    if st is not None and (st.dtype != torch.int32 or st.numel() < 1):
+        raise CCEError("status must be an int32 tensor of at least one element")
+
+
+def _rows(H: torch.Tensor, name: str = "H") -> Tuple[int, int]:
+    if H.dim() != 2 or H.dtype != torch.bfloat16:
+        raise CCEError(f"{name} must be a 2-D bfloat16 tensor, got {H.dtype} {tuple(H.shape)}")
+    return int(H.shape[0]), int(H.shape[1])
+
+
+def _check_head(E: Optional[torch.Tensor], segments, D: int):
+    """E [V, D] bf16, or each segment's E_s [end - begin, D] bf16."""
+    if segments:
+        for k, s in enumerate(segments):
+            b, e = int(s[0]), int(s[1])
+            if e <= b:
+                raise CCEError(f"segment {k} is empty or reversed: [{b}, {e})")
+            if len(s) > 2:
+                _expect(s[2], f"segment {k} E", torch.bfloat16, (e - b, D))
+    elif E is None:
+        raise CCEError("E is required when no segments are given")
+    else:
+        _expect(E, "E", torch.bfloat16, (int(E.shape[0]), D))
+
+
 def _seg_array(segments: Optional[Sequence], dEs=None, comps=None):
     if not segments:
         return None, 0
@@ -177,13 +215,16 @@ def fwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, ignore_inde
     shard=True runs cce_fwd_shard instead and returns (zy_part, lse_part)
     in place of (loss, lse): the correct-token logit when this shard holds
     the target (else 0) and the log-sum-exp over this shard."""
-    N, D = H.shape
+    N, D = _rows(H)
+    _check_head(E, segments, D)
     if segments:
         V = V if V is not None else int(segments[-1][1])
         v_live = sum(int(e) - int(b) for b, e, *_ in segments)
     else:
         V = int(E.shape[0])
         v_live = V
+    _expect(y, "y", torch.int32, (N,))
+    _expect_status(status)
     _require_cuda(H, E, y, *[s[2] for s in (segments or [])])
     dev = H.device
     loss = torch.empty(N, dtype=torch.float32, device=dev)
@@ -218,9 +259,9 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
     exact tile skip when filtering.  fp32_dh=True returns dH in fp32 with dE
     in bf16.  Returns (dH, dE, debug_keep or None).
     """
-    N, D = H.shape
+    N, D = _rows(H)
+    _check_head(E, segments, D)
     dev = H.device
-    _require_cuda(H, E, y, lse, dloss, vocab_perm, colmax)
     gdt = torch.float32 if fp32_grads else torch.bfloat16
     if segments:
         V = V if V is not None else int(segments[-1][1])
@@ -228,15 +269,32 @@ def bwd(H: torch.Tensor, E: Optional[torch.Tensor], y: torch.Tensor, lse: torch.
     else:
         V = int(E.shape[0])
         shapes = [(V, D)]
+    v_live = sum(r for r, _ in shapes)
+    for t, name in ((y, "y"),):
+        _expect(t, name, torch.int32, (N,))
+    for t, name in ((lse, "lse"), (dloss, "dloss")):
+        _expect(t, name, torch.float32, (N,))
+    _expect(vocab_perm, "vocab_perm", torch.int32, (v_live,))
+    _expect(colmax, "colmax", torch.float32, (v_live,))
+    _expect_status(status)
     if dE_out is None:
         if kahan:
             raise CCEError("kahan accumulation needs dE_out and dE_comp")
         dEs = [torch.empty(s, dtype=gdt, device=dev) for s in shapes]
     else:
         dEs = list(dE_out) if isinstance(dE_out, (list, tuple)) else [dE_out]
+        if len(dEs) != len(shapes):
+            raise CCEError(f"dE_out must hold {len(shapes)} tensor(s), one per segment")
+        for k, (t, shp) in enumerate(zip(dEs, shapes)):
+            _expect(t, f"dE_out[{k}]", torch.bfloat16 if kahan else gdt, shp)
     comps = None
     if kahan:
         comps = list(dE_comp) if isinstance(dE_comp, (list, tuple)) else [dE_comp]
+        if len(comps) != len(shapes):
+            raise CCEError(f"dE_comp must hold {len(shapes)} tensor(s), one per segment")
+        for k, (t, shp) in enumerate(zip(comps, shapes)):
+            _expect(t, f"dE_comp[{k}]", torch.bfloat16, shp)
+    _require_cuda(H, E, y, lse, dloss, vocab_perm, colmax, *dEs, *(comps or []))
     dH = torch.empty((N, D), dtype=torch.float32 if fp32_dh else gdt, device=dev)
     flags = ((KAHAN_DE if kahan else 0) | (FP32_GRADS if fp32_grads else 0) |
              (FULL_DE if full_de else 0) | (VOCAB_SHARD if shard else 0) |
@@ -263,6 +321,11 @@ def vocab_sort(colmax: Optional[torch.Tensor], y: torch.Tensor, V: int, ignore_i
     fwd / bwd (the head rows themselves are not read)."""
     dev = y.device
     v_live = sum(int(e) - int(b) for b, e, *_ in segments) if segments else V
+    if y.dim() != 1:
+        raise CCEError("y must be 1-D")
+    _expect(y, "y", torch.int32, (y.numel(),))
+    _expect(colmax, "colmax", torch.float32, (v_live,))
+    _require_cuda(y, colmax)
     perm = torch.empty(v_live, dtype=torch.int32, device=dev)
     segarr, nseg = _seg_array(segments)
     ws = _workspace(vocab_sort_workspace_size(y.numel(), V, nseg), dev, workspace)
@@ -340,12 +403,24 @@ def bf16_from_bits(bits, device) -> torch.Tensor:
     return t.to(device).view(torch.bfloat16)
 
 
+def _check_kl(Hs, Es, Ht, Et, row_mask) -> Tuple[int, int, int]:
+    N, D = _rows(Hs, "Hs")
+    if Es is None or Et is None:
+        raise CCEError("Es and Et are required")
+    V = int(Es.shape[0])
+    _expect(Ht, "Ht", torch.bfloat16, (N, D))
+    _expect(Es, "Es", torch.bfloat16, (V, D))
+    _expect(Et, "Et", torch.bfloat16, (V, D))
+    _expect(row_mask, "row_mask", torch.int32, (N,))
+    return N, D, V
+
+
 def kl_fwd(Hs: torch.Tensor, Es: torch.Tensor, Ht: torch.Tensor, Et: torch.Tensor,
            row_mask: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
            status: Optional[torch.Tensor] = None):
     """Per-row (KL(p_t || p_s), lse_s, lse_t) fp32.  See cce_kl_fwd."""
-    N, D = Hs.shape
-    V = int(Es.shape[0])
+    N, D, V = _check_kl(Hs, Es, Ht, Et, row_mask)
+    _expect_status(status)
     _require_cuda(Hs, Es, Ht, Et, row_mask)
     dev = Hs.device
     kl = torch.empty(N, dtype=torch.float32, device=dev)
@@ -368,9 +443,17 @@ def kl_bwd(Hs: torch.Tensor, Es: torch.Tensor, Ht: torch.Tensor, Et: torch.Tenso
            status: Optional[torch.Tensor] = None):
     """Student gradients (dH, dE) of sum_i dloss_i KL_i.  See cce_kl_bwd.
     With debug_rows > 0 returns (dH, dE, keep bits [debug_rows, ceil(V/32)])."""
-    N, D = Hs.shape
-    V = int(Es.shape[0])
-    _require_cuda(Hs, Es, Ht, Et, lse_s, lse_t, dloss, row_mask)
+    N, D, V = _check_kl(Hs, Es, Ht, Et, row_mask)
+    for t, name in ((lse_s, "lse_s"), (lse_t, "lse_t"), (dloss, "dloss")):
+        _expect(t, name, torch.float32, (N,))
+    _expect_status(status)
+    if dE_out is not None:
+        _expect(dE_out, "dE_out", torch.bfloat16 if kahan else
+                (torch.float32 if fp32_grads else torch.bfloat16), (V, D))
+    if kahan:
+        _expect(dE_comp, "dE_comp", torch.bfloat16, (V, D))
+    _require_cuda(Hs, Es, Ht, Et, lse_s, lse_t, dloss, row_mask, dE_out,
+                  dE_comp if kahan else None)
     dev = Hs.device
     gdt = torch.float32 if fp32_grads else torch.bfloat16
     if kahan and (dE_out is None or dE_comp is None):
