@@ -162,3 +162,46 @@ def test_kl_filter_criterion_per_element(case):
     if mask is not None:  # masked rows keep nothing
         assert not kept[mask == 0].any()
     assert dropped.any() and k.any()  # the criterion is exercised both ways
+
+
+@pytest.mark.parametrize("shared", [True, False])
+def test_kl_kahan_accumulation_beats_plain_bf16_and_is_deterministic(shared):
+    """The KL backward's classifier gradient accumulated with CCE_KAHAN_DE over
+    128 micro-batches (8 batches cycled 16 times): a plain bf16 running sum
+    of the oracle's exact parts drifts past the 1e-2 tolerance, while the
+    GPU's Kahan pair (s, c) gives s - c within half of it and at least 4x
+    closer to the exactly rounded sum; two runs agree bit for bit."""
+    from linear_cross_entropy_cce_b200 import cce
+    N, D, V, K = 256, 128, 1024, 128
+    cases = [_kl_case(N, D, V, 2.0, 3.0, shared, seed=60 + s, masked=False) for s in range(8)]
+    Es, Et = cases[0][1], cases[0][3]  # one student head (and teacher head) for every batch
+    Es_d = _up(Es)
+    Et_d = Es_d if shared else _up(Et)
+    dl = np.full(N, 1.0 / N)
+    dev = []
+    for Hs, _, Ht, _, _ in cases:
+        Hs_d, Ht_d = _up(Hs), _up(Ht)
+        _, ls, lt = cce.kl_fwd(Hs_d, Es_d, Ht_d, Et_d)
+        dev.append((Hs_d, Ht_d, ls, lt))
+    dlt = torch.from_numpy(dl).float().cuda()
+    finals = []
+    for rep in range(2):
+        S = torch.zeros((V, D), dtype=torch.bfloat16, device="cuda")
+        C = torch.zeros_like(S)
+        for k in range(K):
+            Hs_d, Ht_d, ls, lt = dev[k % 8]
+            cce.kl_bwd(Hs_d, Es_d, Ht_d, Et_d, ls, lt, dlt, kahan=True, dE_out=S, dE_comp=C)
+        torch.cuda.synchronize()
+        finals.append((S.clone(), C.clone()))
+    assert torch.equal(finals[0][0], finals[1][0]) and torch.equal(finals[0][1], finals[1][1])
+    parts = [oracle.kl_backward(Hs, Es, Ht, Et, dl)[1] for Hs, _, Ht, _, _ in cases]
+    exact = oracle.kahan_reference([parts[k % 8] for k in range(K)])
+    plain = np.zeros_like(exact)
+    for k in range(K):  # bf16 storage, exact parts, rounded after every add
+        plain = oracle.widen_bf16(syn.fp32_to_bf16_bits((plain + parts[k % 8]).astype(np.float32)))
+    err_plain = normwise(plain, exact)
+    S, C = finals[0]
+    err_kahan = normwise(to_np(S) - to_np(C), exact)
+    assert err_plain > TOL_GRAD, err_plain
+    assert err_kahan <= TOL_GRAD / 2, err_kahan
+    assert err_plain >= 4 * err_kahan, (err_plain, err_kahan)
