@@ -150,20 +150,26 @@ def test_random_vocab_parallel_case_matches_oracle(k):
     rng = np.random.default_rng(9000 + k)
     R = int(rng.integers(2, 6))
     eps = EPS_BF16 if rng.random() < 0.5 else 0.0
+    # filtered cases sort each shard's vocabulary by its column maxima, as
+    # the vocabulary-parallel step of the benchmark does
+    sort = eps > 0 and bool(np.random.default_rng(9500 + k).random() < 0.7)
     x = syn.make_inputs(wl, seed=100 + k)
     H, segs, y = upload(x)
-    parts = []
+    parts, colmaxes = [], []
     shards = [vp.shard_segments(segs, v0, v1) for v0, v1 in vp.shard_ranges(wl.V, R)]
     for local in shards:
         if not local:  # a rank whose range holds no live ids
             parts.append(torch.stack([torch.full((wl.N,), -float("inf"), device="cuda"),
                                       torch.zeros(wl.N, device="cuda")]))
+            colmaxes.append(None)
             continue
-        zy_p, lse_p = cce.fwd(H, None, y, x.ignore_index, segments=local, V=wl.V, shard=True)
-        parts.append(torch.stack([lse_p, zy_p]))
+        out = cce.fwd(H, None, y, x.ignore_index, segments=local, V=wl.V, shard=True,
+                      want_colmax=sort)
+        parts.append(torch.stack([out[1], out[0]]))
+        colmaxes.append(out[2] if sort else None)
     loss, lse = cce.vocab_combine(torch.stack(parts), y, wl.V, x.ignore_index, list(wl.segs()))
     rl, rlse = oracle.forward(x.H, x.segments, x.y, wl.V, x.ignore_index)
-    case = (wl, R, eps)
+    case = (wl, R, eps, sort)
     assert np.max(np.abs(to_np(loss) - rl), initial=0.0) <= TOL_ROW, case
     assert np.max(np.abs(to_np(lse) - rlse), initial=0.0) <= TOL_ROW, case
 
@@ -171,11 +177,14 @@ def test_random_vocab_parallel_case_matches_oracle(k):
     dlt = torch.from_numpy(dl).cuda()
     dH = torch.zeros((wl.N, wl.D), dtype=torch.float32, device="cuda")
     dE = {}
-    for local in shards:
+    for local, cm in zip(shards, colmaxes):
         if not local:
             continue
+        perm = (cce.vocab_sort(cm, y, wl.V, x.ignore_index, segments=[s_[:2] for s_ in local])
+                if sort else None)
         dH_p, dEs, _ = cce.bwd(H, None, y, lse, dlt, x.ignore_index, segments=local, V=wl.V,
-                               filter_eps=eps, fp32_dh=True, shard=True)
+                               filter_eps=eps, vocab_perm=perm, colmax=cm, fp32_dh=True,
+                               shard=True)
         dH += dH_p
         for (b, e, _), g in zip(local, dEs):
             dE[(b, e)] = g
