@@ -439,3 +439,22 @@ def test_maximum_width(eps):
     tol = TOL_GRAD_FILTER if eps > 0 else TOL_GRAD
     assert normwise(to_np(dH), rH) <= tol
     assert normwise(to_np(dEs[0]), rE[0]) <= tol
+
+
+@pytest.mark.parametrize("N,D,V", [(300000, 16, 5), (3, 8, 3000000)])
+@pytest.mark.parametrize("eps", [0.0, EPS_BF16])
+def test_extreme_aspect_ratios(N, D, V, eps):
+    """Very many rows over a tiny head (row compaction, scans and the row
+    gathers at scale: 2344 row blocks) and a handful of rows over a very
+    wide head (11719 vocabulary tiles, many backward chunks and list slots)."""
+    wl = syn.Workload(f"aspect{N}x{V}", N=N, D=D, V=V, logit_std=3.0, ignore_frac=0.3)
+    x = syn.make_inputs(wl, seed=47)
+    H, segs, y, lse = _fwd_check(x)
+    dl = x.dloss_mean()
+    dH, dEs, _ = run_bwd(x, H, segs, y, lse, torch.from_numpy(dl).cuda(), filter_eps=eps)
+    torch.cuda.synchronize()
+    rH, rE = oracle.backward(x.H, x.segments, x.y, V, dl, x.ignore_index, filter_eps=eps)
+    tol = TOL_GRAD_FILTER if eps > 0 else TOL_GRAD
+    assert normwise(to_np(dH), rH) <= tol
+    assert normwise(to_np(dEs[0]), rE[0]) <= tol
+    assert np.all(to_np(dH)[~x.valid] == 0)
