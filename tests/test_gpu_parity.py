@@ -458,3 +458,35 @@ def test_extreme_aspect_ratios(N, D, V, eps):
     assert normwise(to_np(dH), rH) <= tol
     assert normwise(to_np(dEs[0]), rE[0]) <= tol
     assert np.all(to_np(dH)[~x.valid] == 0)
+
+
+@pytest.mark.parametrize("ign", [7, -1])
+def test_other_ignore_index_values(ign):
+    """ignore_index is any int32: a valid vocabulary id (rows whose target is
+    id 7 are then ignored, and id 7 gets no one-hot term) or another negative
+    value (rows with -1 ignored).  Compared with the oracle called with the
+    same ignore_index."""
+    from linear_cross_entropy_cce_b200 import cce
+    wl = syn.Workload("ign", N=400, D=64, V=300, logit_std=2.0, ignore_frac=0.0, targets="uniform")
+    x = syn.make_inputs(wl, seed=51)
+    y = x.y.copy()
+    y[:40] = ign           # forty ignored rows
+    if ign == 7:
+        y[40:45] = 7       # more rows on id 7: ignored too
+    Hd = cce.bf16_from_bits(x.H, "cuda")
+    Ed = cce.bf16_from_bits(x.segments[0][2], "cuda")
+    yd = torch.from_numpy(y).cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    loss, lse = cce.fwd(Hd, Ed, yd, ign, status=st)
+    valid = y != ign
+    dl = np.where(valid, 1.0 / valid.sum(), 0.0).astype(np.float32)
+    dH, dE, _ = cce.bwd(Hd, Ed, yd, lse, torch.from_numpy(dl).cuda(), ign, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rl, rs = oracle.forward(x.H, x.segments, y, wl.V, ign)
+    assert np.max(np.abs(to_np(loss) - rl)) <= TOL_ROW
+    assert np.all(to_np(loss)[~valid] == 0) and np.all(to_np(lse)[~valid] == 0)
+    rH, rE = oracle.backward(x.H, x.segments, y, wl.V, dl, ign)
+    assert normwise(to_np(dH), rH) <= TOL_GRAD
+    assert normwise(to_np(dE), rE[0]) <= TOL_GRAD
+    assert np.all(to_np(dH)[~valid] == 0)
