@@ -205,3 +205,30 @@ def test_kl_kahan_accumulation_beats_plain_bf16_and_is_deterministic(shared):
     assert err_plain > TOL_GRAD, err_plain
     assert err_kahan <= TOL_GRAD / 2, err_kahan
     assert err_plain >= 4 * err_kahan, (err_plain, err_kahan)
+
+
+@pytest.mark.parametrize("N,D,V,shared", [(3, 8, 2000000, True), (200000, 16, 6, False)])
+@pytest.mark.parametrize("eps", [0.0, EPS_BF16])
+def test_kl_extreme_aspect_ratios(N, D, V, shared, eps):
+    """A few rows over a very wide head (shared: the CTA-pair G producer over
+    7813 tiles) and very many rows over a tiny one (separate heads)."""
+    from linear_cross_entropy_cce_b200 import cce
+    Hs, Es, Ht, Et, mask = _kl_case(N, D, V, 3.0, 2.0, shared, seed=71, masked=True)
+    tm = torch.from_numpy(mask).cuda()
+    Hs_d, Es_d, Ht_d = _up(Hs), _up(Es), _up(Ht)
+    Et_d = Es_d if shared else _up(Et)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kl, ls, lt = cce.kl_fwd(Hs_d, Es_d, Ht_d, Et_d, tm, status=st)
+    dl = np.full(N, 1.0 / N)
+    dH, dE = cce.kl_bwd(Hs_d, Es_d, Ht_d, Et_d, ls, lt, torch.from_numpy(dl).float().cuda(), tm,
+                        filter_eps=eps, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rk, rls, rlt = oracle.kl_forward(Hs, Es, Ht, Et, mask)
+    assert np.max(np.abs(to_np(kl) - rk)) <= TOL_ROW
+    assert np.max(np.abs(to_np(ls) - rls)) <= TOL_ROW
+    assert np.max(np.abs(to_np(lt) - rlt)) <= TOL_ROW
+    rH, rE = oracle.kl_backward(Hs, Es, Ht, Et, dl, mask, filter_eps=eps)
+    tol = TOL_GRAD_FILTER if eps > 0 else TOL_GRAD
+    assert normwise(to_np(dH), rH) <= tol
+    assert normwise(to_np(dE), rE) <= tol
