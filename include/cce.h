@@ -178,7 +178,8 @@ int cce_vocab_combine(const float* parts, int32_t R, const int32_t* y, int64_t N
 /* Workspace bytes cce_bwd needs (0 on invalid sizes).  n_segs is the count
  * the cce_bwd call will pass (0 for a contiguous E): each segment can add one
  * partial vocabulary chunk to the sparse lists, so a workspace sized for fewer
- * segments than the call uses is rejected by the call with CCE_EWORKSPACE. */
+ * segments than the call uses is rejected by the call with CCE_EWORKSPACE;
+ * one sized for more (CCE_MAX_SEGMENTS, say) is always enough. */
 size_t cce_bwd_workspace_size(int64_t N, int64_t D, int64_t V, int32_t n_segs,
                               uint32_t flags);
 

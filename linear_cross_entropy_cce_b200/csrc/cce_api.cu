@@ -344,15 +344,20 @@ int64_t best_dE_width(int64_t V, int64_t D, int64_t lo, int64_t hi, int rows, in
 // and are then trimmed to the width below that cap whose dE contraction
 // wastes the least of its last waves.
 // nseg: the head's segments (0: one segment); each adds at most one chunk.
+// The chunk widths are chosen as if the call had CCE_MAX_SEGMENTS segments,
+// so only the list slots depend on nseg: the workspace size never shrinks as
+// nseg grows, and a workspace sized for more segments than a call uses is
+// always enough.
 BwdPlan plan_bwd(int64_t N, int64_t D, int64_t V, uint32_t flags, bool kl = false, int nseg = 0) {
-  BwdPlan p = plan_bwd_widths(N, D, V, flags, kl, INT64_MAX, INT64_MAX, nseg);
+  constexpr int kWidthSegs = CCE_MAX_SEGMENTS;
+  BwdPlan p = plan_bwd_widths(N, D, V, flags, kl, INT64_MAX, INT64_MAX, kWidthSegs);
   const double bound = (double)N * (double)V * 2.0 / 8.0;
   // small problems are left alone: their scratch is a few MB whatever the
   // logits, and narrow chunks would only add launches
-  if (!kCapChunkToEighth || bound < (double)(64u << 20)) return p;
-  if ((double)p.part_logits < bound) return p;
+  if (!kCapChunkToEighth || bound < (double)(64u << 20) || (double)p.part_logits < bound)
+    return plan_bwd_widths(N, D, V, flags, kl, INT64_MAX, INT64_MAX, nseg);
   while ((double)p.part_logits >= bound && p.Vc_f > BN)
-    p = plan_bwd_widths(N, D, V, flags, kl, p.Vc_f - BN, p.Vc_f - BN, nseg);
+    p = plan_bwd_widths(N, D, V, flags, kl, p.Vc_f - BN, p.Vc_f - BN, kWidthSegs);
   // the dE contraction runs on CTA pairs (256-row tiles, kPlanSMs / 2 at
   // once), except the soft-target KL's filtered chunks (single CTAs, 128-row
   // tiles)

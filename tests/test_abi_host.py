@@ -216,3 +216,26 @@ def test_plain_c_consumer(tmp_path):
     out = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert out.returncode == 0, out.stderr
     assert "c abi ok" in out.stdout
+
+
+def test_workspace_plan_invariants_over_random_shapes():
+    """For seeded random shapes, segment counts and flags: the three size
+    classes add up to the workspace size, the size grows with n_segs, and on
+    heads whose bf16 logits exceed 512 MiB (N V 2 / 8 >= 64 MiB) the
+    logits-class buffers stay below an eighth of them (no buffer of the
+    logits' size)."""
+    import numpy as np
+    rng = np.random.default_rng(2024)
+    for _ in range(300):
+        N = int(rng.integers(1, 1 << 16))
+        D = 8 * int(rng.integers(1, 1025))
+        V = int(rng.integers(1, 1 << 19))
+        nseg = int(rng.integers(0, 9))
+        flags = int(rng.choice([0, cce.KAHAN_DE, cce.FULL_DE, cce.FP32_GRADS]))
+        total = cce.bwd_workspace_size(N, D, V, nseg, flags)
+        parts = cce.bwd_workspace_parts(N, D, V, nseg, flags)
+        assert total > 0 and sum(parts.values()) == total, (N, D, V, nseg, flags)
+        assert cce.bwd_workspace_size(N, D, V, min(8, nseg + 1), flags) >= total
+        bound = N * V * 2 / 8
+        if bound >= 64 * 2 ** 20:
+            assert parts["logits"] < bound, (N, D, V, nseg, flags, parts["logits"], bound)
