@@ -251,7 +251,9 @@ FwdPlan plan_fwd(int64_t N, int64_t D, int64_t V, int32_t n_segs) {
   FwdPlan p;
   p.Npad = std::max<int64_t>(BM, cdiv(N, BM) * BM);
   p.T_v_max = (int)(cdiv(V, BN) + std::max(1, (int)n_segs));
-  p.tpi = fwd_tiles_per_item(p.Npad, D, p.T_v_max, kPairFwd);
+  // tiles per item as if the call had the most segments, so the partial
+  // buffer (S_max rows of partials) never shrinks as n_segs grows
+  p.tpi = fwd_tiles_per_item(p.Npad, D, cdiv(V, BN) + CCE_MAX_SEGMENTS, kPairFwd);
   p.S_max = (int)cdiv(p.T_v_max, p.tpi);
   size_t o = 0;
   p.off_nvalid = o; o += align_up(16);

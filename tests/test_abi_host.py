@@ -239,3 +239,7 @@ def test_workspace_plan_invariants_over_random_shapes():
         bound = N * V * 2 / 8
         if bound >= 64 * 2 ** 20:
             assert parts["logits"] < bound, (N, D, V, nseg, flags, parts["logits"], bound)
+        # the forward's and the sort's scratch never shrink with more segments either
+        more = min(8, nseg + 1)
+        assert cce.fwd_workspace_size(N, D, V, more) >= cce.fwd_workspace_size(N, D, V, nseg) > 0
+        assert cce.vocab_sort_workspace_size(N, V, more) >= cce.vocab_sort_workspace_size(N, V, nseg) > 0
